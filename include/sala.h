@@ -1,0 +1,190 @@
+/*
+ * sala.h -- C ABI of the SALA hybrid-attention hot path (libsala, CUDA sm_100a).
+ *
+ * Four operations, after the MiniCPM-SALA pages:
+ *   - Lightning linear attention, prefill and single-token decode
+ *     (state recurrence S_t = S_{t-1} + k_t v_t^T of the summary page,
+ *     "Prerequisites / Linear Attention"; QK-normalisation, GQA-to-MHA and the
+ *     output gate of the tech-report mirror, section 02 (3); RoPE in the linear
+ *     layers from section 02 (4), HyPE);
+ *   - InfLLM-v2-style block selection and block-sparse softmax attention
+ *     (tech-report mirror, section 02 (2): each query attends to a few selected
+ *     key/value blocks, sparse at long length and dense at standard length,
+ *     output gate; NoPE from section 02 (4); sliding window plus global anchors
+ *     from the summary page, "Prerequisites / Sparse Attention").
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Pointers.  Every tensor pointer is a DEVICE pointer on the current CUDA
+ *   device, except where a comment says otherwise.  The caller owns all memory;
+ *   the library never allocates, frees or synchronises (except
+ *   sala_get_device_error), and every launch is asynchronous on `stream`
+ *   (a cudaStream_t passed as void*; NULL = the legacy default stream).
+ * Layout.  Activations are [B, T, H, D] with element strides {b, t, h} given
+ *   in a sala_strides; the D stride is always 1.  Base pointers must be 16-byte
+ *   aligned and every stride times the element size a multiple of 16 bytes.
+ * Types.  SALA_BF16: bf16 activations, outputs written in bf16 (round to
+ *   nearest even).  SALA_F32: fp32 activations and outputs.  Accumulation is
+ *   fp32 everywhere; the Lightning state is always fp32.
+ * Errors.  Argument checks run on the host before any launch and return
+ *   SALA_ERR_INVALID_ARG / SALA_ERR_UNSUPPORTED without touching memory.  A
+ *   failed launch returns SALA_ERR_CUDA.  Conditions only the device can see
+ *   (a value outside the tensor-core operand range, a bounded wait that ran
+ *   out) set a device error word that sala_get_device_error() reports.
+ * Aliasing.  Outputs must not overlap inputs; `state` is read and written.
+ */
+#ifndef SALA_H
+#define SALA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SALA_OK = 0,
+    SALA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, stride or alignment */
+    SALA_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement */
+    SALA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
+    SALA_ERR_TIMEOUT = 4,      /* a device-side bounded wait ran out */
+    SALA_ERR_WORKSPACE = 5,    /* workspace missing or smaller than required */
+    SALA_ERR_RANGE = 6         /* a value left the fp16 operand range on the device */
+} sala_status;
+
+typedef enum { SALA_F32 = 0, SALA_BF16 = 1 } sala_dtype;
+
+/* Element strides of a [B, T, H, D] activation (the D stride is 1). */
+typedef struct {
+    int64_t b, t, h;
+} sala_strides;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *sala_status_string(sala_status s);
+
+/* Library version string, e.g. "sala-b200 0.1 (sm_100a)". */
+const char *sala_version(void);
+
+/*
+ * Lightning attention prefill (chunked).
+ *
+ * For each (b, h) and t = 0..T-1, with p = pos0 + t:
+ *   qh_t = RoPE_p(RMSNorm(q_t) * q_norm_w),  kh_t = RoPE_p(RMSNorm(k_t) * k_norm_w)
+ *   S_t  = S_{t-1} + kh_t v_t^T                  (S_{-1} = initial state)
+ *   o_t  = qh_t^T S_t                            (state inclusive of token t)
+ *   y_t  = sigmoid(g_t) * o_t   (elementwise; y_t = o_t when g == NULL)
+ * RMSNorm(x) = x / sqrt(mean(x^2) + eps) over D; RoPE is rotate-half: for
+ * i < D/2 the pair (x_i, x_{i+D/2}) turns by p * rope_base^(-2i/D).
+ * Chunked evaluation: O_c = (Q_c K_c^T masked s<=t) V_c + Q_c S_{c-1},
+ * S_c = S_{c-1} + K_c^T V_c, on tensor cores for bf16 with D = 128.
+ *
+ *   q, k, v, g  [B,T,H,D] activations (g may be NULL: no gate)
+ *   o           [B,T,H,D] output y
+ *   state       [B,H,D,D] fp32, contiguous, S[b][h][i][j] (i key dim, j value
+ *               dim).  In: the initial state (ignored when init_zero != 0).
+ *               Out: the state after token T-1.
+ *   q_norm_w, k_norm_w  [D] fp32 norm weights, or NULL for weight 1
+ *   D           64 or 128;  T >= 0 (T = 0 only copies/zeroes the state)
+ *   chunk       64 or 128 (tile length of the chunked evaluation)
+ *   pos0        position of token 0 (RoPE), >= 0
+ *   workspace   device scratch of at least sala_lightning_prefill_workspace()
+ *               bytes (may be NULL when that returns 0); contents are scratch
+ *   dt          SALA_BF16 (D = 64 or 128) or SALA_F32 (D = 64 or 128)
+ * Errors: INVALID_ARG (null q/k/v/o/state, bad sizes, strides or alignment),
+ *         UNSUPPORTED (other D/chunk/dtype), WORKSPACE, CUDA.  Device: RANGE
+ *         when a bf16-path tensor-core operand exceeds the fp16 range.
+ */
+size_t sala_lightning_prefill_workspace(int B, int T, int H, int D, int chunk, sala_dtype dt);
+
+sala_status sala_lightning_prefill(const void *q, const void *k, const void *v, const void *g,
+                                   void *o, float *state, const float *q_norm_w,
+                                   const float *k_norm_w, int B, int T, int H, int D,
+                                   sala_strides sq, sala_strides sk, sala_strides sv,
+                                   sala_strides sg, sala_strides so, int chunk, int64_t pos0,
+                                   float rope_base, float eps, int init_zero, void *workspace,
+                                   size_t workspace_bytes, sala_dtype dt, void *stream);
+
+/*
+ * Lightning attention decode: one new token per batch entry.
+ *   qh = RoPE_p(RMSNorm(q) * q_norm_w), kh likewise, p = pos[b]
+ *   S  <- S + kh v^T ;  o = qh^T S (updated state) ;  y = sigmoid(g) * o
+ *
+ *   q, k, v, g  [B,H,D] activations with strides {b, h} taken from the .b and
+ *               .h fields of the sala_strides (.t unused); g may be NULL
+ *   o           [B,H,D] output (strides `so`)
+ *   state       [B,H,D,D] fp32 contiguous, updated in place
+ *   pos         [B] int32 DEVICE array of positions (>= 0)
+ *   dt          SALA_BF16 or SALA_F32;  D = 64 or 128
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA.
+ */
+sala_status sala_lightning_decode(const void *q, const void *k, const void *v, const void *g,
+                                  void *o, float *state, const float *q_norm_w,
+                                  const float *k_norm_w, const int32_t *pos, int B, int H, int D,
+                                  sala_strides sq, sala_strides sk, sala_strides sv,
+                                  sala_strides sg, sala_strides so, float rope_base, float eps,
+                                  sala_dtype dt, void *stream);
+
+/*
+ * Block selection (InfLLM-v2 style, NoPE).
+ * For each (b, kv head hk, query row t), c = floor(t / block):
+ *   Kbar_j  = mean of the `block` keys of complete block j (fp32)
+ *   score_j = (1/sqrt(D)) * sum_{h in group(hk)} q_{t,h} . Kbar_j,
+ *             group(hk) = query heads hk*G .. hk*G+G-1, G = Hq / Hkv
+ *   candidates: complete blocks n_init <= j <= c - n_local
+ *   chosen: the top `topk` candidates (larger score first, ties -> smaller j),
+ *   united with the init blocks {0..n_init-1} and the local window
+ *   {c-n_local+1..c} (clipped to [0, c]); written sorted ascending and padded
+ *   with -1 to n_sel = n_init + topk + n_local entries.
+ * When every candidate fits the budget all causal blocks are chosen, which is
+ * the dense fallback.
+ *
+ *   q           [B,T,Hq,D], k [B,T,Hkv,D] (bf16)
+ *   idx         [B,Hkv,T,n_sel] int32 output, contiguous
+ *   ws          device scratch of >= sala_sparse_select_workspace() bytes
+ *   block = 64, 1 <= topk <= 256, 0 <= n_init, 1 <= n_local, D = 64 or 128,
+ *   Hq % Hkv == 0, Hq / Hkv <= 32.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
+ */
+size_t sala_sparse_select_workspace(int B, int T, int Hq, int Hkv, int D, int block);
+
+sala_status sala_sparse_select(const void *q, const void *k, int B, int T, int Hq, int Hkv,
+                               int D, sala_strides sq, sala_strides sk, int block, int topk,
+                               int n_init, int n_local, int32_t *idx, void *ws, size_t ws_bytes,
+                               sala_dtype dt, void *stream);
+
+/*
+ * Block-sparse softmax attention (NoPE, causal).
+ * For each (b, query head h, row t), hk = h / (Hq / Hkv):
+ *   keys = union of blocks [j*block, (j+1)*block) over the entries j >= 0 of
+ *          idx[b][hk][t][:], restricted to s <= t
+ *   o    = sum_s softmax_s(scale * q_{t,h} . k_s) v_s ;  y = sigmoid(g) * o
+ * An empty key set gives y = 0.  Entries of a row must be distinct; -1 entries
+ * are skipped.  The GQA group of hk shares the row's selection.
+ *
+ *   q, g, o     [B,T,Hq,D] (g may be NULL), k, v [B,T,Hkv,D] (bf16)
+ *   idx         [B,Hkv,T,n_sel] int32, contiguous, entries in [-1, ceil(T/block))
+ *   scale       softmax scale; 0 selects 1/sqrt(D)
+ *   block = 64, D = 64 or 128, Hq / Hkv = 16 (the GQA group fills one
+ *   16-row tensor-core tile).
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA.
+ */
+sala_status sala_sparse_attn(const void *q, const void *k, const void *v, const void *g,
+                             const int32_t *idx, int n_sel, void *o, int B, int T, int Hq,
+                             int Hkv, int D, sala_strides sq, sala_strides sk, sala_strides sv,
+                             sala_strides sg, sala_strides so, int block, float scale,
+                             sala_dtype dt, void *stream);
+
+/*
+ * Synchronise `stream`, then read and clear the device error word of the
+ * current device.  Returns SALA_OK, SALA_ERR_RANGE or SALA_ERR_TIMEOUT (the
+ * first condition raised since the last call), or SALA_ERR_CUDA if the
+ * synchronisation itself failed.
+ */
+sala_status sala_get_device_error(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SALA_H */

@@ -1,1 +1,224 @@
-"""B200-native SALA hybrid-attention hot path (placeholder; binding added with the library)."""
+"""B200-native SALA hybrid-attention hot path: thin Python binding over libsala.
+
+Every call below marshals torch CUDA tensors into the C ABI of ``include/sala.h``
+(pointers, sizes, element strides, the current CUDA stream) and raises
+``SalaError`` on a non-zero status.  All arithmetic runs in the CUDA kernels of
+``libsala.so``; there is no CPU or PyTorch fallback: if the library is missing
+the first call raises.  Outputs and scratch buffers not passed by the caller are
+allocated with torch (device memory is plumbing here).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "SalaError", "load_library", "lightning_prefill", "lightning_prefill_workspace",
+    "lightning_decode", "sparse_select", "sparse_select_workspace", "sparse_attn",
+    "get_device_error", "status_string", "version", "LIB_PATH",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsala.so")
+SALA_F32, SALA_BF16 = 0, 1
+_lib = None
+
+
+class SalaError(RuntimeError):
+    def __init__(self, fn: str, status: int, text: str):
+        super().__init__(f"{fn} failed: {text} ({status})")
+        self.status = status
+
+
+class SalaStrides(ctypes.Structure):
+    _fields_ = [("b", ctypes.c_int64), ("t", ctypes.c_int64), ("h", ctypes.c_int64)]
+
+
+def load_library(path: Optional[str] = None):
+    """Load libsala.so (raises OSError if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise OSError(f"libsala.so not found at {p}; build it with "
+                      "`python -m sparse_attention_long_lightning_b200.build`")
+    lib = ctypes.CDLL(p)
+    vp, i, i64, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    S = SalaStrides
+    lib.sala_status_string.argtypes = [i]
+    lib.sala_status_string.restype = ctypes.c_char_p
+    lib.sala_version.argtypes = []
+    lib.sala_version.restype = ctypes.c_char_p
+    lib.sala_lightning_prefill_workspace.argtypes = [i, i, i, i, i, i]
+    lib.sala_lightning_prefill_workspace.restype = sz
+    lib.sala_lightning_prefill.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, S, S, S, S,
+                                           S, i, i64, f, f, i, vp, sz, i, vp]
+    lib.sala_lightning_prefill.restype = i
+    lib.sala_lightning_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, S, S, S, S,
+                                          S, f, f, i, vp]
+    lib.sala_lightning_decode.restype = i
+    lib.sala_sparse_select_workspace.argtypes = [i, i, i, i, i, i]
+    lib.sala_sparse_select_workspace.restype = sz
+    lib.sala_sparse_select.argtypes = [vp, vp, i, i, i, i, i, S, S, i, i, i, i, vp, vp, sz, i, vp]
+    lib.sala_sparse_select.restype = i
+    lib.sala_sparse_attn.argtypes = [vp, vp, vp, vp, vp, i, vp, i, i, i, i, i, S, S, S, S, S, i, f,
+                                     i, vp]
+    lib.sala_sparse_attn.restype = i
+    lib.sala_get_device_error.argtypes = [vp]
+    lib.sala_get_device_error.restype = i
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().sala_status_string(int(status)).decode()
+
+
+def version() -> str:
+    return load_library().sala_version().decode()
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise SalaError(fn, status, status_string(status))
+
+
+def _p(t: Optional[torch.Tensor]):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SALA_BF16
+    if t.dtype == torch.float32:
+        return SALA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _s4(t: Optional[torch.Tensor]) -> SalaStrides:
+    """Element strides {b, t, h} of a [B, T, H, D] tensor (D stride must be 1)."""
+    if t is None:
+        return SalaStrides(0, 0, 0)
+    if t.dim() != 4 or t.stride(3) != 1:
+        raise ValueError("expected a [B, T, H, D] tensor with unit stride along D")
+    return SalaStrides(t.stride(0), t.stride(1), t.stride(2))
+
+
+def _s3(t: Optional[torch.Tensor]) -> SalaStrides:
+    """Element strides {b, -, h} of a [B, H, D] tensor."""
+    if t is None:
+        return SalaStrides(0, 0, 0)
+    if t.dim() != 3 or t.stride(2) != 1:
+        raise ValueError("expected a [B, H, D] tensor with unit stride along D")
+    return SalaStrides(t.stride(0), 0, t.stride(1))
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors")
+
+
+def lightning_prefill_workspace(B, T, H, D, chunk=128, dtype=torch.bfloat16) -> int:
+    dt = SALA_BF16 if dtype == torch.bfloat16 else SALA_F32
+    return int(load_library().sala_lightning_prefill_workspace(B, T, H, D, chunk, dt))
+
+
+def lightning_prefill(q, k, v, g=None, state=None, q_norm_w=None, k_norm_w=None, *, chunk=128,
+                      pos0=0, rope_base=10000.0, eps=1e-6, out=None, workspace=None,
+                      stream=None):
+    """Lightning attention prefill.  q,k,v,g: [B,T,H,D].  `state` ([B,H,D,D] fp32) is the
+    initial state, updated in place to the final state; None starts from zero.
+    Returns (out [B,T,H,D], state)."""
+    lib = load_library()
+    _cuda(q, k, v, g, state, out)
+    B, T, H, D = q.shape
+    init_zero = 1 if state is None else 0
+    if state is None:
+        state = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
+    if out is None:
+        out = torch.empty((B, T, H, D), dtype=q.dtype, device=q.device)
+    need = lightning_prefill_workspace(B, T, H, D, chunk, q.dtype)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib.sala_lightning_prefill(
+        _p(q), _p(k), _p(v), _p(g), _p(out), _p(state), _p(q_norm_w), _p(k_norm_w), B, T, H, D,
+        _s4(q), _s4(k), _s4(v), _s4(g), _s4(out), int(chunk), int(pos0), float(rope_base),
+        float(eps), init_zero, _p(workspace), wsb, _dt(q), _stream(stream))
+    _check("sala_lightning_prefill", st)
+    return out, state
+
+
+def lightning_decode(q, k, v, g, state, pos, q_norm_w=None, k_norm_w=None, *, rope_base=10000.0,
+                     eps=1e-6, out=None, stream=None):
+    """One decode step.  q,k,v,g: [B,H,D]; state [B,H,D,D] fp32 (updated in place);
+    pos: [B] int32 CUDA tensor.  Returns out [B,H,D]."""
+    lib = load_library()
+    _cuda(q, k, v, g, state, pos, out)
+    B, H, D = q.shape
+    if pos.dtype != torch.int32:
+        raise TypeError("pos must be int32")
+    if out is None:
+        out = torch.empty((B, H, D), dtype=q.dtype, device=q.device)
+    st = lib.sala_lightning_decode(
+        _p(q), _p(k), _p(v), _p(g), _p(out), _p(state), _p(q_norm_w), _p(k_norm_w), _p(pos), B, H,
+        D, _s3(q), _s3(k), _s3(v), _s3(g), _s3(out), float(rope_base), float(eps), _dt(q),
+        _stream(stream))
+    _check("sala_lightning_decode", st)
+    return out
+
+
+def sparse_select_workspace(B, T, Hq, Hkv, D, block=64) -> int:
+    return int(load_library().sala_sparse_select_workspace(B, T, Hq, Hkv, D, block))
+
+
+def sparse_select(q, k, *, topk=64, n_init=1, n_local=2, block=64, out=None, workspace=None,
+                  stream=None):
+    """Block selection.  q [B,T,Hq,D], k [B,T,Hkv,D] -> idx [B,Hkv,T,n_init+topk+n_local] int32."""
+    lib = load_library()
+    _cuda(q, k, out, workspace)
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    n_sel = n_init + topk + n_local
+    if out is None:
+        out = torch.empty((B, Hkv, T, n_sel), dtype=torch.int32, device=q.device)
+    need = sparse_select_workspace(B, T, Hq, Hkv, D, block)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib.sala_sparse_select(_p(q), _p(k), B, T, Hq, Hkv, D, _s4(q), _s4(k), int(block),
+                                int(topk), int(n_init), int(n_local), _p(out), _p(workspace), wsb,
+                                _dt(q), _stream(stream))
+    _check("sala_sparse_select", st)
+    return out
+
+
+def sparse_attn(q, k, v, idx, g=None, *, block=64, scale=0.0, out=None, stream=None):
+    """Block-sparse attention.  q,g [B,T,Hq,D]; k,v [B,T,Hkv,D]; idx [B,Hkv,T,n_sel] int32."""
+    lib = load_library()
+    _cuda(q, k, v, idx, g, out)
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if idx.dtype != torch.int32 or not idx.is_contiguous():
+        raise ValueError("idx must be a contiguous int32 tensor")
+    if out is None:
+        out = torch.empty_like(q, memory_format=torch.contiguous_format)
+    st = lib.sala_sparse_attn(_p(q), _p(k), _p(v), _p(g), _p(idx), int(idx.shape[-1]), _p(out), B,
+                              T, Hq, Hkv, D, _s4(q), _s4(k), _s4(v), _s4(g), _s4(out), int(block),
+                              float(scale), _dt(q), _stream(stream))
+    _check("sala_sparse_attn", st)
+    return out
+
+
+def get_device_error(stream=None) -> int:
+    """Synchronise the stream and read/clear the device error word (0 = none)."""
+    return int(load_library().sala_get_device_error(_stream(stream)))

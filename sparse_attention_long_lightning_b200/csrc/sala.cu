@@ -1,0 +1,345 @@
+// sala.cu -- libsala: C ABI entry points, host-side argument checks and launches.
+//
+// All kernels are compiled into this one translation unit so that they share
+// the device error word.  Host code here does marshalling only: argument
+// validation, tensor-map encoding for TMA, grid sizing and launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "lightning_cc.cuh"
+#include "lightning_decode.cuh"
+#include "lightning_tc.cuh"
+#include "sparse_attn.cuh"
+#include "sparse_select.cuh"
+
+using namespace sala;
+
+namespace {
+
+#define SALA_CHECK_LAUNCH()                                \
+  do {                                                     \
+    if (cudaPeekAtLastError() != cudaSuccess) {            \
+      (void)cudaGetLastError();                            \
+      return SALA_ERR_CUDA;                                \
+    }                                                      \
+  } while (0)
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Strides (elements) of a [B,T,H,D] tensor: non-negative, rows 16-byte aligned.
+inline bool strides_ok(const sala_strides& s, size_t esize) {
+  if (s.b < 0 || s.t < 0 || s.h < 0) return false;
+  return ((s.b * esize) % 16 == 0) && ((s.t * esize) % 16 == 0) && ((s.h * esize) % 16 == 0);
+}
+
+inline size_t esize_of(sala_dtype dt) { return dt == SALA_BF16 ? 2 : 4; }
+
+int num_sms() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 1;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 4-D bf16 tensor map over a [B, T, H, D] activation with a (64, 1, rows, 1)
+// box and 128-byte swizzle (64 bf16 = 128 bytes per box row).
+bool make_tmap_bhtd(CUtensorMap* map, const void* base, int B, int T, int H, int D,
+                    const sala_strides& s, int box_rows) {
+  auto enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)s.h * 2, (cuuint64_t)s.t * 2, (cuuint64_t)s.b * 2};
+  // Degenerate extents get a harmless stride (never stepped over).
+  if (H == 1 && strides[0] == 0) strides[0] = 16;
+  if (B == 1 && strides[2] == 0) strides[2] = 16;
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <typename KernelT>
+bool set_smem(KernelT* k, size_t bytes) {
+  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) ==
+         cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sala_status_string(sala_status s) {
+  switch (s) {
+    case SALA_OK: return "SALA_OK";
+    case SALA_ERR_INVALID_ARG: return "SALA_ERR_INVALID_ARG";
+    case SALA_ERR_UNSUPPORTED: return "SALA_ERR_UNSUPPORTED";
+    case SALA_ERR_CUDA: return "SALA_ERR_CUDA";
+    case SALA_ERR_TIMEOUT: return "SALA_ERR_TIMEOUT";
+    case SALA_ERR_WORKSPACE: return "SALA_ERR_WORKSPACE";
+    case SALA_ERR_RANGE: return "SALA_ERR_RANGE";
+  }
+  return "SALA_ERR_UNKNOWN";
+}
+
+const char* sala_version(void) { return "sala-b200 0.1 (sm_100a)"; }
+
+// ------------------------------------------------------------------ Lightning prefill
+size_t sala_lightning_prefill_workspace(int B, int T, int H, int D, int chunk, sala_dtype dt) {
+  if (dt == SALA_BF16 && D == 128) return lightning_tc_workspace(B, T, H, chunk, num_sms());
+  return 0;
+}
+
+sala_status sala_lightning_prefill(const void* q, const void* k, const void* v, const void* g,
+                                   void* o, float* state, const float* q_norm_w,
+                                   const float* k_norm_w, int B, int T, int H, int D,
+                                   sala_strides sq, sala_strides sk, sala_strides sv,
+                                   sala_strides sg, sala_strides so, int chunk, int64_t pos0,
+                                   float rope_base, float eps, int init_zero, void* workspace,
+                                   size_t workspace_bytes, sala_dtype dt, void* stream) {
+  if (!state || (T > 0 && (!q || !k || !v || !o))) return SALA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || T < 0 || pos0 < 0 || !(rope_base > 1.0f) || !(eps >= 0.0f))
+    return SALA_ERR_INVALID_ARG;
+  if (dt != SALA_BF16 && dt != SALA_F32) return SALA_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128) return SALA_ERR_UNSUPPORTED;
+  if (chunk != 64 && chunk != 128) return SALA_ERR_UNSUPPORTED;
+  const size_t es = esize_of(dt);
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(state) ||
+      (g && !aligned16(g)))
+    return SALA_ERR_INVALID_ARG;
+  if (!strides_ok(sq, es) || !strides_ok(sk, es) || !strides_ok(sv, es) || !strides_ok(so, es) ||
+      (g && !strides_ok(sg, es)))
+    return SALA_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  const double log2_base = std::log2((double)rope_base);
+  if (T == 0) {
+    if (init_zero && cudaMemsetAsync(state, 0, sizeof(float) * (size_t)B * H * D * D, st) !=
+                         cudaSuccess)
+      return SALA_ERR_CUDA;
+    return SALA_OK;
+  }
+  if (dt == SALA_BF16 && D == 128) {
+    const size_t need = lightning_tc_workspace(B, T, H, chunk, num_sms());
+    if (need > 0 && (!workspace || workspace_bytes < need)) return SALA_ERR_WORKSPACE;
+    return lightning_tc_launch(q, k, v, g, o, state, q_norm_w, k_norm_w, B, T, H, sq, sk, sv, sg,
+                               so, chunk, pos0, log2_base, eps, init_zero, workspace, num_sms(),
+                               st);
+  }
+  const int grid = B * H;
+  if (dt == SALA_F32) {
+    if (D == 64) {
+      auto kern = lightning_prefill_cc_kernel<float, 64>;
+      if (!set_smem(kern, CCSmem<64>::bytes)) return SALA_ERR_CUDA;
+      kern<<<grid, kCCThreads, CCSmem<64>::bytes, st>>>(
+          (const float*)q, (const float*)k, (const float*)v, (const float*)g, (float*)o, state,
+          q_norm_w, k_norm_w, H, T, sq, sk, sv, sg, so, pos0, log2_base, eps, init_zero);
+    } else {
+      auto kern = lightning_prefill_cc_kernel<float, 128>;
+      if (!set_smem(kern, CCSmem<128>::bytes)) return SALA_ERR_CUDA;
+      kern<<<grid, kCCThreads, CCSmem<128>::bytes, st>>>(
+          (const float*)q, (const float*)k, (const float*)v, (const float*)g, (float*)o, state,
+          q_norm_w, k_norm_w, H, T, sq, sk, sv, sg, so, pos0, log2_base, eps, init_zero);
+    }
+  } else {
+    auto kern = lightning_prefill_cc_kernel<__nv_bfloat16, 64>;
+    if (!set_smem(kern, CCSmem<64>::bytes)) return SALA_ERR_CUDA;
+    kern<<<grid, kCCThreads, CCSmem<64>::bytes, st>>>(
+        (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
+        (const __nv_bfloat16*)g, (__nv_bfloat16*)o, state, q_norm_w, k_norm_w, H, T, sq, sk, sv,
+        sg, so, pos0, log2_base, eps, init_zero);
+  }
+  SALA_CHECK_LAUNCH();
+  return SALA_OK;
+}
+
+// ------------------------------------------------------------------ Lightning decode
+sala_status sala_lightning_decode(const void* q, const void* k, const void* v, const void* g,
+                                  void* o, float* state, const float* q_norm_w,
+                                  const float* k_norm_w, const int32_t* pos, int B, int H, int D,
+                                  sala_strides sq, sala_strides sk, sala_strides sv,
+                                  sala_strides sg, sala_strides so, float rope_base, float eps,
+                                  sala_dtype dt, void* stream) {
+  if (!q || !k || !v || !o || !state || !pos) return SALA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || !(rope_base > 1.0f) || !(eps >= 0.0f)) return SALA_ERR_INVALID_ARG;
+  if (dt != SALA_BF16 && dt != SALA_F32) return SALA_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128) return SALA_ERR_UNSUPPORTED;
+  const size_t es = esize_of(dt);
+  if (!aligned16(state) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (g && !aligned16(g)))
+    return SALA_ERR_INVALID_ARG;
+  sala_strides z[5] = {sq, sk, sv, sg, so};
+  for (int i = 0; i < 5; ++i) {
+    if (i == 3 && !g) continue;
+    z[i].t = 0;
+    if (!strides_ok(z[i], es)) return SALA_ERR_INVALID_ARG;
+  }
+  cudaStream_t st = as_stream(stream);
+  const double l2b = std::log2((double)rope_base);
+  const int grid = B * H;
+#define SALA_DEC(TT, DD)                                                                    \
+  lightning_decode_kernel<TT, DD><<<grid, kDecThreads, 0, st>>>(                            \
+      (const TT*)q, (const TT*)k, (const TT*)v, (const TT*)g, (TT*)o, state, q_norm_w,      \
+      k_norm_w, pos, H, sq, sk, sv, sg, so, l2b, eps)
+  if (dt == SALA_BF16) {
+    if (D == 128) SALA_DEC(__nv_bfloat16, 128); else SALA_DEC(__nv_bfloat16, 64);
+  } else {
+    if (D == 128) SALA_DEC(float, 128); else SALA_DEC(float, 64);
+  }
+#undef SALA_DEC
+  SALA_CHECK_LAUNCH();
+  return SALA_OK;
+}
+
+// ------------------------------------------------------------------ sparse selection
+size_t sala_sparse_select_workspace(int B, int T, int Hq, int Hkv, int D, int block) {
+  (void)Hq;
+  if (B <= 0 || T <= 0 || Hkv <= 0 || block != kSelBlk || (D != 64 && D != 128)) return 0;
+  return sel_layout(B, T, Hkv, D).total;
+}
+
+sala_status sala_sparse_select(const void* q, const void* k, int B, int T, int Hq, int Hkv,
+                               int D, sala_strides sq, sala_strides sk, int block, int topk,
+                               int n_init, int n_local, int32_t* idx, void* ws, size_t ws_bytes,
+                               sala_dtype dt, void* stream) {
+  if (T > 0 && (!q || !k || !idx)) return SALA_ERR_INVALID_ARG;
+  if (B <= 0 || T < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return SALA_ERR_INVALID_ARG;
+  if (topk < 1 || n_init < 0 || n_local < 1) return SALA_ERR_INVALID_ARG;
+  if (dt != SALA_BF16) return SALA_ERR_UNSUPPORTED;
+  if (block != kSelBlk || (D != 64 && D != 128) || topk > 256 || Hq / Hkv > 32)
+    return SALA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !strides_ok(sq, 2) || !strides_ok(sk, 2))
+    return SALA_ERR_INVALID_ARG;
+  if (T == 0) return SALA_OK;
+  const SelLayout L = sel_layout(B, T, Hkv, D);
+  if (!ws || ws_bytes < L.total) return SALA_ERR_WORKSPACE;
+  cudaStream_t st = as_stream(stream);
+  float* kbar = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.kbar_off);
+  float* scores = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.score_off);
+  const int G = Hq / Hkv;
+  const float inv_sqrt_d = 1.0f / std::sqrt((float)D);
+  if (L.nb > 0) {
+    dim3 gm(L.nb, Hkv, B);
+    if (D == 128)
+      block_means_kernel<128><<<gm, 128, 0, st>>>((const __nv_bfloat16*)k, kbar, L.nb, Hkv, sk);
+    else
+      block_means_kernel<64><<<gm, 64, 0, st>>>((const __nv_bfloat16*)k, kbar, L.nb, Hkv, sk);
+    SALA_CHECK_LAUNCH();
+  }
+  for (int r0 = 0; r0 < T; r0 += L.rows_pass) {
+    const int r1 = std::min(T, r0 + L.rows_pass);
+    if (L.nb > 0) {
+      dim3 gs((r1 - r0 + kScTile - 1) / kScTile, Hkv, B);
+      if (D == 128) {
+        auto kern = block_scores_kernel<128>;
+        if (!set_smem(kern, score_smem_bytes<128>())) return SALA_ERR_CUDA;
+        kern<<<gs, 256, score_smem_bytes<128>(), st>>>((const __nv_bfloat16*)q, kbar, scores,
+                                                        L.nb, Hkv, G, sq, r0, r1, L.rows_pass,
+                                                        n_init, n_local, inv_sqrt_d);
+      } else {
+        auto kern = block_scores_kernel<64>;
+        if (!set_smem(kern, score_smem_bytes<64>())) return SALA_ERR_CUDA;
+        kern<<<gs, 256, score_smem_bytes<64>(), st>>>((const __nv_bfloat16*)q, kbar, scores,
+                                                       L.nb, Hkv, G, sq, r0, r1, L.rows_pass,
+                                                       n_init, n_local, inv_sqrt_d);
+      }
+      SALA_CHECK_LAUNCH();
+    }
+    const int64_t nwarps = (int64_t)B * Hkv * (r1 - r0);
+    const int64_t nblk = (nwarps + kTopkWarps - 1) / kTopkWarps;
+    topk_select_kernel<<<(unsigned)nblk, kTopkWarps * 32, 0, st>>>(
+        scores, idx, B, T, Hkv, L.nb > 0 ? L.nb : 1, r0, r1, L.rows_pass, topk, n_init, n_local);
+    SALA_CHECK_LAUNCH();
+  }
+  return SALA_OK;
+}
+
+// ------------------------------------------------------------------ sparse attention
+sala_status sala_sparse_attn(const void* q, const void* k, const void* v, const void* g,
+                             const int32_t* idx, int n_sel, void* o, int B, int T, int Hq,
+                             int Hkv, int D, sala_strides sq, sala_strides sk, sala_strides sv,
+                             sala_strides sg, sala_strides so, int block, float scale,
+                             sala_dtype dt, void* stream) {
+  if (T > 0 && (!q || !k || !v || !o || !idx)) return SALA_ERR_INVALID_ARG;
+  if (B <= 0 || T < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || n_sel <= 0 || !(scale >= 0.0f))
+    return SALA_ERR_INVALID_ARG;
+  if (dt != SALA_BF16) return SALA_ERR_UNSUPPORTED;
+  if (block != kSaBlk || (D != 64 && D != 128) || Hq / Hkv > 16) return SALA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (g && !aligned16(g)))
+    return SALA_ERR_INVALID_ARG;
+  if (!strides_ok(sq, 2) || !strides_ok(sk, 2) || !strides_ok(sv, 2) || !strides_ok(so, 2) ||
+      (g && !strides_ok(sg, 2)))
+    return SALA_ERR_INVALID_ARG;
+  if (T == 0) return SALA_OK;
+  CUtensorMap tk, tv;
+  if (!make_tmap_bhtd(&tk, k, B, T, Hkv, D, sk, kSaBlk) ||
+      !make_tmap_bhtd(&tv, v, B, T, Hkv, D, sv, kSaBlk))
+    return SALA_ERR_CUDA;
+  SaParams p;
+  p.q = (const __nv_bfloat16*)q;
+  p.g = (const __nv_bfloat16*)g;
+  p.o = (__nv_bfloat16*)o;
+  p.idx = idx;
+  p.sq = sq; p.sg = sg; p.so = so;
+  p.n_sel = n_sel; p.B = B; p.T = T; p.Hq = Hq; p.Hkv = Hkv; p.G = Hq / Hkv;
+  const float sc = scale > 0.0f ? scale : 1.0f / std::sqrt((float)D);
+  p.scale_log2 = sc * 1.4426950408889634f;
+  p.rows = (int64_t)B * Hkv * T;
+  cudaStream_t st = as_stream(stream);
+  const int64_t want = num_sms();
+  const unsigned grid = (unsigned)std::min<int64_t>(want, p.rows);
+  if (D == 128) {
+    constexpr int NS = 5;
+    auto kern = sparse_attn_kernel<128, NS>;
+    if (!set_smem(kern, SaSmem<128, NS>::bytes)) return SALA_ERR_CUDA;
+    kern<<<grid, kSaThreads, SaSmem<128, NS>::bytes, st>>>(tk, tv, p);
+  } else {
+    constexpr int NS = 8;
+    auto kern = sparse_attn_kernel<64, NS>;
+    if (!set_smem(kern, SaSmem<64, NS>::bytes)) return SALA_ERR_CUDA;
+    kern<<<grid, kSaThreads, SaSmem<64, NS>::bytes, st>>>(tk, tv, p);
+  }
+  SALA_CHECK_LAUNCH();
+  return SALA_OK;
+}
+
+// ------------------------------------------------------------------ device error word
+sala_status sala_get_device_error(void* stream) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return SALA_ERR_CUDA;
+  }
+  int h = 0;
+  if (cudaMemcpyFromSymbol(&h, g_device_error, sizeof(int)) != cudaSuccess) return SALA_ERR_CUDA;
+  if (h != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess)
+      return SALA_ERR_CUDA;
+  }
+  return (sala_status)h;
+}
+
+}  // extern "C"

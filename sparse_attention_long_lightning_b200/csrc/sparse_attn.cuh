@@ -1,0 +1,312 @@
+// sparse_attn.cuh -- block-sparse softmax attention over selected KV blocks (NoPE).
+//
+// InfLLM-v2 style sparse layer (MiniCPM-SALA tech-report mirror, section 02 (2)
+// and (4)): every query row t of KV head hk attends to the union of the blocks
+// listed in idx[b][hk][t][:] (keys s <= t only), softmax scaled by `scale`, and
+// the GQA group of hk (query heads hk*G .. hk*G+G-1) shares that selection.
+//
+// Design (sm_100a).  The per-row selections are random-access gathers, so the
+// kernel is bound by moving 64-key K/V blocks from L2/HBM into shared memory,
+// not by arithmetic: each gathered block serves only the group's G <= 16 query
+// rows (16 flop per byte).  A persistent CTA therefore dedicates one producer
+// warp to TMA: it walks the rows assigned to the CTA and, for each selected
+// block, issues tile loads of K and V (128-byte swizzle, no multicast) into an
+// NS-deep ring guarded by mbarriers.  Four consumer warps split each 64-key
+// block 16 keys apiece: the group's 16 query rows form the M = 16 operand of
+// m16n8k16 tensor-core MMAs (Q K^T in bf16, P V in fp16 with fp32
+// accumulation), an online softmax runs per warp in registers, and the four
+// partial (max, sum, O) triples are merged through shared memory at the end of
+// the row.  All waits are bounded; a wait that runs out raises SALA_ERR_TIMEOUT
+// in the device error word and the kernel winds down instead of hanging.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace sala {
+
+constexpr int kSaBlk = 64;          // keys per KV block
+constexpr int kSaConsumers = 4;     // consumer warps (16 keys each)
+constexpr int kSaThreads = (kSaConsumers + 1) * 32;
+
+template <int D, int NS>
+struct SaSmem {
+  static constexpr int kHalf = kSaBlk * 64 * 2;                 // one 64-col box: 8 KB
+  static constexpr int kTile = kSaBlk * D * 2;                  // K or V block
+  static constexpr int kStage = 2 * kTile;                      // K then V
+  static constexpr int kOLd = D + 4;                            // merge row stride (floats)
+  static constexpr int kMerge = kSaConsumers * 16 * kOLd * 4;   // partial O
+  static constexpr int kML = kSaConsumers * 16 * 2 * 4;         // partial m, l
+  static constexpr size_t bytes = 1024 /*align*/ + size_t(NS) * kStage + kMerge + kML +
+                                  (2 * NS + 4) * 8;
+};
+
+struct SaParams {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* g;
+  __nv_bfloat16* o;
+  const int32_t* idx;
+  sala_strides sq, sg, so;
+  int n_sel, B, T, Hq, Hkv, G;
+  float scale_log2;  // softmax scale * log2(e)
+  int64_t rows;      // B * Hkv * T
+};
+
+template <int D, int NS>
+__global__ void __launch_bounds__(kSaThreads, 1)
+sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                   const __grid_constant__ CUtensorMap tmap_v, const SaParams p) {
+  using L = SaSmem<D, NS>;
+  constexpr int kKSteps = D / 16;   // QK^T k-steps
+  constexpr int kNT = D / 8;        // PV n-tiles
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* stages = smem;
+  float* mergeO = reinterpret_cast<float*>(smem + size_t(NS) * L::kStage);
+  float* mergeML = mergeO + L::kMerge / 4;
+  uint64_t* full = reinterpret_cast<uint64_t*>(mergeML + L::kML / 4);
+  uint64_t* empty = full + NS;
+  uint64_t* mrg_full = empty + NS;
+  uint64_t* mrg_empty = mrg_full + 1;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(mrg_empty + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kSaConsumers);
+    }
+    mbar_init(mrg_full, kSaConsumers);
+    mbar_init(mrg_empty, kSaConsumers);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  const int64_t T = p.T;
+  if (warp == kSaConsumers) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tmap_k);
+      prefetch_tmap(&tmap_v);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int64_t r = blockIdx.x; r < p.rows && ok; r += gridDim.x) {
+        const int64_t t = r % T;
+        const int hk = (int)((r / T) % p.Hkv);
+        const int b = (int)(r / (T * p.Hkv));
+        const int32_t* ir = p.idx + r * p.n_sel;
+        for (int e = 0; e < p.n_sel; ++e) {
+          const int j = __ldg(ir + e);
+          if (j < 0 || (int64_t)j * kSaBlk > t) continue;
+          const int s = it % NS;
+          if (*abort_flag || !mbar_wait(&empty[s], ((it / NS) & 1) ^ 1)) { ok = false; break; }
+          uint8_t* st = stages + size_t(s) * L::kStage;
+          mbar_arrive_expect_tx(&full[s], L::kStage);
+#pragma unroll
+          for (int hf = 0; hf < D / 64; ++hf) {
+            tma_load_4d(st + hf * L::kHalf, &tmap_k, &full[s], hf * 64, hk, j * kSaBlk, b);
+            tma_load_4d(st + L::kTile + hf * L::kHalf, &tmap_v, &full[s], hf * 64, hk,
+                        j * kSaBlk, b);
+          }
+          ++it;
+        }
+      }
+      if (!ok) *abort_flag = 1;
+      // Wait (bounded) until every copy this thread issued has landed.
+      const uint32_t n_out = it < (uint32_t)NS ? it : (uint32_t)NS;
+      for (uint32_t u = it - n_out; u < it; ++u) mbar_wait(&full[u % NS], (u / NS) & 1);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int gq = lane >> 2, tq = lane & 3;  // mma group id / thread in group
+  uint32_t it = 0, nrow = 0;
+  float* myO = mergeO + warp * 16 * L::kOLd;
+  float* myML = mergeML + warp * 32;
+  for (int64_t r = blockIdx.x; r < p.rows; r += gridDim.x, ++nrow) {
+    const int64_t t = r % T;
+    const int hk = (int)((r / T) % p.Hkv);
+    const int b = (int)(r / (T * p.Hkv));
+    const int32_t* ir = p.idx + r * p.n_sel;
+
+    // Q fragments: rows = the group's query heads (padded to 16 with zeros).
+    uint32_t qa[kKSteps][4];
+    {
+      const __nv_bfloat16* qr = p.q + b * p.sq.b + t * p.sq.t + (int64_t)(hk * p.G) * p.sq.h;
+#pragma unroll
+      for (int kk = 0; kk < kKSteps; ++kk) {
+#pragma unroll
+        for (int rg = 0; rg < 4; ++rg) {
+          const int row = gq + (rg & 1) * 8;
+          const int col = kk * 16 + tq * 2 + (rg >> 1) * 8;
+          qa[kk][rg] = row < p.G
+                           ? *reinterpret_cast<const uint32_t*>(qr + (int64_t)row * p.sq.h + col)
+                           : 0u;
+        }
+      }
+    }
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // rows gq, gq+8
+    float oacc[kNT][4];
+#pragma unroll
+    for (int nt = 0; nt < kNT; ++nt) oacc[nt][0] = oacc[nt][1] = oacc[nt][2] = oacc[nt][3] = 0.f;
+    uint32_t bad = 0;
+    bool ok = !*abort_flag;
+
+    for (int e = 0; e < p.n_sel && ok; ++e) {
+      const int j = __ldg(ir + e);
+      if (j < 0 || (int64_t)j * kSaBlk > t) continue;
+      const int s = it % NS;
+      if (!mbar_wait(&full[s], (it / NS) & 1)) { ok = false; break; }
+      const uint32_t kb = smem_u32(stages + size_t(s) * L::kStage);
+      const uint32_t vb = kb + L::kTile;
+
+      // ---- S = Q K^T for keys 16*warp .. 16*warp+15 of the block
+      float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      {
+        const int mat = lane >> 3, rin = lane & 7;
+        const uint32_t krow = warp * 16 + (mat >> 1) * 8 + rin;
+#pragma unroll
+        for (int kk = 0; kk < kKSteps; ++kk) {
+          const uint32_t chunk = 2 * kk + (mat & 1);
+          const uint32_t addr = kb + (chunk >> 3) * L::kHalf + swz128(krow, chunk & 7);
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(addr, b0, b1, b2, b3);
+          mma_bf16_16816(sc[0], qa[kk], b0, b1);
+          mma_bf16_16816(sc[1], qa[kk], b2, b3);
+        }
+      }
+      // ---- scale, causal mask, online softmax (log2 domain)
+      const int64_t key0 = (int64_t)j * kSaBlk + warp * 16 + tq * 2;
+      float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int64_t key = key0 + nt * 8 + (c & 1);
+          float x = sc[nt][c] * p.scale_log2;
+          x = key <= t ? x : -INFINITY;
+          sc[nt][c] = x;
+        }
+        mx0 = fmaxf(mx0, fmaxf(sc[nt][0], sc[nt][1]));
+        mx1 = fmaxf(mx1, fmaxf(sc[nt][2], sc[nt][3]));
+      }
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+      const float mu0 = mn0 == -INFINITY ? 0.f : mn0, mu1 = mn1 == -INFINITY ? 0.f : mn1;
+      const float al0 = exp2f(m0 - mu0), al1 = exp2f(m1 - mu1);
+      m0 = mn0;
+      m1 = mn1;
+      uint32_t pa[4];
+      float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const float p0 = exp2f(sc[nt][0] - mu0), p1 = exp2f(sc[nt][1] - mu0);
+        const float p2 = exp2f(sc[nt][2] - mu1), p3 = exp2f(sc[nt][3] - mu1);
+        rs0 += p0 + p1;
+        rs1 += p2 + p3;
+        pa[nt * 2 + 0] = pack_f16x2(p0, p1);
+        pa[nt * 2 + 1] = pack_f16x2(p2, p3);
+      }
+      l0 = l0 * al0 + rs0;
+      l1 = l1 * al1 + rs1;
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt) {
+        oacc[nt][0] *= al0; oacc[nt][1] *= al0;
+        oacc[nt][2] *= al1; oacc[nt][3] *= al1;
+      }
+      // ---- O += P V (V converted bf16 -> fp16 in registers)
+      {
+        const int mat = lane >> 3, rin = lane & 7;
+        const uint32_t vrow = warp * 16 + (mat & 1) * 8 + rin;
+#pragma unroll
+        for (int pp = 0; pp < kNT / 2; ++pp) {
+          const uint32_t chunk = 2 * pp + (mat >> 1);
+          const uint32_t addr = vb + (chunk >> 3) * L::kHalf + swz128(vrow, chunk & 7);
+          uint32_t v0, v1, v2, v3;
+          ldsm_x4_t(addr, v0, v1, v2, v3);
+          v0 = bf16x2_to_f16x2(v0); v1 = bf16x2_to_f16x2(v1);
+          v2 = bf16x2_to_f16x2(v2); v3 = bf16x2_to_f16x2(v3);
+          bad |= f16x2_nonfinite(v0) | f16x2_nonfinite(v1) | f16x2_nonfinite(v2) |
+                 f16x2_nonfinite(v3);
+          mma_f16_16816(oacc[2 * pp], pa, v0, v1);
+          mma_f16_16816(oacc[2 * pp + 1], pa, v2, v3);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      ++it;
+    }
+    if (!ok) { *abort_flag = 1; return; }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) raise_device_error(SALA_ERR_RANGE);
+
+    // ---- merge the four warps' partial softmax states
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    if (nrow > 0 && !mbar_wait(mrg_empty, (nrow - 1) & 1)) { *abort_flag = 1; return; }
+#pragma unroll
+    for (int nt = 0; nt < kNT; ++nt) {
+      const int col = nt * 8 + tq * 2;
+      *reinterpret_cast<float2*>(myO + gq * L::kOLd + col) = make_float2(oacc[nt][0], oacc[nt][1]);
+      *reinterpret_cast<float2*>(myO + (gq + 8) * L::kOLd + col) =
+          make_float2(oacc[nt][2], oacc[nt][3]);
+    }
+    if (tq == 0) {
+      myML[gq] = m0; myML[gq + 8] = m1;
+      myML[16 + gq] = l0; myML[16 + gq + 8] = l1;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(mrg_full);
+    if (!mbar_wait(mrg_full, nrow & 1)) { *abort_flag = 1; return; }
+    {
+      const int ct = threadIdx.x;          // 0..127
+      const int row = ct >> 3;             // query head within the group
+      constexpr int kCols = D / 8;
+      const int c0 = (ct & 7) * kCols;
+      if (row < p.G) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kSaConsumers; ++w) M = fmaxf(M, mergeML[w * 32 + row]);
+        float wgt[kSaConsumers], Lsum = 0.f;
+#pragma unroll
+        for (int w = 0; w < kSaConsumers; ++w) {
+          const float mw = mergeML[w * 32 + row];
+          wgt[w] = (M == -INFINITY) ? 0.f : exp2f(mw - M);
+          Lsum += wgt[w] * mergeML[w * 32 + 16 + row];
+        }
+        const float inv = Lsum > 0.f ? 1.0f / Lsum : 0.f;
+        const int h = hk * p.G + row;
+        const __nv_bfloat16* gr = p.g ? p.g + b * p.sg.b + t * p.sg.t + (int64_t)h * p.sg.h : nullptr;
+        __nv_bfloat16* orow = p.o + b * p.so.b + t * p.so.t + (int64_t)h * p.so.h;
+#pragma unroll
+        for (int c = 0; c < kCols; c += 2) {
+          float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+          for (int w = 0; w < kSaConsumers; ++w) {
+            const float2 ow = *reinterpret_cast<const float2*>(mergeO + (w * 16 + row) * L::kOLd + c0 + c);
+            a0 = fmaf(wgt[w], ow.x, a0);
+            a1 = fmaf(wgt[w], ow.y, a1);
+          }
+          a0 *= inv;
+          a1 *= inv;
+          if (gr) {
+            const __nv_bfloat162 gg = *reinterpret_cast<const __nv_bfloat162*>(gr + c0 + c);
+            a0 *= sigmoidf_(__bfloat162float(gg.x));
+            a1 *= sigmoidf_(__bfloat162float(gg.y));
+          }
+          *reinterpret_cast<__nv_bfloat162*>(orow + c0 + c) = __floats2bfloat162_rn(a0, a1);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(mrg_empty);
+  }
+}
+
+}  // namespace sala

@@ -1,0 +1,109 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, and host-side argument validation rejects bad calls before
+any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_attention_long_lightning_b200 as sala
+from sparse_attention_long_lightning_b200 import build as sala_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sala.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    sala_build.build()
+    return sala.load_library()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sala_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_four_operations():
+    names = declared_symbols()
+    for fn in ("sala_lightning_prefill", "sala_lightning_decode", "sala_sparse_select",
+               "sala_sparse_attn"):
+        assert fn in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    assert sala.status_string(0) == "SALA_OK"
+    assert sala.status_string(1) == "SALA_ERR_INVALID_ARG"
+    assert sala.status_string(6) == "SALA_ERR_RANGE"
+    assert "sm_100a" in sala.version()
+
+
+Z = sala.SalaStrides(0, 0, 0)
+
+
+def _prefill(lib, q=None, D=128, chunk=128, dt=1, T=16, B=1, H=1, base=10000.0, pos0=0):
+    p = ctypes.c_void_p(16) if q is None else q
+    st = sala.SalaStrides(T * H * D, H * D, D)
+    return lib.sala_lightning_prefill(p, p, p, None, p, p, None, None, B, T, H, D, st, st, st, Z,
+                                      st, chunk, pos0, base, 1e-6, 1, None, 0, dt, None)
+
+
+def test_prefill_rejects_bad_arguments(lib):
+    assert _prefill(lib, q=ctypes.c_void_p(0)) == 1          # null pointer
+    assert _prefill(lib, q=ctypes.c_void_p(8)) == 1          # misaligned
+    assert _prefill(lib, D=96) == 2                          # unsupported head dim
+    assert _prefill(lib, chunk=32) == 2                      # unsupported chunk
+    assert _prefill(lib, dt=7) == 2                          # unknown dtype
+    assert _prefill(lib, B=0) == 1
+    assert _prefill(lib, T=-1) == 1
+    assert _prefill(lib, base=1.0) == 1
+    assert _prefill(lib, pos0=-3) == 1
+    p = ctypes.c_void_p(16)
+    bad = sala.SalaStrides(1, 1, 1)                          # rows not 16-byte aligned
+    assert lib.sala_lightning_prefill(p, p, p, None, p, p, None, None, 1, 4, 1, 128, bad, bad,
+                                      bad, Z, bad, 128, 0, 10000.0, 1e-6, 1, None, 0, 1,
+                                      None) == 1
+
+
+def test_decode_rejects_bad_arguments(lib):
+    p = ctypes.c_void_p(16)
+    st = sala.SalaStrides(128, 0, 128)
+    assert lib.sala_lightning_decode(p, p, p, None, p, p, None, None, None, 1, 1, 128, st, st,
+                                     st, Z, st, 10000.0, 1e-6, 1, None) == 1  # null pos
+    assert lib.sala_lightning_decode(p, p, p, None, p, p, None, None, p, 1, 1, 48, st, st, st, Z,
+                                     st, 10000.0, 1e-6, 1, None) == 2
+
+
+def test_select_and_attn_reject_bad_arguments(lib):
+    p = ctypes.c_void_p(16)
+    st = sala.SalaStrides(64 * 2 * 128, 2 * 128, 128)
+    # Hq not a multiple of Hkv
+    assert lib.sala_sparse_select(p, p, 1, 64, 3, 2, 128, st, st, 64, 4, 1, 2, p, p, 1 << 20, 1,
+                                  None) == 1
+    # block size other than 64
+    assert lib.sala_sparse_select(p, p, 1, 64, 2, 2, 128, st, st, 32, 4, 1, 2, p, p, 1 << 20, 1,
+                                  None) == 2
+    # workspace too small
+    assert lib.sala_sparse_select(p, p, 1, 640, 2, 2, 128, st, st, 64, 4, 1, 2, p, p, 16, 1,
+                                  None) == 5
+    # fp32 sparse path is not provided
+    assert lib.sala_sparse_attn(p, p, p, None, p, 67, p, 1, 64, 2, 2, 128, st, st, st, Z, st, 64,
+                                0.0, 0, None) == 2
+    # group larger than one 16-row tile
+    assert lib.sala_sparse_attn(p, p, p, None, p, 67, p, 1, 64, 64, 2, 128, st, st, st, Z, st, 64,
+                                0.0, 1, None) == 2
+
+
+def test_workspace_queries(lib):
+    n = sala.sparse_select_workspace(1, 131072, 32, 2, 128)
+    nb = 131072 // 64
+    assert n >= nb * 2 * 128 * 4                             # block means
+    assert n <= nb * 2 * 128 * 4 + (1 << 30) + 4096          # scores bounded by 1 GiB
+    assert sala.sparse_select_workspace(1, 1 << 20, 32, 2, 128) <= (1 << 30) + (1 << 25)

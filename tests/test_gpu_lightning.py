@@ -1,0 +1,152 @@
+"""GPU parity: Lightning prefill and decode (libsala, through the C ABI) vs the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_attention_long_lightning_b200 import inputs
+from tests._parity import TOL_BF16, TOL_F32, raw_rel_err, rel_err
+
+pytestmark = pytest.mark.gpu
+
+sala = pytest.importorskip("sparse_attention_long_lightning_b200")
+DEV = "cuda"
+
+
+def _np(t):
+    return t.detach().double().cpu().numpy()
+
+
+def test_lightning_small_fp32_full():
+    """Lightning, B1 H2 D64 T1024, fp32, chunk 64, seed 1001: every output and the state."""
+    x = inputs.lightning_inputs(1, 1024, 2, 64, seed=1001, dtype=torch.float32)
+    y, S = sala.lightning_prefill(x.q.cuda(), x.k.cuda(), x.v.cuda(), x.g.cuda(), chunk=64)
+    yr, Sr = oracle.lightning_recurrent(_np(x.q), _np(x.k), _np(x.v), _np(x.g))
+    assert rel_err(_np(y), yr, False) <= TOL_F32
+    assert rel_err(_np(S), Sr, False) <= TOL_F32
+
+
+def _packed(B, T, H, D, dtype, seed):
+    """q, k, v as non-contiguous views of one packed [B, T, 3, H, D] projection."""
+    gen = inputs.generator(seed)
+    qkv = inputs.randn((B, T, 3, H, D), gen, dtype)
+    g = inputs.randn((B, T, H, D), gen, dtype)
+    return qkv, g
+
+
+@pytest.mark.parametrize("T,D,chunk,dtype", [
+    (1, 128, 128, torch.bfloat16), (63, 128, 128, torch.bfloat16), (64, 128, 64, torch.bfloat16),
+    (65, 128, 128, torch.bfloat16), (127, 128, 64, torch.bfloat16), (300, 128, 128, torch.bfloat16),
+    (641, 128, 128, torch.bfloat16), (257, 64, 64, torch.bfloat16), (200, 128, 64, torch.float32),
+    (129, 64, 128, torch.float32)])
+def test_lightning_ragged_strided(T, D, chunk, dtype):
+    """Ragged lengths, packed (strided) q/k/v, norm weights, a non-zero initial
+    state and a position offset, B = 2, H = 3."""
+    B, H = 2, 3
+    qkv, g = _packed(B, T, H, D, dtype, seed=T * 7 + D)
+    gen = inputs.generator(99)
+    S0 = inputs.randn((B, H, D, D), gen, torch.float32, scale=0.05)
+    qw = 1.0 + 0.1 * inputs.randn((D,), gen, torch.float32)
+    kw = 1.0 + 0.1 * inputs.randn((D,), gen, torch.float32)
+    dq = qkv.cuda()
+    st = S0.cuda().clone()
+    y, S = sala.lightning_prefill(dq[:, :, 0], dq[:, :, 1], dq[:, :, 2], g.cuda(), st,
+                                  qw.cuda(), kw.cuda(), chunk=chunk, pos0=5)
+    yr, Sr = oracle.lightning_recurrent(_np(qkv[:, :, 0]), _np(qkv[:, :, 1]), _np(qkv[:, :, 2]),
+                                        _np(g), _np(S0), _np(qw), _np(kw), pos0=5)
+    bf = dtype == torch.bfloat16
+    tol = TOL_BF16 if bf else TOL_F32
+    assert rel_err(_np(y), yr, bf) <= tol
+    assert rel_err(_np(S), Sr, False) <= tol
+    assert sala.get_device_error() == 0
+
+
+def test_lightning_no_gate_zero_length():
+    B, T, H, D = 1, 70, 2, 128
+    x = inputs.lightning_inputs(B, T, H, D, seed=5, gate=False)
+    y, S = sala.lightning_prefill(x.q.cuda(), x.k.cuda(), x.v.cuda(), None, chunk=128)
+    yr, Sr = oracle.lightning_recurrent(_np(x.q), _np(x.k), _np(x.v))
+    assert rel_err(_np(y), yr, True) <= TOL_BF16
+    # T = 0: the state passes through unchanged (or is zeroed when no state is given)
+    st = S.clone()
+    e = torch.empty((B, 0, H, D), dtype=torch.bfloat16, device=DEV)
+    sala.lightning_prefill(e, e, e, None, st)
+    torch.cuda.synchronize()
+    assert torch.equal(st, S)
+
+
+def test_lightning_segments_continue():
+    """prefill(T1) then prefill(T2) from its state at pos0 = T1 equals the oracle on T1+T2."""
+    B, T, H, D = 1, 700, 2, 128
+    x = inputs.lightning_inputs(B, T, H, D, seed=11)
+    dq, dk, dv, dg = (t.cuda() for t in (x.q, x.k, x.v, x.g))
+    ya, S = sala.lightning_prefill(dq[:, :300], dk[:, :300], dv[:, :300], dg[:, :300])
+    yb, S = sala.lightning_prefill(dq[:, 300:], dk[:, 300:], dv[:, 300:], dg[:, 300:], S,
+                                   pos0=300)
+    yr, Sr = oracle.lightning_recurrent(_np(x.q), _np(x.k), _np(x.v), _np(x.g))
+    assert rel_err(_np(torch.cat([ya, yb], 1)), yr, True) <= TOL_BF16
+    assert rel_err(_np(S), Sr, False) <= TOL_BF16
+
+
+def test_lightning_32k_full_size_sampled_heads():
+    """Lightning prefill B1 H32 D128 T32768 bf16, chunk 128, seed 1002 (the launch
+    the benchmark times): four heads compared on every row, plus their final state."""
+    B, T, H, D = 1, 32768, 32, 128
+    x = inputs.lightning_inputs(B, T, H, D, seed=1002, device=DEV)
+    y, S = sala.lightning_prefill(x.q, x.k, x.v, x.g, chunk=128)
+    heads = [0, 7, 19, 31]
+    yr, Sr = oracle.lightning_recurrent(*(_np(t[:, :, heads]) for t in (x.q, x.k, x.v, x.g)))
+    e_y = rel_err(_np(y[:, :, heads]), yr, True)
+    e_s = rel_err(_np(S[:, heads]), Sr, False)
+    print(f"32k: y {e_y:.3e} (raw {raw_rel_err(_np(y[:, :, heads]), yr):.3e}) S {e_s:.3e}")
+    assert e_y <= TOL_BF16 and e_s <= TOL_BF16
+    assert sala.get_device_error() == 0
+
+
+@pytest.mark.parametrize("D,dtype", [(128, torch.bfloat16), (64, torch.float32)])
+def test_decode_steps(D, dtype):
+    B, H, steps = 3, 4, 5
+    gen = inputs.generator(1234)
+    S0 = inputs.randn((B, H, D, D), gen, torch.float32, scale=1.0 / 64)
+    qw = 1.0 + 0.1 * inputs.randn((D,), gen, torch.float32)
+    st = S0.cuda().clone()
+    Sref = _np(S0)
+    for s in range(steps):
+        q, k, v, g = inputs.decode_tokens(B, H, D, seed=77, step=s, dtype=dtype)
+        pos = torch.tensor([s, 1000 + s, 123456 + s], dtype=torch.int32)
+        y = sala.lightning_decode(q.cuda(), k.cuda(), v.cuda(), g.cuda(), st, pos.cuda(),
+                                  qw.cuda(), None)
+        yr, Sref = oracle.lightning_decode(_np(q), _np(k), _np(v), _np(g), Sref, pos.numpy(),
+                                           _np(qw), None)
+        bf = dtype == torch.bfloat16
+        tol = TOL_BF16 if bf else TOL_F32
+        assert rel_err(_np(y), yr, bf) <= tol
+    assert rel_err(_np(st), Sref, False) <= (TOL_BF16 if dtype == torch.bfloat16 else TOL_F32)
+
+
+def test_decode_full_size_steps():
+    """Decode B64 H32 D128, state N(0,1)/64 (seed 1003), first three steps of the
+    256-step workload: every output and the whole state."""
+    B, H, D = 64, 32, 128
+    S0 = inputs.decode_state(B, H, D, seed=1003, device=DEV)
+    st = S0.clone()
+    Sref = _np(S0)
+    for s in range(3):
+        q, k, v, g = inputs.decode_tokens(B, H, D, seed=1003, step=s, device=DEV)
+        pos = torch.full((B,), s, dtype=torch.int32, device=DEV)
+        y = sala.lightning_decode(q, k, v, g, st, pos)
+        yr, Sref = oracle.lightning_decode(_np(q), _np(k), _np(v), _np(g), Sref, np.full(B, s))
+        assert rel_err(_np(y), yr, True) <= TOL_BF16
+    assert rel_err(_np(st), Sref, False) <= TOL_BF16
+
+
+def test_decode_continues_prefill():
+    """GPU prefill(T) then GPU decode at pos T matches oracle prefill(T+1) row T."""
+    B, T, H, D = 1, 200, 2, 128
+    x = inputs.lightning_inputs(B, T + 1, H, D, seed=21)
+    dq, dk, dv, dg = (t.cuda() for t in (x.q, x.k, x.v, x.g))
+    _, S = sala.lightning_prefill(dq[:, :T], dk[:, :T], dv[:, :T], dg[:, :T])
+    pos = torch.full((B,), T, dtype=torch.int32, device=DEV)
+    y = sala.lightning_decode(dq[:, T], dk[:, T], dv[:, T], dg[:, T], S, pos)
+    yr, _ = oracle.lightning_recurrent(*(_np(t) for t in (x.q, x.k, x.v, x.g)), rows=[T])
+    assert rel_err(_np(y), yr[:, 0], True) <= TOL_BF16
