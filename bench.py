@@ -1,0 +1,425 @@
+"""Benchmark: SALA hybrid-attention prefill throughput (tokens/s) at 128K tokens.
+
+One step = one prefill pass of the 8-layer hybrid attention stack (Lightning
+layers 0,1,3,4,5,7; sparse layers 2,6), B=1, T=131072, 32 heads (2 KV heads in
+the sparse layers), head_dim 128, bf16, through the libsala C ABI:
+    Lightning layer: sala_lightning_prefill (chunk 128, fresh zero state)
+    sparse layer:    sala_sparse_select (block 64, top-64 + 1 init + 2 local) then
+                     sala_sparse_attn (gated)
+Inputs are synthetic N(0,1) per layer (seed 1005 + layer), all resident in HBM
+(about 39 GB, far larger than L2, so no flush is needed between steps).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own independent
+sequence (weak scaling, no data-path collective); the step time is the max over
+ranks; value = tokens processed by all ranks / that time.
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
+workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "Hybrid-attn prefill tokens/s at 128K (lightning+sparse); % of roofline"
+B, H, HKV, D = 1, 32, 2, 128
+CHUNK, BLOCK, TOPK, N_INIT, N_LOCAL = 128, 64, 64, 1, 2
+SPARSE_LAYERS = (2, 6)
+NUM_LAYERS = 8
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return (float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]),
+                "measured")
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        return dist, dist.get_rank(), ws
+    torch.cuda.set_device(0)
+    return None, 0, 1
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        loaded = [s for s in sm if mx is None or s >= 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+class Layer:
+    pass
+
+
+def make_layers(T, device, seed=1005):
+    from sparse_attention_long_lightning_b200 import inputs
+    import sparse_attention_long_lightning_b200 as sala
+    layers = []
+    for l in range(NUM_LAYERS):
+        x = inputs.hybrid_layer_inputs(l, T, B, H, HKV, D, device=device, seed=seed)
+        L = Layer()
+        L.index, L.sparse = l, l in SPARSE_LAYERS
+        L.q, L.k, L.v, L.g = x.q, x.k, x.v, x.g
+        L.o = torch.empty_like(x.q)
+        if L.sparse:
+            L.idx = torch.empty((B, HKV, T, N_INIT + TOPK + N_LOCAL), dtype=torch.int32,
+                                device=device)
+            L.ws = torch.empty(sala.sparse_select_workspace(B, T, H, HKV, D, BLOCK),
+                               dtype=torch.uint8, device=device)
+        else:
+            L.state = torch.empty((B, H, D, D), dtype=torch.float32, device=device)
+            n = sala.lightning_prefill_workspace(B, T, H, D, CHUNK, torch.bfloat16)
+            L.ws = torch.empty(max(n, 1), dtype=torch.uint8, device=device)
+        layers.append(L)
+    return layers
+
+
+def run_layer(L, sala, events=None):
+    """One layer of the stack through the C ABI; optional per-op CUDA events."""
+    if L.sparse:
+        if events is not None:
+            events["sel"][0].record()
+        sala.sparse_select(L.q, L.k, topk=TOPK, n_init=N_INIT, n_local=N_LOCAL, block=BLOCK,
+                           out=L.idx, workspace=L.ws)
+        if events is not None:
+            events["sel"][1].record()
+            events["attn"][0].record()
+        sala.sparse_attn(L.q, L.k, L.v, L.idx, L.g, block=BLOCK, out=L.o)
+        if events is not None:
+            events["attn"][1].record()
+    else:
+        if events is not None:
+            events["light"][0].record()
+        # fresh zero initial state each pass (state=None semantics via init_zero)
+        sala.lightning_prefill(L.q, L.k, L.v, L.g, None, chunk=CHUNK, out=L.o, workspace=L.ws)
+        if events is not None:
+            events["light"][1].record()
+
+
+def step(layers, sala, ev=None):
+    for L in layers:
+        run_layer(L, sala, ev)
+
+
+def sparse_attn_flops(L):
+    """Algorithmic flops of one sparse-attention launch: 4*D per (query head, attended key)."""
+    T = L.q.shape[1]
+    idx = L.idx.long()
+    t = torch.arange(T, device=idx.device).view(1, 1, T, 1)
+    valid = (idx >= 0) & (idx * BLOCK <= t)
+    keys = torch.clamp(t - idx * BLOCK + 1, max=BLOCK)
+    keys = torch.where(valid, keys, torch.zeros_like(keys))
+    n = keys.sum().item()  # over (b, hk, t): keys per row, shared by the group
+    return 4.0 * D * n * (H // HKV)
+
+
+def count_launches(layers, sala):
+    """Kernels of libsala launched by one step (profiled once, outside the timed region)."""
+    from torch.profiler import ProfilerActivity, profile
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        step(layers, sala)
+        torch.cuda.synchronize()
+    n = 0
+    for e in prof.events():
+        if e.device_type.name == "CUDA" and "sala::" in e.name:
+            n += 1
+    return n
+
+
+def cpu_baseline(T, small=False):
+    """Time the fp64 oracle on a bounded, stratified sample of the same workload and
+    scale it to tokens/s of the whole 8-layer stack.  Returns (tok/s, info)."""
+    import oracle
+    from sparse_attention_long_lightning_b200 import inputs
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    # Lightning: 16 heads x nt tokens (all cores busy), per token-head cost.
+    nh, nt = 16, (256 if small else 1024)
+    x = inputs.lightning_inputs(1, nt, nh, D, seed=1005)
+    arr = [t.double().numpy() for t in (x.q, x.k, x.v, x.g)]
+    t0 = time.perf_counter()
+    oracle.lightning_recurrent(*arr)
+    light_s_per_tokhead = (time.perf_counter() - t0) / (nh * nt)
+    # Sparse: selection + attention for rows spread evenly over [0, T), both KV heads.
+    s = inputs.sparse_inputs(1, T, H, HKV, D, seed=1007, gate=True)
+    k64, v64 = s.k.double().numpy(), s.v.double().numpy()
+    nrows = 32 if small else 128
+    rows = np.unique(np.linspace(0, T - 1, nrows).astype(np.int64))
+    q_rows, g_rows = s.q[:, rows].double().numpy(), s.g[:, rows].double().numpy()
+    t0 = time.perf_counter()
+    idx, _ = oracle.sparse_select(q_rows, k64, rows=rows, T=T)
+    oracle.attention(q_rows, k64, v64, g_rows, idx=idx, rows=rows)
+    sparse_s_per_row = (time.perf_counter() - t0) / len(rows)
+    per_token = 6 * H * light_s_per_tokhead + 2 * sparse_s_per_row
+    info = {"kind": "oracle", "cores": cores,
+            "sample": f"Lightning: {nh} heads x {nt} tokens; sparse: {len(rows)} rows evenly "
+                      f"spaced over T={T} (select+attention, 2 KV heads); scaled to 6 Lightning "
+                      f"+ 2 sparse layers x {T} tokens"}
+    return 1.0 / per_token, info
+
+
+def run_reference(args):
+    """--impl reference: the fp64 CPU oracle on a bounded sample of the workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    T = args.T
+    times = []
+    info = None
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        tps, info = cpu_baseline(T, small=True)
+        if i >= args.warmup:
+            times.append(T / tps)
+    sec = float(np.mean(times))
+    value = T / sec
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": f"SALA hybrid attention prefill, 8 layers (Lightning 0,1,3,4,5,7;"
+                                   f" sparse 2,6), B1 T{T} H32 Hkv2 D128",
+                       "global_batch": B, "seq_len": T, "parallelism": "cpu"},
+            "cpu_baseline": dict(info, value=value, unit="tokens/s"),
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def e2e_measure(layers, sala, steps, stream):
+    """Same step through the public API with inputs in pinned host memory: every step
+    copies each layer's inputs host->device and the outputs device->host."""
+    host_light = [t.cpu().pin_memory() for t in (layers[0].q, layers[0].k, layers[0].v,
+                                                 layers[0].g)]
+    sp = layers[SPARSE_LAYERS[0]]
+    host_sparse = [t.cpu().pin_memory() for t in (sp.q, sp.k, sp.v, sp.g)]
+    host_out = torch.empty_like(layers[0].o, device="cpu").pin_memory()
+    h2d = sum(sum(t.numel() * t.element_size() for t in (L.q, L.k, L.v, L.g)) for L in layers)
+    d2h = sum(L.o.numel() * L.o.element_size() for L in layers)
+
+    def one():
+        for L in layers:
+            src = host_sparse if L.sparse else host_light
+            for dst, s in zip((L.q, L.k, L.v, L.g), src):
+                dst.copy_(s, non_blocking=True)
+            run_layer(L, sala)
+            host_out.copy_(L.o, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps / 1e3, h2d, d2h
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--T", type=int, default=131072)
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the e2e, CPU-baseline and launch-count legs")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import sparse_attention_long_lightning_b200 as sala
+    sala.load_library()
+    dist, rank, world = _dist()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    hbm, tf_burst, tf_sust, peak_src = _peaks()
+    T = args.T
+    layers = make_layers(T, dev, seed=1005 + 1000 * rank)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        step(layers, sala)
+    torch.cuda.synchronize()
+    err = sala.get_device_error()
+    if err:
+        raise RuntimeError(f"device error after warm-up: {sala.status_string(err)}")
+
+    per_op = {k: [] for k in ("light", "sel", "attn")}
+    n_ops = {"light": 6, "sel": 2, "attn": 2}
+
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        start.record(stream)
+        for _ in range(args.steps):
+            for L in layers:
+                if L.sparse:
+                    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    run_layer(L, sala, {"sel": (s0, s1), "attn": (a0, a1)})
+                    per_op["sel"].append((s0, s1))
+                    per_op["attn"].append((a0, a1))
+                else:
+                    l0, l1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    run_layer(L, sala, {"light": (l0, l1)})
+                    per_op["light"].append((l0, l1))
+        end.record(stream)
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    sec = start.elapsed_time(end) / 1e3 / args.steps
+    if dist is not None:
+        t = torch.tensor([sec], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        sec = float(t.item())
+    err = sala.get_device_error()
+    if err:
+        raise RuntimeError(f"device error in timed region: {sala.status_string(err)}")
+
+    op_ms = {k: float(np.mean([a.elapsed_time(b) for a, b in v])) for k, v in per_op.items()}
+    value = world * T / sec
+
+    # roofline of the dominant kernel and component figures
+    light_bytes = 5 * B * T * H * D * 2 + B * H * D * D * 4
+    sel_bytes = B * T * H * D * 2 + B * T * HKV * D * 2 + B * HKV * T * (N_INIT + TOPK + N_LOCAL) * 4
+    attn_flops = sparse_attn_flops(layers[SPARSE_LAYERS[0]])
+    comps = {
+        "lightning_prefill": {"ms": op_ms["light"], "GB/s": light_bytes / op_ms["light"] / 1e6,
+                              "frac_hbm": light_bytes / op_ms["light"] / 1e6 / hbm},
+        "sparse_select": {"ms": op_ms["sel"], "GB/s": sel_bytes / op_ms["sel"] / 1e6,
+                          "frac_hbm": sel_bytes / op_ms["sel"] / 1e6 / hbm},
+        "sparse_attn": {"ms": op_ms["attn"], "TFLOP/s": attn_flops / op_ms["attn"] / 1e9,
+                        "frac_tensor": attn_flops / op_ms["attn"] / 1e9 / tf_sust},
+    }
+    share = {k: n_ops[k] * op_ms[k] for k in op_ms}
+    dom = max(share, key=share.get)
+    if dom == "attn":
+        roof = {"kernel": "sparse_attn_kernel", "bound": "tensor",
+                "achieved": attn_flops / op_ms["attn"] / 1e9, "peak": tf_sust, "unit": "TFLOP/s",
+                "traffic": None, "peak_source": f"bf16_tflops_sustained ({peak_src})",
+                "per_launch": f"{attn_flops:.4e} flop"}
+    elif dom == "light":
+        roof = {"kernel": "lightning_prefill", "bound": "hbm",
+                "achieved": light_bytes / op_ms["light"] / 1e6, "peak": hbm, "unit": "GB/s",
+                "traffic": None, "peak_source": f"hbm_gbs ({peak_src})",
+                "per_launch": f"{light_bytes:.4e} bytes"}
+    else:
+        roof = {"kernel": "sparse_select", "bound": "hbm",
+                "achieved": sel_bytes / op_ms["sel"] / 1e6, "peak": hbm, "unit": "GB/s",
+                "traffic": None, "peak_source": f"hbm_gbs ({peak_src})",
+                "per_launch": f"{sel_bytes:.4e} bytes"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": "SALA hybrid attention prefill, 8 layers (Lightning 0,1,3,4,5,7; "
+                                   "sparse 2,6), B1 T131072 H32 (sparse: 32q/2kv) D128 bf16",
+                       "global_batch": B * world, "seq_len": T,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "inputs (~39 GB resident) far exceed L2; no flush",
+                       "chunk": CHUNK, "block": BLOCK, "topk": TOPK, "n_init": N_INIT,
+                       "n_local": N_LOCAL},
+            "roofline": roof, "components": comps, "clocks": clk.summary()}
+
+    if not args.no_extras:
+        line["gpu_launches"] = count_launches(layers, sala) * args.steps
+        e2e_sec, h2d, d2h = e2e_measure(layers, sala, args.e2e_steps, stream)
+        line["e2e"] = {"value": world * T / e2e_sec if dist is None else None, "unit": "tokens/s",
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                       "ms_per_step": e2e_sec * 1e3}
+        if dist is not None:
+            t = torch.tensor([e2e_sec], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            line["e2e"]["value"] = world * T / float(t.item())
+            line["e2e"]["ms_per_step"] = float(t.item()) * 1e3
+        if rank == 0 and world == 1:
+            tps, info = cpu_baseline(T)
+            line["cpu_baseline"] = dict(info, value=tps, unit="tokens/s")
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

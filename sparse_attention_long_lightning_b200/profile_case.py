@@ -1,0 +1,67 @@
+"""Run one hot-path operation at a chosen size, for profiler captures and quick timing.
+
+    python -m sparse_attention_long_lightning_b200.profile_case --op attn --T 16384 --iters 3
+
+Ops: lightning (prefill, B1 H32 D128 bf16 chunk 128), decode (B64 H32 D128 bf16),
+select / attn (B1 Hq32 Hkv2 D128 bf16, top-64 + 1 + 2).  Prints the mean CUDA-event
+time per call.
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+import sparse_attention_long_lightning_b200 as sala
+from sparse_attention_long_lightning_b200 import inputs
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--op", required=True, choices=["lightning", "decode", "select", "attn"])
+    ap.add_argument("--T", type=int, default=16384)
+    ap.add_argument("--B", type=int, default=64, help="batch for decode")
+    ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=1)
+    a = ap.parse_args()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    if a.op == "lightning":
+        x = inputs.lightning_inputs(1, a.T, 32, 128, seed=1002, device=dev)
+        o = torch.empty_like(x.q)
+        ws = torch.empty(max(1, sala.lightning_prefill_workspace(1, a.T, 32, 128, 128)),
+                         dtype=torch.uint8, device=dev)
+        fn = lambda: sala.lightning_prefill(x.q, x.k, x.v, x.g, None, chunk=128, out=o,
+                                            workspace=ws)
+    elif a.op == "decode":
+        S = inputs.decode_state(a.B, 32, 128, seed=1003, device=dev)
+        q, k, v, g = inputs.decode_tokens(a.B, 32, 128, seed=1003, step=0, device=dev)
+        pos = torch.zeros(a.B, dtype=torch.int32, device=dev)
+        o = torch.empty_like(q)
+        fn = lambda: sala.lightning_decode(q, k, v, g, S, pos, out=o)
+    else:
+        s = inputs.sparse_inputs(1, a.T, 32, 2, 128, seed=1004, device=dev, gate=True)
+        idx = sala.sparse_select(s.q, s.k)
+        ws = torch.empty(sala.sparse_select_workspace(1, a.T, 32, 2, 128), dtype=torch.uint8,
+                         device=dev)
+        o = torch.empty_like(s.q)
+        if a.op == "select":
+            fn = lambda: sala.sparse_select(s.q, s.k, out=idx, workspace=ws)
+        else:
+            fn = lambda: sala.sparse_attn(s.q, s.k, s.v, idx, s.g, out=o)
+    for _ in range(a.warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(a.iters):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    err = sala.get_device_error()
+    print(f"{a.op} T={a.T}: {e0.elapsed_time(e1) / a.iters:.3f} ms/call, device_error={err}")
+    return 1 if err else 0
+
+
+if __name__ == "__main__":
+    raise SystemExit(main())
