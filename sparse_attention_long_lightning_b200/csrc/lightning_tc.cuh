@@ -1,33 +1,494 @@
-// lightning_tc.cuh -- Lightning prefill for bf16, head_dim 128 (provisional:
-// runs the fp32 CUDA-core chunked kernel).
+// lightning_tc.cuh -- Lightning attention prefill on 5th-gen tensor cores (tcgen05 + TMEM),
+// bf16 activations, head_dim 128, chunk 128.
+//
+// Method: the Lightning state recurrence S_t = S_{t-1} + k_t v_t^T read out as
+// o_t = q_t^T S_t (MiniCPM-SALA summary page, "Prerequisites / Linear Attention"),
+// with per-head QK RMSNorm, rotate-half RoPE and a sigmoid output gate
+// (tech-report mirror, section 02 (3) and (4)), evaluated chunk by chunk:
+//   P_c = (Qh_c Kh_c^T) masked to s <= t,  O_c = P_c V_c + Qh_c S_{c-1},
+//   S_c = S_{c-1} + Kh_c^T V_c,            y_c = sigmoid(g_c) * O_c.
+//
+// Sequence parallelism.  One head has only T/128 sequential chunks, so each
+// head's chunks are split into G contiguous segments and the work runs in three
+// launches:
+//   (A) state pass   -- per segment, dS = sum_c Kh_c^T V_c  (reads k, v only)
+//   (B) scan         -- per head, exclusive prefix of the segment sums (+ S0);
+//                       also writes the final state
+//   (C) output pass  -- per segment, start from its prefix state and emit y.
+//
+// Per chunk inside a CTA (128 threads, one per token row of the chunk):
+//   * TMA brings the raw bf16 q/k/v tiles (128 tokens x 128 dims, 128-byte
+//     swizzle, two 64-column slabs each) into a double-buffered stage.
+//   * Each thread normalises/rotates its q and k row and converts q, k, v to
+//     fp16 IN PLACE (same swizzled layout), so the tile is directly a tcgen05
+//     operand.  fp16 (10-bit mantissa) keeps the rounding of the normalised,
+//     rotated operands well inside the 1e-2 tolerance, where bf16 would not.
+//   * One thread issues the MMAs (fp32 accumulation in tensor memory):
+//       TMEM[P] = Qh Kh^T             (A, B K-major)
+//       TMEM[O] = Qh S_op             (B = fp16 copy of S, MN-major)
+//       TMEM[S] += Kh^T V             (A, B MN-major views of the same tiles)
+//     then, after the threads turned P into a causally masked fp16 copy in
+//     TMEM, TMEM[O] += P V with A read straight from tensor memory.
+//   * The fp16 copy of S is rescaled by a power of two per chunk (2^-e) so it
+//     stays inside the fp16 range at any length; P uses the same factor and
+//     the epilogue multiplies O by 2^e (exact).
 #pragma once
 
 #include "lightning_cc.cuh"
+#include "ptx.cuh"
 
 namespace sala {
 
-inline size_t lightning_tc_workspace(int B, int T, int H, int chunk, int nsm) {
-  (void)B; (void)T; (void)H; (void)chunk; (void)nsm;
-  return 0;
+constexpr int kTcC = 128;                 // chunk (tokens)
+constexpr int kTcThreads = 128;
+constexpr int kTcSlab = 128 * 128;        // one 128-row x 64-col 16-bit slab: 16 KB
+constexpr int kTcTile = 2 * kTcSlab;      // 128 x 128 16-bit tile: 32 KB
+
+template <bool kStateOnly>
+struct TcSmem {
+  static constexpr int kStageBytes = (kStateOnly ? 2 : 3) * kTcTile;
+  static constexpr int kSop = kStateOnly ? 0 : kTcTile;
+  static constexpr int kMisc = 1024;
+  static constexpr size_t bytes = 1024 /*alignment slack*/ + 2 * size_t(kStageBytes) + kSop + kMisc;
+  static constexpr uint32_t kTmemCols = kStateOnly ? 128 : 512;
+};
+
+struct TcParams {
+  const __nv_bfloat16* g;
+  __nv_bfloat16* o;
+  const float* qw;
+  const float* kw;
+  float* ws;  // [B*H][G][128][128] fp32: segment sums, turned into segment start states
+  sala_strides sg, so;
+  int B, T, H, G, NC;
+  int64_t pos0;
+  double log2_base;
+  float eps;
+};
+
+// Block-wide max of |values| -> power-of-two exponent e >= 0 with max * 2^-e < 2^15.
+__device__ __forceinline__ int tc_block_scale_exp(float m, float* red) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  const int warp = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) red[warp] = m;
+  __syncthreads();
+  m = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  __syncthreads();
+  int x = 0;
+  frexpf(m, &x);
+  return x > 15 ? x - 15 : 0;
 }
 
-inline sala_status lightning_tc_launch(const void* q, const void* k, const void* v, const void* g,
-                                       void* o, float* state, const float* qw, const float* kw,
-                                       int B, int T, int H, sala_strides sq, sala_strides sk,
-                                       sala_strides sv, sala_strides sg, sala_strides so,
-                                       int chunk, int64_t pos0, double log2_base, float eps,
-                                       int init_zero, void* ws, int nsm, cudaStream_t st) {
-  (void)chunk; (void)ws; (void)nsm;
-  auto kern = lightning_prefill_cc_kernel<__nv_bfloat16, 128>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)CCSmem<128>::bytes) != cudaSuccess)
-    return SALA_ERR_CUDA;
-  kern<<<B * H, kCCThreads, CCSmem<128>::bytes, st>>>(
-      (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
-      (const __nv_bfloat16*)g, (__nv_bfloat16*)o, state, qw, kw, H, T, sq, sk, sv, sg, so, pos0,
-      log2_base, eps, init_zero);
-  if (cudaPeekAtLastError() != cudaSuccess) { (void)cudaGetLastError(); return SALA_ERR_CUDA; }
-  return SALA_OK;
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* f) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+__device__ __forceinline__ uint4 f32x8_to_f16(const float* f) {
+  return make_uint4(pack_f16x2(f[0], f[1]), pack_f16x2(f[2], f[3]), pack_f16x2(f[4], f[5]),
+                    pack_f16x2(f[6], f[7]));
+}
+__device__ __forceinline__ uint32_t f16x8_nonfinite(const uint4& u) {
+  return f16x2_nonfinite(u.x) | f16x2_nonfinite(u.y) | f16x2_nonfinite(u.z) |
+         f16x2_nonfinite(u.w);
+}
+
+// Normalise + rotate the raw bf16 row r of the k (and q) tile and convert it, and the v
+// row, to fp16 in place.  Tiles are two 64-column slabs of 128 rows x 128 bytes with
+// the 128-byte swizzle.  Returns non-zero if an fp16 value is not finite.
+template <bool kWithQ>
+__device__ __forceinline__ uint32_t tc_prep_row(uint8_t* sQ, uint8_t* sK, uint8_t* sV, int r,
+                                                int64_t pos, const TcParams& p,
+                                                const double* inv_freq) {
+  float ssq = 0.f, ssk = 0.f;
+#pragma unroll
+  for (int cj = 0; cj < 16; ++cj) {
+    const uint32_t a = (cj >> 3) * kTcSlab + swz128(r, cj & 7);
+    float f[8];
+    bf16x8_to_f32(*reinterpret_cast<const uint4*>(sK + a), f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ssk = fmaf(f[e], f[e], ssk);
+    if (kWithQ) {
+      bf16x8_to_f32(*reinterpret_cast<const uint4*>(sQ + a), f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ssq = fmaf(f[e], f[e], ssq);
+    }
+  }
+  const float rk = rsqrtf(ssk * (1.0f / 128.0f) + p.eps);
+  const float rq = rsqrtf(ssq * (1.0f / 128.0f) + p.eps);
+  uint32_t bad = 0;
+  const double two_pi = 6.283185307179586476925286766559;
+  const double inv_two_pi = 0.15915494309189533576888376337251;
+#pragma unroll 1
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t alo = swz128(r, j), ahi = kTcSlab + swz128(r, j);
+    float klo[8], khi[8], qlo[8], qhi[8];
+    bf16x8_to_f32(*reinterpret_cast<const uint4*>(sK + alo), klo);
+    bf16x8_to_f32(*reinterpret_cast<const uint4*>(sK + ahi), khi);
+    if (kWithQ) {
+      bf16x8_to_f32(*reinterpret_cast<const uint4*>(sQ + alo), qlo);
+      bf16x8_to_f32(*reinterpret_cast<const uint4*>(sQ + ahi), qhi);
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int i = 8 * j + e;  // rotation pair (i, i + 64)
+      const double a = (double)pos * inv_freq[i];
+      const float ang = (float)(a - rint(a * inv_two_pi) * two_pi);
+      float s, c;
+      __sincosf(ang, &s, &c);
+      const float wk0 = p.kw ? __ldg(p.kw + i) : 1.f, wk1 = p.kw ? __ldg(p.kw + i + 64) : 1.f;
+      const float k0 = klo[e] * rk * wk0, k1 = khi[e] * rk * wk1;
+      klo[e] = k0 * c - k1 * s;
+      khi[e] = k1 * c + k0 * s;
+      if (kWithQ) {
+        const float wq0 = p.qw ? __ldg(p.qw + i) : 1.f, wq1 = p.qw ? __ldg(p.qw + i + 64) : 1.f;
+        const float q0 = qlo[e] * rq * wq0, q1 = qhi[e] * rq * wq1;
+        qlo[e] = q0 * c - q1 * s;
+        qhi[e] = q1 * c + q0 * s;
+      }
+    }
+    uint4 u = f32x8_to_f16(klo);
+    bad |= f16x8_nonfinite(u);
+    *reinterpret_cast<uint4*>(sK + alo) = u;
+    u = f32x8_to_f16(khi);
+    bad |= f16x8_nonfinite(u);
+    *reinterpret_cast<uint4*>(sK + ahi) = u;
+    if (kWithQ) {
+      u = f32x8_to_f16(qlo);
+      bad |= f16x8_nonfinite(u);
+      *reinterpret_cast<uint4*>(sQ + alo) = u;
+      u = f32x8_to_f16(qhi);
+      bad |= f16x8_nonfinite(u);
+      *reinterpret_cast<uint4*>(sQ + ahi) = u;
+    }
+  }
+#pragma unroll
+  for (int cj = 0; cj < 16; ++cj) {
+    const uint32_t a = (cj >> 3) * kTcSlab + swz128(r, cj & 7);
+    uint4 u = *reinterpret_cast<const uint4*>(sV + a);
+    u.x = bf16x2_to_f16x2(u.x); u.y = bf16x2_to_f16x2(u.y);
+    u.z = bf16x2_to_f16x2(u.z); u.w = bf16x2_to_f16x2(u.w);
+    bad |= f16x8_nonfinite(u);
+    *reinterpret_cast<uint4*>(sV + a) = u;
+  }
+  return bad;
+}
+
+// K-major operand (rows = M or N, 128-byte rows along K), k-step kk of 16 elements.
+__device__ __forceinline__ uint64_t tc_desc_k(const uint8_t* base, int kk) {
+  return umma_desc_sw128(smem_u32(base) + (kk >> 2) * kTcSlab + (kk & 3) * 32, 16, 1024);
+}
+// MN-major operand (rows = K, 128-byte rows along MN, two 64-wide MN slabs), k-step kk.
+__device__ __forceinline__ uint64_t tc_desc_mn(const uint8_t* base, int kk) {
+  return umma_desc_sw128(smem_u32(base) + kk * 2048, kTcSlab, 1024);
+}
+
+template <bool kStateOnly>
+__global__ void __launch_bounds__(kTcThreads, 1)
+lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                    const __grid_constant__ CUtensorMap tmv, const TcParams p) {
+  using L = TcSmem<kStateOnly>;
+  constexpr uint32_t kIdScore = umma_idesc_f16(128, 128, false, false);
+  constexpr uint32_t kIdInter = umma_idesc_f16(128, 128, false, true);
+  constexpr uint32_t kIdState = umma_idesc_f16(128, 128, true, true);
+  constexpr uint32_t kIdPV = umma_idesc_f16(128, 128, false, true);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* stages = smem;
+  uint8_t* sop = smem + 2 * L::kStageBytes;
+  uint8_t* misc = sop + L::kSop;
+  uint64_t* full = reinterpret_cast<uint64_t*>(misc);      // [2]
+  uint64_t* mma_bar = full + 2;                            // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_bar + 1);
+  float* red = reinterpret_cast<float*>(misc + 64);        // [4]
+  double* inv_freq = reinterpret_cast<double*>(misc + 128);  // [64]
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int seg = blockIdx.x % p.G;
+  const int bh = blockIdx.x / p.G;
+  const int b = bh / p.H, h = bh % p.H;
+  const int c_begin = (int)((int64_t)seg * p.NC / p.G);
+  const int c_end = (int)((int64_t)(seg + 1) * p.NC / p.G);
+  const int nchunks = c_end - c_begin;
+
+  if (tid == 0) {
+    mbar_init(&full[0], 1);
+    mbar_init(&full[1], 1);
+    mbar_init(mma_bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) tc_alloc(tmem_slot, L::kTmemCols);
+  if (tid < 64) inv_freq[tid] = exp2(-(2.0 * tid / 128.0) * p.log2_base);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t t_p = tmem, t_o = tmem + 128, t_s = kStateOnly ? tmem : tmem + 256;
+  const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+
+  auto issue = [&](int u) {
+    uint8_t* st = stages + (u & 1) * L::kStageBytes;
+    const int t0 = (c_begin + u) * kTcC;
+    mbar_arrive_expect_tx(&full[u & 1], L::kStageBytes);
+    uint8_t* dk = st + (kStateOnly ? 0 : kTcTile);
+    uint8_t* dv = dk + kTcTile;
+    if (!kStateOnly) {
+      tma_load_4d(st, &tmq, &full[u & 1], 0, h, t0, b);
+      tma_load_4d(st + kTcSlab, &tmq, &full[u & 1], 64, h, t0, b);
+    }
+    tma_load_4d(dk, &tmk, &full[u & 1], 0, h, t0, b);
+    tma_load_4d(dk + kTcSlab, &tmk, &full[u & 1], 64, h, t0, b);
+    tma_load_4d(dv, &tmv, &full[u & 1], 0, h, t0, b);
+    tma_load_4d(dv + kTcSlab, &tmv, &full[u & 1], 64, h, t0, b);
+  };
+  int issued = 0;
+  if (tid == 0) {
+    if (!kStateOnly) prefetch_tmap(&tmq);
+    prefetch_tmap(&tmk);
+    prefetch_tmap(&tmv);
+    for (; issued < 2 && issued < nchunks; ++issued) issue(issued);
+  }
+
+  float* wseg = p.ws + ((size_t)bh * p.G + seg) * (128 * 128);
+  int e_cur = 0;
+  uint32_t bad = 0;
+  if (!kStateOnly) {
+    // segment start state -> TMEM[S] (fp32) and its fp16 operand copy
+    const float* srow = wseg + (size_t)tid * 128;
+    float mx = 0.f;
+#pragma unroll 1
+    for (int gq = 0; gq < 4; ++gq) {
+      uint32_t r[32];
+#pragma unroll
+      for (int v4 = 0; v4 < 8; ++v4) {
+        const float4 x = *reinterpret_cast<const float4*>(srow + 32 * gq + 4 * v4);
+        r[4 * v4 + 0] = __float_as_uint(x.x); r[4 * v4 + 1] = __float_as_uint(x.y);
+        r[4 * v4 + 2] = __float_as_uint(x.z); r[4 * v4 + 3] = __float_as_uint(x.w);
+        mx = fmaxf(mx, fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(x.z), fabsf(x.w))));
+      }
+      tc_st32(t_s + lane_off + 32 * gq, r);
+    }
+    tc_wait_st();
+    e_cur = tc_block_scale_exp(mx, red);
+    const float sc = pow2i(-e_cur);
+#pragma unroll 1
+    for (int cj = 0; cj < 16; ++cj) {
+      float f[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) f[e] = srow[8 * cj + e] * sc;
+      *reinterpret_cast<uint4*>(sop + (cj >> 3) * kTcSlab + swz128(tid, cj & 7)) = f32x8_to_f16(f);
+    }
+    fence_proxy_async_smem();
+  }
+
+  uint32_t mma_phase = 0;
+  bool ok = true;
+  for (int u = 0; u < nchunks; ++u) {
+    const int s = u & 1;
+    uint8_t* st = stages + s * L::kStageBytes;
+    uint8_t* sQ = st;
+    uint8_t* sK = st + (kStateOnly ? 0 : kTcTile);
+    uint8_t* sV = sK + kTcTile;
+    const int64_t t = (int64_t)(c_begin + u) * kTcC + tid;
+    ok = ok && mbar_wait(&full[s], (u >> 1) & 1);
+    if (ok) bad |= tc_prep_row<!kStateOnly>(sQ, sK, sV, tid, p.pos0 + t, p, inv_freq);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    ok = __syncthreads_and(ok);
+    if (!ok) break;
+    if (tid == 0) {
+      tc_fence_after();
+      if (!kStateOnly) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc_mma_ss(t_p, tc_desc_k(sQ, kk), tc_desc_k(sK, kk), kIdScore, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc_mma_ss(t_o, tc_desc_k(sQ, kk), tc_desc_mn(sop, kk), kIdInter, kk > 0);
+      }
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        tc_mma_ss(t_s, tc_desc_mn(sK, kk), tc_desc_mn(sV, kk), kIdState,
+                  (kStateOnly && u == 0 && kk == 0) ? 0u : 1u);
+      tc_commit(mma_bar);
+    }
+    ok = mbar_wait(mma_bar, mma_phase & 1);
+    ++mma_phase;
+    tc_fence_after();
+    if (kStateOnly) {
+      ok = __syncthreads_and(ok);
+      if (!ok) break;
+      if (tid == 0 && issued < nchunks) issue(issued++);
+      continue;
+    }
+    // ---- P -> causally masked fp16 copy (in place, TMEM), scaled by 2^-e
+    {
+      const float ps = pow2i(-e_cur);
+#pragma unroll 1
+      for (int gq = 0; gq < 4; ++gq) {
+        uint32_t r[32], pk[16];
+        tc_ld32(t_p + lane_off + 32 * gq, r);
+        tc_wait_ld();
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+          const int col = 32 * gq + 2 * m;
+          const float a = col <= tid ? __uint_as_float(r[2 * m]) * ps : 0.f;
+          const float c = col + 1 <= tid ? __uint_as_float(r[2 * m + 1]) * ps : 0.f;
+          pk[m] = pack_f16x2(a, c);
+          bad |= f16x2_nonfinite(pk[m]);
+        }
+        tc_st16(t_p + lane_off + 16 * gq, pk);
+      }
+      tc_wait_st();
+    }
+    // ---- S (now inclusive of this chunk) -> fp16 operand copy for the next chunk
+    int e_next = e_cur;
+    if (u + 1 < nchunks) {
+      float mx = 0.f;
+#pragma unroll 1
+      for (int gq = 0; gq < 4; ++gq) {
+        uint32_t r[32];
+        tc_ld32(t_s + lane_off + 32 * gq, r);
+        tc_wait_ld();
+#pragma unroll
+        for (int m = 0; m < 32; ++m) mx = fmaxf(mx, fabsf(__uint_as_float(r[m])));
+      }
+      e_next = tc_block_scale_exp(mx, red);
+      const float sc = pow2i(-e_next);
+#pragma unroll 1
+      for (int gq = 0; gq < 4; ++gq) {
+        uint32_t r[32];
+        tc_ld32(t_s + lane_off + 32 * gq, r);
+        tc_wait_ld();
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          float f[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(r[8 * c4 + e]) * sc;
+          const int cj = 4 * gq + c4;
+          *reinterpret_cast<uint4*>(sop + (cj >> 3) * kTcSlab + swz128(tid, cj & 7)) =
+              f32x8_to_f16(f);
+        }
+      }
+      fence_proxy_async_smem();
+    }
+    tc_fence_before();
+    ok = __syncthreads_and(ok);
+    if (!ok) break;
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) tc_mma_ts(t_o, t_p + 8 * kk, tc_desc_mn(sV, kk), kIdPV, 1u);
+      tc_commit(mma_bar);
+    }
+    ok = mbar_wait(mma_bar, mma_phase & 1);
+    ++mma_phase;
+    tc_fence_after();
+    ok = __syncthreads_and(ok);
+    if (!ok) break;
+    if (tid == 0 && issued < nchunks) issue(issued++);
+    // ---- epilogue: y = sigmoid(g) * 2^e * O
+    {
+      const float os = pow2i(e_cur);
+      const bool live = t < p.T;
+      const __nv_bfloat16* gr = p.g ? p.g + b * p.sg.b + t * p.sg.t + (int64_t)h * p.sg.h : nullptr;
+      __nv_bfloat16* orow = p.o + b * p.so.b + t * p.so.t + (int64_t)h * p.so.h;
+#pragma unroll 1
+      for (int gq = 0; gq < 4; ++gq) {
+        uint32_t r[32];
+        tc_ld32(t_o + lane_off + 32 * gq, r);
+        tc_wait_ld();
+        if (live) {
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            float y[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) y[e] = __uint_as_float(r[8 * c8 + e]) * os;
+            if (gr) {
+              float gf[8];
+              bf16x8_to_f32(*reinterpret_cast<const uint4*>(gr + 32 * gq + 8 * c8), gf);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) y[e] *= sigmoidf_(gf[e]);
+            }
+            uint4 w;
+            __nv_bfloat162 h0 = __floats2bfloat162_rn(y[0], y[1]), h1 = __floats2bfloat162_rn(y[2], y[3]);
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(y[4], y[5]), h3 = __floats2bfloat162_rn(y[6], y[7]);
+            w.x = *reinterpret_cast<uint32_t*>(&h0); w.y = *reinterpret_cast<uint32_t*>(&h1);
+            w.z = *reinterpret_cast<uint32_t*>(&h2); w.w = *reinterpret_cast<uint32_t*>(&h3);
+            *reinterpret_cast<uint4*>(orow + 32 * gq + 8 * c8) = w;
+          }
+        }
+      }
+    }
+    e_cur = e_next;
+    tc_fence_before();
+  }
+
+  if (kStateOnly && ok && nchunks > 0) {
+    float* srow = wseg + (size_t)tid * 128;
+#pragma unroll 1
+    for (int gq = 0; gq < 4; ++gq) {
+      uint32_t r[32];
+      tc_ld32(t_s + lane_off + 32 * gq, r);
+      tc_wait_ld();
+#pragma unroll
+      for (int v4 = 0; v4 < 8; ++v4)
+        *reinterpret_cast<float4*>(srow + 32 * gq + 4 * v4) =
+            make_float4(__uint_as_float(r[4 * v4]), __uint_as_float(r[4 * v4 + 1]),
+                        __uint_as_float(r[4 * v4 + 2]), __uint_as_float(r[4 * v4 + 3]));
+    }
+  }
+  if (__any_sync(0xffffffffu, bad) && (tid & 31) == 0) raise_device_error(SALA_ERR_RANGE);
+  if (!ok && tid == 0) {
+    // wind down: let every issued copy land before the CTA's shared memory goes away
+    for (int u = issued > 2 ? issued - 2 : 0; u < issued; ++u) mbar_wait(&full[u & 1], (u >> 1) & 1);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tc_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+// Exclusive prefix over the segment sums of each (b, h), in place; the final
+// state (initial + all segments) goes to `state`.  grid B*H, 256 threads.
+__global__ void __launch_bounds__(256)
+lightning_scan_kernel(float* __restrict__ ws, float* __restrict__ state, int G, int init_zero) {
+  const int bh = blockIdx.x;
+  float* base = ws + (size_t)bh * G * (128 * 128);
+  float* sg = state + (size_t)bh * (128 * 128);
+  for (int e = threadIdx.x * 4; e < 128 * 128; e += 256 * 4) {
+    float4 run = init_zero ? make_float4(0.f, 0.f, 0.f, 0.f) : *reinterpret_cast<const float4*>(sg + e);
+    for (int s = 0; s < G; ++s) {
+      float4* cell = reinterpret_cast<float4*>(base + (size_t)s * (128 * 128) + e);
+      const float4 d = *cell;
+      *cell = run;
+      run.x += d.x; run.y += d.y; run.z += d.z; run.w += d.w;
+    }
+    *reinterpret_cast<float4*>(sg + e) = run;
+  }
+}
+
+inline int lightning_tc_segments(int B, int H, int T, int nsm) {
+  const int NC = (T + kTcC - 1) / kTcC;
+  int G = (8 * nsm) / (B * H);
+  if (G < 1) G = 1;
+  if (G > NC) G = NC;
+  return G;
+}
+
+inline size_t lightning_tc_workspace(int B, int T, int H, int chunk, int nsm) {
+  if (chunk != kTcC || T <= 0) return 0;
+  return (size_t)B * H * lightning_tc_segments(B, H, T, nsm) * 128 * 128 * sizeof(float);
 }
 
 }  // namespace sala

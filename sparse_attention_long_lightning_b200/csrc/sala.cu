@@ -142,12 +142,39 @@ sala_status sala_lightning_prefill(const void* q, const void* k, const void* v, 
       return SALA_ERR_CUDA;
     return SALA_OK;
   }
-  if (dt == SALA_BF16 && D == 128) {
-    const size_t need = lightning_tc_workspace(B, T, H, chunk, num_sms());
-    if (need > 0 && (!workspace || workspace_bytes < need)) return SALA_ERR_WORKSPACE;
-    return lightning_tc_launch(q, k, v, g, o, state, q_norm_w, k_norm_w, B, T, H, sq, sk, sv, sg,
-                               so, chunk, pos0, log2_base, eps, init_zero, workspace, num_sms(),
-                               st);
+  if (dt == SALA_BF16 && D == 128 && chunk == kTcC) {
+    const int nsm = num_sms();
+    const size_t need = lightning_tc_workspace(B, T, H, chunk, nsm);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return SALA_ERR_WORKSPACE;
+    CUtensorMap tq, tk, tv;
+    if (!make_tmap_bhtd(&tq, q, B, T, H, D, sq, kTcC) || !make_tmap_bhtd(&tk, k, B, T, H, D, sk, kTcC) ||
+        !make_tmap_bhtd(&tv, v, B, T, H, D, sv, kTcC))
+      return SALA_ERR_CUDA;
+    TcParams p;
+    p.g = (const __nv_bfloat16*)g;
+    p.o = (__nv_bfloat16*)o;
+    p.qw = q_norm_w;
+    p.kw = k_norm_w;
+    p.ws = (float*)workspace;
+    p.sg = sg;
+    p.so = so;
+    p.B = B; p.T = T; p.H = H;
+    p.G = lightning_tc_segments(B, H, T, nsm);
+    p.NC = (T + kTcC - 1) / kTcC;
+    p.pos0 = pos0;
+    p.log2_base = log2_base;
+    p.eps = eps;
+    const unsigned grid = (unsigned)(B * H * p.G);
+    auto ka = lightning_tc_kernel<true>;
+    auto kc = lightning_tc_kernel<false>;
+    if (!set_smem(ka, TcSmem<true>::bytes) || !set_smem(kc, TcSmem<false>::bytes)) return SALA_ERR_CUDA;
+    ka<<<grid, kTcThreads, TcSmem<true>::bytes, st>>>(tk, tk, tv, p);
+    SALA_CHECK_LAUNCH();
+    lightning_scan_kernel<<<B * H, 256, 0, st>>>(p.ws, state, p.G, init_zero);
+    SALA_CHECK_LAUNCH();
+    kc<<<grid, kTcThreads, TcSmem<false>::bytes, st>>>(tq, tk, tv, p);
+    SALA_CHECK_LAUNCH();
+    return SALA_OK;
   }
   const int grid = B * H;
   if (dt == SALA_F32) {
@@ -164,10 +191,17 @@ sala_status sala_lightning_prefill(const void* q, const void* k, const void* v, 
           (const float*)q, (const float*)k, (const float*)v, (const float*)g, (float*)o, state,
           q_norm_w, k_norm_w, H, T, sq, sk, sv, sg, so, pos0, log2_base, eps, init_zero);
     }
-  } else {
+  } else if (D == 64) {
     auto kern = lightning_prefill_cc_kernel<__nv_bfloat16, 64>;
     if (!set_smem(kern, CCSmem<64>::bytes)) return SALA_ERR_CUDA;
     kern<<<grid, kCCThreads, CCSmem<64>::bytes, st>>>(
+        (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
+        (const __nv_bfloat16*)g, (__nv_bfloat16*)o, state, q_norm_w, k_norm_w, H, T, sq, sk, sv,
+        sg, so, pos0, log2_base, eps, init_zero);
+  } else {
+    auto kern = lightning_prefill_cc_kernel<__nv_bfloat16, 128>;
+    if (!set_smem(kern, CCSmem<128>::bytes)) return SALA_ERR_CUDA;
+    kern<<<grid, kCCThreads, CCSmem<128>::bytes, st>>>(
         (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
         (const __nv_bfloat16*)g, (__nv_bfloat16*)o, state, q_norm_w, k_norm_w, H, T, sq, sk, sv,
         sg, so, pos0, log2_base, eps, init_zero);
