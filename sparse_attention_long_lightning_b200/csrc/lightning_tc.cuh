@@ -40,7 +40,7 @@
 namespace sala {
 
 constexpr int kTcC = 128;                 // chunk (tokens)
-constexpr int kTcThreads = 128;
+constexpr int kTcThreads = 512;             // 16 warps: 4 per SM sub-partition
 constexpr int kTcSlab = 128 * 128;        // one 128-row x 64-col 16-bit slab: 16 KB
 constexpr int kTcTile = 2 * kTcSlab;      // 128 x 128 16-bit tile: 32 KB
 
@@ -73,7 +73,9 @@ __device__ __forceinline__ int tc_block_scale_exp(float m, float* red) {
   const int warp = threadIdx.x >> 5;
   if ((threadIdx.x & 31) == 0) red[warp] = m;
   __syncthreads();
-  m = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  m = red[0];
+#pragma unroll
+  for (int w = 1; w < kTcThreads / 32; ++w) m = fmaxf(m, red[w]);
   __syncthreads();
   int x = 0;
   frexpf(m, &x);
@@ -99,17 +101,21 @@ __device__ __forceinline__ uint32_t f16x8_nonfinite(const uint4& u) {
          f16x2_nonfinite(u.w);
 }
 
-// Normalise + rotate the raw bf16 row r of the k (and q) tile and convert it, and the v
-// row, to fp16 in place.  Tiles are two 64-column slabs of 128 rows x 128 bytes with
-// the 128-byte swizzle.  Returns non-zero if an fp16 value is not finite.
+// Normalise + rotate a quarter of raw bf16 row r of the k (and q) tile and convert
+// it, and a quarter of the v row, to fp16 in place.  Four consecutive lanes share
+// a row: quarter qd owns rotation pairs i in [16 qd, 16 qd + 16) (chunks 2qd, 2qd+1
+// of both 64-column slabs) and v chunks 4qd..4qd+3.  Tiles are two 64-column slabs
+// of 128 rows x 128 bytes with the 128-byte swizzle.  Returns non-zero if an fp16
+// value is not finite.
 template <bool kWithQ>
-__device__ __forceinline__ uint32_t tc_prep_row(uint8_t* sQ, uint8_t* sK, uint8_t* sV, int r,
-                                                int64_t pos, const TcParams& p,
-                                                const double* inv_freq) {
+__device__ __forceinline__ uint32_t tc_prep_quarter(uint8_t* sQ, uint8_t* sK, uint8_t* sV, int r,
+                                                    int qd, int64_t pos, const TcParams& p,
+                                                    const double* inv_freq) {
   float ssq = 0.f, ssk = 0.f;
 #pragma unroll
-  for (int cj = 0; cj < 16; ++cj) {
-    const uint32_t a = (cj >> 3) * kTcSlab + swz128(r, cj & 7);
+  for (int u = 0; u < 4; ++u) {
+    const int j = 2 * qd + (u & 1);
+    const uint32_t a = (u >> 1) * kTcSlab + swz128(r, j);
     float f[8];
     bf16x8_to_f32(*reinterpret_cast<const uint4*>(sK + a), f);
 #pragma unroll
@@ -120,13 +126,18 @@ __device__ __forceinline__ uint32_t tc_prep_row(uint8_t* sQ, uint8_t* sK, uint8_
       for (int e = 0; e < 8; ++e) ssq = fmaf(f[e], f[e], ssq);
     }
   }
+  ssk += __shfl_xor_sync(0xffffffffu, ssk, 1);
+  ssk += __shfl_xor_sync(0xffffffffu, ssk, 2);
+  ssq += __shfl_xor_sync(0xffffffffu, ssq, 1);
+  ssq += __shfl_xor_sync(0xffffffffu, ssq, 2);
   const float rk = rsqrtf(ssk * (1.0f / 128.0f) + p.eps);
   const float rq = rsqrtf(ssq * (1.0f / 128.0f) + p.eps);
   uint32_t bad = 0;
   const double two_pi = 6.283185307179586476925286766559;
   const double inv_two_pi = 0.15915494309189533576888376337251;
-#pragma unroll 1
-  for (int j = 0; j < 8; ++j) {
+#pragma unroll
+  for (int jj = 0; jj < 2; ++jj) {
+    const int j = 2 * qd + jj;
     const uint32_t alo = swz128(r, j), ahi = kTcSlab + swz128(r, j);
     float klo[8], khi[8], qlo[8], qhi[8];
     bf16x8_to_f32(*reinterpret_cast<const uint4*>(sK + alo), klo);
@@ -140,17 +151,17 @@ __device__ __forceinline__ uint32_t tc_prep_row(uint8_t* sQ, uint8_t* sK, uint8_
       const int i = 8 * j + e;  // rotation pair (i, i + 64)
       const double a = (double)pos * inv_freq[i];
       const float ang = (float)(a - rint(a * inv_two_pi) * two_pi);
-      float s, c;
-      __sincosf(ang, &s, &c);
+      float sn, cs;
+      __sincosf(ang, &sn, &cs);
       const float wk0 = p.kw ? __ldg(p.kw + i) : 1.f, wk1 = p.kw ? __ldg(p.kw + i + 64) : 1.f;
       const float k0 = klo[e] * rk * wk0, k1 = khi[e] * rk * wk1;
-      klo[e] = k0 * c - k1 * s;
-      khi[e] = k1 * c + k0 * s;
+      klo[e] = k0 * cs - k1 * sn;
+      khi[e] = k1 * cs + k0 * sn;
       if (kWithQ) {
         const float wq0 = p.qw ? __ldg(p.qw + i) : 1.f, wq1 = p.qw ? __ldg(p.qw + i + 64) : 1.f;
         const float q0 = qlo[e] * rq * wq0, q1 = qhi[e] * rq * wq1;
-        qlo[e] = q0 * c - q1 * s;
-        qhi[e] = q1 * c + q0 * s;
+        qlo[e] = q0 * cs - q1 * sn;
+        qhi[e] = q1 * cs + q0 * sn;
       }
     }
     uint4 u = f32x8_to_f16(klo);
@@ -169,13 +180,14 @@ __device__ __forceinline__ uint32_t tc_prep_row(uint8_t* sQ, uint8_t* sK, uint8_
     }
   }
 #pragma unroll
-  for (int cj = 0; cj < 16; ++cj) {
+  for (int u = 0; u < 4; ++u) {
+    const int cj = 4 * qd + u;
     const uint32_t a = (cj >> 3) * kTcSlab + swz128(r, cj & 7);
-    uint4 u = *reinterpret_cast<const uint4*>(sV + a);
-    u.x = bf16x2_to_f16x2(u.x); u.y = bf16x2_to_f16x2(u.y);
-    u.z = bf16x2_to_f16x2(u.z); u.w = bf16x2_to_f16x2(u.w);
-    bad |= f16x8_nonfinite(u);
-    *reinterpret_cast<uint4*>(sV + a) = u;
+    uint4 x = *reinterpret_cast<const uint4*>(sV + a);
+    x.x = bf16x2_to_f16x2(x.x); x.y = bf16x2_to_f16x2(x.y);
+    x.z = bf16x2_to_f16x2(x.z); x.w = bf16x2_to_f16x2(x.w);
+    bad |= f16x8_nonfinite(x);
+    *reinterpret_cast<uint4*>(sV + a) = x;
   }
   return bad;
 }
@@ -208,10 +220,15 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   uint64_t* full = reinterpret_cast<uint64_t*>(misc);      // [2]
   uint64_t* mma_bar = full + 2;                            // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_bar + 1);
-  float* red = reinterpret_cast<float*>(misc + 64);        // [4]
+  float* red = reinterpret_cast<float*>(misc + 64);        // [16]
   double* inv_freq = reinterpret_cast<double*>(misc + 128);  // [64]
 
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // prep mapping: 4 lanes per token row
+  const int prow = 8 * warp + (lane >> 2), pqd = lane & 3;
+  // TMEM mapping: warp w reads lanes 32*(w%4).. (rows), columns 32*(w/4)..
+  const int lq = warp & 3, cg = warp >> 2;
+  const int trow = 32 * lq + lane;
   const int seg = blockIdx.x % p.G;
   const int bh = blockIdx.x / p.G;
   const int b = bh / p.H, h = bh % p.H;
@@ -231,8 +248,10 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // columns: P fp32 [0,128), O [128,256), S [256,384), P fp16 copy [384,448)
   const uint32_t t_p = tmem, t_o = tmem + 128, t_s = kStateOnly ? tmem : tmem + 256;
-  const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+  const uint32_t t_p16 = tmem + 384;
+  const uint32_t lane_off = (uint32_t)(32 * lq) << 16;
 
   auto issue = [&](int u) {
     uint8_t* st = stages + (u & 1) * L::kStageBytes;
@@ -262,29 +281,27 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   uint32_t bad = 0;
   if (!kStateOnly) {
     // segment start state -> TMEM[S] (fp32) and its fp16 operand copy
-    const float* srow = wseg + (size_t)tid * 128;
+    const float* src = wseg + (size_t)trow * 128 + 32 * cg;
+    uint32_t r[32];
     float mx = 0.f;
-#pragma unroll 1
-    for (int gq = 0; gq < 4; ++gq) {
-      uint32_t r[32];
 #pragma unroll
-      for (int v4 = 0; v4 < 8; ++v4) {
-        const float4 x = *reinterpret_cast<const float4*>(srow + 32 * gq + 4 * v4);
-        r[4 * v4 + 0] = __float_as_uint(x.x); r[4 * v4 + 1] = __float_as_uint(x.y);
-        r[4 * v4 + 2] = __float_as_uint(x.z); r[4 * v4 + 3] = __float_as_uint(x.w);
-        mx = fmaxf(mx, fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(x.z), fabsf(x.w))));
-      }
-      tc_st32(t_s + lane_off + 32 * gq, r);
+    for (int v4 = 0; v4 < 8; ++v4) {
+      const float4 x = *reinterpret_cast<const float4*>(src + 4 * v4);
+      r[4 * v4 + 0] = __float_as_uint(x.x); r[4 * v4 + 1] = __float_as_uint(x.y);
+      r[4 * v4 + 2] = __float_as_uint(x.z); r[4 * v4 + 3] = __float_as_uint(x.w);
+      mx = fmaxf(mx, fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(x.z), fabsf(x.w))));
     }
+    tc_st32(t_s + lane_off + 32 * cg, r);
     tc_wait_st();
     e_cur = tc_block_scale_exp(mx, red);
     const float sc = pow2i(-e_cur);
-#pragma unroll 1
-    for (int cj = 0; cj < 16; ++cj) {
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) {
       float f[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) f[e] = srow[8 * cj + e] * sc;
-      *reinterpret_cast<uint4*>(sop + (cj >> 3) * kTcSlab + swz128(tid, cj & 7)) = f32x8_to_f16(f);
+      for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(r[8 * c4 + e]) * sc;
+      const int cj = 4 * cg + c4;
+      *reinterpret_cast<uint4*>(sop + (cj >> 3) * kTcSlab + swz128(trow, cj & 7)) = f32x8_to_f16(f);
     }
     fence_proxy_async_smem();
   }
@@ -297,9 +314,11 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     uint8_t* sQ = st;
     uint8_t* sK = st + (kStateOnly ? 0 : kTcTile);
     uint8_t* sV = sK + kTcTile;
-    const int64_t t = (int64_t)(c_begin + u) * kTcC + tid;
+    const int64_t chunk_t0 = (int64_t)(c_begin + u) * kTcC;
     ok = ok && mbar_wait(&full[s], (u >> 1) & 1);
-    if (ok) bad |= tc_prep_row<!kStateOnly>(sQ, sK, sV, tid, p.pos0 + t, p, inv_freq);
+    if (ok)
+      bad |= tc_prep_quarter<!kStateOnly>(sQ, sK, sV, prow, pqd, p.pos0 + chunk_t0 + prow, p,
+                                          inv_freq);
     fence_proxy_async_smem();
     tc_fence_before();
     ok = __syncthreads_and(ok);
@@ -329,54 +348,42 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       if (tid == 0 && issued < nchunks) issue(issued++);
       continue;
     }
-    // ---- P -> causally masked fp16 copy (in place, TMEM), scaled by 2^-e
+    // ---- P -> causally masked fp16 copy in TMEM, scaled by 2^-e
     {
       const float ps = pow2i(-e_cur);
-#pragma unroll 1
-      for (int gq = 0; gq < 4; ++gq) {
-        uint32_t r[32], pk[16];
-        tc_ld32(t_p + lane_off + 32 * gq, r);
-        tc_wait_ld();
+      uint32_t r[32], pk[16];
+      tc_ld32(t_p + lane_off + 32 * cg, r);
+      tc_wait_ld();
 #pragma unroll
-        for (int m = 0; m < 16; ++m) {
-          const int col = 32 * gq + 2 * m;
-          const float a = col <= tid ? __uint_as_float(r[2 * m]) * ps : 0.f;
-          const float c = col + 1 <= tid ? __uint_as_float(r[2 * m + 1]) * ps : 0.f;
-          pk[m] = pack_f16x2(a, c);
-          bad |= f16x2_nonfinite(pk[m]);
-        }
-        tc_st16(t_p + lane_off + 16 * gq, pk);
+      for (int m = 0; m < 16; ++m) {
+        const int col = 32 * cg + 2 * m;
+        const float a = col <= trow ? __uint_as_float(r[2 * m]) * ps : 0.f;
+        const float c = col + 1 <= trow ? __uint_as_float(r[2 * m + 1]) * ps : 0.f;
+        pk[m] = pack_f16x2(a, c);
+        bad |= f16x2_nonfinite(pk[m]);
       }
+      tc_st16(t_p16 + lane_off + 16 * cg, pk);
       tc_wait_st();
     }
     // ---- S (now inclusive of this chunk) -> fp16 operand copy for the next chunk
     int e_next = e_cur;
     if (u + 1 < nchunks) {
+      uint32_t r[32];
+      tc_ld32(t_s + lane_off + 32 * cg, r);
+      tc_wait_ld();
       float mx = 0.f;
-#pragma unroll 1
-      for (int gq = 0; gq < 4; ++gq) {
-        uint32_t r[32];
-        tc_ld32(t_s + lane_off + 32 * gq, r);
-        tc_wait_ld();
 #pragma unroll
-        for (int m = 0; m < 32; ++m) mx = fmaxf(mx, fabsf(__uint_as_float(r[m])));
-      }
+      for (int m = 0; m < 32; ++m) mx = fmaxf(mx, fabsf(__uint_as_float(r[m])));
       e_next = tc_block_scale_exp(mx, red);
       const float sc = pow2i(-e_next);
-#pragma unroll 1
-      for (int gq = 0; gq < 4; ++gq) {
-        uint32_t r[32];
-        tc_ld32(t_s + lane_off + 32 * gq, r);
-        tc_wait_ld();
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          float f[8];
+      for (int c4 = 0; c4 < 4; ++c4) {
+        float f[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(r[8 * c4 + e]) * sc;
-          const int cj = 4 * gq + c4;
-          *reinterpret_cast<uint4*>(sop + (cj >> 3) * kTcSlab + swz128(tid, cj & 7)) =
-              f32x8_to_f16(f);
-        }
+        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(r[8 * c4 + e]) * sc;
+        const int cj = 4 * cg + c4;
+        *reinterpret_cast<uint4*>(sop + (cj >> 3) * kTcSlab + swz128(trow, cj & 7)) =
+            f32x8_to_f16(f);
       }
       fence_proxy_async_smem();
     }
@@ -386,7 +393,8 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) tc_mma_ts(t_o, t_p + 8 * kk, tc_desc_mn(sV, kk), kIdPV, 1u);
+      for (int kk = 0; kk < 8; ++kk)
+        tc_mma_ts(t_o, t_p16 + 8 * kk, tc_desc_mn(sV, kk), kIdPV, 1u);
       tc_commit(mma_bar);
     }
     ok = mbar_wait(mma_bar, mma_phase & 1);
@@ -398,33 +406,31 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     // ---- epilogue: y = sigmoid(g) * 2^e * O
     {
       const float os = pow2i(e_cur);
-      const bool live = t < p.T;
-      const __nv_bfloat16* gr = p.g ? p.g + b * p.sg.b + t * p.sg.t + (int64_t)h * p.sg.h : nullptr;
-      __nv_bfloat16* orow = p.o + b * p.so.b + t * p.so.t + (int64_t)h * p.so.h;
-#pragma unroll 1
-      for (int gq = 0; gq < 4; ++gq) {
-        uint32_t r[32];
-        tc_ld32(t_o + lane_off + 32 * gq, r);
-        tc_wait_ld();
-        if (live) {
+      const int64_t t = chunk_t0 + trow;
+      uint32_t r[32];
+      tc_ld32(t_o + lane_off + 32 * cg, r);
+      tc_wait_ld();
+      if (t < p.T) {
+        const __nv_bfloat16* gr =
+            p.g ? p.g + b * p.sg.b + t * p.sg.t + (int64_t)h * p.sg.h + 32 * cg : nullptr;
+        __nv_bfloat16* orow = p.o + b * p.so.b + t * p.so.t + (int64_t)h * p.so.h + 32 * cg;
 #pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8) {
-            float y[8];
+        for (int c8 = 0; c8 < 4; ++c8) {
+          float y[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) y[e] = __uint_as_float(r[8 * c8 + e]) * os;
-            if (gr) {
-              float gf[8];
-              bf16x8_to_f32(*reinterpret_cast<const uint4*>(gr + 32 * gq + 8 * c8), gf);
+          for (int e = 0; e < 8; ++e) y[e] = __uint_as_float(r[8 * c8 + e]) * os;
+          if (gr) {
+            float gf[8];
+            bf16x8_to_f32(*reinterpret_cast<const uint4*>(gr + 8 * c8), gf);
 #pragma unroll
-              for (int e = 0; e < 8; ++e) y[e] *= sigmoidf_(gf[e]);
-            }
-            uint4 w;
-            __nv_bfloat162 h0 = __floats2bfloat162_rn(y[0], y[1]), h1 = __floats2bfloat162_rn(y[2], y[3]);
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(y[4], y[5]), h3 = __floats2bfloat162_rn(y[6], y[7]);
-            w.x = *reinterpret_cast<uint32_t*>(&h0); w.y = *reinterpret_cast<uint32_t*>(&h1);
-            w.z = *reinterpret_cast<uint32_t*>(&h2); w.w = *reinterpret_cast<uint32_t*>(&h3);
-            *reinterpret_cast<uint4*>(orow + 32 * gq + 8 * c8) = w;
+            for (int e = 0; e < 8; ++e) y[e] *= sigmoidf_(gf[e]);
           }
+          uint4 w;
+          __nv_bfloat162 h0 = __floats2bfloat162_rn(y[0], y[1]), h1 = __floats2bfloat162_rn(y[2], y[3]);
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(y[4], y[5]), h3 = __floats2bfloat162_rn(y[6], y[7]);
+          w.x = *reinterpret_cast<uint32_t*>(&h0); w.y = *reinterpret_cast<uint32_t*>(&h1);
+          w.z = *reinterpret_cast<uint32_t*>(&h2); w.w = *reinterpret_cast<uint32_t*>(&h3);
+          *reinterpret_cast<uint4*>(orow + 8 * c8) = w;
         }
       }
     }
@@ -433,22 +439,19 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   }
 
   if (kStateOnly && ok && nchunks > 0) {
-    float* srow = wseg + (size_t)tid * 128;
-#pragma unroll 1
-    for (int gq = 0; gq < 4; ++gq) {
-      uint32_t r[32];
-      tc_ld32(t_s + lane_off + 32 * gq, r);
-      tc_wait_ld();
+    float* dst = wseg + (size_t)trow * 128 + 32 * cg;
+    uint32_t r[32];
+    tc_ld32(t_s + lane_off + 32 * cg, r);
+    tc_wait_ld();
 #pragma unroll
-      for (int v4 = 0; v4 < 8; ++v4)
-        *reinterpret_cast<float4*>(srow + 32 * gq + 4 * v4) =
-            make_float4(__uint_as_float(r[4 * v4]), __uint_as_float(r[4 * v4 + 1]),
-                        __uint_as_float(r[4 * v4 + 2]), __uint_as_float(r[4 * v4 + 3]));
-    }
+    for (int v4 = 0; v4 < 8; ++v4)
+      *reinterpret_cast<float4*>(dst + 4 * v4) =
+          make_float4(__uint_as_float(r[4 * v4]), __uint_as_float(r[4 * v4 + 1]),
+                      __uint_as_float(r[4 * v4 + 2]), __uint_as_float(r[4 * v4 + 3]));
   }
-  if (__any_sync(0xffffffffu, bad) && (tid & 31) == 0) raise_device_error(SALA_ERR_RANGE);
+  if (__any_sync(0xffffffffu, bad) && lane == 0) raise_device_error(SALA_ERR_RANGE);
   if (!ok && tid == 0) {
-    // wind down: let every issued copy land before the CTA's shared memory goes away
+    // wind down: let the last issued copies land before the CTA's shared memory goes away
     for (int u = issued > 2 ? issued - 2 : 0; u < issued; ++u) mbar_wait(&full[u & 1], (u >> 1) & 1);
   }
   tc_fence_before();

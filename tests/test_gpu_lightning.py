@@ -150,3 +150,34 @@ def test_decode_continues_prefill():
     y = sala.lightning_decode(dq[:, T], dk[:, T], dv[:, T], dg[:, T], S, pos)
     yr, _ = oracle.lightning_recurrent(*(_np(t) for t in (x.q, x.k, x.v, x.g)), rows=[T])
     assert rel_err(_np(y), yr[:, 0], True) <= TOL_BF16
+
+
+def test_lightning_large_state_rescaling():
+    """Keys nearly constant and values ~500: the state grows past the fp16 range
+    within one chunk, so the tensor-core path must rescale its fp16 copy of S by
+    powers of two; the result must still match the oracle."""
+    B, T, H, D = 1, 1000, 2, 128
+    gen = inputs.generator(4242)
+    base = inputs.randn((1, 1, H, D), gen, torch.float32)
+    k = (base + 0.01 * inputs.randn((B, T, H, D), gen, torch.float32)).to(torch.bfloat16)
+    q = inputs.randn((B, T, H, D), gen)
+    v = (500.0 + inputs.randn((B, T, H, D), gen, torch.float32)).to(torch.bfloat16)
+    g = inputs.randn((B, T, H, D), gen)
+    y, S = sala.lightning_prefill(q.cuda(), k.cuda(), v.cuda(), g.cuda(), chunk=128)
+    yr, Sr = oracle.lightning_recurrent(_np(q), _np(k), _np(v), _np(g))
+    assert float(np.abs(Sr).max()) > 65504.0  # the state really left the fp16 range
+    assert rel_err(_np(y), yr, True) <= TOL_BF16
+    assert rel_err(_np(S), Sr, False) <= TOL_BF16
+    assert sala.get_device_error() == 0
+
+
+def test_lightning_flags_fp16_range():
+    """A value outside the fp16 operand range sets SALA_ERR_RANGE in the device word."""
+    B, T, H, D = 1, 256, 1, 128
+    x = inputs.lightning_inputs(B, T, H, D, seed=3)
+    v = x.v.clone()
+    v[0, 17, 0, 5] = 1.0e6
+    sala.get_device_error()
+    sala.lightning_prefill(x.q.cuda(), x.k.cuda(), v.cuda(), x.g.cuda(), chunk=128)
+    assert sala.get_device_error() == 6
+    assert sala.get_device_error() == 0
