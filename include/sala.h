@@ -176,6 +176,38 @@ sala_status sala_sparse_attn(const void *q, const void *k, const void *v, const 
                              sala_dtype dt, void *stream);
 
 /*
+ * Lightning prefill that allocates nothing (no counterpart in the paper: this is
+ * a library convenience).  Some callers cannot hand the library a workspace:
+ * code embedded in a host framework that owns all device memory and offers its
+ * plugins no allocator, or a serving loop whose memory pool is frozen after
+ * start-up and must not call cudaMalloc on the hot path.  This entry point takes
+ * the same arguments as sala_lightning_prefill minus the workspace and keeps its
+ * per-segment state scratch in a fixed 16 MiB array that lives in the library's
+ * device image (every GPU that loads the library holds it until exit).
+ *
+ * Limits: the bf16 / head_dim 128 / chunk 128 path needs B*H <= 256 (one 64 KiB
+ * state per segment, at least one segment per head); larger B*H returns
+ * SALA_ERR_WORKSPACE before any launch.  With fewer segments than the regular
+ * entry point it runs fewer CTAs, so it is slower for small B*H.  Other
+ * dtype/head_dim/chunk combinations need no scratch and behave exactly like
+ * sala_lightning_prefill.
+ * Set-up: the first call on each device looks up the device address of the
+ * scratch array (so make that first call before any stream capture).
+ * Concurrency: every call on a device shares the one scratch array and leaves
+ * its contents behind; calls that can overlap on the GPU (different streams,
+ * or several threads) race on it and must be serialised by the caller.
+ * Calls no cudaMalloc/cudaFree and no allocating library routine.
+ */
+sala_status sala_lightning_prefill_noalloc(const void *q, const void *k, const void *v,
+                                           const void *g, void *o, float *state,
+                                           const float *q_norm_w, const float *k_norm_w, int B,
+                                           int T, int H, int D, sala_strides sq,
+                                           sala_strides sk, sala_strides sv, sala_strides sg,
+                                           sala_strides so, int chunk, int64_t pos0,
+                                           float rope_base, float eps, int init_zero,
+                                           sala_dtype dt, void *stream);
+
+/*
  * Synchronise `stream`, then read and clear the device error word of the
  * current device.  Returns SALA_OK, SALA_ERR_RANGE or SALA_ERR_TIMEOUT (the
  * first condition raised since the last call), or SALA_ERR_CUDA if the

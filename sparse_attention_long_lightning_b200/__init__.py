@@ -17,6 +17,7 @@ import torch
 
 __all__ = [
     "SalaError", "load_library", "lightning_prefill", "lightning_prefill_workspace",
+    "lightning_prefill_noalloc",
     "lightning_decode", "sparse_select", "sparse_select_workspace", "sparse_attn",
     "get_device_error", "status_string", "version", "LIB_PATH",
 ]
@@ -57,6 +58,9 @@ def load_library(path: Optional[str] = None):
     lib.sala_lightning_prefill.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, S, S, S, S,
                                            S, i, i64, f, f, i, vp, sz, i, vp]
     lib.sala_lightning_prefill.restype = i
+    lib.sala_lightning_prefill_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, S,
+                                                   S, S, S, S, i, i64, f, f, i, i, vp]
+    lib.sala_lightning_prefill_noalloc.restype = i
     lib.sala_lightning_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, S, S, S, S,
                                           S, f, f, i, vp]
     lib.sala_lightning_decode.restype = i
@@ -155,6 +159,28 @@ def lightning_prefill(q, k, v, g=None, state=None, q_norm_w=None, k_norm_w=None,
         _s4(q), _s4(k), _s4(v), _s4(g), _s4(out), int(chunk), int(pos0), float(rope_base),
         float(eps), init_zero, _p(workspace), wsb, _dt(q), _stream(stream))
     _check("sala_lightning_prefill", st)
+    return out, state
+
+
+def lightning_prefill_noalloc(q, k, v, g, state, out, q_norm_w=None, k_norm_w=None, *, chunk=128,
+                              pos0=0, rope_base=10000.0, eps=1e-6, init_zero=False, stream=None):
+    """Lightning prefill through the entry point that allocates nothing.
+
+    For callers that cannot give the library a workspace (a host framework that
+    owns all device memory, or a serving loop whose pool is frozen): the library
+    keeps the per-segment scratch in a fixed 16 MiB device array instead.  The
+    caller passes preallocated `state` ([B,H,D,D] fp32, in/out) and `out`; with
+    init_zero the incoming state is ignored.  Calls that may overlap on the GPU
+    share that array and must be serialised.  B*H above 256 raises SalaError
+    (SALA_ERR_WORKSPACE) for the bf16 / head_dim 128 / chunk 128 path."""
+    lib = load_library()
+    _cuda(q, k, v, g, state, out)
+    B, T, H, D = q.shape
+    st = lib.sala_lightning_prefill_noalloc(
+        _p(q), _p(k), _p(v), _p(g), _p(out), _p(state), _p(q_norm_w), _p(k_norm_w), B, T, H, D,
+        _s4(q), _s4(k), _s4(v), _s4(g), _s4(out), int(chunk), int(pos0), float(rope_base),
+        float(eps), 1 if init_zero else 0, _dt(q), _stream(stream))
+    _check("sala_lightning_prefill_noalloc", st)
     return out, state
 
 

@@ -367,6 +367,102 @@ sala_status sala_sparse_attn(const void* q, const void* k, const void* v, const 
   return SALA_OK;
 }
 
+// ------------------------------------------------------------------ no-allocation prefill
+}  // extern "C"
+
+namespace {
+
+// Fixed scratch for sala_lightning_prefill_noalloc: room for 256 fp32 128x128
+// segment states.  Host code may not use the symbol itself as a device address;
+// the per-device address comes from cudaGetSymbolAddress below.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[256] = {};
+
+// Device address of the scratch array for the current device (looked up once).
+void* noalloc_scratch_address() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return nullptr;
+    }
+    g_noalloc_addr[dev] = ptr;
+  }
+  return g_noalloc_addr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+sala_status sala_lightning_prefill_noalloc(const void* q, const void* k, const void* v,
+                                           const void* g, void* o, float* state,
+                                           const float* q_norm_w, const float* k_norm_w, int B,
+                                           int T, int H, int D, sala_strides sq,
+                                           sala_strides sk, sala_strides sv, sala_strides sg,
+                                           sala_strides so, int chunk, int64_t pos0,
+                                           float rope_base, float eps, int init_zero,
+                                           sala_dtype dt, void* stream) {
+  const bool tc_path = dt == SALA_BF16 && D == 128 && chunk == kTcC;
+  if (!tc_path || T <= 0)  // these paths use no scratch at all
+    return sala_lightning_prefill(q, k, v, g, o, state, q_norm_w, k_norm_w, B, T, H, D, sq, sk,
+                                  sv, sg, so, chunk, pos0, rope_base, eps, init_zero, nullptr, 0,
+                                  dt, stream);
+  if (!state || !q || !k || !v || !o) return SALA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || pos0 < 0 || !(rope_base > 1.0f) || !(eps >= 0.0f))
+    return SALA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(state) ||
+      (g && !aligned16(g)))
+    return SALA_ERR_INVALID_ARG;
+  if (!strides_ok(sq, 2) || !strides_ok(sk, 2) || !strides_ok(sv, 2) || !strides_ok(so, 2) ||
+      (g && !strides_ok(sg, 2)))
+    return SALA_ERR_INVALID_ARG;
+  constexpr int64_t kStateBytes = 128 * 128 * sizeof(float);
+  const int64_t capacity = (int64_t)(kNoAllocScratchBytes / kStateBytes);  // segment states
+  if ((int64_t)B * H > capacity) return SALA_ERR_WORKSPACE;
+  void* scratch = noalloc_scratch_address();
+  if (!scratch) return SALA_ERR_CUDA;
+  cudaStream_t st = as_stream(stream);
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_bhtd(&tq, q, B, T, H, D, sq, kTcC) || !make_tmap_bhtd(&tk, k, B, T, H, D, sk, kTcC) ||
+      !make_tmap_bhtd(&tv, v, B, T, H, D, sv, kTcC))
+    return SALA_ERR_CUDA;
+  TcParams p;
+  p.g = (const __nv_bfloat16*)g;
+  p.o = (__nv_bfloat16*)o;
+  p.qw = q_norm_w;
+  p.kw = k_norm_w;
+  p.ws = (float*)scratch;
+  p.sg = sg;
+  p.so = so;
+  p.B = B; p.T = T; p.H = H;
+  p.NC = (T + kTcC - 1) / kTcC;
+  int G = lightning_tc_segments(B, H, T, num_sms());
+  const int g_cap = (int)(capacity / ((int64_t)B * H));
+  if (G > g_cap) G = g_cap;
+  p.G = G;
+  p.pos0 = pos0;
+  p.log2_base = std::log2((double)rope_base);
+  p.eps = eps;
+  const unsigned grid = (unsigned)(B * H * p.G);
+  auto ka = lightning_tc_kernel<true>;
+  auto kc = lightning_tc_kernel<false>;
+  if (!set_smem(ka, TcSmem<true>::bytes) || !set_smem(kc, TcSmem<false>::bytes)) return SALA_ERR_CUDA;
+  ka<<<grid, kTcThreads, TcSmem<true>::bytes, st>>>(tk, tk, tv, p);
+  SALA_CHECK_LAUNCH();
+  lightning_scan_kernel<<<B * H, 256, 0, st>>>(p.ws, state, p.G, init_zero);
+  SALA_CHECK_LAUNCH();
+  kc<<<grid, kTcThreads, TcSmem<false>::bytes, st>>>(tq, tk, tv, p);
+  SALA_CHECK_LAUNCH();
+  return SALA_OK;
+}
+
 // ------------------------------------------------------------------ device error word
 sala_status sala_get_device_error(void* stream) {
   if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) {

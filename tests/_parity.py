@@ -26,6 +26,18 @@ def rel_err(out, ref, bf16_out: bool) -> float:
     return float(err.max() / rms) if rms > 0 else float(err.max())
 
 
+def rel_err_bf16_pair(a, b) -> float:
+    """Same 1e-2 rule for two bf16 OUTPUTS of the library (no fp64 reference):
+    each side was rounded to bf16 once, so half an ulp of each is allowed."""
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    def half_ulp(x):
+        return np.exp2(np.floor(np.log2(np.maximum(np.abs(x), 1e-30))) - 8)
+    err = np.maximum(np.abs(a - b) - half_ulp(a) - half_ulp(b), 0.0)
+    rms = np.sqrt(np.mean(b * b))
+    return float(err.max() / rms) if rms > 0 else float(err.max())
+
+
 def raw_rel_err(out, ref) -> float:
     out = np.asarray(out, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
