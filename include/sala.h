@@ -165,8 +165,8 @@ sala_status sala_sparse_select(const void *q, const void *k, int B, int T, int H
  *   q, g, o     [B,T,Hq,D] (g may be NULL), k, v [B,T,Hkv,D] (bf16)
  *   idx         [B,Hkv,T,n_sel] int32, contiguous, entries in [-1, ceil(T/block))
  *   scale       softmax scale; 0 selects 1/sqrt(D)
- *   block = 64, D = 64 or 128, Hq / Hkv = 16 (the GQA group fills one
- *   16-row tensor-core tile).
+ *   block = 64, D = 64 or 128, 1 <= Hq / Hkv <= 16 (the GQA group fills one
+ *   16-row tensor-core tile, padded with zero rows when smaller).
  * Errors: INVALID_ARG, UNSUPPORTED, CUDA.
  */
 sala_status sala_sparse_attn(const void *q, const void *k, const void *v, const void *g,

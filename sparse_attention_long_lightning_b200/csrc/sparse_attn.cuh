@@ -14,8 +14,9 @@
 // K and V (128-byte swizzle, no multicast) into the group's NS-deep ring,
 // recording the block id beside the stage.  Each group has four consumer
 // warps that split every 64-key block 16 keys apiece: the group's 16 query
-// heads form the M = 16 operand of m16n8k16 tensor-core MMAs (Q K^T in bf16,
-// P V in fp16, fp32 accumulation), the online softmax runs per warp in
+// heads form the M = 16 operand of m16n8k16 tensor-core MMAs (Q K^T in bf16;
+// P V with P split into bf16 high and low parts, so V is used exactly as
+// stored; fp32 accumulation), the online softmax runs per warp in
 // registers with a lazily raised reference maximum (rescaling only when a
 // score exceeds it by more than 2^8), and the four partial (max, sum, O)
 // triples are merged through shared memory at the end of the row.  All waits
@@ -201,9 +202,10 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
       const uint32_t kb = smem_u32(stages + size_t(s) * L::kStage);
       const uint32_t vb = kb + L::kTile;
 
-      // ---- S = Q K^T for keys 16*wq .. 16*wq+15 of the block
-      float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      // ---- S = Q K^T for keys 16*wq .. 16*wq+15 of the block (4 independent chains)
+      float sc[2][4];
       {
+        float sx[2][2][4] = {};
         const int mat = lane >> 3, rin = lane & 7;
         const uint32_t krow = wq * 16 + (mat >> 1) * 8 + rin;
 #pragma unroll
@@ -212,9 +214,13 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
           const uint32_t addr = kb + (chunk >> 3) * L::kHalf + swz128(krow, chunk & 7);
           uint32_t b0, b1, b2, b3;
           ldsm_x4(addr, b0, b1, b2, b3);
-          mma_bf16_16816(sc[0], qa[kk], b0, b1);
-          mma_bf16_16816(sc[1], qa[kk], b2, b3);
+          mma_bf16_16816(sx[0][kk & 1], qa[kk], b0, b1);
+          mma_bf16_16816(sx[1][kk & 1], qa[kk], b2, b3);
         }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) sc[nt][c] = sx[nt][0][c] + sx[nt][1][c];
       }
       // ---- scale; causal mask only where the block reaches past t
       const bool straddle = (int64_t)j * kSaBlk + kSaBlk - 1 > t;
@@ -251,17 +257,24 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
         }
       }
       const float mu0 = m0 == -INFINITY ? 0.f : m0, mu1 = m1 == -INFINITY ? 0.f : m1;
-      uint32_t pa[4];
+      // P = P_hi + P_lo, both bf16 (exact to 2^-16 relative), so V stays bf16
+      uint32_t ph[4], pl[4];
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
         const float p0 = exp2f(sc[nt][0] - mu0), p1 = exp2f(sc[nt][1] - mu0);
         const float p2 = exp2f(sc[nt][2] - mu1), p3 = exp2f(sc[nt][3] - mu1);
         l0 += p0 + p1;
         l1 += p2 + p3;
-        pa[nt * 2 + 0] = pack_f16x2(p0, p1);
-        pa[nt * 2 + 1] = pack_f16x2(p2, p3);
+        const __nv_bfloat162 h01 = __floats2bfloat162_rn(p0, p1);
+        const __nv_bfloat162 h23 = __floats2bfloat162_rn(p2, p3);
+        const __nv_bfloat162 l01 = __floats2bfloat162_rn(p0 - __low2float(h01), p1 - __high2float(h01));
+        const __nv_bfloat162 l23 = __floats2bfloat162_rn(p2 - __low2float(h23), p3 - __high2float(h23));
+        ph[nt * 2 + 0] = *reinterpret_cast<const uint32_t*>(&h01);
+        ph[nt * 2 + 1] = *reinterpret_cast<const uint32_t*>(&h23);
+        pl[nt * 2 + 0] = *reinterpret_cast<const uint32_t*>(&l01);
+        pl[nt * 2 + 1] = *reinterpret_cast<const uint32_t*>(&l23);
       }
-      // ---- O += P V (V converted bf16 -> fp16 in registers)
+      // ---- O += P V
       {
         const int mat = lane >> 3, rin = lane & 7;
         const uint32_t vrow = wq * 16 + (mat & 1) * 8 + rin;
@@ -271,8 +284,10 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
           const uint32_t addr = vb + (chunk >> 3) * L::kHalf + swz128(vrow, chunk & 7);
           uint32_t v0, v1, v2, v3;
           ldsm_x4_t(addr, v0, v1, v2, v3);
-          mma_f16_16816(oacc[2 * pp], pa, bf16x2_to_f16x2(v0), bf16x2_to_f16x2(v1));
-          mma_f16_16816(oacc[2 * pp + 1], pa, bf16x2_to_f16x2(v2), bf16x2_to_f16x2(v3));
+          mma_bf16_16816(oacc[2 * pp], ph, v0, v1);
+          mma_bf16_16816(oacc[2 * pp + 1], ph, v2, v3);
+          mma_bf16_16816(oacc[2 * pp], pl, v0, v1);
+          mma_bf16_16816(oacc[2 * pp + 1], pl, v2, v3);
         }
       }
       __syncwarp();
@@ -363,30 +378,6 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s_last]);
   }
-}
-
-// Values of a bf16 [B, T, H, D] tensor that would not survive conversion to the
-// fp16 tensor-core operand (|x| >= 65536 in bf16, inf or NaN) raise SALA_ERR_RANGE.
-__global__ void __launch_bounds__(256)
-f16_range_check_kernel(const __nv_bfloat16* __restrict__ x, sala_strides s, int B, int T, int H,
-                       int D) {
-  const int64_t rows = (int64_t)B * T * H;
-  const int per_row = D / 8;
-  uint32_t bad = 0;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < rows * per_row;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t row = i / per_row;
-    const int c = (int)(i % per_row);
-    const int h = (int)(row % H);
-    const int64_t t = (row / H) % T;
-    const int b = (int)(row / ((int64_t)H * T));
-    const uint4 u = *reinterpret_cast<const uint4*>(x + b * s.b + t * s.t + h * s.h + 8 * c);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-      bad |= ((w[k] & 0x7fffu) >= 0x4780u) | (((w[k] >> 16) & 0x7fffu) >= 0x4780u);
-  }
-  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) raise_device_error(SALA_ERR_RANGE);
 }
 
 }  // namespace sala
