@@ -48,7 +48,7 @@ template <bool kStateOnly>
 struct TcSmem {
   static constexpr int kStageBytes = (kStateOnly ? 2 : 3) * kTcTile;
   static constexpr int kSop = kStateOnly ? 0 : kTcTile;
-  static constexpr int kMisc = 1024;
+  static constexpr int kMisc = 2048;
   static constexpr size_t bytes = 1024 /*alignment slack*/ + 2 * size_t(kStageBytes) + kSop + kMisc;
   static constexpr uint32_t kTmemCols = kStateOnly ? 128 : 512;
 };
@@ -109,8 +109,8 @@ __device__ __forceinline__ uint32_t f16x8_nonfinite(const uint4& u) {
 // value is not finite.
 template <bool kWithQ>
 __device__ __forceinline__ uint32_t tc_prep_quarter(uint8_t* sQ, uint8_t* sK, uint8_t* sV, int r,
-                                                    int qd, int64_t pos, const TcParams& p,
-                                                    const double* inv_freq) {
+                                                    int qd, const TcParams& p,
+                                                    const float2* ang_base) {
   float ssq = 0.f, ssk = 0.f;
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
@@ -133,8 +133,7 @@ __device__ __forceinline__ uint32_t tc_prep_quarter(uint8_t* sQ, uint8_t* sK, ui
   const float rk = rsqrtf(ssk * (1.0f / 128.0f) + p.eps);
   const float rq = rsqrtf(ssq * (1.0f / 128.0f) + p.eps);
   uint32_t bad = 0;
-  const double two_pi = 6.283185307179586476925286766559;
-  const double inv_two_pi = 0.15915494309189533576888376337251;
+  const float two_pi = 6.28318530717958647692f, inv_two_pi = 0.15915494309189533577f;
 #pragma unroll
   for (int jj = 0; jj < 2; ++jj) {
     const int j = 2 * qd + jj;
@@ -149,8 +148,10 @@ __device__ __forceinline__ uint32_t tc_prep_quarter(uint8_t* sQ, uint8_t* sK, ui
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const int i = 8 * j + e;  // rotation pair (i, i + 64)
-      const double a = (double)pos * inv_freq[i];
-      const float ang = (float)(a - rint(a * inv_two_pi) * two_pi);
+      // angle = (chunk base angle, reduced in fp64) + r * inv_freq_i, re-reduced in fp32
+      const float2 bf = ang_base[i];
+      float ang = fmaf((float)r, bf.y, bf.x);
+      ang = fmaf(-rintf(ang * inv_two_pi), two_pi, ang);
       float sn, cs;
       __sincosf(ang, &sn, &cs);
       const float wk0 = p.kw ? __ldg(p.kw + i) : 1.f, wk1 = p.kw ? __ldg(p.kw + i + 64) : 1.f;
@@ -201,6 +202,41 @@ __device__ __forceinline__ uint64_t tc_desc_mn(const uint8_t* base, int kk) {
   return umma_desc_sw128(smem_u32(base) + kk * 2048, kTcSlab, 1024);
 }
 
+// Gated bf16 epilogue of one chunk: thread (trow, cg) reads 32 fp32 columns of O from
+// TMEM, scales by 2^e, multiplies by sigmoid(g) (prefetched) and stores 64 bytes.
+__device__ __forceinline__ void tc_epilogue(uint32_t t_o, const uint4 (&gv)[4], bool gated,
+                                            float os, __nv_bfloat16* orow, bool live) {
+  uint32_t r[32];
+  tc_ld32(t_o, r);
+  tc_wait_ld();
+  if (!live) return;
+#pragma unroll
+  for (int c8 = 0; c8 < 4; ++c8) {
+    float y[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) y[e] = __uint_as_float(r[8 * c8 + e]) * os;
+    if (gated) {
+      float gf[8];
+      bf16x8_to_f32(gv[c8], gf);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) y[e] *= sigmoidf_(gf[e]);
+    }
+    uint4 w;
+    __nv_bfloat162 h0 = __floats2bfloat162_rn(y[0], y[1]), h1 = __floats2bfloat162_rn(y[2], y[3]);
+    __nv_bfloat162 h2 = __floats2bfloat162_rn(y[4], y[5]), h3 = __floats2bfloat162_rn(y[6], y[7]);
+    w.x = *reinterpret_cast<uint32_t*>(&h0); w.y = *reinterpret_cast<uint32_t*>(&h1);
+    w.z = *reinterpret_cast<uint32_t*>(&h2); w.w = *reinterpret_cast<uint32_t*>(&h3);
+    *reinterpret_cast<uint4*>(orow + 8 * c8) = w;
+  }
+}
+
+// Software pipeline per CTA (one segment of one head), chunk u:
+//   A  wait TMA(u); prep(u) in place                      [tensor core: PV(u-1)]
+//   B  wait PV(u-1); TMA(u+1) into the freed stage; issue score/inter/state MMAs of u
+//   C  epilogue(u-1) from the other O buffer             [tensor core: MMAs of u]
+//   D  wait MMAs of u; P -> masked fp16 (in place, TMEM); S -> fp16 operand for u+1
+//   E  issue PV(u)
+// TMEM columns: P fp32 [0,128) with its fp16 copy in [0,64), O[2] [128,384), S [384,512).
 template <bool kStateOnly>
 __global__ void __launch_bounds__(kTcThreads, 1)
 lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
@@ -218,16 +254,16 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   uint8_t* sop = smem + 2 * L::kStageBytes;
   uint8_t* misc = sop + L::kSop;
   uint64_t* full = reinterpret_cast<uint64_t*>(misc);      // [2]
-  uint64_t* mma_bar = full + 2;                            // [1]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_bar + 1);
+  uint64_t* mma1_bar = full + 2;                           // score/inter/state done
+  uint64_t* mma2_bar = full + 3;                           // PV done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(full + 4);
   float* red = reinterpret_cast<float*>(misc + 64);        // [16]
   double* inv_freq = reinterpret_cast<double*>(misc + 128);  // [64]
+  float2* ang_tab = reinterpret_cast<float2*>(misc + 640);   // [2][64]: (base angle, inv_freq)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // prep mapping: 4 lanes per token row
-  const int prow = 8 * warp + (lane >> 2), pqd = lane & 3;
-  // TMEM mapping: warp w reads lanes 32*(w%4).. (rows), columns 32*(w/4)..
-  const int lq = warp & 3, cg = warp >> 2;
+  const int prow = 8 * warp + (lane >> 2), pqd = lane & 3;  // prep: 4 lanes per row
+  const int lq = warp & 3, cg = warp >> 2;                  // TMEM: lanes 32lq.., cols 32cg..
   const int trow = 32 * lq + lane;
   const int seg = blockIdx.x % p.G;
   const int bh = blockIdx.x / p.G;
@@ -239,7 +275,8 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   if (tid == 0) {
     mbar_init(&full[0], 1);
     mbar_init(&full[1], 1);
-    mbar_init(mma_bar, 1);
+    mbar_init(mma1_bar, 1);
+    mbar_init(mma2_bar, 1);
     fence_mbar_init();
   }
   if (warp == 0) tc_alloc(tmem_slot, L::kTmemCols);
@@ -248,11 +285,18 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // columns: P fp32 [0,128), O [128,256), S [256,384), P fp16 copy [384,448)
-  const uint32_t t_p = tmem, t_o = tmem + 128, t_s = kStateOnly ? tmem : tmem + 256;
-  const uint32_t t_p16 = tmem + 384;
+  const uint32_t t_p = tmem, t_o0 = tmem + 128, t_s = kStateOnly ? tmem : tmem + 384;
   const uint32_t lane_off = (uint32_t)(32 * lq) << 16;
 
+  // base angle of each rotation pair at the first token of chunk u (fp64 reduction)
+  auto fill_angles = [&](int u) {
+    if (tid < 64) {
+      const double a = (double)(p.pos0 + (int64_t)(c_begin + u) * kTcC) * inv_freq[tid];
+      const double two_pi = 6.283185307179586476925286766559;
+      const double red_a = a - rint(a * (1.0 / two_pi)) * two_pi;
+      ang_tab[(u & 1) * 64 + tid] = make_float2((float)red_a, (float)inv_freq[tid]);
+    }
+  };
   auto issue = [&](int u) {
     uint8_t* st = stages + (u & 1) * L::kStageBytes;
     const int t0 = (c_begin + u) * kTcC;
@@ -275,9 +319,11 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     prefetch_tmap(&tmv);
     for (; issued < 2 && issued < nchunks; ++issued) issue(issued);
   }
+  __syncthreads();  // inv_freq visible
+  fill_angles(0);
 
   float* wseg = p.ws + ((size_t)bh * p.G + seg) * (128 * 128);
-  int e_cur = 0;
+  int e_cur = 0, e_prev = 0;
   uint32_t bad = 0;
   if (!kStateOnly) {
     // segment start state -> TMEM[S] (fp32) and its fp16 operand copy
@@ -305,30 +351,38 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     }
     fence_proxy_async_smem();
   }
+  __syncthreads();  // angle table for chunk 0 visible
 
-  uint32_t mma_phase = 0;
+  uint32_t ph1 = 0, ph2 = 0;  // completed-phase counters of mma1_bar / mma2_bar
   bool ok = true;
+  uint4 gv[4] = {};           // gate of this thread's row/columns for the pending epilogue
+  const bool gated = p.g != nullptr;
   for (int u = 0; u < nchunks; ++u) {
     const int s = u & 1;
     uint8_t* st = stages + s * L::kStageBytes;
     uint8_t* sQ = st;
     uint8_t* sK = st + (kStateOnly ? 0 : kTcTile);
     uint8_t* sV = sK + kTcTile;
-    const int64_t chunk_t0 = (int64_t)(c_begin + u) * kTcC;
+    // ---- A: prep(u) while the tensor core runs PV(u-1)
     ok = ok && mbar_wait(&full[s], (u >> 1) & 1);
-    if (ok)
-      bad |= tc_prep_quarter<!kStateOnly>(sQ, sK, sV, prow, pqd, p.pos0 + chunk_t0 + prow, p,
-                                          inv_freq);
+    if (ok) bad |= tc_prep_quarter<!kStateOnly>(sQ, sK, sV, prow, pqd, p, ang_tab + s * 64);
     fence_proxy_async_smem();
+    // angles of chunk u+1 (other parity; prep(u-1), the last reader, is behind a barrier)
+    if (u + 1 < nchunks) fill_angles(u + 1);
+    // ---- B: wait for the previous chunk's last MMAs, refill its stage, issue this chunk's
+    if (u > 0) {
+      ok = ok && mbar_wait(kStateOnly ? mma1_bar : mma2_bar,
+                           (kStateOnly ? ph1 : ph2) & 1);
+      if (kStateOnly) ++ph1; else ++ph2;
+    }
     tc_fence_before();
     ok = __syncthreads_and(ok);
     if (!ok) break;
+    tc_fence_after();
     if (tid == 0) {
-      tc_fence_after();
+      if (u > 0 && issued < nchunks) issue(issued++);  // stage of chunk u-1 is free
+      const uint32_t t_o = t_o0 + 128 * (u & 1);
       if (!kStateOnly) {
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          tc_mma_ss(t_p, tc_desc_k(sQ, kk), tc_desc_k(sK, kk), kIdScore, kk > 0);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           tc_mma_ss(t_o, tc_desc_k(sQ, kk), tc_desc_mn(sop, kk), kIdInter, kk > 0);
@@ -337,23 +391,45 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       for (int kk = 0; kk < 8; ++kk)
         tc_mma_ss(t_s, tc_desc_mn(sK, kk), tc_desc_mn(sV, kk), kIdState,
                   (kStateOnly && u == 0 && kk == 0) ? 0u : 1u);
-      tc_commit(mma_bar);
+      if (!kStateOnly) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc_mma_ss(t_p, tc_desc_k(sQ, kk), tc_desc_k(sK, kk), kIdScore, kk > 0);
+      }
+      tc_commit(mma1_bar);
     }
-    ok = mbar_wait(mma_bar, mma_phase & 1);
-    ++mma_phase;
-    tc_fence_after();
-    if (kStateOnly) {
-      ok = __syncthreads_and(ok);
-      if (!ok) break;
-      if (tid == 0 && issued < nchunks) issue(issued++);
-      continue;
+    if (kStateOnly) continue;
+    // ---- C: epilogue(u-1) while the tensor core runs this chunk's MMAs
+    if (u > 0) {
+      const int64_t t = (int64_t)(c_begin + u - 1) * kTcC + trow;
+      __nv_bfloat16* orow = p.o + b * p.so.b + t * p.so.t + (int64_t)h * p.so.h + 32 * cg;
+      tc_epilogue(t_o0 + 128 * ((u - 1) & 1) + lane_off + 32 * cg, gv, gated, pow2i(e_prev),
+                  orow, t < p.T);
     }
-    // ---- P -> causally masked fp16 copy in TMEM, scaled by 2^-e
     {
-      const float ps = pow2i(-e_cur);
-      uint32_t r[32], pk[16];
+      // prefetch this chunk's gate for its epilogue (next iteration)
+      const int64_t t = (int64_t)(c_begin + u) * kTcC + trow;
+      if (gated && t < p.T) {
+        const uint4* gp = reinterpret_cast<const uint4*>(p.g + b * p.sg.b + t * p.sg.t +
+                                                         (int64_t)h * p.sg.h + 32 * cg);
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8) gv[c8] = __ldg(gp + c8);
+      }
+    }
+    // ---- D: P -> masked fp16 copy (in place), S -> fp16 operand for the next chunk
+    ok = mbar_wait(mma1_bar, ph1 & 1);
+    ++ph1;
+    tc_fence_after();
+    {
+      uint32_t r[32];
       tc_ld32(t_p + lane_off + 32 * cg, r);
       tc_wait_ld();
+      tc_fence_before();
+      ok = __syncthreads_and(ok);  // every P column read before any fp16 copy lands on it
+      if (!ok) break;
+      tc_fence_after();
+      const float ps = pow2i(-e_cur);
+      uint32_t pk[16];
 #pragma unroll
       for (int m = 0; m < 16; ++m) {
         const int col = 32 * cg + 2 * m;
@@ -362,11 +438,10 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         pk[m] = pack_f16x2(a, c);
         bad |= f16x2_nonfinite(pk[m]);
       }
-      tc_st16(t_p16 + lane_off + 16 * cg, pk);
+      tc_st16(t_p + lane_off + 16 * cg, pk);
       tc_wait_st();
     }
-    // ---- S (now inclusive of this chunk) -> fp16 operand copy for the next chunk
-    int e_next = e_cur;
+    e_prev = e_cur;
     if (u + 1 < nchunks) {
       uint32_t r[32];
       tc_ld32(t_s + lane_off + 32 * cg, r);
@@ -374,7 +449,7 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       float mx = 0.f;
 #pragma unroll
       for (int m = 0; m < 32; ++m) mx = fmaxf(mx, fabsf(__uint_as_float(r[m])));
-      e_next = tc_block_scale_exp(mx, red);
+      const int e_next = tc_block_scale_exp(mx, red);
       const float sc = pow2i(-e_next);
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) {
@@ -386,68 +461,44 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
             f32x8_to_f16(f);
       }
       fence_proxy_async_smem();
+      e_cur = e_next;
     }
+    // ---- E: PV(u)
     tc_fence_before();
     ok = __syncthreads_and(ok);
     if (!ok) break;
     if (tid == 0) {
       tc_fence_after();
+      const uint32_t t_o = t_o0 + 128 * (u & 1);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        tc_mma_ts(t_o, t_p16 + 8 * kk, tc_desc_mn(sV, kk), kIdPV, 1u);
-      tc_commit(mma_bar);
+      for (int kk = 0; kk < 8; ++kk) tc_mma_ts(t_o, t_p + 8 * kk, tc_desc_mn(sV, kk), kIdPV, 1u);
+      tc_commit(mma2_bar);
     }
-    ok = mbar_wait(mma_bar, mma_phase & 1);
-    ++mma_phase;
-    tc_fence_after();
-    ok = __syncthreads_and(ok);
-    if (!ok) break;
-    if (tid == 0 && issued < nchunks) issue(issued++);
-    // ---- epilogue: y = sigmoid(g) * 2^e * O
-    {
-      const float os = pow2i(e_cur);
-      const int64_t t = chunk_t0 + trow;
-      uint32_t r[32];
-      tc_ld32(t_o + lane_off + 32 * cg, r);
-      tc_wait_ld();
-      if (t < p.T) {
-        const __nv_bfloat16* gr =
-            p.g ? p.g + b * p.sg.b + t * p.sg.t + (int64_t)h * p.sg.h + 32 * cg : nullptr;
-        __nv_bfloat16* orow = p.o + b * p.so.b + t * p.so.t + (int64_t)h * p.so.h + 32 * cg;
-#pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {
-          float y[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) y[e] = __uint_as_float(r[8 * c8 + e]) * os;
-          if (gr) {
-            float gf[8];
-            bf16x8_to_f32(*reinterpret_cast<const uint4*>(gr + 8 * c8), gf);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) y[e] *= sigmoidf_(gf[e]);
-          }
-          uint4 w;
-          __nv_bfloat162 h0 = __floats2bfloat162_rn(y[0], y[1]), h1 = __floats2bfloat162_rn(y[2], y[3]);
-          __nv_bfloat162 h2 = __floats2bfloat162_rn(y[4], y[5]), h3 = __floats2bfloat162_rn(y[6], y[7]);
-          w.x = *reinterpret_cast<uint32_t*>(&h0); w.y = *reinterpret_cast<uint32_t*>(&h1);
-          w.z = *reinterpret_cast<uint32_t*>(&h2); w.w = *reinterpret_cast<uint32_t*>(&h3);
-          *reinterpret_cast<uint4*>(orow + 8 * c8) = w;
-        }
-      }
-    }
-    e_cur = e_next;
-    tc_fence_before();
   }
 
-  if (kStateOnly && ok && nchunks > 0) {
-    float* dst = wseg + (size_t)trow * 128 + 32 * cg;
-    uint32_t r[32];
-    tc_ld32(t_s + lane_off + 32 * cg, r);
-    tc_wait_ld();
+  // drain: the last chunk's MMAs, then its epilogue / the segment sum
+  if (ok && nchunks > 0) {
+    ok = mbar_wait(kStateOnly ? mma1_bar : mma2_bar, (kStateOnly ? ph1 : ph2) & 1);
+    tc_fence_after();
+    if (ok) {
+      if (kStateOnly) {
+        float* dst = wseg + (size_t)trow * 128 + 32 * cg;
+        uint32_t r[32];
+        tc_ld32(t_s + lane_off + 32 * cg, r);
+        tc_wait_ld();
 #pragma unroll
-    for (int v4 = 0; v4 < 8; ++v4)
-      *reinterpret_cast<float4*>(dst + 4 * v4) =
-          make_float4(__uint_as_float(r[4 * v4]), __uint_as_float(r[4 * v4 + 1]),
-                      __uint_as_float(r[4 * v4 + 2]), __uint_as_float(r[4 * v4 + 3]));
+        for (int v4 = 0; v4 < 8; ++v4)
+          *reinterpret_cast<float4*>(dst + 4 * v4) =
+              make_float4(__uint_as_float(r[4 * v4]), __uint_as_float(r[4 * v4 + 1]),
+                          __uint_as_float(r[4 * v4 + 2]), __uint_as_float(r[4 * v4 + 3]));
+      } else {
+        const int u = nchunks;
+        const int64_t t = (int64_t)(c_begin + u - 1) * kTcC + trow;
+        __nv_bfloat16* orow = p.o + b * p.so.b + t * p.so.t + (int64_t)h * p.so.h + 32 * cg;
+        tc_epilogue(t_o0 + 128 * ((u - 1) & 1) + lane_off + 32 * cg, gv, gated, pow2i(e_prev),
+                    orow, t < p.T);
+      }
+    }
   }
   if (__any_sync(0xffffffffu, bad) && lane == 0) raise_device_error(SALA_ERR_RANGE);
   if (!ok && tid == 0) {

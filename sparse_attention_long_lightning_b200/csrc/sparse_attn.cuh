@@ -274,20 +274,26 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
         pl[nt * 2 + 0] = *reinterpret_cast<const uint32_t*>(&l01);
         pl[nt * 2 + 1] = *reinterpret_cast<const uint32_t*>(&l23);
       }
-      // ---- O += P V
+      // ---- O += P V; the low-part MMA of each accumulator trails its high-part MMA by
+      // two iterations so dependent MMAs are never issued back to back
       {
         const int mat = lane >> 3, rin = lane & 7;
         const uint32_t vrow = wq * 16 + (mat & 1) * 8 + rin;
+        uint32_t vv[kNT / 2][4];
 #pragma unroll
-        for (int pp = 0; pp < kNT / 2; ++pp) {
-          const uint32_t chunk = 2 * pp + (mat >> 1);
-          const uint32_t addr = vb + (chunk >> 3) * L::kHalf + swz128(vrow, chunk & 7);
-          uint32_t v0, v1, v2, v3;
-          ldsm_x4_t(addr, v0, v1, v2, v3);
-          mma_bf16_16816(oacc[2 * pp], ph, v0, v1);
-          mma_bf16_16816(oacc[2 * pp + 1], ph, v2, v3);
-          mma_bf16_16816(oacc[2 * pp], pl, v0, v1);
-          mma_bf16_16816(oacc[2 * pp + 1], pl, v2, v3);
+        for (int pp = 0; pp < kNT / 2 + 2; ++pp) {
+          if (pp < kNT / 2) {
+            const uint32_t chunk = 2 * pp + (mat >> 1);
+            const uint32_t addr = vb + (chunk >> 3) * L::kHalf + swz128(vrow, chunk & 7);
+            ldsm_x4_t(addr, vv[pp][0], vv[pp][1], vv[pp][2], vv[pp][3]);
+            mma_bf16_16816(oacc[2 * pp], ph, vv[pp][0], vv[pp][1]);
+            mma_bf16_16816(oacc[2 * pp + 1], ph, vv[pp][2], vv[pp][3]);
+          }
+          if (pp >= 2) {
+            const int qq = pp - 2;
+            mma_bf16_16816(oacc[2 * qq], pl, vv[qq][0], vv[qq][1]);
+            mma_bf16_16816(oacc[2 * qq + 1], pl, vv[qq][2], vv[qq][3]);
+          }
         }
       }
       __syncwarp();
