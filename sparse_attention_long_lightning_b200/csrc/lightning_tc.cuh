@@ -265,8 +265,11 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   const int prow = 8 * warp + (lane >> 2), pqd = lane & 3;  // prep: 4 lanes per row
   const int lq = warp & 3, cg = warp >> 2;                  // TMEM: lanes 32lq.., cols 32cg..
   const int trow = 32 * lq + lane;
-  const int seg = blockIdx.x % p.G;
-  const int bh = blockIdx.x / p.G;
+  // Heads vary fastest across the grid: CTAs running at the same time cover all heads
+  // of the same token range, so whole [H, D] token rows are fetched together (DRAM
+  // row locality) instead of one 256-byte head slice per 8 KB row.
+  const int bh = blockIdx.x % (p.B * p.H);
+  const int seg = blockIdx.x / (p.B * p.H);
   const int b = bh / p.H, h = bh % p.H;
   const int c_begin = (int)((int64_t)seg * p.NC / p.G);
   const int c_end = (int)((int64_t)(seg + 1) * p.NC / p.G);
