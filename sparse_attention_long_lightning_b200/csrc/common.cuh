@@ -40,7 +40,9 @@ __device__ __forceinline__ float ld(const T* p) { return Elem<T>::load(p); }
 template <typename T>
 __device__ __forceinline__ void st(T* p, float x) { Elem<T>::store(p, x); }
 
-__device__ __forceinline__ float sigmoidf_(float z) { return 1.0f / (1.0f + __expf(-z)); }
+// Logistic sigmoid with the fast approximate divide (a few ulp; an exact IEEE
+// division here costs a multi-instruction sequence per output element).
+__device__ __forceinline__ float sigmoidf_(float z) { return __fdividef(1.0f, 1.0f + __expf(-z)); }
 
 // Rotary angle for position `pos` and pair i of a D-dim head, reduced to
 // [-pi, pi] in double precision before the fp32 sine/cosine, so that long
