@@ -17,6 +17,7 @@
 #include "lightning_decode.cuh"
 #include "lightning_tc.cuh"
 #include "sparse_attn.cuh"
+#include "sparse_attn_tc.cuh"
 #include "sparse_select.cuh"
 
 using namespace sala;
@@ -64,10 +65,10 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
-// 4-D bf16 tensor map over a [B, T, H, D] activation with a (64, 1, rows, 1)
+// 4-D bf16 tensor map over a [B, T, H, D] activation with a (64, box_h, rows, 1)
 // box and 128-byte swizzle (64 bf16 = 128 bytes per box row).
 bool make_tmap_bhtd(CUtensorMap* map, const void* base, int B, int T, int H, int D,
-                    const sala_strides& s, int box_rows) {
+                    const sala_strides& s, int box_rows, int box_h = 1) {
   auto enc = get_encode_fn();
   if (!enc) return false;
   cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
@@ -75,7 +76,7 @@ bool make_tmap_bhtd(CUtensorMap* map, const void* base, int B, int T, int H, int
   // Degenerate extents get a harmless stride (never stepped over).
   if (H == 1 && strides[0] == 0) strides[0] = 16;
   if (B == 1 && strides[2] == 0) strides[2] = 16;
-  cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
+  cuuint32_t box[4] = {64, (cuuint32_t)box_h, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -342,10 +343,19 @@ sala_status sala_sparse_attn(const void* q, const void* k, const void* v, const 
   const float sc = scale > 0.0f ? scale : 1.0f / std::sqrt((float)D);
   p.scale_log2 = sc * 1.4426950408889634f;
   p.rows = (int64_t)B * Hkv * T;
+  p.q_box_h = 16;
   cudaStream_t st = as_stream(stream);
   const int64_t want = num_sms();
   const unsigned grid = (unsigned)std::min<int64_t>(want, p.rows);
-  if (D == 128) {
+  if (D == 128 && n_sel <= kStMaxSel) {
+    // tcgen05 path: keys as the MMA M dimension
+    CUtensorMap tq;
+    p.q_box_h = Hq < 16 ? Hq : 16;
+    if (!make_tmap_bhtd(&tq, q, B, T, Hq, D, sq, 1, p.q_box_h)) return SALA_ERR_CUDA;
+    auto kern = sparse_attn_tc_kernel;
+    if (!set_smem(kern, StSmem::bytes)) return SALA_ERR_CUDA;
+    kern<<<grid, kStThreads, StSmem::bytes, st>>>(tq, tk, tv, p);
+  } else if (D == 128) {
     constexpr int NS = 3;
     auto kern = sparse_attn_kernel<128, NS>;
     if (!set_smem(kern, SaSmem<128, NS>::bytes)) return SALA_ERR_CUDA;

@@ -47,7 +47,8 @@ def test_select_batched_strided():
 
 @pytest.mark.parametrize("T,Hq,Hkv,D,topk,gate", [
     (64 * 20 + 17, 16, 2, 128, 4, True), (64 * 9 + 63, 8, 1, 64, 3, False),
-    (33, 16, 1, 128, 64, True), (64 * 12, 16, 1, 128, 64, False)])
+    (33, 16, 1, 128, 64, True), (64 * 12, 16, 1, 128, 64, False),
+    (64 * 9 + 63, 8, 1, 128, 3, True), (64 * 30 + 1, 24, 2, 128, 5, True)])
 def test_sparse_attn_small(T, Hq, Hkv, D, topk, gate):
     s = inputs.sparse_inputs(1, T, Hq, Hkv, D, seed=3 * T + D, gate=gate)
     dq, dk, dv = s.q.cuda(), s.k.cuda(), s.v.cuda()
