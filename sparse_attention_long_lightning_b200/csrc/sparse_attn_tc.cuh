@@ -16,8 +16,9 @@
 // precision.  Accumulators live in tensor memory, so the softmax warps hold no
 // accumulator registers.
 //
-// Roles (192 threads): warps 0-3 softmax + epilogue (thread = TMEM lane: a key of the
-// pair, later a head dimension), warp 4 TMA producer, warp 5 MMA issuer.  The
+// Roles (320 threads): warps 0-7 softmax + epilogue (thread = TMEM lane: a key of the
+// pair, later a head dimension; warps w and w+4 share the lanes and take heads 0-7 and
+// 8-15), warp 8 TMA producer, warp 9 MMA issuer.  The
 // softmax keeps a per-head reference maximum that is raised only when a score
 // exceeds it by more than 2^8 (then O^T and the running sums are rescaled); row sums
 // accumulate per thread and are reduced once per row.  S^T, P^T, Q and O^T are
@@ -29,7 +30,8 @@
 namespace sala {
 
 constexpr int kStNS = 3;                  // K/V pair stages
-constexpr int kStThreads = 192;
+constexpr int kStThreads = 320;          // 8 softmax warps, producer, MMA issuer
+constexpr int kStSoft = 256;
 constexpr int kStHalf = 128 * 128;        // [128 rows x 64 cols] bf16 slab: 16 KB
 constexpr int kStStage = 4 * kStHalf;     // K d-half 0, K d-half 1, V d-half 0, V d-half 1
 constexpr int kStPBuf = 2 * 32 * 128;     // P^T: two 64-key halves of [32 rows x 128 B]
@@ -43,7 +45,7 @@ struct StSmem {
   static constexpr size_t kQ = kP + 2 * kStPBuf;
   static constexpr size_t kList = kQ + 2 * kStQBuf;
   static constexpr size_t kRed = kList + kStMaxSel * 4;     // [4][16] floats
-  static constexpr size_t kFlag = kRed + 4 * 16 * 4;        // [2][4] ints
+  static constexpr size_t kFlag = kRed + 4 * 16 * 4;        // [16] ints
   static constexpr size_t kBars = kFlag + 64;
   static constexpr int kNumBars = 2 * kStNS + 16;
   static constexpr size_t kSlot = kBars + kNumBars * 8;
@@ -91,16 +93,16 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_cons
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);
-      mbar_init(&p_ready[i], 4);
+      mbar_init(&s_free[i], kStSoft / 32);
+      mbar_init(&p_ready[i], kStSoft / 32);
       mbar_init(&p_free[i], 1);
       mbar_init(&o_full[i], 1);
-      mbar_init(&o_free[i], 4);
+      mbar_init(&o_free[i], kStSoft / 32);
     }
     for (int i = 0; i < 8; ++i) flags[i] = 0;  // abort flag, vote slots, block count
     fence_mbar_init();
   }
-  if (warp == 5) tc_alloc(tmem_slot, 128);
+  if (warp == 9) tc_alloc(tmem_slot, 128);
   // Q rows past the group (G < 16) are never loaded: keep them zero
   for (int i = tid; i < 2 * kStQBuf / 16; i += kStThreads)
     reinterpret_cast<uint4*>(qbuf)[i] = make_uint4(0u, 0u, 0u, 0u);
@@ -119,7 +121,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_cons
     b = (int)(r / (T * p.Hkv));
   };
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tmap(&tmq);
@@ -168,7 +170,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_cons
       }
       if (!ok) flags[0] = 1;
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       uint32_t kv_it = 0, pr = 0, qrow = 0, orow = 0;
@@ -228,18 +230,20 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_cons
       if (ok && have_prev && !issue_pv()) ok = false;
       if (!ok) flags[0] = 1;
     }
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------------------ softmax + epilogue
-    const int kl = tid;  // key of the pair (softmax) / head dimension (epilogue)
-    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+    const int kl = tid & 127;       // key of the pair (softmax) / head dimension (epilogue)
+    const int hh = tid >> 7;        // head half: heads 8*hh .. 8*hh+7
+    const int wq = warp & 3;        // TMEM lane quadrant
+    const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
     uint32_t pr = 0, orow = 0;
-    int vote = 0;  // cross-warp votes taken so far
+    int vote = 0;                   // cross-warp votes taken so far
     bool ok = true;
     for (int64_t r = blockIdx.x; r < p.rows && ok; r += gridDim.x) {
       int64_t t; int hk, b;
       row_coords(r, t, hk, b);
       // compact the row's live blocks into shared memory (warp 0), count them
-      named_bar_sync(1, 128);  // previous row finished reading the list
+      named_bar_sync(1, kStSoft);  // previous row finished reading the list
       if (warp == 0) {
         const int32_t* ir = p.idx + r * p.n_sel;
         int base = 0;
@@ -253,36 +257,41 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_cons
         }
         if (lane == 0) flags[7] = base;
       }
-      named_bar_sync(1, 128);
+      named_bar_sync(1, kStSoft);
       const int nblk = flags[7];
       const int npairs = (nblk + 1) >> 1;
-      // gate of this thread's dimension for every head of the group (prefetched)
-      uint32_t graw[8] = {};
       const int d = kl;
+      const int h0 = 8 * hh;
+      // gate of this thread's dimension for its 8 heads (prefetched)
+      uint32_t graw[4] = {};
       if (p.g != nullptr && nblk > 0) {
-        const __nv_bfloat16* gr = p.g + b * p.sg.b + t * p.sg.t + (int64_t)(hk * p.G) * p.sg.h + d;
+        const __nv_bfloat16* gr =
+            p.g + b * p.sg.b + t * p.sg.t + (int64_t)(hk * p.G + h0) * p.sg.h + d;
 #pragma unroll
-        for (int h = 0; h < 16; h += 2) {
-          const uint16_t a = h < p.G ? __ldg(reinterpret_cast<const uint16_t*>(gr + (int64_t)h * p.sg.h)) : 0;
-          const uint16_t c = h + 1 < p.G ? __ldg(reinterpret_cast<const uint16_t*>(gr + (int64_t)(h + 1) * p.sg.h)) : 0;
+        for (int h = 0; h < 8; h += 2) {
+          const uint16_t a = h0 + h < p.G ? __ldg(reinterpret_cast<const uint16_t*>(gr + (int64_t)h * p.sg.h)) : 0;
+          const uint16_t c = h0 + h + 1 < p.G ? __ldg(reinterpret_cast<const uint16_t*>(gr + (int64_t)(h + 1) * p.sg.h)) : 0;
           graw[h >> 1] = (uint32_t)a | ((uint32_t)c << 16);
         }
       }
-      __nv_bfloat16* orow_ptr = p.o + b * p.so.b + t * p.so.t + (int64_t)(hk * p.G) * p.so.h + d;
+      __nv_bfloat16* orow_ptr =
+          p.o + b * p.so.b + t * p.so.t + (int64_t)(hk * p.G + h0) * p.so.h + d;
       if (nblk == 0) {
-        for (int h = 0; h < p.G; ++h) orow_ptr[(int64_t)h * p.so.h] = __float2bfloat16_rn(0.f);
+        for (int h = 0; h < 8 && h0 + h < p.G; ++h)
+          orow_ptr[(int64_t)h * p.so.h] = __float2bfloat16_rn(0.f);
         continue;
       }
-      float m_ref[16], l_part[16];
+      float m_ref[8], l_part[8];
 #pragma unroll
-      for (int h = 0; h < 16; ++h) { m_ref[h] = -INFINITY; l_part[h] = 0.f; }
+      for (int h = 0; h < 8; ++h) { m_ref[h] = -INFINITY; l_part[h] = 0.f; }
       const uint32_t ob = orow & 1;
+      const uint32_t t_o = tmem + 32 + 32 * ob + lane_off;
       for (int i = 0; i < npairs && ok; ++i) {
         const uint32_t sb = pr & 1;
         if (!mbar_wait(&s_full[sb], (pr >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
-        uint32_t sv[16];
-        tc_ld16(tmem + 16 * sb + lane_off, sv);
+        uint32_t sv[8];
+        tc_ld8(tmem + 16 * sb + h0 + lane_off, sv);
         tc_wait_ld();
         tc_fence_before();
         __syncwarp();
@@ -292,10 +301,10 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_cons
         const int64_t key = kl < 64 ? (int64_t)jA * kSaBlk + kl
                                     : (jB >= 0 ? (int64_t)jB * kSaBlk + kl - 64 : INT64_MAX);
         const bool valid = key <= t;
-        float x[16];
+        float x[8];
         bool raise = false;
 #pragma unroll
-        for (int h = 0; h < 16; ++h) {
+        for (int h = 0; h < 8; ++h) {
           x[h] = valid ? __uint_as_float(sv[h]) * p.scale_log2 : -INFINITY;
           raise |= x[h] > m_ref[h] + kStLazy;
         }
@@ -304,60 +313,63 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_cons
         const int slot = 1 + vote % 3;
         if (tid == 0) flags[1 + (vote + 1) % 3] = 0;
         if (__any_sync(0xffffffffu, raise) && lane == 0) flags[slot] = 1;
-        named_bar_sync(1, 128);
+        named_bar_sync(1, kStSoft);
         const bool any_raise = flags[slot] != 0;
         ++vote;
         if (any_raise) {
 #pragma unroll
-          for (int h = 0; h < 16; ++h) {
+          for (int h = 0; h < 8; ++h) {
             float mh = x[h];
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) mh = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, off));
-            if (lane == 0) red[warp * 16 + h] = mh;
+            if (lane == 0) red[wq * 16 + h0 + h] = mh;
           }
-          named_bar_sync(1, 128);
-          float alpha[16];
+          named_bar_sync(1, kStSoft);
+          float alpha[8];
 #pragma unroll
-          for (int h = 0; h < 16; ++h) {
-            const float bm = fmaxf(fmaxf(red[h], red[16 + h]), fmaxf(red[32 + h], red[48 + h]));
+          for (int h = 0; h < 8; ++h) {
+            const int hd = h0 + h;
+            const float bm = fmaxf(fmaxf(red[hd], red[16 + hd]), fmaxf(red[32 + hd], red[48 + hd]));
             const float nm = fmaxf(m_ref[h], bm);
             alpha[h] = (nm == -INFINITY || m_ref[h] == -INFINITY) ? 0.f : exp2f(m_ref[h] - nm);
             if (m_ref[h] == nm) alpha[h] = 1.f;
             m_ref[h] = nm;
             l_part[h] *= alpha[h];
           }
-          named_bar_sync(1, 128);  // everyone read red[]
+          named_bar_sync(1, kStSoft);  // everyone read red[]
           if (i > 0) {
             // rescale this row's partial O^T once the previous pair's P.V has landed
             const uint32_t pp = pr - 1;
             if (!mbar_wait(&p_free[pp & 1], (pp >> 1) & 1)) { ok = false; break; }
             tc_fence_after();
-            uint32_t ov[32];
-            tc_ld32(tmem + 32 + 32 * ob + lane_off, ov);
+            uint32_t ohi[8], olo[8];
+            tc_ld8(t_o + h0, ohi);
+            tc_ld8(t_o + 16 + h0, olo);
             tc_wait_ld();
 #pragma unroll
-            for (int h = 0; h < 16; ++h) {
-              ov[h] = __float_as_uint(__uint_as_float(ov[h]) * alpha[h]);
-              ov[16 + h] = __float_as_uint(__uint_as_float(ov[16 + h]) * alpha[h]);
+            for (int h = 0; h < 8; ++h) {
+              ohi[h] = __float_as_uint(__uint_as_float(ohi[h]) * alpha[h]);
+              olo[h] = __float_as_uint(__uint_as_float(olo[h]) * alpha[h]);
             }
-            tc_st32(tmem + 32 + 32 * ob + lane_off, ov);
+            tc_st8(t_o + h0, ohi);
+            tc_st8(t_o + 16 + h0, olo);
             tc_wait_st();
             tc_fence_before();
           }
         }
-        // P^T (bf16 high / low parts) for this key
+        // P^T (bf16 high / low parts) for this key and these heads
         if (pr >= 2 && !mbar_wait(&p_free[sb], ((pr >> 1) & 1) ^ 1)) { ok = false; break; }
         uint8_t* pt = pbuf + sb * kStPBuf + (kl >> 6) * 4096;
         const int kk = kl & 63;
         const uint32_t col = (uint32_t)(kk & 7) << 1;
 #pragma unroll
-        for (int h = 0; h < 16; ++h) {
+        for (int h = 0; h < 8; ++h) {
           const float mu = m_ref[h] == -INFINITY ? 0.f : m_ref[h];
           const float pv = exp2f(x[h] - mu);
           l_part[h] += pv;
           const __nv_bfloat16 hi = __float2bfloat16_rn(pv);
           const __nv_bfloat16 lo = __float2bfloat16_rn(pv - __bfloat162float(hi));
-          const uint32_t n0 = h, n1 = 16 + h;
+          const uint32_t n0 = h0 + h, n1 = 16 + h0 + h;
           *reinterpret_cast<__nv_bfloat16*>(pt + n0 * 128 + ((((kk >> 3) ^ (n0 & 7)) << 4) | col)) = hi;
           *reinterpret_cast<__nv_bfloat16*>(pt + n1 * 128 + ((((kk >> 3) ^ (n1 & 7)) << 4) | col)) = lo;
         }
@@ -370,31 +382,33 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_cons
       if (!ok) break;
       // ---- epilogue: row sums, normalise, gate, store
 #pragma unroll
-      for (int h = 0; h < 16; ++h) {
+      for (int h = 0; h < 8; ++h) {
         float ls = l_part[h];
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, off);
-        if (lane == 0) red[warp * 16 + h] = ls;
+        if (lane == 0) red[wq * 16 + h0 + h] = ls;
       }
-      named_bar_sync(1, 128);
-      float inv_l[16];
+      named_bar_sync(1, kStSoft);
+      float inv_l[8];
 #pragma unroll
-      for (int h = 0; h < 16; ++h) {
-        const float L = red[h] + red[16 + h] + red[32 + h] + red[48 + h];
+      for (int h = 0; h < 8; ++h) {
+        const int hd = h0 + h;
+        const float L = red[hd] + red[16 + hd] + red[32 + hd] + red[48 + hd];
         inv_l[h] = L > 0.f ? 1.0f / L : 0.f;
       }
       if (!mbar_wait(&o_full[ob], (orow >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
-      uint32_t ov[32];
-      tc_ld32(tmem + 32 + 32 * ob + lane_off, ov);
+      uint32_t ohi[8], olo[8];
+      tc_ld8(t_o + h0, ohi);
+      tc_ld8(t_o + 16 + h0, olo);
       tc_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&o_free[ob]);
 #pragma unroll
-      for (int h = 0; h < 16; ++h) {
-        if (h < p.G) {
-          float y = (__uint_as_float(ov[h]) + __uint_as_float(ov[16 + h])) * inv_l[h];
+      for (int h = 0; h < 8; ++h) {
+        if (h0 + h < p.G) {
+          float y = (__uint_as_float(ohi[h]) + __uint_as_float(olo[h])) * inv_l[h];
           if (p.g != nullptr) {
             const uint32_t gbits = (graw[h >> 1] >> (16 * (h & 1))) & 0xffffu;
             y *= sigmoidf_(__uint_as_float(gbits << 16));
@@ -409,7 +423,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_cons
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tc_dealloc(tmem, 128);
   }
