@@ -344,10 +344,14 @@ sala_status sala_sparse_attn(const void* q, const void* k, const void* v, const 
   p.scale_log2 = sc * 1.4426950408889634f;
   p.rows = (int64_t)B * Hkv * T;
   p.q_box_h = 16;
+  // The mma.sync kernel is faster on this workload (it frees each K/V stage right after
+  // the Q.K^T MMAs because V fragments can be held in registers); the tcgen05 kernel
+  // must keep every stage until its P.V MMA has read V from shared memory.
+  const bool use_tc_sparse = false;
   cudaStream_t st = as_stream(stream);
   const int64_t want = num_sms();
   const unsigned grid = (unsigned)std::min<int64_t>(want, p.rows);
-  if (D == 128 && n_sel <= kStMaxSel) {
+  if (D == 128 && n_sel <= kStMaxSel && use_tc_sparse) {
     // tcgen05 path: keys as the MMA M dimension
     CUtensorMap tq;
     p.q_box_h = Hq < 16 ? Hq : 16;

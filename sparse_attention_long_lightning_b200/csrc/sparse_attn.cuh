@@ -203,10 +203,9 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
       const uint32_t kb = smem_u32(stages + size_t(s) * L::kStage);
       const uint32_t vb = kb + L::kTile;
 
-      // ---- S = Q K^T for keys 16*wq .. 16*wq+15 of the block (4 independent chains)
-      float sc[2][4];
+      // ---- S = Q K^T for keys 16*wq .. 16*wq+15 of the block
+      float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
       {
-        float sx[2][2][4] = {};
         const int mat = lane >> 3, rin = lane & 7;
         const uint32_t krow = wq * 16 + (mat >> 1) * 8 + rin;
 #pragma unroll
@@ -215,13 +214,28 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
           const uint32_t addr = kb + (chunk >> 3) * L::kHalf + swz128(krow, chunk & 7);
           uint32_t b0, b1, b2, b3;
           ldsm_x4(addr, b0, b1, b2, b3);
-          mma_bf16_16816(sx[0][kk & 1], qa[kk], b0, b1);
-          mma_bf16_16816(sx[1][kk & 1], qa[kk], b2, b3);
+          mma_bf16_16816(sc[0], qa[kk], b0, b1);
+          mma_bf16_16816(sc[1], qa[kk], b2, b3);
         }
+      }
+      // ---- this warp's V fragments go to registers, then the stage is released at once
+      // (except the row's last block, whose stage is reused for the merge)
+      uint32_t vv[kNT / 2][4];
+      {
+        const int mat = lane >> 3, rin = lane & 7;
+        const uint32_t vrow = wq * 16 + (mat & 1) * 8 + rin;
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) sc[nt][c] = sx[nt][0][c] + sx[nt][1][c];
+        for (int pp = 0; pp < kNT / 2; ++pp) {
+          const uint32_t chunk = 2 * pp + (mat >> 1);
+          const uint32_t addr = vb + (chunk >> 3) * L::kHalf + swz128(vrow, chunk & 7);
+          ldsm_x4_t(addr, vv[pp][0], vv[pp][1], vv[pp][2], vv[pp][3]);
+        }
+      }
+      __syncwarp();
+      if (e + 1 < nblk) {
+        if (lane == 0) mbar_arrive(&empty[s]);
+      } else {
+        s_last = s;
       }
       // ---- scale; causal mask only where the block reaches past t
       const bool straddle = (int64_t)j * kSaBlk + kSaBlk - 1 > t;
@@ -275,33 +289,16 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
         pl[nt * 2 + 0] = *reinterpret_cast<const uint32_t*>(&l01);
         pl[nt * 2 + 1] = *reinterpret_cast<const uint32_t*>(&l23);
       }
-      // ---- O += P V; the low-part MMA of each accumulator trails its high-part MMA by
-      // two iterations so dependent MMAs are never issued back to back
-      {
-        const int mat = lane >> 3, rin = lane & 7;
-        const uint32_t vrow = wq * 16 + (mat & 1) * 8 + rin;
-        uint32_t vv[kNT / 2][4];
+      // ---- O += P V from the register copy of V: all high parts, then all low parts
 #pragma unroll
-        for (int pp = 0; pp < kNT / 2 + 2; ++pp) {
-          if (pp < kNT / 2) {
-            const uint32_t chunk = 2 * pp + (mat >> 1);
-            const uint32_t addr = vb + (chunk >> 3) * L::kHalf + swz128(vrow, chunk & 7);
-            ldsm_x4_t(addr, vv[pp][0], vv[pp][1], vv[pp][2], vv[pp][3]);
-            mma_bf16_16816(oacc[2 * pp], ph, vv[pp][0], vv[pp][1]);
-            mma_bf16_16816(oacc[2 * pp + 1], ph, vv[pp][2], vv[pp][3]);
-          }
-          if (pp >= 2) {
-            const int qq = pp - 2;
-            mma_bf16_16816(oacc[2 * qq], pl, vv[qq][0], vv[qq][1]);
-            mma_bf16_16816(oacc[2 * qq + 1], pl, vv[qq][2], vv[qq][3]);
-          }
-        }
+      for (int pp = 0; pp < kNT / 2; ++pp) {
+        mma_bf16_16816(oacc[2 * pp], ph, vv[pp][0], vv[pp][1]);
+        mma_bf16_16816(oacc[2 * pp + 1], ph, vv[pp][2], vv[pp][3]);
       }
-      __syncwarp();
-      if (e + 1 < nblk) {
-        if (lane == 0) mbar_arrive(&empty[s]);
-      } else {
-        s_last = s;  // released after the merge, which reuses it
+#pragma unroll
+      for (int pp = 0; pp < kNT / 2; ++pp) {
+        mma_bf16_16816(oacc[2 * pp], pl, vv[pp][0], vv[pp][1]);
+        mma_bf16_16816(oacc[2 * pp + 1], pl, vv[pp][2], vv[pp][3]);
       }
       ++it;
     }
