@@ -14,9 +14,9 @@
 // K and V (128-byte swizzle, no multicast) into the group's NS-deep ring,
 // recording the block id beside the stage.  Each group has four consumer
 // warps that split every 64-key block 16 keys apiece: the group's 16 query
-// heads form the M = 16 operand of m16n8k16 tensor-core MMAs (Q K^T in bf16;
-// P V with P split into bf16 high and low parts, so V is used exactly as
-// stored; fp32 accumulation), the online softmax runs per warp in
+// heads form the M = 16 operand of m16n8k16 tensor-core MMAs (Q K^T in bf16,
+// P V in fp16 with V converted in registers; fp32 accumulation; a pre-pass
+// flags V values outside the fp16 range), the online softmax runs per warp in
 // registers with a lazily raised reference maximum (rescaling only when a
 // score exceeds it by more than 2^8), and the four partial (max, sum, O)
 // triples are merged through shared memory at the end of the row.  All waits
@@ -272,33 +272,22 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
         }
       }
       const float mu0 = m0 == -INFINITY ? 0.f : m0, mu1 = m1 == -INFINITY ? 0.f : m1;
-      // P = P_hi + P_lo, both bf16 (exact to 2^-16 relative), so V stays bf16
-      uint32_t ph[4], pl[4];
+      // P in fp16 (10-bit mantissa); V converted to fp16 in registers
+      uint32_t pa[4];
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
         const float p0 = exp2f(sc[nt][0] - mu0), p1 = exp2f(sc[nt][1] - mu0);
         const float p2 = exp2f(sc[nt][2] - mu1), p3 = exp2f(sc[nt][3] - mu1);
         l0 += p0 + p1;
         l1 += p2 + p3;
-        const __nv_bfloat162 h01 = __floats2bfloat162_rn(p0, p1);
-        const __nv_bfloat162 h23 = __floats2bfloat162_rn(p2, p3);
-        const __nv_bfloat162 l01 = __floats2bfloat162_rn(p0 - __low2float(h01), p1 - __high2float(h01));
-        const __nv_bfloat162 l23 = __floats2bfloat162_rn(p2 - __low2float(h23), p3 - __high2float(h23));
-        ph[nt * 2 + 0] = *reinterpret_cast<const uint32_t*>(&h01);
-        ph[nt * 2 + 1] = *reinterpret_cast<const uint32_t*>(&h23);
-        pl[nt * 2 + 0] = *reinterpret_cast<const uint32_t*>(&l01);
-        pl[nt * 2 + 1] = *reinterpret_cast<const uint32_t*>(&l23);
+        pa[nt * 2 + 0] = pack_f16x2(p0, p1);
+        pa[nt * 2 + 1] = pack_f16x2(p2, p3);
       }
-      // ---- O += P V from the register copy of V: all high parts, then all low parts
+      // ---- O += P V
 #pragma unroll
       for (int pp = 0; pp < kNT / 2; ++pp) {
-        mma_bf16_16816(oacc[2 * pp], ph, vv[pp][0], vv[pp][1]);
-        mma_bf16_16816(oacc[2 * pp + 1], ph, vv[pp][2], vv[pp][3]);
-      }
-#pragma unroll
-      for (int pp = 0; pp < kNT / 2; ++pp) {
-        mma_bf16_16816(oacc[2 * pp], pl, vv[pp][0], vv[pp][1]);
-        mma_bf16_16816(oacc[2 * pp + 1], pl, vv[pp][2], vv[pp][3]);
+        mma_f16_16816(oacc[2 * pp], pa, bf16x2_to_f16x2(vv[pp][0]), bf16x2_to_f16x2(vv[pp][1]));
+        mma_f16_16816(oacc[2 * pp + 1], pa, bf16x2_to_f16x2(vv[pp][2]), bf16x2_to_f16x2(vv[pp][3]));
       }
       ++it;
     }
@@ -382,6 +371,30 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s_last]);
   }
+}
+
+// Values of a bf16 [B, T, H, D] tensor that would not survive conversion to the
+// fp16 tensor-core operand (|x| >= 65536 in bf16, inf or NaN) raise SALA_ERR_RANGE.
+__global__ void __launch_bounds__(256)
+f16_range_check_kernel(const __nv_bfloat16* __restrict__ x, sala_strides s, int B, int T, int H,
+                       int D) {
+  const int64_t rows = (int64_t)B * T * H;
+  const int per_row = D / 8;
+  uint32_t bad = 0;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < rows * per_row;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = i / per_row;
+    const int c = (int)(i % per_row);
+    const int h = (int)(row % H);
+    const int64_t t = (row / H) % T;
+    const int b = (int)(row / ((int64_t)H * T));
+    const uint4 u = *reinterpret_cast<const uint4*>(x + b * s.b + t * s.t + h * s.h + 8 * c);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      bad |= ((w[k] & 0x7fffu) >= 0x4780u) | (((w[k] >> 16) & 0x7fffu) >= 0x4780u);
+  }
+  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) raise_device_error(SALA_ERR_RANGE);
 }
 
 }  // namespace sala
