@@ -46,10 +46,11 @@ constexpr int kTcTile = 2 * kTcSlab;      // 128 x 128 16-bit tile: 32 KB
 
 template <bool kStateOnly>
 struct TcSmem {
+  static constexpr int kStages = kStateOnly ? 3 : 2;
   static constexpr int kStageBytes = (kStateOnly ? 2 : 3) * kTcTile;
   static constexpr int kSop = kStateOnly ? 0 : kTcTile;
   static constexpr int kMisc = 2048;
-  static constexpr size_t bytes = 1024 /*alignment slack*/ + 2 * size_t(kStageBytes) + kSop + kMisc;
+  static constexpr size_t bytes = 1024 /*alignment slack*/ + size_t(kStages) * kStageBytes + kSop + kMisc;
   static constexpr uint32_t kTmemCols = kStateOnly ? 128 : 512;
 };
 
@@ -105,10 +106,10 @@ __device__ __forceinline__ uint32_t f16x8_nonfinite(const uint4& u) {
 // it, and a quarter of the v row, to fp16 in place.  Four consecutive lanes share
 // a row: quarter qd owns rotation pairs i in [16 qd, 16 qd + 16) (chunks 2qd, 2qd+1
 // of both 64-column slabs) and v chunks 4qd..4qd+3.  Tiles are two 64-column slabs
-// of 128 rows x 128 bytes with the 128-byte swizzle.  Returns non-zero if an fp16
-// value is not finite.
+// of 128 rows x 128 bytes with the 128-byte swizzle.  An fp16 overflow here shows up
+// downstream as a non-finite output or state, which the epilogue reports.
 template <bool kWithQ>
-__device__ __forceinline__ uint32_t tc_prep_quarter(uint8_t* sQ, uint8_t* sK, uint8_t* sV, int r,
+__device__ __forceinline__ void tc_prep_quarter(uint8_t* sQ, uint8_t* sK, uint8_t* sV, int r,
                                                     int qd, const TcParams& p,
                                                     const float2* ang_base) {
   float ssq = 0.f, ssk = 0.f;
@@ -132,7 +133,6 @@ __device__ __forceinline__ uint32_t tc_prep_quarter(uint8_t* sQ, uint8_t* sK, ui
   ssq += __shfl_xor_sync(0xffffffffu, ssq, 2);
   const float rk = rsqrtf(ssk * (1.0f / 128.0f) + p.eps);
   const float rq = rsqrtf(ssq * (1.0f / 128.0f) + p.eps);
-  uint32_t bad = 0;
   const float two_pi = 6.28318530717958647692f, inv_two_pi = 0.15915494309189533577f;
 #pragma unroll
   for (int jj = 0; jj < 2; ++jj) {
@@ -165,19 +165,11 @@ __device__ __forceinline__ uint32_t tc_prep_quarter(uint8_t* sQ, uint8_t* sK, ui
         qhi[e] = q1 * cs + q0 * sn;
       }
     }
-    uint4 u = f32x8_to_f16(klo);
-    bad |= f16x8_nonfinite(u);
-    *reinterpret_cast<uint4*>(sK + alo) = u;
-    u = f32x8_to_f16(khi);
-    bad |= f16x8_nonfinite(u);
-    *reinterpret_cast<uint4*>(sK + ahi) = u;
+    *reinterpret_cast<uint4*>(sK + alo) = f32x8_to_f16(klo);
+    *reinterpret_cast<uint4*>(sK + ahi) = f32x8_to_f16(khi);
     if (kWithQ) {
-      u = f32x8_to_f16(qlo);
-      bad |= f16x8_nonfinite(u);
-      *reinterpret_cast<uint4*>(sQ + alo) = u;
-      u = f32x8_to_f16(qhi);
-      bad |= f16x8_nonfinite(u);
-      *reinterpret_cast<uint4*>(sQ + ahi) = u;
+      *reinterpret_cast<uint4*>(sQ + alo) = f32x8_to_f16(qlo);
+      *reinterpret_cast<uint4*>(sQ + ahi) = f32x8_to_f16(qhi);
     }
   }
 #pragma unroll
@@ -187,10 +179,8 @@ __device__ __forceinline__ uint32_t tc_prep_quarter(uint8_t* sQ, uint8_t* sK, ui
     uint4 x = *reinterpret_cast<const uint4*>(sV + a);
     x.x = bf16x2_to_f16x2(x.x); x.y = bf16x2_to_f16x2(x.y);
     x.z = bf16x2_to_f16x2(x.z); x.w = bf16x2_to_f16x2(x.w);
-    bad |= f16x8_nonfinite(x);
     *reinterpret_cast<uint4*>(sV + a) = x;
   }
-  return bad;
 }
 
 // K-major operand (rows = M or N, 128-byte rows along K), k-step kk of 16 elements.
@@ -205,7 +195,8 @@ __device__ __forceinline__ uint64_t tc_desc_mn(const uint8_t* base, int kk) {
 // Gated bf16 epilogue of one chunk: thread (trow, cg) reads 32 fp32 columns of O from
 // TMEM, scales by 2^e, multiplies by sigmoid(g) (prefetched) and stores 64 bytes.
 __device__ __forceinline__ void tc_epilogue(uint32_t t_o, const uint4 (&gv)[4], bool gated,
-                                            float os, __nv_bfloat16* orow, bool live) {
+                                            float os, __nv_bfloat16* orow, bool live,
+                                            uint32_t& bad) {
   uint32_t r[32];
   tc_ld32(t_o, r);
   tc_wait_ld();
@@ -221,6 +212,8 @@ __device__ __forceinline__ void tc_epilogue(uint32_t t_o, const uint4 (&gv)[4], 
 #pragma unroll
       for (int e = 0; e < 8; ++e) y[e] *= sigmoidf_(gf[e]);
     }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) bad |= (__float_as_uint(y[e]) & 0x7f800000u) == 0x7f800000u;
     uint4 w;
     __nv_bfloat162 h0 = __floats2bfloat162_rn(y[0], y[1]), h1 = __floats2bfloat162_rn(y[2], y[3]);
     __nv_bfloat162 h2 = __floats2bfloat162_rn(y[4], y[5]), h3 = __floats2bfloat162_rn(y[6], y[7]);
@@ -251,12 +244,12 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* stages = smem;
-  uint8_t* sop = smem + 2 * L::kStageBytes;
+  uint8_t* sop = smem + L::kStages * L::kStageBytes;
   uint8_t* misc = sop + L::kSop;
-  uint64_t* full = reinterpret_cast<uint64_t*>(misc);      // [2]
-  uint64_t* mma1_bar = full + 2;                           // score/inter/state done
-  uint64_t* mma2_bar = full + 3;                           // PV done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(full + 4);
+  uint64_t* full = reinterpret_cast<uint64_t*>(misc);      // [kStages]
+  uint64_t* mma1_bar = full + 3;                           // score/inter/state done
+  uint64_t* mma2_bar = full + 4;                           // PV done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(full + 5);
   float* red = reinterpret_cast<float*>(misc + 64);        // [16]
   double* inv_freq = reinterpret_cast<double*>(misc + 128);  // [64]
   float2* ang_tab = reinterpret_cast<float2*>(misc + 640);   // [2][64]: (base angle, inv_freq)
@@ -276,8 +269,7 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   const int nchunks = c_end - c_begin;
 
   if (tid == 0) {
-    mbar_init(&full[0], 1);
-    mbar_init(&full[1], 1);
+    for (int i = 0; i < L::kStages; ++i) mbar_init(&full[i], 1);
     mbar_init(mma1_bar, 1);
     mbar_init(mma2_bar, 1);
     fence_mbar_init();
@@ -301,26 +293,27 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     }
   };
   auto issue = [&](int u) {
-    uint8_t* st = stages + (u & 1) * L::kStageBytes;
+    const int si = u % L::kStages;
+    uint8_t* st = stages + si * L::kStageBytes;
     const int t0 = (c_begin + u) * kTcC;
-    mbar_arrive_expect_tx(&full[u & 1], L::kStageBytes);
+    mbar_arrive_expect_tx(&full[si], L::kStageBytes);
     uint8_t* dk = st + (kStateOnly ? 0 : kTcTile);
     uint8_t* dv = dk + kTcTile;
     if (!kStateOnly) {
-      tma_load_4d(st, &tmq, &full[u & 1], 0, h, t0, b);
-      tma_load_4d(st + kTcSlab, &tmq, &full[u & 1], 64, h, t0, b);
+      tma_load_4d(st, &tmq, &full[si], 0, h, t0, b);
+      tma_load_4d(st + kTcSlab, &tmq, &full[si], 64, h, t0, b);
     }
-    tma_load_4d(dk, &tmk, &full[u & 1], 0, h, t0, b);
-    tma_load_4d(dk + kTcSlab, &tmk, &full[u & 1], 64, h, t0, b);
-    tma_load_4d(dv, &tmv, &full[u & 1], 0, h, t0, b);
-    tma_load_4d(dv + kTcSlab, &tmv, &full[u & 1], 64, h, t0, b);
+    tma_load_4d(dk, &tmk, &full[si], 0, h, t0, b);
+    tma_load_4d(dk + kTcSlab, &tmk, &full[si], 64, h, t0, b);
+    tma_load_4d(dv, &tmv, &full[si], 0, h, t0, b);
+    tma_load_4d(dv + kTcSlab, &tmv, &full[si], 64, h, t0, b);
   };
   int issued = 0;
   if (tid == 0) {
     if (!kStateOnly) prefetch_tmap(&tmq);
     prefetch_tmap(&tmk);
     prefetch_tmap(&tmv);
-    for (; issued < 2 && issued < nchunks; ++issued) issue(issued);
+    for (; issued < L::kStages && issued < nchunks; ++issued) issue(issued);
   }
   __syncthreads();  // inv_freq visible
   fill_angles(0);
@@ -361,14 +354,14 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   uint4 gv[4] = {};           // gate of this thread's row/columns for the pending epilogue
   const bool gated = p.g != nullptr;
   for (int u = 0; u < nchunks; ++u) {
-    const int s = u & 1;
+    const int s = u % L::kStages;
     uint8_t* st = stages + s * L::kStageBytes;
     uint8_t* sQ = st;
     uint8_t* sK = st + (kStateOnly ? 0 : kTcTile);
     uint8_t* sV = sK + kTcTile;
     // ---- A: prep(u) while the tensor core runs PV(u-1)
-    ok = ok && mbar_wait(&full[s], (u >> 1) & 1);
-    if (ok) bad |= tc_prep_quarter<!kStateOnly>(sQ, sK, sV, prow, pqd, p, ang_tab + s * 64);
+    ok = ok && mbar_wait(&full[s], (u / L::kStages) & 1);
+    if (ok) tc_prep_quarter<!kStateOnly>(sQ, sK, sV, prow, pqd, p, ang_tab + (u & 1) * 64);
     fence_proxy_async_smem();
     // angles of chunk u+1 (other parity; prep(u-1), the last reader, is behind a barrier)
     if (u + 1 < nchunks) fill_angles(u + 1);
@@ -407,7 +400,7 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       const int64_t t = (int64_t)(c_begin + u - 1) * kTcC + trow;
       __nv_bfloat16* orow = p.o + b * p.so.b + t * p.so.t + (int64_t)h * p.so.h + 32 * cg;
       tc_epilogue(t_o0 + 128 * ((u - 1) & 1) + lane_off + 32 * cg, gv, gated, pow2i(e_prev),
-                  orow, t < p.T);
+                  orow, t < p.T, bad);
     }
     {
       // prefetch this chunk's gate for its epilogue (next iteration)
@@ -433,13 +426,21 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       tc_fence_after();
       const float ps = pow2i(-e_cur);
       uint32_t pk[16];
+      if (lq > cg) {          // rows 32lq.. all lie below columns 32cg..32cg+31: no mask
 #pragma unroll
-      for (int m = 0; m < 16; ++m) {
-        const int col = 32 * cg + 2 * m;
-        const float a = col <= trow ? __uint_as_float(r[2 * m]) * ps : 0.f;
-        const float c = col + 1 <= trow ? __uint_as_float(r[2 * m + 1]) * ps : 0.f;
-        pk[m] = pack_f16x2(a, c);
-        bad |= f16x2_nonfinite(pk[m]);
+        for (int m = 0; m < 16; ++m)
+          pk[m] = pack_f16x2(__uint_as_float(r[2 * m]) * ps, __uint_as_float(r[2 * m + 1]) * ps);
+      } else if (lq < cg) {   // strictly above the diagonal: all masked
+#pragma unroll
+        for (int m = 0; m < 16; ++m) pk[m] = 0u;
+      } else {                // diagonal block: keep s <= t
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+          const int col = 2 * m;
+          const float a = col <= lane ? __uint_as_float(r[2 * m]) * ps : 0.f;
+          const float c = col + 1 <= lane ? __uint_as_float(r[2 * m + 1]) * ps : 0.f;
+          pk[m] = pack_f16x2(a, c);
+        }
       }
       tc_st16(t_p + lane_off + 16 * cg, pk);
       tc_wait_st();
@@ -452,6 +453,7 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       float mx = 0.f;
 #pragma unroll
       for (int m = 0; m < 32; ++m) mx = fmaxf(mx, fabsf(__uint_as_float(r[m])));
+      bad |= !(mx <= 3.0e38f);  // inf or NaN in the state
       const int e_next = tc_block_scale_exp(mx, red);
       const float sc = pow2i(-e_next);
 #pragma unroll
@@ -499,14 +501,15 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         const int64_t t = (int64_t)(c_begin + u - 1) * kTcC + trow;
         __nv_bfloat16* orow = p.o + b * p.so.b + t * p.so.t + (int64_t)h * p.so.h + 32 * cg;
         tc_epilogue(t_o0 + 128 * ((u - 1) & 1) + lane_off + 32 * cg, gv, gated, pow2i(e_prev),
-                    orow, t < p.T);
+                    orow, t < p.T, bad);
       }
     }
   }
   if (__any_sync(0xffffffffu, bad) && lane == 0) raise_device_error(SALA_ERR_RANGE);
   if (!ok && tid == 0) {
     // wind down: let the last issued copies land before the CTA's shared memory goes away
-    for (int u = issued > 2 ? issued - 2 : 0; u < issued; ++u) mbar_wait(&full[u & 1], (u >> 1) & 1);
+    for (int u = issued > L::kStages ? issued - L::kStages : 0; u < issued; ++u)
+      mbar_wait(&full[u % L::kStages], (u / L::kStages) & 1);
   }
   tc_fence_before();
   __syncthreads();
@@ -517,22 +520,24 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
 }
 
 // Exclusive prefix over the segment sums of each (b, h), in place; the final
-// state (initial + all segments) goes to `state`.  grid B*H, 256 threads.
+// state (initial + all segments) goes to `state`.  grid (B*H, 16), 256 threads:
+// each thread owns one float4 of the 128x128 state and walks the G segments.
 __global__ void __launch_bounds__(256)
 lightning_scan_kernel(float* __restrict__ ws, float* __restrict__ state, int G, int init_zero) {
   const int bh = blockIdx.x;
-  float* base = ws + (size_t)bh * G * (128 * 128);
-  float* sg = state + (size_t)bh * (128 * 128);
-  for (int e = threadIdx.x * 4; e < 128 * 128; e += 256 * 4) {
-    float4 run = init_zero ? make_float4(0.f, 0.f, 0.f, 0.f) : *reinterpret_cast<const float4*>(sg + e);
-    for (int s = 0; s < G; ++s) {
-      float4* cell = reinterpret_cast<float4*>(base + (size_t)s * (128 * 128) + e);
-      const float4 d = *cell;
-      *cell = run;
-      run.x += d.x; run.y += d.y; run.z += d.z; run.w += d.w;
-    }
-    *reinterpret_cast<float4*>(sg + e) = run;
+  const int e = (blockIdx.y * 256 + threadIdx.x) * 4;
+  float* base = ws + (size_t)bh * G * (128 * 128) + e;
+  float* sg = state + (size_t)bh * (128 * 128) + e;
+  float4 run = init_zero ? make_float4(0.f, 0.f, 0.f, 0.f) : *reinterpret_cast<const float4*>(sg);
+  float4 nxt = G > 0 ? *reinterpret_cast<const float4*>(base) : run;
+  for (int s = 0; s < G; ++s) {
+    float4* cell = reinterpret_cast<float4*>(base + (size_t)s * (128 * 128));
+    const float4 d = nxt;
+    if (s + 1 < G) nxt = *reinterpret_cast<const float4*>(base + (size_t)(s + 1) * (128 * 128));
+    *cell = run;
+    run.x += d.x; run.y += d.y; run.z += d.z; run.w += d.w;
   }
+  *reinterpret_cast<float4*>(sg) = run;
 }
 
 inline int lightning_tc_segments(int B, int H, int T, int nsm) {

@@ -171,7 +171,7 @@ sala_status sala_lightning_prefill(const void* q, const void* k, const void* v, 
     if (!set_smem(ka, TcSmem<true>::bytes) || !set_smem(kc, TcSmem<false>::bytes)) return SALA_ERR_CUDA;
     ka<<<grid, kTcThreads, TcSmem<true>::bytes, st>>>(tk, tk, tv, p);
     SALA_CHECK_LAUNCH();
-    lightning_scan_kernel<<<B * H, 256, 0, st>>>(p.ws, state, p.G, init_zero);
+    lightning_scan_kernel<<<dim3(B * H, 16), 256, 0, st>>>(p.ws, state, p.G, init_zero);
     SALA_CHECK_LAUNCH();
     kc<<<grid, kTcThreads, TcSmem<false>::bytes, st>>>(tq, tk, tv, p);
     SALA_CHECK_LAUNCH();
@@ -470,7 +470,7 @@ sala_status sala_lightning_prefill_noalloc(const void* q, const void* k, const v
   if (!set_smem(ka, TcSmem<true>::bytes) || !set_smem(kc, TcSmem<false>::bytes)) return SALA_ERR_CUDA;
   ka<<<grid, kTcThreads, TcSmem<true>::bytes, st>>>(tk, tk, tv, p);
   SALA_CHECK_LAUNCH();
-  lightning_scan_kernel<<<B * H, 256, 0, st>>>(p.ws, state, p.G, init_zero);
+  lightning_scan_kernel<<<dim3(B * H, 16), 256, 0, st>>>(p.ws, state, p.G, init_zero);
   SALA_CHECK_LAUNCH();
   kc<<<grid, kTcThreads, TcSmem<false>::bytes, st>>>(tq, tk, tv, p);
   SALA_CHECK_LAUNCH();
