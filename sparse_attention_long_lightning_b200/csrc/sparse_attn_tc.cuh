@@ -29,25 +29,26 @@
 
 namespace sala {
 
-constexpr int kStNS = 3;                  // K/V pair stages
+constexpr int kStNS = 3;                  // K ring and V ring depth (pairs)
 constexpr int kStThreads = 320;          // 8 softmax warps, producer, MMA issuer
 constexpr int kStSoft = 256;
 constexpr int kStHalf = 128 * 128;        // [128 rows x 64 cols] bf16 slab: 16 KB
-constexpr int kStStage = 4 * kStHalf;     // K d-half 0, K d-half 1, V d-half 0, V d-half 1
+constexpr int kStTile = 2 * kStHalf;      // K or V of a pair: d-half 0, d-half 1 (32 KB)
 constexpr int kStPBuf = 2 * 32 * 128;     // P^T: two 64-key halves of [32 rows x 128 B]
 constexpr int kStQBuf = 2 * 16 * 128;     // Q: two 64-dim halves of [16 heads x 128 B]
 constexpr int kStMaxSel = 256;            // selected-block list capacity of one row
 constexpr float kStLazy = 8.0f;
 
 struct StSmem {
-  static constexpr size_t kStages = 0;
-  static constexpr size_t kP = kStages + size_t(kStNS) * kStStage;
+  static constexpr size_t kKRing = 0;
+  static constexpr size_t kVRing = kKRing + size_t(kStNS) * kStTile;
+  static constexpr size_t kP = kVRing + size_t(kStNS) * kStTile;
   static constexpr size_t kQ = kP + 2 * kStPBuf;
   static constexpr size_t kList = kQ + 2 * kStQBuf;
   static constexpr size_t kRed = kList + kStMaxSel * 4;     // [4][16] floats
   static constexpr size_t kFlag = kRed + 4 * 16 * 4;        // [16] ints
   static constexpr size_t kBars = kFlag + 64;
-  static constexpr int kNumBars = 2 * kStNS + 16;
+  static constexpr int kNumBars = 4 * kStNS + 16;
   static constexpr size_t kSlot = kBars + kNumBars * 8;
   static constexpr size_t bytes = 1024 + kSlot + 16;
 };
@@ -64,16 +65,19 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_cons
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* stages = smem + StSmem::kStages;
+  uint8_t* kring = smem + StSmem::kKRing;
+  uint8_t* vring = smem + StSmem::kVRing;
   uint8_t* pbuf = smem + StSmem::kP;
   uint8_t* qbuf = smem + StSmem::kQ;
   int32_t* list = reinterpret_cast<int32_t*>(smem + StSmem::kList);
   float* red = reinterpret_cast<float*>(smem + StSmem::kRed);
   volatile int* flags = reinterpret_cast<volatile int*>(smem + StSmem::kFlag);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + StSmem::kBars);
-  uint64_t* kv_full = bars;
-  uint64_t* kv_empty = kv_full + kStNS;
-  uint64_t* q_full = kv_empty + kStNS;   // [2]
+  uint64_t* k_full = bars;
+  uint64_t* k_empty = k_full + kStNS;
+  uint64_t* v_full = k_empty + kStNS;
+  uint64_t* v_empty = v_full + kStNS;
+  uint64_t* q_full = v_empty + kStNS;    // [2]
   uint64_t* q_empty = q_full + 2;        // [2]
   uint64_t* s_full = q_empty + 2;        // [2]
   uint64_t* s_free = s_full + 2;         // [2]
@@ -86,8 +90,10 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_cons
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     for (int s = 0; s < kStNS; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
@@ -123,12 +129,21 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_cons
 
   if (warp == 8) {
     // ------------------------------------------------------------------ producer
-    if (lane == 0) {
-      prefetch_tmap(&tmq);
-      prefetch_tmap(&tmk);
-      prefetch_tmap(&tmv);
-      uint32_t kv_it = 0, qrow = 0;
+    // lane 0 streams Q and the K ring, lane 1 the V ring, so K can run ahead of V
+    if (lane < 2) {
+      const bool is_k = lane == 0;
+      if (is_k) {
+        prefetch_tmap(&tmq);
+        prefetch_tmap(&tmk);
+      } else {
+        prefetch_tmap(&tmv);
+      }
+      uint32_t it = 0, qrow = 0;
       bool ok = true;
+      uint64_t* fullb = is_k ? k_full : v_full;
+      uint64_t* emptyb = is_k ? k_empty : v_empty;
+      uint8_t* ring = is_k ? kring : vring;
+      const CUtensorMap* map = is_k ? &tmk : &tmv;
       for (int64_t r = blockIdx.x; r < p.rows && ok; r += gridDim.x) {
         int64_t t; int hk, b;
         row_coords(r, t, hk, b);
@@ -136,12 +151,14 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_cons
         int nblk = 0;
         for (int e = 0; e < p.n_sel; ++e) nblk += sa_block_live(__ldg(ir + e), t);
         if (nblk == 0) continue;
-        const int qs = qrow & 1;
-        if (flags[0] || !mbar_wait(&q_empty[qs], ((qrow >> 1) & 1) ^ 1)) { ok = false; break; }
-        mbar_arrive_expect_tx(&q_full[qs], 2 * 128 * p.q_box_h);
-        tma_load_4d(qbuf + qs * kStQBuf, &tmq, &q_full[qs], 0, hk * p.G, (int)t, b);
-        tma_load_4d(qbuf + qs * kStQBuf + 2048, &tmq, &q_full[qs], 64, hk * p.G, (int)t, b);
-        ++qrow;
+        if (is_k) {
+          const int qs = qrow & 1;
+          if (flags[0] || !mbar_wait(&q_empty[qs], ((qrow >> 1) & 1) ^ 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(&q_full[qs], 2 * 128 * p.q_box_h);
+          tma_load_4d(qbuf + qs * kStQBuf, &tmq, &q_full[qs], 0, hk * p.G, (int)t, b);
+          tma_load_4d(qbuf + qs * kStQBuf + 2048, &tmq, &q_full[qs], 64, hk * p.G, (int)t, b);
+          ++qrow;
+        }
         int e = 0, got = 0;
         while (got < nblk && ok) {
           int jA = -1, jB = -1;
@@ -153,19 +170,16 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_cons
           } else {
             jB = jA;  // odd tail: repeat a real block; its keys are masked out
           }
-          const int s = kv_it % kStNS;
-          if (flags[0] || !mbar_wait(&kv_empty[s], ((kv_it / kStNS) & 1) ^ 1)) { ok = false; break; }
-          uint8_t* st = stages + size_t(s) * kStStage;
-          mbar_arrive_expect_tx(&kv_full[s], kStStage);
+          const int s = it % kStNS;
+          if (flags[0] || !mbar_wait(&emptyb[s], ((it / kStNS) & 1) ^ 1)) { ok = false; break; }
+          uint8_t* st = ring + size_t(s) * kStTile;
+          mbar_arrive_expect_tx(&fullb[s], kStTile);
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {
-            tma_load_4d(st + hf * kStHalf, &tmk, &kv_full[s], hf * 64, hk, jA * kSaBlk, b);
-            tma_load_4d(st + hf * kStHalf + 8192, &tmk, &kv_full[s], hf * 64, hk, jB * kSaBlk, b);
-            tma_load_4d(st + (2 + hf) * kStHalf, &tmv, &kv_full[s], hf * 64, hk, jA * kSaBlk, b);
-            tma_load_4d(st + (2 + hf) * kStHalf + 8192, &tmv, &kv_full[s], hf * 64, hk,
-                        jB * kSaBlk, b);
+            tma_load_4d(st + hf * kStHalf, map, &fullb[s], hf * 64, hk, jA * kSaBlk, b);
+            tma_load_4d(st + hf * kStHalf + 8192, map, &fullb[s], hf * 64, hk, jB * kSaBlk, b);
           }
-          ++kv_it;
+          ++it;
         }
       }
       if (!ok) flags[0] = 1;
@@ -173,24 +187,25 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_cons
   } else if (warp == 9) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      uint32_t kv_it = 0, pr = 0, qrow = 0, orow = 0;
+      uint32_t pr = 0, qrow = 0, orow = 0;
       bool ok = true;
       // the previous pair's P.V, issued after the next pair's Q.K^T
       bool have_prev = false;
-      uint32_t pv_stage = 0, pv_pr = 0, pv_orow = 0;
+      uint32_t pv_pr = 0, pv_orow = 0;
       bool pv_first = false, pv_last = false;
       auto issue_pv = [&]() -> bool {
-        const uint32_t pb = pv_pr & 1, ob = pv_orow & 1;
+        const uint32_t pb = pv_pr & 1, ob = pv_orow & 1, vs = pv_pr % kStNS;
+        if (!mbar_wait(&v_full[vs], (pv_pr / kStNS) & 1)) return false;
         if (!mbar_wait(&p_ready[pb], (pv_pr >> 1) & 1)) return false;
         if (pv_first && !mbar_wait(&o_free[ob], ((pv_orow >> 1) & 1) ^ 1)) return false;
         tc_fence_after();
-        const uint32_t vb = smem_u32(stages + size_t(pv_stage) * kStStage + 2 * kStHalf);
+        const uint32_t vb = smem_u32(vring + size_t(vs) * kStTile);
         const uint32_t pbb = smem_u32(pbuf + pb * kStPBuf);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           tc_mma_ss(tmem + 32 + 32 * ob, umma_desc_sw128(vb + kk * 2048, kStHalf, 1024),
                     st_desc_k(pbb, kk, 4096), kIdPV, (pv_first && kk == 0) ? 0u : 1u);
-        tc_commit(&kv_empty[pv_stage]);
+        tc_commit(&v_empty[vs]);
         tc_commit(&p_free[pb]);
         if (pv_last) tc_commit(&o_full[ob]);
         return true;
@@ -206,23 +221,24 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_cons
         const uint32_t qs = qrow & 1;
         if (flags[0] || !mbar_wait(&q_full[qs], (qrow >> 1) & 1)) { ok = false; break; }
         for (int i = 0; i < npairs; ++i) {
-          const uint32_t s = kv_it % kStNS, sb = pr & 1;
-          if (!mbar_wait(&kv_full[s], (kv_it / kStNS) & 1) ||
+          const uint32_t s = pr % kStNS, sb = pr & 1;
+          if (!mbar_wait(&k_full[s], (pr / kStNS) & 1) ||
               !mbar_wait(&s_free[sb], ((pr >> 1) & 1) ^ 1)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t kb = smem_u32(stages + size_t(s) * kStStage);
+          const uint32_t kb = smem_u32(kring + size_t(s) * kStTile);
           const uint32_t qb = smem_u32(qbuf + qs * kStQBuf);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             tc_mma_ss(tmem + 16 * sb, st_desc_k(kb, kk, kStHalf), st_desc_k(qb, kk, 2048), kIdQK,
                       kk > 0);
           tc_commit(&s_full[sb]);
+          tc_commit(&k_empty[s]);
           if (i == npairs - 1) tc_commit(&q_empty[qs]);
           if (have_prev && !issue_pv()) { ok = false; break; }
           have_prev = true;
-          pv_stage = s; pv_pr = pr; pv_orow = orow;
+          pv_pr = pr; pv_orow = orow;
           pv_first = (i == 0); pv_last = (i == npairs - 1);
-          ++kv_it; ++pr;
+          ++pr;
         }
         ++qrow;
         ++orow;
