@@ -351,7 +351,7 @@ sala_status sala_sparse_attn(const void* q, const void* k, const void* v, const 
   cudaStream_t st = as_stream(stream);
   const int64_t want = num_sms();
   const unsigned grid = (unsigned)std::min<int64_t>(want, p.rows);
-  if (!use_tc_sparse) {
+  if (!(D == 128 && n_sel <= kStMaxSel && use_tc_sparse)) {
     // values that would not survive the fp16 P.V operand conversion raise SALA_ERR_RANGE
     const int64_t n = (int64_t)B * T * Hkv * (D / 8);
     const unsigned cg = (unsigned)std::min<int64_t>((n + 255) / 256, 4 * want);
