@@ -347,7 +347,7 @@ sala_status sala_sparse_attn(const void* q, const void* k, const void* v, const 
   // The mma.sync kernel is faster on this workload (it frees each K/V stage right after
   // the Q.K^T MMAs because V fragments can be held in registers); the tcgen05 kernel
   // must keep every stage until its P.V MMA has read V from shared memory.
-  const bool use_tc_sparse = true;
+  const bool use_tc_sparse = false;
   cudaStream_t st = as_stream(stream);
   const int64_t want = num_sms();
   const unsigned grid = (unsigned)std::min<int64_t>(want, p.rows);
