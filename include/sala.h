@@ -167,8 +167,8 @@ sala_status sala_sparse_select(const void *q, const void *k, int B, int T, int H
  *   scale       softmax scale; 0 selects 1/sqrt(D)
  *   block = 64, D = 64 or 128, 1 <= Hq / Hkv <= 16 (the GQA group fills one
  *   16-row tensor-core tile, padded with zero rows when smaller).
- * Errors: INVALID_ARG, UNSUPPORTED, CUDA.  Device (D = 64 only, where V becomes an
- *   fp16 operand): RANGE when a v value has |v| >= 65536.  D = 128 uses v exactly.
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA.  Device: RANGE when a v value does not
+ *   fit the fp16 tensor-core operand (|v| >= 65536).
  */
 sala_status sala_sparse_attn(const void *q, const void *k, const void *v, const void *g,
                              const int32_t *idx, int n_sel, void *o, int B, int T, int Hq,

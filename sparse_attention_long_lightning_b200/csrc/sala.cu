@@ -17,7 +17,6 @@
 #include "lightning_decode.cuh"
 #include "lightning_tc.cuh"
 #include "sparse_attn.cuh"
-#include "sparse_attn_tc.cuh"
 #include "sparse_select.cuh"
 
 using namespace sala;
@@ -343,30 +342,17 @@ sala_status sala_sparse_attn(const void* q, const void* k, const void* v, const 
   const float sc = scale > 0.0f ? scale : 1.0f / std::sqrt((float)D);
   p.scale_log2 = sc * 1.4426950408889634f;
   p.rows = (int64_t)B * Hkv * T;
-  p.q_box_h = 16;
-  // The mma.sync kernel is faster on this workload (it frees each K/V stage right after
-  // the Q.K^T MMAs because V fragments can be held in registers); the tcgen05 kernel
-  // must keep every stage until its P.V MMA has read V from shared memory.
-  const bool use_tc_sparse = false;
   cudaStream_t st = as_stream(stream);
   const int64_t want = num_sms();
   const unsigned grid = (unsigned)std::min<int64_t>(want, p.rows);
-  if (!(D == 128 && n_sel <= kStMaxSel && use_tc_sparse)) {
+  {
     // values that would not survive the fp16 P.V operand conversion raise SALA_ERR_RANGE
     const int64_t n = (int64_t)B * T * Hkv * (D / 8);
     const unsigned cg = (unsigned)std::min<int64_t>((n + 255) / 256, 4 * want);
     f16_range_check_kernel<<<cg, 256, 0, st>>>((const __nv_bfloat16*)v, sv, B, T, Hkv, D);
     SALA_CHECK_LAUNCH();
   }
-  if (D == 128 && n_sel <= kStMaxSel && use_tc_sparse) {
-    // tcgen05 path: keys as the MMA M dimension
-    CUtensorMap tq;
-    p.q_box_h = Hq < 16 ? Hq : 16;
-    if (!make_tmap_bhtd(&tq, q, B, T, Hq, D, sq, 1, p.q_box_h)) return SALA_ERR_CUDA;
-    auto kern = sparse_attn_tc_kernel;
-    if (!set_smem(kern, StSmem::bytes)) return SALA_ERR_CUDA;
-    kern<<<grid, kStThreads, StSmem::bytes, st>>>(tq, tk, tv, p);
-  } else if (D == 128) {
+  if (D == 128) {
     constexpr int NS = 3;
     auto kern = sparse_attn_kernel<128, NS>;
     if (!set_smem(kern, SaSmem<128, NS>::bytes)) return SALA_ERR_CUDA;

@@ -56,7 +56,6 @@ struct SaParams {
   int n_sel, B, T, Hq, Hkv, G;
   float scale_log2;  // softmax scale * log2(e)
   int64_t rows;      // B * Hkv * T
-  int q_box_h;       // query heads per Q tile load (tensor-core path)
 };
 
 // A selected block j takes part in row t iff j >= 0 and its first key is <= t.
