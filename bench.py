@@ -65,6 +65,20 @@ def _dist():
     return None, 0, 1
 
 
+def max_over_ranks(dist, seconds, device):
+    """Step time of the whole job: the slowest rank's device-timed seconds."""
+    if dist is None:
+        return seconds
+    t = torch.tensor([seconds], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(world, tokens_per_rank, seconds_max):
+    """Whole-job tokens/s: every rank processes its own sequence of tokens_per_rank."""
+    return world * tokens_per_rank / seconds_max
+
+
 class ClockSampler:
     """nvidia-smi clock/throttle samples while the timed region runs."""
 
@@ -343,17 +357,13 @@ def main():
         torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
-    sec = start.elapsed_time(end) / 1e3 / args.steps
-    if dist is not None:
-        t = torch.tensor([sec], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        sec = float(t.item())
+    sec = max_over_ranks(dist, start.elapsed_time(end) / 1e3 / args.steps, dev)
     err = sala.get_device_error()
     if err:
         raise RuntimeError(f"device error in timed region: {sala.status_string(err)}")
 
     op_ms = {k: float(np.mean([a.elapsed_time(b) for a, b in v])) for k, v in per_op.items()}
-    value = world * T / sec
+    value = weak_scaling_value(world, T, sec)
 
     # roofline of the dominant kernel and component figures
     light_bytes = 5 * B * T * H * D * 2 + B * H * D * D * 4
@@ -402,14 +412,10 @@ def main():
     if not args.no_extras:
         line["gpu_launches"] = count_launches(layers, sala) * args.steps
         e2e_sec, h2d, d2h = e2e_measure(layers, sala, args.e2e_steps, stream)
-        line["e2e"] = {"value": world * T / e2e_sec if dist is None else None, "unit": "tokens/s",
+        e2e_sec = max_over_ranks(dist, e2e_sec, dev)
+        line["e2e"] = {"value": weak_scaling_value(world, T, e2e_sec), "unit": "tokens/s",
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                        "ms_per_step": e2e_sec * 1e3}
-        if dist is not None:
-            t = torch.tensor([e2e_sec], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            line["e2e"]["value"] = world * T / float(t.item())
-            line["e2e"]["ms_per_step"] = float(t.item()) * 1e3
         if rank == 0 and world == 1:
             tps, info = cpu_baseline(T)
             line["cpu_baseline"] = dict(info, value=tps, unit="tokens/s")

@@ -209,6 +209,16 @@ sala_status sala_lightning_prefill_noalloc(const void *q, const void *k, const v
                                            sala_dtype dt, void *stream);
 
 /*
+ * Failure-path self-test (a library diagnostic, no counterpart on the pages): runs
+ * the bounded mbarrier wait every kernel uses on a barrier that never completes,
+ * with a budget of `cycles` SM clock cycles (1 .. 4e9), so the wait runs out, sets
+ * SALA_ERR_TIMEOUT in the device error word and returns.  Nothing faults or hangs;
+ * read the result with sala_get_device_error().
+ * Errors: INVALID_ARG (cycles out of range), CUDA.
+ */
+sala_status sala_selftest_wait_timeout(long long cycles, void *stream);
+
+/*
  * Synchronise `stream`, then read and clear the device error word of the
  * current device.  Returns SALA_OK, SALA_ERR_RANGE or SALA_ERR_TIMEOUT (the
  * first condition raised since the last call), or SALA_ERR_CUDA if the

@@ -19,7 +19,7 @@ __all__ = [
     "SalaError", "load_library", "lightning_prefill", "lightning_prefill_workspace",
     "lightning_prefill_noalloc",
     "lightning_decode", "sparse_select", "sparse_select_workspace", "sparse_attn",
-    "get_device_error", "status_string", "version", "LIB_PATH",
+    "get_device_error", "selftest_wait_timeout", "status_string", "version", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsala.so")
@@ -73,6 +73,8 @@ def load_library(path: Optional[str] = None):
     lib.sala_sparse_attn.restype = i
     lib.sala_get_device_error.argtypes = [vp]
     lib.sala_get_device_error.restype = i
+    lib.sala_selftest_wait_timeout.argtypes = [ctypes.c_longlong, vp]
+    lib.sala_selftest_wait_timeout.restype = i
     _lib = lib
     return lib
 
@@ -243,6 +245,14 @@ def sparse_attn(q, k, v, idx, g=None, *, block=64, scale=0.0, out=None, stream=N
                               float(scale), _dt(q), _stream(stream))
     _check("sala_sparse_attn", st)
     return out
+
+
+def selftest_wait_timeout(cycles=20_000_000, stream=None):
+    """Run the bounded-wait failure path on the GPU: a wait that can never complete
+    gives up after `cycles` clock cycles and sets SALA_ERR_TIMEOUT (read it with
+    get_device_error)."""
+    _check("sala_selftest_wait_timeout",
+           load_library().sala_selftest_wait_timeout(int(cycles), _stream(stream)))
 
 
 def get_device_error(stream=None) -> int:

@@ -42,11 +42,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 // Bounded wait: returns false (and raises SALA_ERR_TIMEOUT) if the phase with
 // the given parity has not completed within the cycle budget.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          long long budget = kSpinCycleBudget) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kSpinCycleBudget) {
+    if (clock64() - t0 > budget) {
       raise_device_error(SALA_ERR_TIMEOUT);
       return false;
     }

@@ -463,6 +463,31 @@ sala_status sala_lightning_prefill_noalloc(const void* q, const void* k, const v
   return SALA_OK;
 }
 
+// ------------------------------------------------------------------ failure-path self-test
+}  // extern "C"
+
+namespace {
+// One thread waits, with the kernels' own bounded wait, on an mbarrier whose phase
+// never completes (nothing arrives), then returns having raised SALA_ERR_TIMEOUT.
+__global__ void selftest_wait_timeout_kernel(long long budget) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    (void)mbar_wait(&bar, 0, budget);
+  }
+}
+}  // namespace
+
+extern "C" {
+
+sala_status sala_selftest_wait_timeout(long long cycles, void* stream) {
+  if (cycles < 1 || cycles > kSpinCycleBudget) return SALA_ERR_INVALID_ARG;
+  selftest_wait_timeout_kernel<<<1, 32, 0, as_stream(stream)>>>(cycles);
+  SALA_CHECK_LAUNCH();
+  return SALA_OK;
+}
+
 // ------------------------------------------------------------------ device error word
 sala_status sala_get_device_error(void* stream) {
   if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) {

@@ -123,3 +123,19 @@ def test_sparse_128k_full_size_sampled_rows():
           f"(raw {raw_rel_err(_np(o[:, rows]), ref_o):.3e})")
     assert e <= TOL_BF16
     assert sala.get_device_error() == 0
+
+
+def test_bounded_wait_reports_timeout():
+    """A device wait that can never complete gives up after its cycle budget and
+    reports SALA_ERR_TIMEOUT through the device error word; the context stays usable."""
+    sala.get_device_error()
+    sala.selftest_wait_timeout(20_000_000)
+    assert sala.get_device_error() == 4
+    assert sala.get_device_error() == 0
+    # the GPU still computes correctly afterwards
+    T, Hq, Hkv, D = 200, 16, 1, 128
+    s = inputs.sparse_inputs(1, T, Hq, Hkv, D, seed=8)
+    idx = sala.sparse_select(s.q.cuda(), s.k.cuda(), topk=2)
+    o = sala.sparse_attn(s.q.cuda(), s.k.cuda(), s.v.cuda(), idx)
+    ref = oracle.attention(_np(s.q), _np(s.k), _np(s.v), idx=idx.cpu().numpy())
+    assert rel_err(_np(o), ref, True) <= TOL_BF16
