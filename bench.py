@@ -150,7 +150,9 @@ def make_layers(T, device, seed=1005):
         if L.sparse:
             L.idx = torch.empty((B, HKV, T, N_INIT + TOPK + N_LOCAL), dtype=torch.int32,
                                 device=device)
-            L.ws = torch.empty(sala.sparse_select_workspace(B, T, H, HKV, D, BLOCK),
+            # one scratch serves both calls (selection, then the fp16 copy of v)
+            L.ws = torch.empty(max(sala.sparse_select_workspace(B, T, H, HKV, D, BLOCK),
+                                   sala.sparse_attn_workspace(B, T, HKV, D)),
                                dtype=torch.uint8, device=device)
         else:
             L.state = torch.empty((B, H, D, D), dtype=torch.float32, device=device)
@@ -170,7 +172,7 @@ def run_layer(L, sala, events=None):
         if events is not None:
             events["sel"][1].record()
             events["attn"][0].record()
-        sala.sparse_attn(L.q, L.k, L.v, L.idx, L.g, block=BLOCK, out=L.o)
+        sala.sparse_attn(L.q, L.k, L.v, L.idx, L.g, block=BLOCK, out=L.o, workspace=L.ws)
         if events is not None:
             events["attn"][1].record()
     else:

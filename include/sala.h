@@ -165,16 +165,21 @@ sala_status sala_sparse_select(const void *q, const void *k, int B, int T, int H
  *   q, g, o     [B,T,Hq,D] (g may be NULL), k, v [B,T,Hkv,D] (bf16)
  *   idx         [B,Hkv,T,n_sel] int32, contiguous, entries in [-1, ceil(T/block))
  *   scale       softmax scale; 0 selects 1/sqrt(D)
+ *   ws          device scratch of >= sala_sparse_attn_workspace() bytes, 16-byte
+ *               aligned, caller-owned; it receives an fp16 copy of v (the P.V
+ *               tensor-core operand) and may be reused once the call has run
  *   block = 64, D = 64 or 128, 1 <= Hq / Hkv <= 16 (the GQA group fills one
  *   16-row tensor-core tile, padded with zero rows when smaller).
- * Errors: INVALID_ARG, UNSUPPORTED, CUDA.  Device: RANGE when a v value does not
- *   fit the fp16 tensor-core operand (|v| >= 65536).
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.  Device: RANGE when a v value
+ *   does not fit the fp16 tensor-core operand (|v| >= 65536).
  */
+size_t sala_sparse_attn_workspace(int B, int T, int Hkv, int D);
+
 sala_status sala_sparse_attn(const void *q, const void *k, const void *v, const void *g,
                              const int32_t *idx, int n_sel, void *o, int B, int T, int Hq,
                              int Hkv, int D, sala_strides sq, sala_strides sk, sala_strides sv,
                              sala_strides sg, sala_strides so, int block, float scale,
-                             sala_dtype dt, void *stream);
+                             void *ws, size_t ws_bytes, sala_dtype dt, void *stream);
 
 /*
  * Lightning prefill that allocates nothing (no counterpart in the paper: this is

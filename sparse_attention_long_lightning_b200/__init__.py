@@ -19,6 +19,7 @@ __all__ = [
     "SalaError", "load_library", "lightning_prefill", "lightning_prefill_workspace",
     "lightning_prefill_noalloc",
     "lightning_decode", "sparse_select", "sparse_select_workspace", "sparse_attn",
+    "sparse_attn_workspace",
     "get_device_error", "selftest_wait_timeout", "status_string", "version", "LIB_PATH",
 ]
 
@@ -68,8 +69,10 @@ def load_library(path: Optional[str] = None):
     lib.sala_sparse_select_workspace.restype = sz
     lib.sala_sparse_select.argtypes = [vp, vp, i, i, i, i, i, S, S, i, i, i, i, vp, vp, sz, i, vp]
     lib.sala_sparse_select.restype = i
+    lib.sala_sparse_attn_workspace.argtypes = [i, i, i, i]
+    lib.sala_sparse_attn_workspace.restype = sz
     lib.sala_sparse_attn.argtypes = [vp, vp, vp, vp, vp, i, vp, i, i, i, i, i, S, S, S, S, S, i, f,
-                                     i, vp]
+                                     vp, sz, i, vp]
     lib.sala_sparse_attn.restype = i
     lib.sala_get_device_error.argtypes = [vp]
     lib.sala_get_device_error.restype = i
@@ -230,19 +233,28 @@ def sparse_select(q, k, *, topk=64, n_init=1, n_local=2, block=64, out=None, wor
     return out
 
 
-def sparse_attn(q, k, v, idx, g=None, *, block=64, scale=0.0, out=None, stream=None):
+def sparse_attn_workspace(B, T, Hkv, D) -> int:
+    return int(load_library().sala_sparse_attn_workspace(B, T, Hkv, D))
+
+
+def sparse_attn(q, k, v, idx, g=None, *, block=64, scale=0.0, out=None, workspace=None,
+                stream=None):
     """Block-sparse attention.  q,g [B,T,Hq,D]; k,v [B,T,Hkv,D]; idx [B,Hkv,T,n_sel] int32."""
     lib = load_library()
-    _cuda(q, k, v, idx, g, out)
+    _cuda(q, k, v, idx, g, out, workspace)
     B, T, Hq, D = q.shape
     Hkv = k.shape[2]
     if idx.dtype != torch.int32 or not idx.is_contiguous():
         raise ValueError("idx must be a contiguous int32 tensor")
     if out is None:
         out = torch.empty_like(q, memory_format=torch.contiguous_format)
+    need = sparse_attn_workspace(B, T, Hkv, D)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
     st = lib.sala_sparse_attn(_p(q), _p(k), _p(v), _p(g), _p(idx), int(idx.shape[-1]), _p(out), B,
                               T, Hq, Hkv, D, _s4(q), _s4(k), _s4(v), _s4(g), _s4(out), int(block),
-                              float(scale), _dt(q), _stream(stream))
+                              float(scale), _p(workspace), wsb, _dt(q), _stream(stream))
     _check("sala_sparse_attn", st)
     return out
 

@@ -64,10 +64,11 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
-// 4-D bf16 tensor map over a [B, T, H, D] activation with a (64, box_h, rows, 1)
-// box and 128-byte swizzle (64 bf16 = 128 bytes per box row).
+// 4-D 16-bit (bf16, or fp16 when `f16`) tensor map over a [B, T, H, D] activation
+// with a (64, box_h, rows, 1) box and 128-byte swizzle (64 elements = 128 bytes
+// per box row).
 bool make_tmap_bhtd(CUtensorMap* map, const void* base, int B, int T, int H, int D,
-                    const sala_strides& s, int box_rows, int box_h = 1) {
+                    const sala_strides& s, int box_rows, int box_h = 1, bool f16 = false) {
   auto enc = get_encode_fn();
   if (!enc) return false;
   cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
@@ -77,7 +78,7 @@ bool make_tmap_bhtd(CUtensorMap* map, const void* base, int B, int T, int H, int
   if (B == 1 && strides[2] == 0) strides[2] = 16;
   cuuint32_t box[4] = {64, (cuuint32_t)box_h, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+  CUresult r = enc(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -312,11 +313,16 @@ sala_status sala_sparse_select(const void* q, const void* k, int B, int T, int H
 }
 
 // ------------------------------------------------------------------ sparse attention
+size_t sala_sparse_attn_workspace(int B, int T, int Hkv, int D) {
+  if (B <= 0 || T <= 0 || Hkv <= 0 || D <= 0) return 0;
+  return ((size_t)B * T * Hkv * D * 2 + 255) / 256 * 256;  // fp16 copy of v
+}
+
 sala_status sala_sparse_attn(const void* q, const void* k, const void* v, const void* g,
                              const int32_t* idx, int n_sel, void* o, int B, int T, int Hq,
                              int Hkv, int D, sala_strides sq, sala_strides sk, sala_strides sv,
                              sala_strides sg, sala_strides so, int block, float scale,
-                             sala_dtype dt, void* stream) {
+                             void* ws, size_t ws_bytes, sala_dtype dt, void* stream) {
   if (T > 0 && (!q || !k || !v || !o || !idx)) return SALA_ERR_INVALID_ARG;
   if (B <= 0 || T < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || n_sel <= 0 || !(scale >= 0.0f))
     return SALA_ERR_INVALID_ARG;
@@ -328,9 +334,13 @@ sala_status sala_sparse_attn(const void* q, const void* k, const void* v, const 
       (g && !strides_ok(sg, 2)))
     return SALA_ERR_INVALID_ARG;
   if (T == 0) return SALA_OK;
+  if (!ws || !aligned16(ws) || ws_bytes < sala_sparse_attn_workspace(B, T, Hkv, D))
+    return SALA_ERR_WORKSPACE;
+  // the fp16 copy of v: contiguous [B, T, Hkv, D]
+  const sala_strides sv16 = {(int64_t)T * Hkv * D, (int64_t)Hkv * D, (int64_t)D};
   CUtensorMap tk, tv;
   if (!make_tmap_bhtd(&tk, k, B, T, Hkv, D, sk, kSaBlk) ||
-      !make_tmap_bhtd(&tv, v, B, T, Hkv, D, sv, kSaBlk))
+      !make_tmap_bhtd(&tv, ws, B, T, Hkv, D, sv16, kSaBlk, 1, true))
     return SALA_ERR_CUDA;
   SaParams p;
   p.q = (const __nv_bfloat16*)q;
@@ -346,10 +356,11 @@ sala_status sala_sparse_attn(const void* q, const void* k, const void* v, const 
   const int64_t want = num_sms();
   const unsigned grid = (unsigned)std::min<int64_t>(want, p.rows);
   {
-    // values that would not survive the fp16 P.V operand conversion raise SALA_ERR_RANGE
+    // fp16 copy of v for the P.V MMAs; values that would not survive raise SALA_ERR_RANGE
     const int64_t n = (int64_t)B * T * Hkv * (D / 8);
     const unsigned cg = (unsigned)std::min<int64_t>((n + 255) / 256, 4 * want);
-    f16_range_check_kernel<<<cg, 256, 0, st>>>((const __nv_bfloat16*)v, sv, B, T, Hkv, D);
+    to_f16_copy_kernel<<<cg, 256, 0, st>>>((const __nv_bfloat16*)v, sv, B, T, Hkv, D,
+                                           (__half*)ws);
     SALA_CHECK_LAUNCH();
   }
   if (D == 128) {

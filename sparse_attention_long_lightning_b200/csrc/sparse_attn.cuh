@@ -15,8 +15,8 @@
 // recording the block id beside the stage.  Each group has four consumer
 // warps that split every 64-key block 16 keys apiece: the group's 16 query
 // heads form the M = 16 operand of m16n8k16 tensor-core MMAs (Q K^T in bf16,
-// P V in fp16 with V converted in registers; fp32 accumulation; a pre-pass
-// flags V values outside the fp16 range), the online softmax runs per warp in
+// P V in fp16 on an fp16 copy of V that a pre-pass writes once and checks for
+// values outside the fp16 range; fp32 accumulation), the online softmax runs per warp in
 // registers with a lazily raised reference maximum (rescaling only when a
 // score exceeds it by more than 2^8), and the four partial (max, sum, O)
 // triples are merged through shared memory at the end of the row.  All waits
@@ -271,7 +271,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
         }
       }
       const float mu0 = m0 == -INFINITY ? 0.f : m0, mu1 = m1 == -INFINITY ? 0.f : m1;
-      // P in fp16 (10-bit mantissa); V converted to fp16 in registers
+      // P in fp16 (10-bit mantissa), V is the fp16 copy
       uint32_t pa[4];
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
@@ -285,8 +285,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
       // ---- O += P V
 #pragma unroll
       for (int pp = 0; pp < kNT / 2; ++pp) {
-        mma_f16_16816(oacc[2 * pp], pa, bf16x2_to_f16x2(vv[pp][0]), bf16x2_to_f16x2(vv[pp][1]));
-        mma_f16_16816(oacc[2 * pp + 1], pa, bf16x2_to_f16x2(vv[pp][2]), bf16x2_to_f16x2(vv[pp][3]));
+        mma_f16_16816(oacc[2 * pp], pa, vv[pp][0], vv[pp][1]);
+        mma_f16_16816(oacc[2 * pp + 1], pa, vv[pp][2], vv[pp][3]);
       }
       ++it;
     }
@@ -372,11 +372,14 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
   }
 }
 
-// Values of a bf16 [B, T, H, D] tensor that would not survive conversion to the
-// fp16 tensor-core operand (|x| >= 65536 in bf16, inf or NaN) raise SALA_ERR_RANGE.
+// Writes the fp16 copy of a bf16 [B, T, H, D] tensor (contiguous [B, T, H, D]
+// output) that the P.V MMAs read.  bf16 -> fp16 is exact for normal values
+// below 65504 (8 significant bits fit in 11); values that would not survive
+// (|x| >= 65536 in bf16, inf or NaN) raise SALA_ERR_RANGE.  Tiny values become
+// fp16 subnormals (absolute error below 2^-25).
 __global__ void __launch_bounds__(256)
-f16_range_check_kernel(const __nv_bfloat16* __restrict__ x, sala_strides s, int B, int T, int H,
-                       int D) {
+to_f16_copy_kernel(const __nv_bfloat16* __restrict__ x, sala_strides s, int B, int T, int H,
+                   int D, __half* __restrict__ y) {
   const int64_t rows = (int64_t)B * T * H;
   const int per_row = D / 8;
   uint32_t bad = 0;
@@ -389,9 +392,13 @@ f16_range_check_kernel(const __nv_bfloat16* __restrict__ x, sala_strides s, int 
     const int b = (int)(row / ((int64_t)H * T));
     const uint4 u = *reinterpret_cast<const uint4*>(x + b * s.b + t * s.t + h * s.h + 8 * c);
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    uint32_t hv[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
+    for (int k = 0; k < 4; ++k) {
       bad |= ((w[k] & 0x7fffu) >= 0x4780u) | (((w[k] >> 16) & 0x7fffu) >= 0x4780u);
+      hv[k] = bf16x2_to_f16x2(w[k]);
+    }
+    *reinterpret_cast<uint4*>(y + i * 8) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
   }
   if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) raise_device_error(SALA_ERR_RANGE);
 }

@@ -42,13 +42,14 @@ def main():
     else:
         s = inputs.sparse_inputs(1, a.T, 32, 2, 128, seed=1004, device=dev, gate=True)
         idx = sala.sparse_select(s.q, s.k)
-        ws = torch.empty(sala.sparse_select_workspace(1, a.T, 32, 2, 128), dtype=torch.uint8,
+        ws = torch.empty(max(sala.sparse_select_workspace(1, a.T, 32, 2, 128),
+                             sala.sparse_attn_workspace(1, a.T, 2, 128)), dtype=torch.uint8,
                          device=dev)
         o = torch.empty_like(s.q)
         if a.op == "select":
             fn = lambda: sala.sparse_select(s.q, s.k, out=idx, workspace=ws)
         else:
-            fn = lambda: sala.sparse_attn(s.q, s.k, s.v, idx, s.g, out=o)
+            fn = lambda: sala.sparse_attn(s.q, s.k, s.v, idx, s.g, out=o, workspace=ws)
     for _ in range(a.warmup):
         fn()
     torch.cuda.synchronize()

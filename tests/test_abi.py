@@ -95,10 +95,13 @@ def test_select_and_attn_reject_bad_arguments(lib):
                                   None) == 5
     # fp32 sparse path is not provided
     assert lib.sala_sparse_attn(p, p, p, None, p, 67, p, 1, 64, 2, 2, 128, st, st, st, Z, st, 64,
-                                0.0, 0, None) == 2
+                                0.0, p, 1 << 20, 0, None) == 2
     # group larger than one 16-row tile
     assert lib.sala_sparse_attn(p, p, p, None, p, 67, p, 1, 64, 64, 2, 128, st, st, st, Z, st, 64,
-                                0.0, 1, None) == 2
+                                0.0, p, 1 << 20, 1, None) == 2
+    # workspace too small for the fp16 copy of v
+    assert lib.sala_sparse_attn(p, p, p, None, p, 67, p, 1, 64, 2, 2, 128, st, st, st, Z, st, 64,
+                                0.0, p, 16, 1, None) == 5
 
 
 def test_workspace_queries(lib):
@@ -107,3 +110,5 @@ def test_workspace_queries(lib):
     assert n >= nb * 2 * 128 * 4                             # block means
     assert n <= nb * 2 * 128 * 4 + (1 << 30) + 4096          # scores bounded by 1 GiB
     assert sala.sparse_select_workspace(1, 1 << 20, 32, 2, 128) <= (1 << 30) + (1 << 25)
+    assert sala.sparse_attn_workspace(1, 131072, 2, 128) == 131072 * 2 * 128 * 2
+    assert sala.sparse_attn_workspace(1, 0, 2, 128) == 0
