@@ -14,10 +14,11 @@
 // K and V (128-byte swizzle, no multicast) into the group's NS-deep ring,
 // recording the block id beside the stage.  Each group has four consumer
 // warps that split every 64-key block 16 keys apiece: the group's 16 query
-// heads form the M = 16 operand of m16n8k16 tensor-core MMAs (Q K^T in bf16,
-// P V in fp16 on an fp16 copy of V that a pre-pass writes once and checks for
-// values outside the fp16 range; fp32 accumulation), the online softmax runs per warp in
-// registers with a lazily raised reference maximum (rescaling only when a
+// heads form the M = 16 operand of m16n8k16 tensor-core MMAs (Q K^T in bf16
+// with four independent accumulator chains, P V in fp16 on an fp16 copy of V
+// that a pre-pass writes once and checks for values outside the fp16 range;
+// fp32 accumulation), the online softmax runs per warp in registers with a
+// lazily raised reference maximum (rescaling only when a
 // score exceeds it by more than 2^8), and the four partial (max, sum, O)
 // triples are merged through shared memory at the end of the row.  All waits
 // are bounded; a wait that runs out raises SALA_ERR_TIMEOUT in the device
@@ -205,6 +206,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
       // ---- S = Q K^T for keys 16*wq .. 16*wq+15 of the block
       float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
       {
+        float sd[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         const int mat = lane >> 3, rin = lane & 7;
         const uint32_t krow = wq * 16 + (mat >> 1) * 8 + rin;
 #pragma unroll
@@ -213,9 +215,18 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
           const uint32_t addr = kb + (chunk >> 3) * L::kHalf + swz128(krow, chunk & 7);
           uint32_t b0, b1, b2, b3;
           ldsm_x4(addr, b0, b1, b2, b3);
-          mma_bf16_16816(sc[0], qa[kk], b0, b1);
-          mma_bf16_16816(sc[1], qa[kk], b2, b3);
+          if (kk & 1) {
+            mma_bf16_16816(sd[0], qa[kk], b0, b1);
+            mma_bf16_16816(sd[1], qa[kk], b2, b3);
+          } else {
+            mma_bf16_16816(sc[0], qa[kk], b0, b1);
+            mma_bf16_16816(sc[1], qa[kk], b2, b3);
+          }
         }
+#pragma unroll
+        for (int a = 0; a < 2; ++a)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) sc[a][c] += sd[a][c];
       }
       // ---- this warp's V fragments go to registers, then the stage is released at once
       // (except the row's last block, whose stage is reused for the merge)
