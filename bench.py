@@ -151,7 +151,7 @@ def make_layers(T, device, seed=1005):
             L.idx = torch.empty((B, HKV, T, N_INIT + TOPK + N_LOCAL), dtype=torch.int32,
                                 device=device)
             # one scratch serves both calls (selection, then the fp16 copy of v)
-            L.ws = torch.empty(max(sala.sparse_select_workspace(B, T, H, HKV, D, BLOCK),
+            L.ws = torch.empty(max(sala.sparse_select_workspace(B, T, H, HKV, D, BLOCK, TOPK),
                                    sala.sparse_attn_workspace(B, T, HKV, D)),
                                dtype=torch.uint8, device=device)
         else:

@@ -137,16 +137,21 @@ sala_status sala_lightning_decode(const void *q, const void *k, const void *v, c
  *   {c-n_local+1..c} (clipped to [0, c]); written sorted ascending and padded
  *   with -1 to n_sel = n_init + topk + n_local entries.
  * When every candidate fits the budget all causal blocks are chosen, which is
- * the dense fallback.
+ * the dense fallback.  Scores are computed in fp32-equivalent precision (bf16
+ * high/low operand splits on tensor cores, or fp32 for topk > 64); a decision
+ * between two scores closer than about 1e-5 may differ from exact arithmetic.
  *
  *   q           [B,T,Hq,D], k [B,T,Hkv,D] (bf16)
  *   idx         [B,Hkv,T,n_sel] int32 output, contiguous
- *   ws          device scratch of >= sala_sparse_select_workspace() bytes
+ *   ws          device scratch of >= sala_sparse_select_workspace(..., topk) bytes,
+ *               caller-owned, free again when the call has run; block means only
+ *               for topk <= 64 (T / 64 <= 65535), plus a score scratch of at most
+ *               1 GiB otherwise
  *   block = 64, 1 <= topk <= 256, 0 <= n_init, 1 <= n_local, D = 64 or 128,
  *   Hq % Hkv == 0, Hq / Hkv <= 32.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
  */
-size_t sala_sparse_select_workspace(int B, int T, int Hq, int Hkv, int D, int block);
+size_t sala_sparse_select_workspace(int B, int T, int Hq, int Hkv, int D, int block, int topk);
 
 sala_status sala_sparse_select(const void *q, const void *k, int B, int T, int Hq, int Hkv,
                                int D, sala_strides sq, sala_strides sk, int block, int topk,

@@ -65,7 +65,7 @@ def load_library(path: Optional[str] = None):
     lib.sala_lightning_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, S, S, S, S,
                                           S, f, f, i, vp]
     lib.sala_lightning_decode.restype = i
-    lib.sala_sparse_select_workspace.argtypes = [i, i, i, i, i, i]
+    lib.sala_sparse_select_workspace.argtypes = [i, i, i, i, i, i, i]
     lib.sala_sparse_select_workspace.restype = sz
     lib.sala_sparse_select.argtypes = [vp, vp, i, i, i, i, i, S, S, i, i, i, i, vp, vp, sz, i, vp]
     lib.sala_sparse_select.restype = i
@@ -208,8 +208,8 @@ def lightning_decode(q, k, v, g, state, pos, q_norm_w=None, k_norm_w=None, *, ro
     return out
 
 
-def sparse_select_workspace(B, T, Hq, Hkv, D, block=64) -> int:
-    return int(load_library().sala_sparse_select_workspace(B, T, Hq, Hkv, D, block))
+def sparse_select_workspace(B, T, Hq, Hkv, D, block=64, topk=64) -> int:
+    return int(load_library().sala_sparse_select_workspace(B, T, Hq, Hkv, D, block, topk))
 
 
 def sparse_select(q, k, *, topk=64, n_init=1, n_local=2, block=64, out=None, workspace=None,
@@ -222,7 +222,7 @@ def sparse_select(q, k, *, topk=64, n_init=1, n_local=2, block=64, out=None, wor
     n_sel = n_init + topk + n_local
     if out is None:
         out = torch.empty((B, Hkv, T, n_sel), dtype=torch.int32, device=q.device)
-    need = sparse_select_workspace(B, T, Hq, Hkv, D, block)
+    need = sparse_select_workspace(B, T, Hq, Hkv, D, block, topk)
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0

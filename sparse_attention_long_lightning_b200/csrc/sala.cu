@@ -250,10 +250,16 @@ sala_status sala_lightning_decode(const void* q, const void* k, const void* v, c
 }
 
 // ------------------------------------------------------------------ sparse selection
-size_t sala_sparse_select_workspace(int B, int T, int Hq, int Hkv, int D, int block) {
+// The fused path scores and selects in one kernel: topk <= kSelFusedMaxK and block
+// indices that fit 16 bits.  Otherwise scores go through a bounded scratch.
+static bool sel_fused(int T, int topk) { return topk <= kSelFusedMaxK && T / kSelBlk <= 65535; }
+
+size_t sala_sparse_select_workspace(int B, int T, int Hq, int Hkv, int D, int block, int topk) {
   (void)Hq;
-  if (B <= 0 || T <= 0 || Hkv <= 0 || block != kSelBlk || (D != 64 && D != 128)) return 0;
-  return sel_layout(B, T, Hkv, D).total;
+  if (B <= 0 || T <= 0 || Hkv <= 0 || block != kSelBlk || (D != 64 && D != 128) || topk < 1)
+    return 0;
+  const SelLayout L = sel_layout(B, T, Hkv, D);
+  return sel_fused(T, topk) ? L.total_fused : L.total;
 }
 
 sala_status sala_sparse_select(const void* q, const void* k, int B, int T, int Hq, int Hkv,
@@ -270,19 +276,43 @@ sala_status sala_sparse_select(const void* q, const void* k, int B, int T, int H
     return SALA_ERR_INVALID_ARG;
   if (T == 0) return SALA_OK;
   const SelLayout L = sel_layout(B, T, Hkv, D);
-  if (!ws || ws_bytes < L.total) return SALA_ERR_WORKSPACE;
+  const bool fused = sel_fused(T, topk);
+  if (!ws || ws_bytes < (fused ? L.total_fused : L.total)) return SALA_ERR_WORKSPACE;
   cudaStream_t st = as_stream(stream);
-  float* kbar = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.kbar_off);
-  float* scores = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.score_off);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  float* kbar = reinterpret_cast<float*>(wsb + L.kbar_off);
+  __nv_bfloat16* khi = reinterpret_cast<__nv_bfloat16*>(wsb + L.khi_off);
+  __nv_bfloat16* klo = reinterpret_cast<__nv_bfloat16*>(wsb + L.klo_off);
+  float* scores = reinterpret_cast<float*>(wsb + L.score_off);
   const int G = Hq / Hkv;
   const float inv_sqrt_d = 1.0f / std::sqrt((float)D);
   if (L.nb > 0) {
     dim3 gm(L.nb, Hkv, B);
     if (D == 128)
-      block_means_kernel<128><<<gm, 128, 0, st>>>((const __nv_bfloat16*)k, kbar, L.nb, Hkv, sk);
+      block_means_kernel<128><<<gm, 128, 0, st>>>((const __nv_bfloat16*)k, kbar, khi, klo, L.nb,
+                                                   Hkv, sk);
     else
-      block_means_kernel<64><<<gm, 64, 0, st>>>((const __nv_bfloat16*)k, kbar, L.nb, Hkv, sk);
+      block_means_kernel<64><<<gm, 64, 0, st>>>((const __nv_bfloat16*)k, kbar, khi, klo, L.nb,
+                                                 Hkv, sk);
     SALA_CHECK_LAUNCH();
+  }
+  if (fused) {
+    dim3 gf((T + kSelBlk - 1) / kSelBlk, Hkv, B);
+    if (D == 128) {
+      auto kern = select_fused_kernel<128>;
+      if (!set_smem(kern, SfSmem<128>::bytes)) return SALA_ERR_CUDA;
+      kern<<<gf, kSfThreads, SfSmem<128>::bytes, st>>>((const __nv_bfloat16*)q, khi, klo, idx, T,
+                                                       L.nb, Hkv, G, sq, topk, n_init, n_local,
+                                                       inv_sqrt_d);
+    } else {
+      auto kern = select_fused_kernel<64>;
+      if (!set_smem(kern, SfSmem<64>::bytes)) return SALA_ERR_CUDA;
+      kern<<<gf, kSfThreads, SfSmem<64>::bytes, st>>>((const __nv_bfloat16*)q, khi, klo, idx, T,
+                                                      L.nb, Hkv, G, sq, topk, n_init, n_local,
+                                                      inv_sqrt_d);
+    }
+    SALA_CHECK_LAUNCH();
+    return SALA_OK;
   }
   for (int r0 = 0; r0 < T; r0 += L.rows_pass) {
     const int r1 = std::min(T, r0 + L.rows_pass);

@@ -42,7 +42,7 @@ def main():
     else:
         s = inputs.sparse_inputs(1, a.T, 32, 2, 128, seed=1004, device=dev, gate=True)
         idx = sala.sparse_select(s.q, s.k)
-        ws = torch.empty(max(sala.sparse_select_workspace(1, a.T, 32, 2, 128),
+        ws = torch.empty(max(sala.sparse_select_workspace(1, a.T, 32, 2, 128, 64, 64),
                              sala.sparse_attn_workspace(1, a.T, 2, 128)), dtype=torch.uint8,
                          device=dev)
         o = torch.empty_like(s.q)

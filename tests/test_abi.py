@@ -105,10 +105,14 @@ def test_select_and_attn_reject_bad_arguments(lib):
 
 
 def test_workspace_queries(lib):
-    n = sala.sparse_select_workspace(1, 131072, 32, 2, 128)
     nb = 131072 // 64
-    assert n >= nb * 2 * 128 * 4                             # block means
-    assert n <= nb * 2 * 128 * 4 + (1 << 30) + 4096          # scores bounded by 1 GiB
-    assert sala.sparse_select_workspace(1, 1 << 20, 32, 2, 128) <= (1 << 30) + (1 << 25)
+    means = nb * 2 * 128 * (4 + 2 + 2)                       # fp32 means + bf16 hi / lo
+    # topk <= 64: block means only (scores and top-k fused)
+    n = sala.sparse_select_workspace(1, 131072, 32, 2, 128, 64, 64)
+    assert means <= n <= means + 1024
+    # larger topk: plus a score scratch bounded by 1 GiB
+    n = sala.sparse_select_workspace(1, 131072, 32, 2, 128, 64, 100)
+    assert means + (1 << 29) <= n <= means + (1 << 30) + 4096
+    assert sala.sparse_select_workspace(1, 1 << 20, 32, 2, 128, 64, 200) <= (1 << 30) + (1 << 26)
     assert sala.sparse_attn_workspace(1, 131072, 2, 128) == 131072 * 2 * 128 * 2
     assert sala.sparse_attn_workspace(1, 0, 2, 128) == 0

@@ -33,6 +33,26 @@ def test_select_small(T, Hq, Hkv, D, topk):
     check_index_sets(idx.cpu().numpy(), ref, gap)
 
 
+def test_select_topk_above_fused_limit():
+    """topk > 64 takes the score-scratch path (scores in fp32, per-row radix select)."""
+    T, Hq, Hkv, D, topk = 64 * 200 + 9, 16, 2, 128, 100
+    s = inputs.sparse_inputs(1, T, Hq, Hkv, D, seed=77)
+    idx = sala.sparse_select(s.q.cuda(), s.k.cuda(), topk=topk)
+    ref, gap = oracle.sparse_select(_np(s.q), _np(s.k), topk=topk)
+    check_index_sets(idx.cpu().numpy(), ref, gap)
+
+
+def test_select_exact_ties_take_smaller_blocks():
+    """Every block holds the same keys, so all candidate scores of a row are equal:
+    the selection must be the topk smallest candidate indices, exactly."""
+    T, Hq, Hkv, D, topk = 64 * 300 + 10, 16, 2, 128, 64
+    s = inputs.sparse_inputs(1, T, Hq, Hkv, D, seed=78)
+    k = s.k[:, :64].repeat(1, (T + 63) // 64, 1, 1)[:, :T].contiguous()
+    idx = sala.sparse_select(s.q.cuda(), k.cuda(), topk=topk).cpu().numpy()
+    ref, _ = oracle.sparse_select(_np(s.q), _np(k), topk=topk)
+    assert np.array_equal(idx, ref)
+
+
 def test_select_batched_strided():
     """B = 2 with q, k as views of a packed tensor (non-contiguous strides)."""
     B, T, Hq, Hkv, D = 2, 64 * 13 + 30, 16, 2, 128
