@@ -201,6 +201,7 @@ __device__ __forceinline__ void tc_epilogue(uint32_t t_o, const uint4 (&gv)[4], 
   tc_ld32(t_o, r);
   tc_wait_ld();
   if (!live) return;
+  float chk = 0.f;
 #pragma unroll
   for (int c8 = 0; c8 < 4; ++c8) {
     float y[8];
@@ -212,8 +213,9 @@ __device__ __forceinline__ void tc_epilogue(uint32_t t_o, const uint4 (&gv)[4], 
 #pragma unroll
       for (int e = 0; e < 8; ++e) y[e] *= sigmoidf_(gf[e]);
     }
+    // inf or NaN anywhere makes the running sum non-finite
 #pragma unroll
-    for (int e = 0; e < 8; ++e) bad |= (__float_as_uint(y[e]) & 0x7f800000u) == 0x7f800000u;
+    for (int e = 0; e < 8; ++e) chk += y[e];
     uint4 w;
     __nv_bfloat162 h0 = __floats2bfloat162_rn(y[0], y[1]), h1 = __floats2bfloat162_rn(y[2], y[3]);
     __nv_bfloat162 h2 = __floats2bfloat162_rn(y[4], y[5]), h3 = __floats2bfloat162_rn(y[6], y[7]);
@@ -221,6 +223,7 @@ __device__ __forceinline__ void tc_epilogue(uint32_t t_o, const uint4 (&gv)[4], 
     w.z = *reinterpret_cast<uint32_t*>(&h2); w.w = *reinterpret_cast<uint32_t*>(&h3);
     *reinterpret_cast<uint4*>(orow + 8 * c8) = w;
   }
+  bad |= !(fabsf(chk) <= 3.0e38f);
 }
 
 // Software pipeline per CTA (one segment of one head), chunk u:
@@ -253,6 +256,7 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   float* red = reinterpret_cast<float*>(misc + 64);        // [16]
   double* inv_freq = reinterpret_cast<double*>(misc + 128);  // [64]
   float2* ang_tab = reinterpret_cast<float2*>(misc + 640);   // [2][64]: (base angle, inv_freq)
+  uint32_t* smax = reinterpret_cast<uint32_t*>(misc + 1792);  // [2] bits of the |S| maximum
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int prow = 8 * warp + (lane >> 2), pqd = lane & 3;  // prep: 4 lanes per row
@@ -269,6 +273,8 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   const int nchunks = c_end - c_begin;
 
   if (tid == 0) {
+    smax[0] = 0u;
+    smax[1] = 0u;
     for (int i = 0; i < L::kStages; ++i) mbar_init(&full[i], 1);
     mbar_init(mma1_bar, 1);
     mbar_init(mma2_bar, 1);
@@ -376,6 +382,7 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     if (!ok) break;
     tc_fence_after();
     if (tid == 0) {
+      smax[(u + 1) & 1] = 0u;  // last read before this barrier; next written after the next one
       if (u > 0 && issued < nchunks) issue(issued++);  // stage of chunk u-1 is free
       const uint32_t t_o = t_o0 + 128 * (u & 1);
       if (!kStateOnly) {
@@ -447,6 +454,8 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     }
     e_prev = e_cur;
     if (u + 1 < nchunks) {
+      // |S| maximum of the block through one shared atomic per warp; it is read after
+      // the next barrier, so the scale needs no barrier of its own
       uint32_t r[32];
       tc_ld32(t_s + lane_off + 32 * cg, r);
       tc_wait_ld();
@@ -454,7 +463,31 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
 #pragma unroll
       for (int m = 0; m < 32; ++m) mx = fmaxf(mx, fabsf(__uint_as_float(r[m])));
       bad |= !(mx <= 3.0e38f);  // inf or NaN in the state
-      const int e_next = tc_block_scale_exp(mx, red);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      if (lane == 0) atomicMax(&smax[u & 1], __float_as_uint(mx));
+    }
+    // ---- E: PV(u)
+    tc_fence_before();
+    ok = __syncthreads_and(ok);
+    if (!ok) break;
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t t_o = t_o0 + 128 * (u & 1);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) tc_mma_ts(t_o, t_p + 8 * kk, tc_desc_mn(sV, kk), kIdPV, 1u);
+      tc_commit(mma2_bar);
+    }
+    // ---- S -> fp16 operand for chunk u+1 (its last reader, the inter MMA of chunk u,
+    // completed before D; the state MMA of chunk u+1 is issued only after the next barrier)
+    if (u + 1 < nchunks) {
+      tc_fence_after();
+      uint32_t r[32];
+      tc_ld32(t_s + lane_off + 32 * cg, r);
+      tc_wait_ld();
+      int x = 0;
+      frexpf(__uint_as_float(smax[u & 1]), &x);
+      const int e_next = x > 15 ? x - 15 : 0;
       const float sc = pow2i(-e_next);
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) {
@@ -467,17 +500,6 @@ lightning_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       }
       fence_proxy_async_smem();
       e_cur = e_next;
-    }
-    // ---- E: PV(u)
-    tc_fence_before();
-    ok = __syncthreads_and(ok);
-    if (!ok) break;
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t t_o = t_o0 + 128 * (u & 1);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) tc_mma_ts(t_o, t_p + 8 * kk, tc_desc_mn(sV, kk), kIdPV, 1u);
-      tc_commit(mma2_bar);
     }
   }
 
