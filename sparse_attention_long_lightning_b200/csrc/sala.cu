@@ -16,6 +16,7 @@
 #include "lightning_cc.cuh"
 #include "lightning_decode.cuh"
 #include "lightning_tc.cuh"
+#include "lightning_out.cuh"
 #include "sparse_attn.cuh"
 #include "sparse_select.cuh"
 
@@ -166,10 +167,10 @@ sala_status sala_lightning_prefill(const void* q, const void* k, const void* v, 
     p.log2_base = log2_base;
     p.eps = eps;
     const unsigned grid = (unsigned)(B * H * p.G);
-    auto ka = lightning_tc_kernel<true>;
-    auto kc = lightning_tc_kernel<false>;
+    auto ka = lightning_state_kernel;
+    auto kc = lightning_out_kernel;
     if (!set_smem(ka, TcSmem<true>::bytes) || !set_smem(kc, TcSmem<false>::bytes)) return SALA_ERR_CUDA;
-    ka<<<grid, kTcThreads, TcSmem<true>::bytes, st>>>(tk, tk, tv, p);
+    ka<<<grid, kTcThreads, TcSmem<true>::bytes, st>>>(tk, tv, p);
     SALA_CHECK_LAUNCH();
     lightning_scan_kernel<<<dim3(B * H, 16), 256, 0, st>>>(p.ws, state, p.G, init_zero);
     SALA_CHECK_LAUNCH();
@@ -492,10 +493,10 @@ sala_status sala_lightning_prefill_noalloc(const void* q, const void* k, const v
   p.log2_base = std::log2((double)rope_base);
   p.eps = eps;
   const unsigned grid = (unsigned)(B * H * p.G);
-  auto ka = lightning_tc_kernel<true>;
-  auto kc = lightning_tc_kernel<false>;
+  auto ka = lightning_state_kernel;
+  auto kc = lightning_out_kernel;
   if (!set_smem(ka, TcSmem<true>::bytes) || !set_smem(kc, TcSmem<false>::bytes)) return SALA_ERR_CUDA;
-  ka<<<grid, kTcThreads, TcSmem<true>::bytes, st>>>(tk, tk, tv, p);
+  ka<<<grid, kTcThreads, TcSmem<true>::bytes, st>>>(tk, tv, p);
   SALA_CHECK_LAUNCH();
   lightning_scan_kernel<<<dim3(B * H, 16), 256, 0, st>>>(p.ws, state, p.G, init_zero);
   SALA_CHECK_LAUNCH();
