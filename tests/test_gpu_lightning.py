@@ -103,6 +103,26 @@ def test_lightning_32k_full_size_sampled_heads():
     assert sala.get_device_error() == 0
 
 
+def test_lightning_1m_full_size_sampled_head():
+    """One Lightning layer of the 1M-token hybrid stack: B1 H32 D128 T1048576 bf16,
+    chunk 128 (seed 1012).  One head is compared on 4096 spread rows plus the last 128,
+    and its final state, against the full 1M-token recurrence."""
+    B, T, H, D = 1, 1 << 20, 32, 128
+    x = inputs.lightning_inputs(B, T, H, D, seed=1012, device=DEV)
+    y, S = sala.lightning_prefill(x.q, x.k, x.v, x.g, chunk=128)
+    head = 13
+    rng = np.random.default_rng(7)
+    rows = np.unique(np.concatenate([rng.choice(T - 128, size=4096, replace=False),
+                                     np.arange(T - 128, T)]))
+    yr, Sr = oracle.lightning_recurrent(*(_np(t[:, :, [head]]) for t in (x.q, x.k, x.v, x.g)),
+                                        rows=rows)
+    e_y = rel_err(_np(y[:, rows][:, :, [head]]), yr, True)
+    e_s = rel_err(_np(S[:, [head]]), Sr, False)
+    print(f"1m: y {e_y:.3e} S {e_s:.3e}")
+    assert e_y <= TOL_BF16 and e_s <= TOL_BF16
+    assert sala.get_device_error() == 0
+
+
 @pytest.mark.parametrize("D,dtype", [(128, torch.bfloat16), (64, torch.float32)])
 def test_decode_steps(D, dtype):
     B, H, steps = 3, 4, 5

@@ -145,6 +145,27 @@ def test_sparse_128k_full_size_sampled_rows():
     assert sala.get_device_error() == 0
 
 
+def test_sparse_1m_full_size_sampled_rows():
+    """One sparse layer of the 1M-token hybrid stack: B1 T1048576 Hq32 Hkv2 D128 (seed
+    1011), selection (16383 candidate blocks per late row) and attention compared on
+    sampled rows of both KV heads (first/last 256 rows and 256 spread rows)."""
+    T, Hq, Hkv, D = 1 << 20, 32, 2, 128
+    s = inputs.sparse_inputs(1, T, Hq, Hkv, D, seed=1011, device=DEV, gate=True)
+    idx = sala.sparse_select(s.q, s.k)
+    o = sala.sparse_attn(s.q, s.k, s.v, idx, s.g)
+    rows = _sampled_rows(T, 256, seed=5)
+    q_rows = _np(s.q[:, rows])
+    k_np, v_np = _np(s.k), _np(s.v)
+    ref_idx, gap = oracle.sparse_select(q_rows, k_np, rows=rows, T=T)
+    gi = idx[:, :, rows].cpu().numpy()
+    ndiff, nrow = check_index_sets(gi, ref_idx, gap)
+    ref_o = oracle.attention(q_rows, k_np, v_np, _np(s.g[:, rows]), idx=gi, rows=rows)
+    e = rel_err(_np(o[:, rows]), ref_o, True)
+    print(f"1m sparse: index rows differing at near-ties {ndiff}/{nrow}; attn {e:.3e}")
+    assert e <= TOL_BF16
+    assert sala.get_device_error() == 0
+
+
 def test_bounded_wait_reports_timeout():
     """A device wait that can never complete gives up after its cycle budget and
     reports SALA_ERR_TIMEOUT through the device error word; the context stays usable."""
