@@ -370,26 +370,132 @@ __device__ __forceinline__ int sf_compact(float* bs, uint16_t* bj, int m, int k,
     jv[i] = valid[i] ? (int)bj[e] : 0;
     key[i] = valid[i] ? order_key(sv[i]) : 0u;
   }
-  uint32_t prefix = 0, pmask = 0;
-  int rem = 0;
-  warp_kth_prefix<PER>(key, valid, k, hist, lane, &prefix, &pmask, &rem);
-  int n_eq = 0;
-#pragma unroll
-  for (int i = 0; i < PER; ++i)
-    n_eq += __popc(__ballot_sync(0xffffffffu, valid[i] && (key[i] & pmask) == prefix));
+  const uint32_t lt_mask = (1u << lane) - 1u;
   bool take[PER];
+  bool done = false;
+  {
+    // Fast path: one histogram over 256 value bins between the smallest and the largest
+    // score.  The bin is a monotone function of the score, so every bin above the one
+    // holding the k-th best is kept whole; inside that boundary bin (usually a few
+    // entries) the exact order (larger score, then smaller block) decides.
+    float lo = INFINITY, hi = -INFINITY;
 #pragma unroll
-  for (int i = 0; i < PER; ++i)
-    take[i] = valid[i] && ((key[i] & pmask) > prefix || ((key[i] & pmask) == prefix && n_eq == rem));
-  if (n_eq != rem) {
-    // (pmask is all ones here) exact score ties at the boundary: keep the `rem`
-    // smallest block indices among them
+    for (int i = 0; i < PER; ++i)
+      if (valid[i]) {
+        lo = fminf(lo, sv[i]);
+        hi = fmaxf(hi, sv[i]);
+      }
 #pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      if (valid[i] && key[i] == prefix) {
+    for (int off = 16; off > 0; off >>= 1) {
+      lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+      hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+    }
+    const float scale = 255.0f / (hi - lo);
+    if (hi > lo && scale < 1.0e30f) {
+      int bin[PER];
+#pragma unroll
+      for (int i = 0; i < PER; ++i) bin[i] = valid[i] ? min(255, (int)((sv[i] - lo) * scale)) : -1;
+      for (int e = lane; e < 256; e += 32) hist[e] = 0;
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < PER; ++i)
+        if (bin[i] >= 0) atomicAdd(&hist[bin[i]], 1u);
+      __syncwarp();
+      uint32_t hv[8];
+      uint32_t local = 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        hv[u] = hist[lane * 8 + u];
+        local += hv[u];
+      }
+      uint32_t incl = local;  // suffix sum over lanes >= lane
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t o = __shfl_down_sync(0xffffffffu, incl, off);
+        if (lane + off < 32) incl += o;
+      }
+      const uint32_t above = incl - local;
+      const bool mine = above < (uint32_t)k && (uint32_t)k <= incl;
+      int bucket = 0, rem_b = 0, n_b = 0;
+      if (mine) {
+        uint32_t cntv = above;
+#pragma unroll
+        for (int u = 7; u >= 0; --u) {
+          if (rem_b == 0 && cntv + hv[u] >= (uint32_t)k) {
+            bucket = lane * 8 + u;
+            rem_b = k - (int)cntv;
+            n_b = (int)hv[u];
+          }
+          cntv += hv[u];
+        }
+      }
+      const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+      bucket = __shfl_sync(0xffffffffu, bucket, src);
+      rem_b = __shfl_sync(0xffffffffu, rem_b, src);
+      n_b = __shfl_sync(0xffffffffu, n_b, src);
+      if (rem_b == n_b) {
+#pragma unroll
+        for (int i = 0; i < PER; ++i) take[i] = bin[i] >= bucket;
+        done = true;
+      } else if (n_b <= 32) {
+        // gather the boundary bin into lanes 0..n_b-1 (through the histogram area)
+        float* xs = reinterpret_cast<float*>(hist);
+        int* xj = reinterpret_cast<int*>(hist) + 32;
+        int pos[PER];
+        int cnt = 0;
+        __syncwarp();  // every lane has read the histogram
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+          const bool in_b = bin[i] == bucket;
+          const uint32_t bm = __ballot_sync(0xffffffffu, in_b);
+          pos[i] = cnt + __popc(bm & lt_mask);
+          if (in_b) {
+            xs[pos[i]] = sv[i];
+            xj[pos[i]] = jv[i];
+          }
+          cnt += __popc(bm);
+        }
+        __syncwarp();
+        const float s_me = lane < n_b ? xs[lane] : -INFINITY;
+        const int j_me = lane < n_b ? xj[lane] : 0x7fffffff;
         int rank = 0;
-        for (int e2 = 0; e2 < m; ++e2) rank += (order_key(bs[e2]) == prefix && (int)bj[e2] < jv[i]);
-        take[i] = rank < rem;
+        for (int l2 = 0; l2 < n_b; ++l2) {
+          const float s2 = __shfl_sync(0xffffffffu, s_me, l2);
+          const int j2 = __shfl_sync(0xffffffffu, j_me, l2);
+          rank += (s2 > s_me || (s2 == s_me && j2 < j_me));
+        }
+        const bool win = lane < n_b && rank < rem_b;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+          const bool w = __shfl_sync(0xffffffffu, win, bin[i] == bucket ? pos[i] : 0);
+          take[i] = bin[i] > bucket || (bin[i] == bucket && w);
+        }
+        done = true;
+      }
+    }
+  }
+  if (!done) {
+    // general path (equal scores filling the boundary): radix select on the order keys
+    uint32_t prefix = 0, pmask = 0;
+    int rem = 0;
+    warp_kth_prefix<PER>(key, valid, k, hist, lane, &prefix, &pmask, &rem);
+    int n_eq = 0;
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+      n_eq += __popc(__ballot_sync(0xffffffffu, valid[i] && (key[i] & pmask) == prefix));
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+      take[i] = valid[i] && ((key[i] & pmask) > prefix || ((key[i] & pmask) == prefix && n_eq == rem));
+    if (n_eq != rem) {
+      // (pmask is all ones here) exact score ties at the boundary: keep the `rem`
+      // smallest block indices among them
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        if (valid[i] && key[i] == prefix) {
+          int rank = 0;
+          for (int e2 = 0; e2 < m; ++e2) rank += (order_key(bs[e2]) == prefix && (int)bj[e2] < jv[i]);
+          take[i] = rank < rem;
+        }
       }
     }
   }
@@ -401,7 +507,6 @@ __device__ __forceinline__ int sf_compact(float* bs, uint16_t* bj, int m, int k,
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, off));
   __syncwarp();  // every lane has read the buffer
-  const uint32_t lt_mask = (1u << lane) - 1u;
   int pos = 0;
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
