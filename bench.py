@@ -276,29 +276,55 @@ def run_reference(args):
 
 def e2e_measure(layers, sala, steps, stream):
     """Same step through the public API with inputs in pinned host memory: every step
-    copies each layer's inputs host->device and the outputs device->host."""
+    copies each layer's inputs host->device and its output device->host.  Copies run on
+    their own streams, so layer l+1's inputs cross PCIe while layer l computes and layer
+    l-1's output comes back; each layer's device buffers are reused only after their
+    previous copies and kernels have finished (events)."""
     host_light = [t.cpu().pin_memory() for t in (layers[0].q, layers[0].k, layers[0].v,
                                                  layers[0].g)]
     sp = layers[SPARSE_LAYERS[0]]
     host_sparse = [t.cpu().pin_memory() for t in (sp.q, sp.k, sp.v, sp.g)]
-    host_out = torch.empty_like(layers[0].o, device="cpu").pin_memory()
+    host_out = [torch.empty_like(L.o, device="cpu").pin_memory() for L in layers]
     h2d = sum(sum(t.numel() * t.element_size() for t in (L.q, L.k, L.v, L.g)) for L in layers)
     d2h = sum(L.o.numel() * L.o.element_size() for L in layers)
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    n = len(layers)
+    ev = lambda: torch.cuda.Event()
+    computed = [ev() for _ in range(n)]   # layer l's kernels finished (its inputs are free)
+    copied_out = [ev() for _ in range(n)]  # layer l's output is on the host (o is free)
+    first = [True]
 
     def one():
-        for L in layers:
-            src = host_sparse if L.sparse else host_light
-            for dst, s in zip((L.q, L.k, L.v, L.g), src):
-                dst.copy_(s, non_blocking=True)
-            run_layer(L, sala)
-            host_out.copy_(L.o, non_blocking=True)
+        for l, L in enumerate(layers):
+            arrived = ev()
+            with torch.cuda.stream(s_in):
+                if not first[0]:
+                    s_in.wait_event(computed[l])
+                src = host_sparse if L.sparse else host_light
+                for dst, h in zip((L.q, L.k, L.v, L.g), src):
+                    dst.copy_(h, non_blocking=True)
+                arrived.record(s_in)
+            stream.wait_event(arrived)
+            if not first[0]:
+                stream.wait_event(copied_out[l])
+            with torch.cuda.stream(stream):
+                run_layer(L, sala)
+                computed[l].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(computed[l])
+                host_out[l].copy_(L.o, non_blocking=True)
+                copied_out[l].record(s_out)
+        first[0] = False
 
     one()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    s_in.wait_event(e0)
     for _ in range(steps):
         one()
+    stream.wait_stream(s_out)
+    stream.wait_stream(s_in)
     e1.record(stream)
     torch.cuda.synchronize()
     return e0.elapsed_time(e1) / steps / 1e3, h2d, d2h
