@@ -19,6 +19,7 @@
 #include "lightning_out.cuh"
 #include "sparse_attn.cuh"
 #include "sparse_select.cuh"
+#include "sparse_select_tc.cuh"
 
 using namespace sala;
 
@@ -251,8 +252,9 @@ sala_status sala_lightning_decode(const void* q, const void* k, const void* v, c
 }
 
 // ------------------------------------------------------------------ sparse selection
-// The fused path scores and selects in one kernel: topk <= kSelFusedMaxK and block
-// indices that fit 16 bits.  Otherwise scores go through a bounded scratch.
+// The fused path (select_tc_kernel) scores and selects in one persistent kernel: topk <=
+// kSelFusedMaxK and block indices that fit 16 bits.  Otherwise scores go through a
+// bounded scratch.
 static bool sel_fused(int T, int topk) { return topk <= kSelFusedMaxK && T / kSelBlk <= 65535; }
 
 size_t sala_sparse_select_workspace(int B, int T, int Hq, int Hkv, int D, int block, int topk) {
@@ -298,19 +300,27 @@ sala_status sala_sparse_select(const void* q, const void* k, int B, int T, int H
     SALA_CHECK_LAUNCH();
   }
   if (fused) {
-    dim3 gf((T + kSelBlk - 1) / kSelBlk, Hkv, B);
+    // block means (bf16 hi / lo) as a [B, nb, Hkv, D] tensor, 32-candidate boxes
+    const int nbm = L.nb > 0 ? L.nb : 1;
+    const sala_strides skb{(int64_t)nbm * Hkv * D, (int64_t)Hkv * D, (int64_t)D};
+    CUtensorMap th, tl;
+    if (!make_tmap_bhtd(&th, khi, B, nbm, Hkv, D, skb, kStcN) ||
+        !make_tmap_bhtd(&tl, klo, B, nbm, Hkv, D, skb, kStcN))
+      return SALA_ERR_CUDA;
+    const int nitems = (T + kStcRows - 1) / kStcRows * Hkv * B;
+    const int grid = std::min(nitems, num_sms());
     if (D == 128) {
-      auto kern = select_fused_kernel<128>;
-      if (!set_smem(kern, SfSmem<128>::bytes)) return SALA_ERR_CUDA;
-      kern<<<gf, kSfThreads, SfSmem<128>::bytes, st>>>((const __nv_bfloat16*)q, khi, klo, idx, T,
-                                                       L.nb, Hkv, G, sq, topk, n_init, n_local,
-                                                       inv_sqrt_d);
+      auto kern = select_tc_kernel<128>;
+      if (!set_smem(kern, StcSmem<128>::bytes)) return SALA_ERR_CUDA;
+      kern<<<grid, kStcThreads, StcSmem<128>::bytes, st>>>(th, tl, (const __nv_bfloat16*)q, idx,
+                                                          T, L.nb, Hkv, B, G, sq, topk, n_init,
+                                                          n_local);
     } else {
-      auto kern = select_fused_kernel<64>;
-      if (!set_smem(kern, SfSmem<64>::bytes)) return SALA_ERR_CUDA;
-      kern<<<gf, kSfThreads, SfSmem<64>::bytes, st>>>((const __nv_bfloat16*)q, khi, klo, idx, T,
-                                                      L.nb, Hkv, G, sq, topk, n_init, n_local,
-                                                      inv_sqrt_d);
+      auto kern = select_tc_kernel<64>;
+      if (!set_smem(kern, StcSmem<64>::bytes)) return SALA_ERR_CUDA;
+      kern<<<grid, kStcThreads, StcSmem<64>::bytes, st>>>(th, tl, (const __nv_bfloat16*)q, idx,
+                                                         T, L.nb, Hkv, B, G, sq, topk, n_init,
+                                                         n_local);
     }
     SALA_CHECK_LAUNCH();
     return SALA_OK;

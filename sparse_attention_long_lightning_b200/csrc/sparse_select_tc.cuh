@@ -1,0 +1,518 @@
+// sparse_select_tc.cuh -- block selection on tcgen05, one query row per TMEM lane.
+//
+// Same selection as sparse_select.cuh (InfLLM-v2 style, MiniCPM-SALA tech-report
+// mirror, section 02 (2); summary page, "Prerequisites / Sparse Attention"):
+//   score_j = (1/sqrt(D)) (sum_{h in group(hk)} q_{t,h}) . Kbar_j  over the candidates
+//   n_init <= j <= c - n_local, top `topk` (larger score first, ties -> smaller j),
+//   plus the init blocks and the local window, sorted, -1 padded.
+//
+// Design (sm_100a).  A work item is 128 consecutive query rows (two query blocks) of
+// one KV head; the 128 rows are the M dimension of tcgen05 MMAs, so TMEM lane = query
+// row.  CTAs are persistent (one per SM) and take items in a snake order over the
+// long-rows-first item list.  Each CTA has two warpgroups:
+//   producers (warps 4-7): thread p sums the group's queries of row p in fp32, splits
+//     the sum into bf16 high / low parts and stores them to its TMEM lane: the A
+//     operand of the NEXT item (two A buffers), so the query reads overlap the scan;
+//   issuer (warp 8, one thread): streams 32-candidate tiles of the block means (bf16
+//     high / low, written by block_means_kernel) through a 3-stage shared-memory ring
+//     by TMA and issues S = qs_lo.Kb_hi + qs_hi.Kb_lo + qs_hi.Kb_hi into one of 8 fp32
+//     TMEM score buffers;
+//   consumers (warps 0-3): thread r reads its row's 32 scores of a tile, releases the
+//     score buffer (per-warp arrival, so the warps run decoupled) and appends the
+//     scores above its row threshold to a per-row buffer (shared memory, block order).
+// When a buffer could overflow on the next tile, the rows of that warp compact their
+// buffers (each thread its own row, in step): the topk-th best is located by bucketing
+// the scores' order-preserving integer keys (64 bins per pass, counted with shared
+// atomics; the bin holding the boundary is refined until it is resolved), then the
+// kept entries are packed in place, which preserves block order.  The threshold becomes the smallest kept score:
+// a later candidate with an equal score has a larger block index and loses the tie.
+// At the end each row's buffer is compacted to topk and written out as it stands.
+#pragma once
+
+#include "sparse_select.cuh"
+
+namespace sala {
+
+constexpr int kStcRows = 128;   // query rows per item (= TMEM lanes = consumer threads)
+constexpr int kStcN = 32;       // candidates per tile
+constexpr int kStcCap = 214;    // buffered candidates per row
+constexpr int kStcBins = 64;    // histogram bins per compaction pass
+constexpr int kStcStages = 3;   // block-mean tile ring
+constexpr int kStcAcc = 8;      // TMEM score buffers
+constexpr int kStcCoarse = 150;  // entries a compaction during the scan may keep
+constexpr int kStcThreads = 2 * kStcRows + 32;  // consumers, producers, issuer
+
+template <int D>
+struct StcSmem {
+  static constexpr int kHalfB = kStcN * 128;                 // 32 rows x 64 dims bf16: 4 KB
+  static constexpr int kTileB = (D / 64) * kHalfB;           // one hi or lo tile
+  static constexpr int kStage = 2 * kTileB;                  // hi then lo
+  static constexpr size_t kB = 0;                                     // [stages]
+  static constexpr size_t kBufS = kB + kStcStages * size_t(kStage);   // [entry][row] f32
+  static constexpr size_t kBufJ = kBufS + size_t(kStcCap) * kStcRows * 4;  // [entry][row] u16
+  // [bin][row % 64] u32, rows r and r + 64 in the low / high 16 bits
+  static constexpr size_t kHist = kBufJ + size_t(kStcCap) * kStcRows * 2;
+  static constexpr size_t kBars = kHist + size_t(kStcBins) * 64 * 4;
+  static constexpr int kNumBars = 2 * kStcStages + 2 * kStcAcc + 4 + 1;
+  // full[S], stage_free[S], mma_done[A], acc_free[A], a_full[2], a_free[2], drain;
+  // then the tmem slot and the abort flag
+  static constexpr size_t bytes = 1024 + kBars + kNumBars * 8 + 8;
+  static_assert(bytes <= 232448, "fits one CTA per SM");
+};
+
+// Compact one row's m > k buffered entries (shared addresses: sA / jA the scores (f32)
+// and block indices (u16), entry e at + e * kStcRows * size; hA the row's 64 histogram
+// bins, bin b in the 16 bits at `sh16` of the word at hA + b * 256), in buffer order.
+// smin / smax: the smallest and largest buffered score.  Every entry among the k best
+// (larger score first, ties -> smaller block index) is kept; with keep_max == k exactly
+// those are kept, with keep_max > k a coarser cut that keeps at most keep_max entries
+// may be taken instead.  Returns the kept count and sets *thr to the smallest kept score.
+//
+// Each score gets a fine index f in [0, 4096) linear in (s - smin), monotone in s.  Pass
+// A counts f / 64 (64 coarse bins) and finds the bin holding the k-th best; pass B counts
+// f % 64 inside it; if the fine cell holding the boundary still has more entries than
+// needed, their order-preserving integer keys are bucketed (64 bins of the key range,
+// refined until the boundary is resolved or only equal scores remain, where the earliest
+// = smallest block index win).
+__device__ __noinline__ int stc_compact(uint32_t sA, uint32_t jA, uint32_t hA, int sh16, int m,
+                                        int k, float smin, float smax, int keep_max, float* thr) {
+  constexpr uint32_t kSs = kStcRows * 4, kJs = kStcRows * 2, kHs = 64 * 4;  // strides
+  constexpr int kU = 8;  // loads in flight per pass
+  const uint32_t other = sh16 ? 0x0000ffffu : 0xffff0000u;
+  const uint32_t one = 1u << sh16;
+  const float range = smax - smin;
+  const float scale = 4096.0f / range;
+  const bool linear = range > 0.f && scale <= 3.0e38f;
+  auto fine_of = [&](float s) { return linear ? min(4095, (int)((s - smin) * scale)) : 0; };
+  auto clear = [&](int top) {
+    for (int b = 0; b <= top; ++b) red_and_shared(hA + b * kHs, other);
+  };
+  // bin holding the need-th best counting down from `top`; *above: entries in higher bins
+  auto scan = [&](int top, int need, int* above, int* cnt) {
+    int b = -1, ab = 0, cb_at = 0;
+    for (int b0 = top; b0 >= 0 && b < 0; b0 -= kU) {
+      uint32_t hw[kU];
+#pragma unroll
+      for (int x = 0; x < kU; ++x) hw[x] = lds_u32(hA + max(b0 - x, 0) * kHs);
+#pragma unroll
+      for (int x = 0; x < kU; ++x) {
+        const int bb = b0 - x;
+        const int cb = (int)((hw[x] >> sh16) & 0xffffu);
+        if (b < 0 && bb >= 0) {
+          if (ab + cb >= need || bb == 0) {
+            b = bb;
+            cb_at = cb;
+          } else {
+            ab += cb;
+          }
+        }
+      }
+    }
+    *above = ab;
+    *cnt = cb_at;
+    return b;
+  };
+  // one pass over the entries: bin_of(f, key) < 0 skips the entry
+  auto count = [&](auto bin_of) {
+    for (int e0 = 0; e0 < m; e0 += kU) {
+      float v[kU];
+#pragma unroll
+      for (int x = 0; x < kU; ++x) v[x] = lds_f32(sA + min(e0 + x, m - 1) * kSs);
+#pragma unroll
+      for (int x = 0; x < kU; ++x) {
+        const int bin = bin_of(fine_of(v[x]), order_key(v[x]));
+        if (e0 + x < m && bin >= 0) red_add_shared(hA + bin * kHs, one);
+      }
+    }
+  };
+
+  // keep rule: f > fcut, or f == fcut and (key > kh, or key >= kl and among the first
+  // need_last such entries)
+  int fcut, need_last = 0;
+  uint32_t kl = 0u, kh = 0xffffffffu;
+  clear(63);
+  count([&](int f, uint32_t) { return f >> 6; });
+  int above, c;
+  const int bA = scan(63, k, &above, &c);
+  int need = k - above;
+  fcut = bA * 64 - 1;  // keep the whole coarse bin and above
+  if (c != need && above + c > keep_max) {
+    clear(63);
+    count([&](int f, uint32_t) { return (f >> 6) == bA ? (f & 63) : -1; });
+    const int kept_above = above;
+    const int bB = scan(63, need, &above, &c);
+    need -= above;
+    const int fs = bA * 64 + bB;
+    fcut = fs - 1;  // keep the whole fine cell and above
+    if (c != need && kept_above + above + c > keep_max) {
+      // key range of the fine cell's entries
+      kl = 0xffffffffu;
+      kh = 0u;
+      for (int e = 0; e < m; ++e) {
+        const float v = lds_f32(sA + e * kSs);
+        if (fine_of(v) == fs) {
+          kl = min(kl, order_key(v));
+          kh = max(kh, order_key(v));
+        }
+      }
+      int inplay = c;
+      while (inplay > need && kl < kh) {
+        const uint32_t span = kh - kl;
+        const int sh = span < (uint32_t)kStcBins ? 0 : 32 - __clz(span) - 6;  // span >> sh < 64
+        const int top = (int)(span >> sh);
+        const uint32_t l0 = kl, h0 = kh;
+        clear(top);
+        count([&](int f, uint32_t key) {
+          return (f == fs && key >= l0 && key <= h0) ? (int)((key - l0) >> sh) : -1;
+        });
+        const int b = scan(top, need, &above, &c);
+        need -= above;
+        inplay = c;
+        const uint32_t lo = kl + ((uint32_t)b << sh);
+        const uint32_t width = (1u << sh) - 1u;
+        kh = (kh - lo <= width) ? kh : lo + width;
+        kl = lo;
+      }
+      fcut = fs;
+      need_last = need;
+    }
+  }
+  // pack the kept entries in place; every store goes to an entry at or below the ones
+  // already loaded
+  int w = 0, taken = 0;
+  float mn = INFINITY;
+  for (int e0 = 0; e0 < m; e0 += kU) {
+    float v[kU];
+    uint32_t jv[kU];
+#pragma unroll
+    for (int x = 0; x < kU; ++x) {
+      const int e = min(e0 + x, m - 1);
+      v[x] = lds_f32(sA + e * kSs);
+      jv[x] = lds_u16(jA + e * kJs);
+    }
+#pragma unroll
+    for (int x = 0; x < kU; ++x) {
+      const int f = fine_of(v[x]);
+      const uint32_t key = order_key(v[x]);
+      bool keep = f > fcut;
+      if (!keep && f == fcut && e0 + x < m) {
+        if (key > kh) {
+          keep = true;
+        } else if (key >= kl && taken < need_last) {
+          keep = true;
+          ++taken;
+        }
+      }
+      if (keep && e0 + x < m) {
+        sts_f32(sA + w * kSs, v[x]);
+        sts_u16(jA + w * kJs, jv[x]);
+        ++w;
+        mn = fminf(mn, v[x]);
+      }
+    }
+  }
+  *thr = mn;
+  return w;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kStcThreads, 1)
+select_tc_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constant__ CUtensorMap tm_lo,
+                 const __nv_bfloat16* __restrict__ q, int32_t* __restrict__ idx, int T, int nb,
+                 int Hkv, int B, int G, sala_strides sq, int topk, int n_init, int n_local) {
+  using L = StcSmem<D>;
+  constexpr int kK = D / 16;     // k-steps
+  constexpr int kAcols = D / 2;  // TMEM columns of one A operand (bf16 pairs)
+  constexpr uint32_t kId = umma_idesc_bf16(128, kStcN, false, false);
+  constexpr uint32_t kCols = 4 * kAcols + kStcAcc * kStcN <= 256 ? 256 : 512;
+  static_assert(4 * kAcols + kStcAcc * kStcN <= 512, "TMEM columns");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBars);  // [S] tile landed
+  uint64_t* stage_free = full + kStcStages;                      // [S] tile's MMAs done
+  uint64_t* mma_done = stage_free + kStcStages;                  // [A] scores ready
+  uint64_t* acc_free = mma_done + kStcAcc;                       // [A] scores read
+  uint64_t* a_full = acc_free + kStcAcc;                         // [2] queries in TMEM
+  uint64_t* a_free = a_full + 2;                                 // [2] queries consumed
+  uint64_t* drain = a_free + 2;                                  // every MMA done (exit)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 1) + 1;
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int nq2 = (T + kStcRows - 1) / kStcRows;
+  const int hb = Hkv * B;
+  const int nitems = nq2 * hb;
+  const int nrounds = (nitems + (int)gridDim.x - 1) / (int)gridDim.x;
+  const int n_sel = n_init + topk + n_local;
+  // item of round r for this CTA (snake order over the long-rows-first item list)
+  auto item_of = [&](int r) {
+    return r * (int)gridDim.x + ((r & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x);
+  };
+  struct Item {
+    int t0, hk, b, ntiles;
+  };
+  auto info = [&](int k) {
+    Item it;
+    const int x = k / hb, rem = k % hb;
+    it.t0 = (nq2 - 1 - x) * kStcRows;
+    it.hk = rem % Hkv;
+    it.b = rem / Hkv;
+    const int t_last = min(it.t0 + kStcRows - 1, T - 1);
+    const int jhi = min(t_last / kSelBlk - n_local, nb - 1);  // last candidate of the item
+    const int n_item = jhi >= n_init ? jhi - n_init + 1 : 0;
+    it.ntiles = n_item > topk ? (n_item + kStcN - 1) / kStcN : 0;  // 0: nothing to score
+    return it;
+  };
+
+  if (tid == 0) {
+    for (int i = 0; i < kStcStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&stage_free[i], 1);
+    }
+    for (int i = 0; i < kStcAcc; ++i) {
+      mbar_init(&mma_done[i], 1);
+      mbar_init(&acc_free[i], kStcRows / 32);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&a_full[i], kStcRows);
+      mbar_init(&a_free[i], 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) tc_alloc(tmem_slot, kCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tD = tmem + 4 * kAcols;  // [kStcAcc] x 32 columns of scores
+
+  if (warp >= 4 && warp < 8) {
+    // ================= producers: group-summed queries of the CTA's scoring items
+    const int p = tid - kStcRows;
+    const uint32_t lane_off = (uint32_t)(32 * (warp - 4)) << 16;
+    int u = 0;
+    for (int r = 0; r < nrounds; ++r) {
+      const int k = item_of(r);
+      if (k >= nitems) continue;
+      const Item it = info(k);
+      if (it.ntiles == 0) continue;
+      const int buf = u & 1;
+      if (*abort_flag || (u >= 2 && !mbar_wait(&a_free[buf], ((u - 2) >> 1) & 1))) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tA = tmem + buf * 2 * kAcols;
+      const int t = it.t0 + p;
+      const bool in = t < T;
+      const __nv_bfloat16* qp = q + it.b * sq.b + (int64_t)(in ? t : 0) * sq.t +
+                                (int64_t)it.hk * G * sq.h;
+#pragma unroll 1
+      for (int half = 0; half < D / 64; ++half) {
+        float acc[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+        const __nv_bfloat16* base = qp + half * 64;
+#pragma unroll 2
+        for (int h = 0; h < G; ++h) {
+          uint4 w[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            w[c] = __ldg(reinterpret_cast<const uint4*>(base + (int64_t)h * sq.h + 8 * c));
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t ww[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              acc[8 * c + 2 * i] += __uint_as_float(ww[i] << 16);
+              acc[8 * c + 2 * i + 1] += __uint_as_float(ww[i] & 0xffff0000u);
+            }
+          }
+        }
+        uint32_t hw[32], lw[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float x0 = in ? acc[2 * i] : 0.f, x1 = in ? acc[2 * i + 1] : 0.f;
+          const float h0 = __bfloat162float(__float2bfloat16_rn(x0));
+          const float h1 = __bfloat162float(__float2bfloat16_rn(x1));
+          hw[i] = pack_bf16x2(h0, h1);
+          lw[i] = pack_bf16x2(x0 - h0, x1 - h1);
+        }
+        tc_st32(tA + lane_off + 32 * half, hw);
+        tc_st32(tA + kAcols + lane_off + 32 * half, lw);
+      }
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(&a_full[buf]);
+      ++u;
+    }
+  } else if (warp == 8) {
+    // ================= issuer: block-mean tiles by TMA, score MMAs
+    if ((tid & 31) == 0) {
+      prefetch_tmap(&tm_hi);
+      prefetch_tmap(&tm_lo);
+      int g = 0, u = 0, n_issued = 0;
+      bool ok = true;
+      // tile i of `it` as global tile gg, into stage gg % S once that stage's previous
+      // tile has been scored
+      auto issue_tma = [&](const Item& it, int i, int gg) {
+        const int st = gg % kStcStages;
+        if (gg >= kStcStages && !mbar_wait(&stage_free[st], ((gg / kStcStages) + 1) & 1))
+          return false;
+        uint8_t* dst = smem + L::kB + st * L::kStage;
+        const int j0 = n_init + i * kStcN;
+        mbar_arrive_expect_tx(&full[st], L::kStage);
+#pragma unroll
+        for (int hf = 0; hf < D / 64; ++hf) {
+          tma_load_4d(dst + hf * L::kHalfB, &tm_hi, &full[st], hf * 64, it.hk, j0, it.b);
+          tma_load_4d(dst + L::kTileB + hf * L::kHalfB, &tm_lo, &full[st], hf * 64, it.hk, j0,
+                      it.b);
+        }
+        n_issued = gg + 1;
+        return true;
+      };
+      auto desc_b = [&](uint32_t base, int kk) {
+        return umma_desc_sw128(base + (kk >> 2) * L::kHalfB + (kk & 3) * 32, 16, 1024);
+      };
+      for (int r = 0; r < nrounds && ok; ++r) {
+        const int k = item_of(r);
+        if (k >= nitems) continue;
+        const Item it = info(k);
+        if (it.ntiles == 0) continue;
+        const int buf = u & 1;
+        const uint32_t tA = tmem + buf * 2 * kAcols;
+        ok = !*abort_flag && issue_tma(it, 0, g) && (it.ntiles < 2 || issue_tma(it, 1, g + 1)) &&
+             mbar_wait(&a_full[buf], (u >> 1) & 1);
+        tc_fence_after();
+        for (int i = 0; i < it.ntiles && ok; ++i) {
+          const int gg = g + i, st = gg % kStcStages, ab = gg % kStcAcc;
+          ok = mbar_wait(&full[st], (gg / kStcStages) & 1) &&
+               (gg < kStcAcc || mbar_wait(&acc_free[ab], ((gg / kStcAcc) + 1) & 1));
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t bh = smem_u32(smem + L::kB + st * L::kStage), bl = bh + L::kTileB;
+          const uint32_t d = tD + kStcN * ab;
+#pragma unroll
+          for (int kk = 0; kk < kK; ++kk)
+            tc_mma_ts(d, tA + kAcols + 8 * kk, desc_b(bh, kk), kId, kk > 0 ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < kK; ++kk) tc_mma_ts(d, tA + 8 * kk, desc_b(bl, kk), kId, 1u);
+#pragma unroll
+          for (int kk = 0; kk < kK; ++kk) tc_mma_ts(d, tA + 8 * kk, desc_b(bh, kk), kId, 1u);
+          tc_commit(&mma_done[ab]);
+          tc_commit(&stage_free[st]);
+          if (i + 2 < it.ntiles) ok = issue_tma(it, i + 2, gg + 2);
+        }
+        if (!ok) break;
+        tc_commit(&a_free[buf]);  // the item's queries are free once its MMAs complete
+        g += it.ntiles;
+        ++u;
+      }
+      if (!ok) *abort_flag = 1;
+      // wind down: every MMA complete and every copy landed before resources are released
+      tc_commit(drain);
+      mbar_wait(drain, 0);
+      for (int x = n_issued > kStcStages ? n_issued - kStcStages : 0; x < n_issued; ++x)
+        mbar_wait(&full[x % kStcStages], (x / kStcStages) & 1);
+    }
+  } else if (warp < 4) {
+    // ================= consumers: scores, per-row buffers, output
+    const int row = tid;
+    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+    const uint32_t sA = smem_u32(smem + L::kBufS) + row * 4;  // entry e at + e * 512
+    const uint32_t jA = smem_u32(smem + L::kBufJ) + row * 2;  // entry e at + e * 256
+    const uint32_t hA = smem_u32(smem + L::kHist) + (row & 63) * 4;  // bin b at + b * 256
+    const int sh16 = (row >> 6) * 16;
+    int g = 0;  // tiles consumed so far: score buffer g % kStcAcc
+    for (int r = 0; r < nrounds; ++r) {
+      const int k = item_of(r);
+      if (k >= nitems) continue;
+      const Item it = info(k);
+      const int t = it.t0 + row;
+      const bool live = t < T;
+      const int c = t / kSelBlk;
+      const int jmax = min(c - n_local, nb - 1);  // last candidate of this row
+      const int n_row = jmax >= n_init ? jmax - n_init + 1 : 0;
+      const bool buffered = live && n_row > topk;
+      int cnt = 0;
+      float thr = -INFINITY, smin = INFINITY, smax = -INFINITY;
+      bool dead = false;
+      for (int i = 0; i < it.ntiles; ++i) {
+        const int gg = g + i, ab = gg % kStcAcc;
+        const bool landed = !*abort_flag && mbar_wait(&mma_done[ab], (gg / kStcAcc) & 1);
+        if (__any_sync(0xffffffffu, !landed)) {
+          dead = true;
+          break;
+        }
+        tc_fence_after();
+        uint32_t sv[kStcN];
+        tc_ld32(tD + kStcN * ab + lane_off, sv);
+        tc_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if ((tid & 31) == 0) mbar_arrive(&acc_free[ab]);  // this warp is done with it
+        if (buffered) {
+          // scores compared as raw dot products: the 1/sqrt(D) factor preserves the order
+          const int j0 = n_init + i * kStcN;
+          auto append = [&](int cc, bool in_range) {
+            const float sc = __uint_as_float(sv[cc]);
+            if (in_range && sc > thr) {
+              sts_f32(sA + cnt * (kStcRows * 4), sc);
+              sts_u16(jA + cnt * (kStcRows * 2), (uint32_t)(j0 + cc));
+              ++cnt;
+              smin = fminf(smin, sc);
+              smax = fmaxf(smax, sc);
+            }
+          };
+          if (j0 + kStcN - 1 <= jmax) {
+#pragma unroll
+            for (int cc = 0; cc < kStcN; ++cc) append(cc, true);
+          } else {
+#pragma unroll
+            for (int cc = 0; cc < kStcN; ++cc) append(cc, j0 + cc <= jmax);
+          }
+        }
+        if (__any_sync(0xffffffffu, cnt > kStcCap - kStcN) && cnt > topk) {
+          // a cut that keeps at most kStcCoarse entries (all of the topk best)
+          cnt = stc_compact(sA, jA, hA, sh16, cnt, topk, smin, smax, max(kStcCoarse, topk), &thr);
+          smin = thr;
+        }
+      }
+      if (dead) {
+        *abort_flag = 1;
+        break;
+      }
+      g += it.ntiles;
+      if (buffered && cnt > topk)
+        cnt = stc_compact(sA, jA, hA, sh16, cnt, topk, smin, smax, topk, &thr);  // exact
+      // ---- this thread's row: init blocks, the kept candidates in block order, local window
+      if (live) {
+        int32_t* out = idx + (((int64_t)it.b * Hkv + it.hk) * T + t) * n_sel;
+        const int n_first = min(n_init, c + 1);
+        for (int e = 0; e < n_first; ++e) out[e] = e;
+        int pos = n_first;
+        if (!buffered) {
+          for (int e = 0; e < n_row; ++e) out[pos + e] = n_init + e;
+          pos += n_row;
+        } else {
+          for (int e = 0; e < cnt; ++e) out[pos + e] = (int)lds_u16(jA + e * (kStcRows * 2));
+          pos += cnt;
+        }
+        const int lo = max(n_init, c - n_local + 1);
+        for (int j = lo; j <= c; ++j) out[pos++] = j;
+        for (int e = pos; e < n_sel; ++e) out[e] = -1;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tc_dealloc(tmem, kCols);
+  }
+}
+
+}  // namespace sala
