@@ -79,6 +79,19 @@ __device__ __forceinline__ void sts_f32(uint32_t a, float v) {
 __device__ __forceinline__ void sts_u16(uint32_t a, uint32_t v) {
   asm volatile("st.shared.u16 [%0], %1;" ::"r"(a), "h"((unsigned short)v) : "memory");
 }
+// Stores that happen only where `p` holds (a predicated instruction, no branch).
+__device__ __forceinline__ void sts_f32_if(bool p, uint32_t a, float v) {
+  asm volatile(
+      "{\n .reg .pred q;\n setp.ne.b32 q, %2, 0;\n @q st.shared.f32 [%0], %1;\n}\n" ::"r"(a),
+      "f"(v), "r"((uint32_t)p)
+      : "memory");
+}
+__device__ __forceinline__ void sts_u16_if(bool p, uint32_t a, uint32_t v) {
+  asm volatile(
+      "{\n .reg .pred q;\n setp.ne.b32 q, %2, 0;\n @q st.shared.u16 [%0], %1;\n}\n" ::"r"(a),
+      "h"((unsigned short)v), "r"((uint32_t)p)
+      : "memory");
+}
 __device__ __forceinline__ void red_add_shared(uint32_t a, uint32_t v) {
   asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }

@@ -62,152 +62,156 @@ struct StcSmem {
 
 // Compact one row's m > k buffered entries (shared addresses: sA / jA the scores (f32)
 // and block indices (u16), entry e at + e * kStcRows * size; hA the row's 64 histogram
-// bins, bin b in the 16 bits at `sh16` of the word at hA + b * 256), in buffer order.
-// smin / smax: the smallest and largest buffered score.  Every entry among the k best
-// (larger score first, ties -> smaller block index) is kept; with keep_max == k exactly
-// those are kept, with keep_max > k a coarser cut that keeps at most keep_max entries
-// may be taken instead.  Returns the kept count and sets *thr to the smallest kept score.
+// bins for the rare key refinement, bin b in the 16 bits at `sh16` of the word at
+// hA + b * 256), in buffer order.  smin / smax: the smallest and largest buffered score.
+// Every entry among the k best (larger score first, ties -> smaller block index) is
+// kept; with keep_max == k exactly those are kept, with keep_max > k a coarser cut that
+// keeps at most keep_max entries may be taken instead.  Returns the kept count and sets
+// *thr to the smallest kept score.
 //
-// Each score gets a fine index f in [0, 4096) linear in (s - smin), monotone in s.  Pass
-// A counts f / 64 (64 coarse bins) and finds the bin holding the k-th best; pass B counts
-// f % 64 inside it; if the fine cell holding the boundary still has more entries than
-// needed, their order-preserving integer keys are bucketed (64 bins of the key range,
-// refined until the boundary is resolved or only equal scores remain, where the earliest
-// = smallest block index win).
+// Each score gets a fine index f in [0, 65536) linear in (s - smin), monotone in s.  Up
+// to four counting passes of 16 bins (f's bits 15-12, then 11-8 inside the boundary bin,
+// and so on), each histogram held in two 64-bit registers of 8-bit counters, locate the
+// cell holding the k-th best, stopping as soon as the cut is resolved (or, for a coarse
+// cut, small enough).  If the final cell still holds more entries than needed, their
+// order-preserving integer keys are bucketed (64 bins in shared memory, refined until
+// the boundary is resolved or only equal scores remain, where the earliest = smallest
+// block index win).
 __device__ __noinline__ int stc_compact(uint32_t sA, uint32_t jA, uint32_t hA, int sh16, int m,
                                         int k, float smin, float smax, int keep_max, float* thr) {
   constexpr uint32_t kSs = kStcRows * 4, kJs = kStcRows * 2, kHs = 64 * 4;  // strides
   constexpr int kU = 8;  // loads in flight per pass
-  const uint32_t other = sh16 ? 0x0000ffffu : 0xffff0000u;
-  const uint32_t one = 1u << sh16;
   const float range = smax - smin;
-  const float scale = 4096.0f / range;
+  const float scale = 65536.0f / range;
   const bool linear = range > 0.f && scale <= 3.0e38f;
-  auto fine_of = [&](float s) { return linear ? min(4095, (int)((s - smin) * scale)) : 0; };
-  auto clear = [&](int top) {
-    for (int b = 0; b <= top; ++b) red_and_shared(hA + b * kHs, other);
-  };
-  // bin holding the need-th best counting down from `top`; *above: entries in higher bins
-  auto scan = [&](int top, int need, int* above, int* cnt) {
-    int b = -1, ab = 0, cb_at = 0;
-    for (int b0 = top; b0 >= 0 && b < 0; b0 -= kU) {
-      uint32_t hw[kU];
-#pragma unroll
-      for (int x = 0; x < kU; ++x) hw[x] = lds_u32(hA + max(b0 - x, 0) * kHs);
-#pragma unroll
-      for (int x = 0; x < kU; ++x) {
-        const int bb = b0 - x;
-        const int cb = (int)((hw[x] >> sh16) & 0xffffu);
-        if (b < 0 && bb >= 0) {
-          if (ab + cb >= need || bb == 0) {
-            b = bb;
-            cb_at = cb;
-          } else {
-            ab += cb;
-          }
-        }
-      }
-    }
-    *above = ab;
-    *cnt = cb_at;
-    return b;
-  };
-  // one pass over the entries: bin_of(f, key) < 0 skips the entry
-  auto count = [&](auto bin_of) {
+  auto fine_of = [&](float s) { return linear ? min(65535, (int)((s - smin) * scale)) : 0; };
+
+  // ---- fine-index levels: bin = (f >> sh) & 15 among entries with f >> (sh + 4) == prefix
+  int need = k, kept = 0, prefix = 0, cut_sh = 0, c = m;
+  bool done = false;
+#pragma unroll 1
+  for (int sh = 12; sh >= 0; sh -= 4) {
+    uint32_t h[4] = {0u, 0u, 0u, 0u};  // bin b in byte b % 4 of h[b / 4] (m <= 255)
     for (int e0 = 0; e0 < m; e0 += kU) {
       float v[kU];
 #pragma unroll
       for (int x = 0; x < kU; ++x) v[x] = lds_f32(sA + min(e0 + x, m - 1) * kSs);
 #pragma unroll
       for (int x = 0; x < kU; ++x) {
-        const int bin = bin_of(fine_of(v[x]), order_key(v[x]));
-        if (e0 + x < m && bin >= 0) red_add_shared(hA + bin * kHs, one);
+        const int f = fine_of(v[x]);
+        const int bin = (f >> sh) & 15;
+        const bool in = (e0 + x < m) & ((f >> (sh + 4)) == prefix);
+        const uint32_t inc = (uint32_t)in << ((bin & 3) * 8);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) h[i] += (bin >> 2) == i ? inc : 0u;
       }
     }
-  };
-
-  // keep rule: f > fcut, or f == fcut and (key > kh, or key >= kl and among the first
-  // need_last such entries)
-  int fcut, need_last = 0;
-  uint32_t kl = 0u, kh = 0xffffffffu;
-  clear(63);
-  count([&](int f, uint32_t) { return f >> 6; });
-  int above, c;
-  const int bA = scan(63, k, &above, &c);
-  int need = k - above;
-  fcut = bA * 64 - 1;  // keep the whole coarse bin and above
-  if (c != need && above + c > keep_max) {
-    clear(63);
-    count([&](int f, uint32_t) { return (f >> 6) == bA ? (f & 63) : -1; });
-    const int kept_above = above;
-    const int bB = scan(63, need, &above, &c);
+    // bin holding the need-th best, from the top (selects, no branches)
+    int above = 0, b = 0, cb_at = 0;
+    bool found = false;
+#pragma unroll
+    for (int bb = 15; bb >= 0; --bb) {
+      const int cb = (int)((h[bb >> 2] >> ((bb & 3) * 8)) & 0xffu);
+      const bool take = !found & ((above + cb >= need) | (bb == 0));
+      b = take ? bb : b;
+      cb_at = take ? cb : cb_at;
+      above += (!found & !take) ? cb : 0;
+      found = found | take;
+    }
     need -= above;
-    const int fs = bA * 64 + bB;
-    fcut = fs - 1;  // keep the whole fine cell and above
-    if (c != need && kept_above + above + c > keep_max) {
-      // key range of the fine cell's entries
-      kl = 0xffffffffu;
-      kh = 0u;
-      for (int e = 0; e < m; ++e) {
-        const float v = lds_f32(sA + e * kSs);
-        if (fine_of(v) == fs) {
-          kl = min(kl, order_key(v));
-          kh = max(kh, order_key(v));
-        }
-      }
-      int inplay = c;
-      while (inplay > need && kl < kh) {
-        const uint32_t span = kh - kl;
-        const int sh = span < (uint32_t)kStcBins ? 0 : 32 - __clz(span) - 6;  // span >> sh < 64
-        const int top = (int)(span >> sh);
-        const uint32_t l0 = kl, h0 = kh;
-        clear(top);
-        count([&](int f, uint32_t key) {
-          return (f == fs && key >= l0 && key <= h0) ? (int)((key - l0) >> sh) : -1;
-        });
-        const int b = scan(top, need, &above, &c);
-        need -= above;
-        inplay = c;
-        const uint32_t lo = kl + ((uint32_t)b << sh);
-        const uint32_t width = (1u << sh) - 1u;
-        kh = (kh - lo <= width) ? kh : lo + width;
-        kl = lo;
-      }
-      fcut = fs;
-      need_last = need;
+    kept += above;
+    c = cb_at;
+    prefix = prefix * 16 + b;
+    if (c == need || kept + c <= keep_max) {  // keep every cell from `prefix` up
+      cut_sh = sh;
+      done = true;
+      break;
     }
   }
-  // pack the kept entries in place; every store goes to an entry at or below the ones
-  // already loaded
-  int w = 0, taken = 0;
+  const int fcut = done ? prefix - 1 : prefix;  // keep (f >> cut_sh) > fcut (+ ties below)
+
+  int w = 0;
   float mn = INFINITY;
-  for (int e0 = 0; e0 < m; e0 += kU) {
-    float v[kU];
-    uint32_t jv[kU];
+  if (done) {
+    // ---- pack (common path): keep f >> cut_sh > fcut; every store goes to an entry at or
+    // below the ones already loaded
+    for (int e0 = 0; e0 < m; e0 += kU) {
+      float v[kU];
+      uint32_t jv[kU];
 #pragma unroll
-    for (int x = 0; x < kU; ++x) {
-      const int e = min(e0 + x, m - 1);
-      v[x] = lds_f32(sA + e * kSs);
-      jv[x] = lds_u16(jA + e * kJs);
+      for (int x = 0; x < kU; ++x) {
+        const int e = min(e0 + x, m - 1);
+        v[x] = lds_f32(sA + e * kSs);
+        jv[x] = lds_u16(jA + e * kJs);
+      }
+#pragma unroll
+      for (int x = 0; x < kU; ++x) {
+        const bool keep = (e0 + x < m) & ((fine_of(v[x]) >> cut_sh) > fcut);
+        sts_f32_if(keep, sA + w * kSs, v[x]);
+        sts_u16_if(keep, jA + w * kJs, jv[x]);
+        w += keep ? 1 : 0;
+        mn = keep ? fminf(mn, v[x]) : mn;
+      }
     }
-#pragma unroll
-    for (int x = 0; x < kU; ++x) {
-      const int f = fine_of(v[x]);
-      const uint32_t key = order_key(v[x]);
-      bool keep = f > fcut;
-      if (!keep && f == fcut && e0 + x < m) {
+  } else {
+    // ---- the final fine cell holds near-equal scores: bucket their keys
+    const uint32_t other = sh16 ? 0x0000ffffu : 0xffff0000u;
+    const uint32_t one = 1u << sh16;
+    const int fs = prefix;
+    uint32_t kl = 0xffffffffu, kh = 0u;
+    for (int e = 0; e < m; ++e) {
+      const float v = lds_f32(sA + e * kSs);
+      if (fine_of(v) == fs) {
+        kl = min(kl, order_key(v));
+        kh = max(kh, order_key(v));
+      }
+    }
+    int inplay = c;
+    while (inplay > need && kl < kh) {
+      const uint32_t span = kh - kl;
+      const int sh = span < (uint32_t)kStcBins ? 0 : 32 - __clz(span) - 6;  // span >> sh < 64
+      const int top = (int)(span >> sh);
+      for (int bb = 0; bb <= top; ++bb) red_and_shared(hA + bb * kHs, other);
+      for (int e = 0; e < m; ++e) {
+        const float v = lds_f32(sA + e * kSs);
+        const uint32_t key = order_key(v);
+        if (fine_of(v) == fs && key >= kl && key <= kh)
+          red_add_shared(hA + ((key - kl) >> sh) * kHs, one);
+      }
+      int above = 0, b = top;
+      for (; b > 0; --b) {
+        const int cb = (int)((lds_u32(hA + b * kHs) >> sh16) & 0xffffu);
+        if (above + cb >= need) break;
+        above += cb;
+      }
+      need -= above;
+      inplay = (int)((lds_u32(hA + b * kHs) >> sh16) & 0xffffu);
+      const uint32_t lo = kl + ((uint32_t)b << sh);
+      const uint32_t width = (1u << sh) - 1u;
+      kh = (kh - lo <= width) ? kh : lo + width;
+      kl = lo;
+    }
+    // keep f > fs; at f == fs keys above kh, then the first `need` keys in [kl, kh]
+    int taken = 0;
+    for (int e = 0; e < m; ++e) {
+      const float v = lds_f32(sA + e * kSs);
+      const uint32_t j = lds_u16(jA + e * kJs);
+      const int f = fine_of(v);
+      const uint32_t key = order_key(v);
+      bool keep = f > fs;
+      if (!keep && f == fs) {
         if (key > kh) {
           keep = true;
-        } else if (key >= kl && taken < need_last) {
+        } else if (key >= kl && taken < need) {
           keep = true;
           ++taken;
         }
       }
-      if (keep && e0 + x < m) {
-        sts_f32(sA + w * kSs, v[x]);
-        sts_u16(jA + w * kJs, jv[x]);
+      if (keep) {
+        sts_f32(sA + w * kSs, v);
+        sts_u16(jA + w * kJs, j);
         ++w;
-        mn = fminf(mn, v[x]);
+        mn = fminf(mn, v);
       }
     }
   }
@@ -457,15 +461,14 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constan
         if (buffered) {
           // scores compared as raw dot products: the 1/sqrt(D) factor preserves the order
           const int j0 = n_init + i * kStcN;
-          auto append = [&](int cc, bool in_range) {
+          auto append = [&](int cc, bool in_range) {  // predicated, no branch
             const float sc = __uint_as_float(sv[cc]);
-            if (in_range && sc > thr) {
-              sts_f32(sA + cnt * (kStcRows * 4), sc);
-              sts_u16(jA + cnt * (kStcRows * 2), (uint32_t)(j0 + cc));
-              ++cnt;
-              smin = fminf(smin, sc);
-              smax = fmaxf(smax, sc);
-            }
+            const bool p = in_range & (sc > thr);
+            sts_f32_if(p, sA + cnt * (kStcRows * 4), sc);
+            sts_u16_if(p, jA + cnt * (kStcRows * 2), (uint32_t)(j0 + cc));
+            cnt += p ? 1 : 0;
+            smin = p ? fminf(smin, sc) : smin;
+            smax = p ? fmaxf(smax, sc) : smax;
           };
           if (j0 + kStcN - 1 <= jmax) {
 #pragma unroll
