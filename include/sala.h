@@ -187,6 +187,53 @@ sala_status sala_sparse_attn(const void *q, const void *k, const void *v, const 
                              void *ws, size_t ws_bytes, sala_dtype dt, void *stream);
 
 /*
+ * Sparse-layer decode (InfLLM-v2 style, NoPE): one new query per sequence.
+ * For sequence b at position p = pos[b], whose cache already holds the new token's key
+ * and value at row p, the step computes row t = p of the prefill pair
+ * sala_sparse_select + sala_sparse_attn over cache rows 0..p:
+ *   c = p / block; candidates n_init <= j <= c - n_local scored against the block means
+ *   kbar (score_j = sum_{h in group(hk)} q_h . kbar_j), the top `topk` (ties -> smaller
+ *   j) plus the init blocks and the local window, sorted and -1 padded; then softmax
+ *   attention of every query head of the group over those blocks' keys s <= p, gated.
+ * Block means are a cache the caller keeps beside the KV cache: on entry kbar must hold
+ * the means of the complete blocks 0..c-1 (sala_sparse_block_means fills them for a
+ * prefilled cache); when p completes block c ((p + 1) % block == 0) the call writes
+ * kbar[b][c] (summed in key order, bit-identical to sala_sparse_block_means).
+ *
+ *   q, g, o     [B,Hq,D] bf16 (strides .b, .h; .t unused), g may be NULL
+ *   k_cache, v_cache  [B,Tmax,Hkv,D] bf16 (strides b, t, h); rows 0..pos[b] valid
+ *   kbar        [B, Tmax/block, Hkv, D] fp32 contiguous, in/out as above
+ *   pos         [B] int32 DEVICE array, 0 <= pos[b] < Tmax
+ *   idx_out     [B,Hkv,n_init+topk+n_local] int32 (the selection), or NULL
+ *   scale       softmax scale; 0 selects 1/sqrt(D)
+ *   ws          device scratch of >= sala_sparse_decode_workspace() bytes, 16-byte
+ *               aligned, caller-owned (scores, selection, split partials)
+ *   block = 64, Tmax a multiple of 64, D = 64 or 128, 1 <= Hq / Hkv <= 16.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.  Device: RANGE when a pos[b] lies
+ *   outside [0, Tmax) (that sequence is skipped) or a v value does not fit the fp16
+ *   tensor-core operand (|v| >= 65536).
+ */
+size_t sala_sparse_decode_workspace(int B, int Tmax, int Hq, int Hkv, int D, int n_sel);
+
+sala_status sala_sparse_decode(const void *q, const void *k_cache, const void *v_cache,
+                               const void *g, float *kbar, const int32_t *pos, void *o,
+                               int32_t *idx_out, int B, int Tmax, int Hq, int Hkv, int D,
+                               sala_strides sq, sala_strides sk, sala_strides sv, sala_strides sg,
+                               sala_strides so, int block, int topk, int n_init, int n_local,
+                               float scale, void *ws, size_t ws_bytes, sala_dtype dt,
+                               void *stream);
+
+/*
+ * Block means of the complete blocks of a filled cache, the kbar operand of
+ * sala_sparse_decode: kbar[b][j][hk][:] = mean of keys j*64 .. j*64+63 for j < T / 64.
+ *   k       [B,T,Hkv,D] bf16 (strides b, t, h)
+ *   kbar    [B, kbar_blocks, Hkv, D] fp32 contiguous, kbar_blocks >= T / 64
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA.
+ */
+sala_status sala_sparse_block_means(const void *k, int B, int T, int Hkv, int D, sala_strides sk,
+                                    float *kbar, int kbar_blocks, sala_dtype dt, void *stream);
+
+/*
  * Lightning prefill that allocates nothing (no counterpart in the paper: this is
  * a library convenience).  Some callers cannot hand the library a workspace:
  * code embedded in a host framework that owns all device memory and offers its

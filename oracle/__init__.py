@@ -210,3 +210,30 @@ def attention(q, k, v, g=None, idx=None, *, blk=64, scale=None, rows=None):
     lib.oracle_attention(qp, kp, vp, gp, ip, n_sel, B, T, Hq, Hkv, D, blk, sc, rp, nrows,
                          y.ctypes.data_as(_dp))
     return y
+
+
+def sparse_decode(q, k_cache, v_cache, pos, g=None, *, blk=64, topk=64, n_init=1, n_local=2,
+                  scale=None):
+    """Sparse-layer decode step: for each sequence b, row p = pos[b] of the prefill
+    computation (sparse_select then attention) over cache rows 0..p only.
+    q, g: [B, Hq, D]; k_cache, v_cache: [B, Tmax, Hkv, D]; pos: [B] ints.
+    Returns (y [B, Hq, D], idx [B, Hkv, n_sel] int32, gap [B, Hkv])."""
+    q = np.asarray(q, dtype=np.float64)
+    B, Hq, D = q.shape
+    Hkv = np.shape(k_cache)[2]
+    n_sel = n_init + topk + n_local
+    y = np.zeros((B, Hq, D))
+    idx = np.zeros((B, Hkv, n_sel), dtype=np.int32)
+    gap = np.zeros((B, Hkv))
+    for b in range(B):
+        p = int(pos[b])
+        kk = np.asarray(k_cache[b:b + 1, :p + 1], dtype=np.float64)
+        vv = np.asarray(v_cache[b:b + 1, :p + 1], dtype=np.float64)
+        qr = q[b][None, None]
+        gr = None if g is None else np.asarray(g[b], dtype=np.float64)[None, None]
+        ib, gb = sparse_select(qr, kk, blk=blk, topk=topk, n_init=n_init, n_local=n_local,
+                               rows=[p], T=p + 1)
+        y[b] = attention(qr, kk, vv, gr, idx=ib, blk=blk, scale=scale, rows=[p])[0, 0]
+        idx[b] = ib[0, :, 0]
+        gap[b] = gb[0, :, 0]
+    return y, idx, gap

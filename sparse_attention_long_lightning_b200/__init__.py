@@ -20,7 +20,8 @@ __all__ = [
     "lightning_prefill_noalloc",
     "lightning_decode", "sparse_select", "sparse_select_workspace", "sparse_attn",
     "sparse_attn_workspace",
-    "get_device_error", "selftest_wait_timeout", "status_string", "version", "LIB_PATH",
+    "get_device_error", "selftest_wait_timeout", "sparse_decode", "sparse_decode_workspace",
+    "sparse_block_means", "status_string", "version", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsala.so")
@@ -69,6 +70,13 @@ def load_library(path: Optional[str] = None):
     lib.sala_sparse_select_workspace.restype = sz
     lib.sala_sparse_select.argtypes = [vp, vp, i, i, i, i, i, S, S, i, i, i, i, vp, vp, sz, i, vp]
     lib.sala_sparse_select.restype = i
+    lib.sala_sparse_decode_workspace.argtypes = [i, i, i, i, i, i]
+    lib.sala_sparse_decode_workspace.restype = sz
+    lib.sala_sparse_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, S, S, S, S, S,
+                                       i, i, i, i, f, vp, sz, i, vp]
+    lib.sala_sparse_decode.restype = i
+    lib.sala_sparse_block_means.argtypes = [vp, i, i, i, i, S, vp, i, i, vp]
+    lib.sala_sparse_block_means.restype = i
     lib.sala_sparse_attn_workspace.argtypes = [i, i, i, i]
     lib.sala_sparse_attn_workspace.restype = sz
     lib.sala_sparse_attn.argtypes = [vp, vp, vp, vp, vp, i, vp, i, i, i, i, i, S, S, S, S, S, i, f,
@@ -257,6 +265,57 @@ def sparse_attn(q, k, v, idx, g=None, *, block=64, scale=0.0, out=None, workspac
                               float(scale), _p(workspace), wsb, _dt(q), _stream(stream))
     _check("sala_sparse_attn", st)
     return out
+
+
+def sparse_decode_workspace(B, Tmax, Hq, Hkv, D, n_sel) -> int:
+    return int(load_library().sala_sparse_decode_workspace(B, Tmax, Hq, Hkv, D, n_sel))
+
+
+def sparse_decode(q, k_cache, v_cache, kbar, pos, g=None, *, topk=64, n_init=1, n_local=2,
+                  block=64, scale=0.0, out=None, idx_out=None, workspace=None, stream=None):
+    """One sparse-layer decode step.  q,g [B,Hq,D]; k_cache,v_cache [B,Tmax,Hkv,D] with the
+    new token already at row pos[b]; kbar [B,Tmax/64,Hkv,D] fp32 block-mean cache (updated
+    when the token completes a block); pos [B] int32 CUDA.  Returns out [B,Hq,D]."""
+    lib = load_library()
+    _cuda(q, k_cache, v_cache, kbar, pos, g, out, idx_out, workspace)
+    B, Hq, D = q.shape
+    Tmax, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if pos.dtype != torch.int32:
+        raise TypeError("pos must be int32")
+    if kbar.dtype != torch.float32 or not kbar.is_contiguous():
+        raise ValueError("kbar must be a contiguous float32 tensor")
+    n_sel = n_init + topk + n_local
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=q.dtype, device=q.device)
+    if idx_out is not None and (idx_out.dtype != torch.int32 or not idx_out.is_contiguous()):
+        raise ValueError("idx_out must be a contiguous int32 tensor")
+    need = sparse_decode_workspace(B, Tmax, Hq, Hkv, D, n_sel)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib.sala_sparse_decode(
+        _p(q), _p(k_cache), _p(v_cache), _p(g), _p(kbar), _p(pos), _p(out), _p(idx_out), B, Tmax,
+        Hq, Hkv, D, _s3(q), _s4(k_cache), _s4(v_cache), _s3(g), _s3(out), int(block), int(topk),
+        int(n_init), int(n_local), float(scale), _p(workspace), wsb, _dt(q), _stream(stream))
+    _check("sala_sparse_decode", st)
+    return out
+
+
+def sparse_block_means(k, kbar=None, *, kbar_blocks=None, stream=None):
+    """Block means of the complete blocks of k [B,T,Hkv,D] into kbar [B,kbar_blocks,Hkv,D]
+    fp32 (allocated with kbar_blocks = T // 64 when not given)."""
+    lib = load_library()
+    _cuda(k, kbar)
+    B, T, Hkv, D = k.shape
+    if kbar is None:
+        nb = T // 64 if kbar_blocks is None else int(kbar_blocks)
+        kbar = torch.zeros((B, nb, Hkv, D), dtype=torch.float32, device=k.device)
+    if kbar.dtype != torch.float32 or not kbar.is_contiguous():
+        raise ValueError("kbar must be a contiguous float32 tensor")
+    st = lib.sala_sparse_block_means(_p(k), B, T, Hkv, D, _s4(k), _p(kbar), int(kbar.shape[1]),
+                                     _dt(k), _stream(stream))
+    _check("sala_sparse_block_means", st)
+    return kbar
 
 
 def selftest_wait_timeout(cycles=20_000_000, stream=None):

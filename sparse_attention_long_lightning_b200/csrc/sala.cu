@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -18,6 +19,7 @@
 #include "lightning_tc.cuh"
 #include "lightning_out.cuh"
 #include "sparse_attn.cuh"
+#include "sparse_decode.cuh"
 #include "sparse_select.cuh"
 #include "sparse_select_tc.cuh"
 
@@ -415,6 +417,122 @@ sala_status sala_sparse_attn(const void* q, const void* k, const void* v, const 
     if (!set_smem(kern, SaSmem<64, NS>::bytes)) return SALA_ERR_CUDA;
     kern<<<grid, kSaThreads, SaSmem<64, NS>::bytes, st>>>(tk, tv, p);
   }
+  SALA_CHECK_LAUNCH();
+  return SALA_OK;
+}
+
+// ------------------------------------------------------------------ sparse-layer decode
+namespace {
+struct SdLayout {
+  size_t scores_off, idx_off, part_off, total;
+};
+SdLayout sd_layout(int B, int Tmax, int Hkv, int D, int n_sel) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  const size_t nbcap = (size_t)(Tmax / kSdBlk);
+  SdLayout L{};
+  L.scores_off = 0;
+  L.idx_off = up((size_t)B * Hkv * nbcap * 4);
+  L.part_off = L.idx_off + up((size_t)B * Hkv * n_sel * 4);
+  L.total = L.part_off + up((size_t)B * Hkv * kSdMaxSplit * 16 * (D + 2) * 4);
+  return L;
+}
+}  // namespace
+
+size_t sala_sparse_decode_workspace(int B, int Tmax, int Hq, int Hkv, int D, int n_sel) {
+  (void)Hq;
+  if (B <= 0 || Tmax < kSdBlk || Tmax % kSdBlk != 0 || Hkv <= 0 || n_sel <= 0 ||
+      (D != 64 && D != 128))
+    return 0;
+  return sd_layout(B, Tmax, Hkv, D, n_sel).total;
+}
+
+sala_status sala_sparse_decode(const void* q, const void* k_cache, const void* v_cache,
+                               const void* g, float* kbar, const int32_t* pos, void* o,
+                               int32_t* idx_out, int B, int Tmax, int Hq, int Hkv, int D,
+                               sala_strides sq, sala_strides sk, sala_strides sv, sala_strides sg,
+                               sala_strides so, int block, int topk, int n_init, int n_local,
+                               float scale, void* ws, size_t ws_bytes, sala_dtype dt,
+                               void* stream) {
+  if (!q || !k_cache || !v_cache || !kbar || !pos || !o) return SALA_ERR_INVALID_ARG;
+  if (B <= 0 || Tmax < kSdBlk || Tmax % kSdBlk != 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 ||
+      topk < 1 || n_init < 0 || n_local < 1 || !(scale >= 0.0f))
+    return SALA_ERR_INVALID_ARG;
+  if (dt != SALA_BF16) return SALA_ERR_UNSUPPORTED;
+  if (block != kSdBlk || (D != 64 && D != 128) || Hq / Hkv > 16) return SALA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+      !aligned16(kbar) || (g && !aligned16(g)) ||
+      (idx_out && (reinterpret_cast<uintptr_t>(idx_out) & 3u)))
+    return SALA_ERR_INVALID_ARG;
+  if (!strides_ok(sq, 2) || !strides_ok(sk, 2) || !strides_ok(sv, 2) || !strides_ok(so, 2) ||
+      (g && !strides_ok(sg, 2)))
+    return SALA_ERR_INVALID_ARG;
+  const int n_sel = n_init + topk + n_local;
+  const SdLayout L = sd_layout(B, Tmax, Hkv, D, n_sel);
+  if (!ws || !aligned16(ws) || ws_bytes < L.total) return SALA_ERR_WORKSPACE;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  SdParams p;
+  p.q = (const __nv_bfloat16*)q;
+  p.g = (const __nv_bfloat16*)g;
+  p.o = (__nv_bfloat16*)o;
+  p.k = (const __nv_bfloat16*)k_cache;
+  p.v = (const __nv_bfloat16*)v_cache;
+  p.kbar = kbar;
+  p.pos = pos;
+  p.idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(wsb + L.idx_off);
+  p.scores = reinterpret_cast<float*>(wsb + L.scores_off);
+  p.part = reinterpret_cast<float*>(wsb + L.part_off);
+  p.sq = sq; p.sg = sg; p.so = so; p.sk = sk; p.sv = sv;
+  p.B = B; p.Tmax = Tmax; p.Hq = Hq; p.Hkv = Hkv; p.G = Hq / Hkv; p.D = D;
+  p.nbcap = Tmax / kSdBlk;
+  p.n_init = n_init; p.topk = topk; p.n_local = n_local; p.n_sel = n_sel;
+  const int rows = B * Hkv;
+  p.nsplit = std::max(1, std::min({(2 * num_sms() + rows - 1) / rows, kSdMaxSplit, n_sel}));
+  const float sc = scale > 0.0f ? scale : 1.0f / std::sqrt((float)D);
+  p.scale_log2 = sc * 1.4426950408889634f;
+  cudaStream_t st = as_stream(stream);
+  const dim3 gs((p.nbcap + kSdScoreChunk - 1) / kSdScoreChunk, Hkv, B);
+  const dim3 ga(p.nsplit, Hkv, B);
+  if (D == 128) {
+    sd_score_kernel<128><<<gs, 256, 0, st>>>(p);
+  } else {
+    sd_score_kernel<64><<<gs, 256, 0, st>>>(p);
+  }
+  SALA_CHECK_LAUNCH();
+  sd_topk_kernel<<<dim3(Hkv, B), kSdTopkThreads, 0, st>>>(p);
+  SALA_CHECK_LAUNCH();
+  if (D == 128) {
+    auto kern = sd_attn_kernel<128>;
+    if (!set_smem(kern, SdAttnSmem<128>::bytes)) return SALA_ERR_CUDA;
+    kern<<<ga, kSdAttnWarps * 32, SdAttnSmem<128>::bytes, st>>>(p);
+    SALA_CHECK_LAUNCH();
+    sd_combine_kernel<128><<<dim3(Hq, B), 128, 0, st>>>(p);
+  } else {
+    auto kern = sd_attn_kernel<64>;
+    if (!set_smem(kern, SdAttnSmem<64>::bytes)) return SALA_ERR_CUDA;
+    kern<<<ga, kSdAttnWarps * 32, SdAttnSmem<64>::bytes, st>>>(p);
+    SALA_CHECK_LAUNCH();
+    sd_combine_kernel<64><<<dim3(Hq, B), 64, 0, st>>>(p);
+  }
+  SALA_CHECK_LAUNCH();
+  return SALA_OK;
+}
+
+sala_status sala_sparse_block_means(const void* k, int B, int T, int Hkv, int D, sala_strides sk,
+                                    float* kbar, int kbar_blocks, sala_dtype dt, void* stream) {
+  if (T > 0 && (!k || !kbar)) return SALA_ERR_INVALID_ARG;
+  if (B <= 0 || T < 0 || Hkv <= 0 || kbar_blocks < T / kSdBlk) return SALA_ERR_INVALID_ARG;
+  if (dt != SALA_BF16) return SALA_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128) return SALA_ERR_UNSUPPORTED;
+  if (T / kSdBlk == 0) return SALA_OK;
+  if (!aligned16(k) || !aligned16(kbar) || !strides_ok(sk, 2)) return SALA_ERR_INVALID_ARG;
+  const dim3 grid(T / kSdBlk, Hkv, B);
+  cudaStream_t st = as_stream(stream);
+  if (D == 128)
+    sd_block_means_kernel<128><<<grid, 128, 0, st>>>((const __nv_bfloat16*)k, sk, kbar_blocks,
+                                                      Hkv, kbar);
+  else
+    sd_block_means_kernel<64><<<grid, 64, 0, st>>>((const __nv_bfloat16*)k, sk, kbar_blocks, Hkv,
+                                                    kbar);
   SALA_CHECK_LAUNCH();
   return SALA_OK;
 }

@@ -3,8 +3,9 @@
     python -m sparse_attention_long_lightning_b200.profile_case --op attn --T 16384 --iters 3
 
 Ops: lightning (prefill, B1 H32 D128 bf16 chunk 128), decode (B64 H32 D128 bf16),
-select / attn (B1 Hq32 Hkv2 D128 bf16, top-64 + 1 + 2).  Prints the mean CUDA-event
-time per call.
+select / attn (B1 Hq32 Hkv2 D128 bf16, top-64 + 1 + 2), sparse_decode (B sequences,
+Hq32 Hkv2 D128 bf16, KV caches of T tokens, one step at positions near the end).
+Prints the mean CUDA-event time per call.
 """
 from __future__ import annotations
 
@@ -18,7 +19,8 @@ from sparse_attention_long_lightning_b200 import inputs
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", required=True, choices=["lightning", "decode", "select", "attn"])
+    ap.add_argument("--op", required=True, choices=["lightning", "decode", "select", "attn",
+                                                       "sparse_decode"])
     ap.add_argument("--T", type=int, default=16384)
     ap.add_argument("--B", type=int, default=64, help="batch for decode")
     ap.add_argument("--iters", type=int, default=3)
@@ -39,6 +41,24 @@ def main():
         pos = torch.zeros(a.B, dtype=torch.int32, device=dev)
         o = torch.empty_like(q)
         fn = lambda: sala.lightning_decode(q, k, v, g, S, pos, out=o)
+    elif a.op == "sparse_decode":
+        B, Tmax = a.B, a.T
+        gen = inputs.generator(1006, dev)
+        k = inputs.randn((B, Tmax, 2, 128), gen, device=dev)
+        v = inputs.randn((B, Tmax, 2, 128), gen, device=dev)
+        q = inputs.randn((B, 32, 128), gen, device=dev)
+        g = inputs.randn((B, 32, 128), gen, device=dev)
+        kbar = sala.sparse_block_means(k)
+        pos = torch.tensor([Tmax - 1 - 13 * b for b in range(B)], dtype=torch.int32, device=dev)
+        ws = torch.empty(sala.sparse_decode_workspace(B, Tmax, 32, 2, 128, 67), dtype=torch.uint8,
+                         device=dev)
+        o = torch.empty_like(q)
+        fn = lambda: sala.sparse_decode(q, k, v, kbar, pos, g, out=o, workspace=ws)
+        cand = sum(max(0, (Tmax - 1 - 13 * b) // 64 - 2) for b in range(B))
+        nbytes = cand * 2 * 128 * 4 + B * 2 * 67 * 64 * 128 * 2 * 2 + 3 * B * 32 * 128 * 2
+        print(f"sparse_decode: algorithmic bytes per step {nbytes / 1e6:.1f} MB "
+              f"(block means {cand * 2 * 128 * 4 / 1e6:.1f} MB, K/V blocks "
+              f"{B * 2 * 67 * 64 * 128 * 4 / 1e6:.1f} MB)")
     else:
         s = inputs.sparse_inputs(1, a.T, 32, 2, 128, seed=1004, device=dev, gate=True)
         idx = sala.sparse_select(s.q, s.k)

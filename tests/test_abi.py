@@ -104,6 +104,35 @@ def test_select_and_attn_reject_bad_arguments(lib):
                                 0.0, p, 16, 1, None) == 5
 
 
+def test_sparse_decode_rejects_bad_arguments(lib):
+    p = ctypes.c_void_p(16)
+    sq = sala.SalaStrides(32 * 128, 0, 128)
+    sk = sala.SalaStrides(4096 * 2 * 128, 2 * 128, 128)
+
+    def call(pos=p, Tmax=4096, Hq=32, Hkv=2, D=128, ws_bytes=1 << 26, dt=1, block=64):
+        return lib.sala_sparse_decode(p, p, p, None, p, pos, p, None, 1, Tmax, Hq, Hkv, D, sq, sk,
+                                      sk, Z, sq, block, 64, 1, 2, 0.0, p, ws_bytes, dt, None)
+    assert call(pos=None) == 1                 # null pos
+    assert call(Tmax=4000) == 1                # cache length not a multiple of 64
+    assert call(Hq=33) == 1                    # Hq not a multiple of Hkv
+    assert call(D=48) == 2                     # head_dim
+    assert call(Hq=64) == 2                    # group of 32 heads > one 16-row tile
+    assert call(block=32) == 2
+    assert call(dt=0) == 2                     # fp32 not provided
+    assert call(ws_bytes=16) == 5              # workspace too small
+    # block means: kbar too short for the cache
+    assert lib.sala_sparse_block_means(p, 1, 4096, 2, 128, sk, p, 63, 1, None) == 1
+    assert lib.sala_sparse_block_means(p, 1, 4096, 2, 96, sk, p, 64, 1, None) == 2
+
+
+def test_sparse_decode_workspace_query():
+    up = lambda x: (x + 255) // 256 * 256
+    n = sala.sparse_decode_workspace(64, 131072, 32, 2, 128, 67)
+    scores, idx, part = 64 * 2 * 2048 * 4, 64 * 2 * 67 * 4, 64 * 2 * 16 * 16 * 130 * 4
+    assert n == up(scores) + up(idx) + up(part)
+    assert sala.sparse_decode_workspace(1, 100, 32, 2, 128, 67) == 0
+
+
 def test_workspace_queries(lib):
     nb = 131072 // 64
     means = nb * 2 * 128 * (4 + 2 + 2)                       # fp32 means + bf16 hi / lo

@@ -424,3 +424,79 @@ def test_attention_rows_subset_and_empty_set():
     np.testing.assert_array_equal(oracle.attention(q[:, rows], k, v, rows=rows), yf[:, rows])
     empty = -np.ones((1, Hkv, T, 3), dtype=np.int32)
     assert np.all(oracle.attention(q, k, v, idx=empty, blk=blk) == 0.0)
+
+
+# ----------------------------------------------------------------------------
+# Sparse-layer decode (one query at position p over cache rows 0..p)
+# ----------------------------------------------------------------------------
+
+def _dense_row(q, k, v, p, g=None):
+    """Plain numpy softmax attention of one query row over keys 0..p (GQA by repeat)."""
+    Hq, D = q.shape
+    Hkv = k.shape[1]
+    grp = Hq // Hkv
+    y = np.zeros((Hq, D))
+    for h in range(Hq):
+        s = k[:p + 1, h // grp] @ q[h] / math.sqrt(D)
+        w = np.exp(s - s.max())
+        y[h] = (w / w.sum()) @ v[:p + 1, h // grp]
+        if g is not None:
+            y[h] *= 1.0 / (1.0 + np.exp(-g[h]))
+    return y
+
+
+def test_decode_within_budget_is_dense_row():
+    """While p + 1 <= (n_init + topk + n_local) * blk every causal block is chosen, so
+    the decode output is the dense causal softmax row (numpy closed form)."""
+    rng = np.random.default_rng(21)
+    blk, Hq, Hkv, D, Tmax = 8, 4, 2, 8, 96
+    q, g = rng.standard_normal((3, Hq, D)), rng.standard_normal((3, Hq, D))
+    k, v = rng.standard_normal((3, Tmax, Hkv, D)), rng.standard_normal((3, Tmax, Hkv, D))
+    pos = [0, 37, 8 * 5 - 1]  # topk 2 + init 1 + local 2 = 5 blocks of 8
+    y, idx, _ = oracle.sparse_decode(q, k, v, pos, g, blk=blk, topk=2)
+    for b, p in enumerate(pos):
+        np.testing.assert_allclose(y[b], _dense_row(q[b], k[b], v[b], p, g[b]), rtol=1e-12,
+                                   atol=1e-13)
+        c = p // blk
+        live = idx[b, 0][idx[b, 0] >= 0]
+        np.testing.assert_array_equal(live, np.arange(c + 1))
+
+
+def test_decode_ignores_rows_past_p():
+    """Cache rows after p (here NaN) never reach the output or the selection."""
+    rng = np.random.default_rng(22)
+    blk, Hq, Hkv, D, Tmax, p = 8, 4, 2, 8, 200, 133
+    q = rng.standard_normal((1, Hq, D))
+    k, v = rng.standard_normal((1, Tmax, Hkv, D)), rng.standard_normal((1, Tmax, Hkv, D))
+    y0, i0, _ = oracle.sparse_decode(q, k, v, [p], blk=blk, topk=3)
+    k[:, p + 1:] = np.nan
+    v[:, p + 1:] = np.nan
+    y1, i1, _ = oracle.sparse_decode(q, k, v, [p], blk=blk, topk=3)
+    np.testing.assert_array_equal(i0, i1)
+    np.testing.assert_array_equal(y0, y1)
+    assert np.all(np.isfinite(y1))
+
+
+def test_decode_selection_bruteforce():
+    """The decode selection is the brute-force top-k of the block-mean scores over the
+    candidates n_init <= j <= c - n_local, united with the init and local blocks."""
+    rng = np.random.default_rng(23)
+    blk, Hq, Hkv, D, Tmax = 4, 4, 2, 6, 160
+    q = rng.standard_normal((4, Hq, D))
+    k, v = rng.standard_normal((4, Tmax, Hkv, D)), rng.standard_normal((4, Tmax, Hkv, D))
+    pos = [159, 100, 63, 17]
+    topk, n_init, n_local = 5, 1, 2
+    _, idx, _ = oracle.sparse_decode(q, k, v, pos, blk=blk, topk=topk, n_init=n_init,
+                                     n_local=n_local)
+    G = Hq // Hkv
+    for b, p in enumerate(pos):
+        c = p // blk
+        for hk in range(Hkv):
+            qs = q[b, hk * G:(hk + 1) * G].sum(0)
+            cand = list(range(n_init, c - n_local + 1))
+            score = {j: qs @ k[b, j * blk:(j + 1) * blk, hk].mean(0) for j in cand}
+            best = sorted(cand, key=lambda j: (-score[j], j))[:topk]
+            want = sorted(set(range(min(n_init, c + 1))) | set(best) |
+                          set(range(max(n_init, c - n_local + 1), c + 1)))
+            got = idx[b, hk][idx[b, hk] >= 0].tolist()
+            assert got == want, (b, hk)
