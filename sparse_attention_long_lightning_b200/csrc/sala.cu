@@ -423,6 +423,33 @@ sala_status sala_sparse_attn(const void* q, const void* k, const void* v, const 
 
 // ------------------------------------------------------------------ sparse-layer decode
 namespace {
+// Resident CTAs per SM of sd_attn_kernel<D> after its shared-memory opt-in, per device
+// (the opt-in is a per-device function attribute); 0 on failure.
+int sd_attn_occupancy(int D) {
+  constexpr int kDev = 64;
+  static std::mutex mu;
+  static int cache[2][kDev] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDev) return 0;
+  const int w = D == 128 ? 1 : 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[w][dev] == 0) {
+    int occ = 0;
+    bool ok;
+    if (D == 128)
+      ok = set_smem(sd_attn_kernel<128>, SdAttnSmem<128>::bytes) &&
+           cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+               &occ, sd_attn_kernel<128>, kSdAttnWarps * 32, SdAttnSmem<128>::bytes) == cudaSuccess;
+    else
+      ok = set_smem(sd_attn_kernel<64>, SdAttnSmem<64>::bytes) &&
+           cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+               &occ, sd_attn_kernel<64>, kSdAttnWarps * 32, SdAttnSmem<64>::bytes) == cudaSuccess;
+    if (!ok || occ < 1) return 0;
+    cache[w][dev] = occ;
+  }
+  return cache[w][dev];
+}
+
 struct SdLayout {
   size_t scores_off, idx_off, part_off, total;
 };
@@ -485,12 +512,22 @@ sala_status sala_sparse_decode(const void* q, const void* k_cache, const void* v
   p.B = B; p.Tmax = Tmax; p.Hq = Hq; p.Hkv = Hkv; p.G = Hq / Hkv; p.D = D;
   p.nbcap = Tmax / kSdBlk;
   p.n_init = n_init; p.topk = topk; p.n_local = n_local; p.n_sel = n_sel;
-  const int rows = B * Hkv;
-  p.nsplit = std::max(1, std::min({(2 * num_sms() + rows - 1) / rows, kSdMaxSplit, n_sel}));
+  const int rows = B * Hkv, nsm = num_sms();
+  // attention splits: fill the resident CTA slots once (cp.async tiles take 64 KB per CTA
+  // at D = 128); score chunks: the score grid covers the SMs twice.  The shared-memory
+  // opt-in and the occupancy are looked up once per device and kernel.
+  int occ = sd_attn_occupancy(D);
+  if (occ < 1) return SALA_ERR_CUDA;
+  const int slots = std::max(1, occ) * nsm;
+  p.nsplit = std::max(1, std::min({(slots + rows / 2) / rows, kSdMaxSplit, n_sel}));
+  {
+    const int64_t want = ((int64_t)p.nbcap * rows + 2 * nsm - 1) / (2 * nsm);
+    p.chunk = (int)std::max<int64_t>(64, std::min<int64_t>(kSdScoreChunk, (want + 31) / 32 * 32));
+  }
   const float sc = scale > 0.0f ? scale : 1.0f / std::sqrt((float)D);
   p.scale_log2 = sc * 1.4426950408889634f;
   cudaStream_t st = as_stream(stream);
-  const dim3 gs((p.nbcap + kSdScoreChunk - 1) / kSdScoreChunk, Hkv, B);
+  const dim3 gs((p.nbcap + p.chunk - 1) / p.chunk, Hkv, B);
   const dim3 ga(p.nsplit, Hkv, B);
   if (D == 128) {
     sd_score_kernel<128><<<gs, 256, 0, st>>>(p);
@@ -501,15 +538,11 @@ sala_status sala_sparse_decode(const void* q, const void* k_cache, const void* v
   sd_topk_kernel<<<dim3(Hkv, B), kSdTopkThreads, 0, st>>>(p);
   SALA_CHECK_LAUNCH();
   if (D == 128) {
-    auto kern = sd_attn_kernel<128>;
-    if (!set_smem(kern, SdAttnSmem<128>::bytes)) return SALA_ERR_CUDA;
-    kern<<<ga, kSdAttnWarps * 32, SdAttnSmem<128>::bytes, st>>>(p);
+    sd_attn_kernel<128><<<ga, kSdAttnWarps * 32, SdAttnSmem<128>::bytes, st>>>(p);
     SALA_CHECK_LAUNCH();
     sd_combine_kernel<128><<<dim3(Hq, B), 128, 0, st>>>(p);
   } else {
-    auto kern = sd_attn_kernel<64>;
-    if (!set_smem(kern, SdAttnSmem<64>::bytes)) return SALA_ERR_CUDA;
-    kern<<<ga, kSdAttnWarps * 32, SdAttnSmem<64>::bytes, st>>>(p);
+    sd_attn_kernel<64><<<ga, kSdAttnWarps * 32, SdAttnSmem<64>::bytes, st>>>(p);
     SALA_CHECK_LAUNCH();
     sd_combine_kernel<64><<<dim3(Hq, B), 64, 0, st>>>(p);
   }

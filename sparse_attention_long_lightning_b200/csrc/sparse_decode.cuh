@@ -20,7 +20,7 @@
 //   sd_topk_kernel    one CTA per (KV head, sequence): CTA radix select over the scores'
 //                     order-preserving keys, then a stable compaction in block order
 //   sd_attn_kernel    one CTA per (split, KV head, sequence): the split's share of the
-//                     chosen blocks, cp.async double-buffered K/V tiles, the group's query
+//                     chosen blocks, a cp.async ring of K/V tiles, the group's query
 //                     heads as the M = 16 operand of m16n8k16 tensor-core MMAs (Q K^T in
 //                     bf16; P in fp16 on V converted to fp16 in registers), online softmax
 //                     per warp, the four warps merged into one partial (max, sum, O)
@@ -34,9 +34,13 @@
 namespace sala {
 
 constexpr int kSdBlk = 64;           // keys per block
-constexpr int kSdScoreChunk = 512;   // candidates per score CTA
+constexpr int kSdScoreChunk = 512;   // most candidates per score CTA
 constexpr int kSdMaxSplit = 16;      // attention splits per (sequence, KV head)
 constexpr int kSdAttnWarps = 4;      // 16 keys of a block each
+#ifndef SALA_SD_STAGES
+#define SALA_SD_STAGES 3
+#endif
+constexpr int kSdStages = SALA_SD_STAGES;  // K/V tile ring depth of the attention kernel
 
 struct SdParams {
   const __nv_bfloat16* q;   // [B, Hq, D]  (strides sq.b, sq.h)
@@ -51,7 +55,7 @@ struct SdParams {
   float* part;              // [B, Hkv, nsplit, 16 * (D + 2)]
   sala_strides sq, sg, so, sk, sv;
   int B, Tmax, Hq, Hkv, G, D, nbcap;
-  int n_init, topk, n_local, n_sel, nsplit;
+  int n_init, topk, n_local, n_sel, nsplit, chunk;
   float scale_log2;         // softmax scale * log2(e)
 };
 
@@ -86,8 +90,8 @@ __global__ void __launch_bounds__(256) sd_score_kernel(const SdParams p) {
     }
   }
   const int jhi = c - p.n_local;                      // last candidate (complete blocks)
-  const int j0 = p.n_init + blockIdx.x * kSdScoreChunk;
-  const int j1 = min(jhi, j0 + kSdScoreChunk - 1);
+  const int j0 = p.n_init + blockIdx.x * p.chunk;
+  const int j1 = min(jhi, j0 + p.chunk - 1);
   if (j1 < j0) return;
   for (int d = tid; d < D; d += 256) {
     const __nv_bfloat16* qr = p.q + b * p.sq.b + (int64_t)hk * p.G * p.sq.h + d;
@@ -133,12 +137,37 @@ __global__ void __launch_bounds__(256) sd_score_kernel(const SdParams p) {
 
 // ---- top-k of the candidates, written with the init blocks and the local window
 constexpr int kSdTopkThreads = 256;
+constexpr int kSdTopkStage = 8192;  // candidates staged in shared memory (else read from L2)
+
+// Exclusive prefix sum of one int per thread over the CTA; *total gets the sum.
+__device__ __forceinline__ int sd_cta_exscan(int x, int* wbuf, int* total) {
+  constexpr int kW = kSdTopkThreads / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = x;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  if (lane == 31) wbuf[warp] = incl;
+  __syncthreads();
+  int before = 0, tot = 0;
+#pragma unroll
+  for (int w = 0; w < kW; ++w) {
+    const int v = wbuf[w];
+    before += w < warp ? v : 0;
+    tot += v;
+  }
+  __syncthreads();  // wbuf may be reused
+  *total = tot;
+  return before + incl - x;
+}
 
 __global__ void __launch_bounds__(kSdTopkThreads) sd_topk_kernel(const SdParams p) {
-  constexpr int kW = kSdTopkThreads / 32;
+  __shared__ float stage[kSdTopkStage];
   __shared__ uint32_t hist[256];
   __shared__ uint32_t s_prefix, s_rem;
-  __shared__ int wsum[2][kW];
+  __shared__ int wbuf[kSdTopkThreads / 32];
   const int b = blockIdx.y, hk = blockIdx.x, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int t = sd_pos(p, b);
@@ -155,6 +184,12 @@ __global__ void __launch_bounds__(kSdTopkThreads) sd_topk_kernel(const SdParams 
     for (int e = tid; e < n; e += kSdTopkThreads) out[pos + e] = p.n_init + e;
     pos += n;
   } else {
+    const float* src = sc;
+    if (n <= kSdTopkStage) {
+      for (int e = tid; e < n; e += kSdTopkThreads) stage[e] = sc[e];
+      src = stage;
+      __syncthreads();
+    }
     // radix select, 8 bits per pass from the top: the topk-th largest key
     uint32_t prefix = 0, pmask = 0;
     int remaining = p.topk;
@@ -162,7 +197,7 @@ __global__ void __launch_bounds__(kSdTopkThreads) sd_topk_kernel(const SdParams 
       hist[tid] = 0;
       __syncthreads();
       for (int e = tid; e < n; e += kSdTopkThreads) {
-        const uint32_t key = order_key(sc[e]);
+        const uint32_t key = order_key(src[e]);
         if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
       }
       __syncthreads();
@@ -196,35 +231,28 @@ __global__ void __launch_bounds__(kSdTopkThreads) sd_topk_kernel(const SdParams 
       pmask |= 255u << shift;
     }
     // keys above `prefix` are in; of the keys equal to it, the first `remaining` in block
-    // order.  Stable compaction, kSdTopkThreads candidates per round.
-    int eq_before = 0;
-    for (int base = 0; base < n; base += kSdTopkThreads) {
-      const int e = base + tid;
-      const uint32_t key = e < n ? order_key(sc[e]) : 0u;
-      const bool gt = e < n && key > prefix;
-      const bool eq = e < n && key == prefix;
-      const uint32_t lt = (1u << lane) - 1u;
-      const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
-      if (lane == 0) wsum[0][warp] = __popc(eqm);
-      __syncthreads();
-      int eq_off = eq_before;
-      for (int w = 0; w < warp; ++w) eq_off += wsum[0][w];
-      int eq_tot = 0;
-      for (int w = 0; w < kW; ++w) eq_tot += wsum[0][w];
-      const bool take = gt || (eq && eq_off + __popc(eqm & lt) < remaining);
-      const uint32_t selm = __ballot_sync(0xffffffffu, take);
-      if (lane == 0) wsum[1][warp] = __popc(selm);
-      __syncthreads();
-      int sel_off = 0, sel_tot = 0;
-      for (int w = 0; w < kW; ++w) {
-        sel_tot += wsum[1][w];
-        if (w < warp) sel_off += wsum[1][w];
-      }
-      if (take) out[pos + sel_off + __popc(selm & lt)] = p.n_init + e;
-      pos += sel_tot;
-      eq_before += eq_tot;
-      __syncthreads();  // wsum reused next round
+    // order.  Each thread owns a contiguous run of candidates: one scan of the counts
+    // places every thread's selections.
+    const int per = (n + kSdTopkThreads - 1) / kSdTopkThreads;
+    const int e0 = min(n, tid * per), e1 = min(n, e0 + per);
+    int ngt = 0, neq = 0;
+    for (int e = e0; e < e1; ++e) {
+      const uint32_t key = order_key(src[e]);
+      ngt += key > prefix;
+      neq += key == prefix;
     }
+    int tot;
+    const int gt_before = sd_cta_exscan(ngt, wbuf, &tot);
+    const int eq_before = sd_cta_exscan(neq, wbuf, &tot);
+    int w = pos + gt_before + min(eq_before, remaining);
+    int eq_seen = eq_before;
+    for (int e = e0; e < e1; ++e) {
+      const uint32_t key = order_key(src[e]);
+      bool take = key > prefix;
+      if (key == prefix) take = eq_seen++ < remaining;
+      if (take) out[w++] = p.n_init + e;
+    }
+    pos += p.topk;
   }
   const int lo = max(p.n_init, c - p.n_local + 1);
   for (int j = lo + tid; j <= c; j += kSdTopkThreads) out[pos + (j - lo)] = j;
@@ -239,8 +267,8 @@ struct SdAttnSmem {
   static constexpr int kTile = kSdBlk * D * 2;       // K or V block
   static constexpr int kBuf = 2 * kTile;             // K then V
   static constexpr int kMerge = kSdAttnWarps * 16 * D * 4 + kSdAttnWarps * 32 * 4;
-  static_assert(kMerge <= 2 * kBuf, "merge area fits in the tile buffers");
-  static constexpr size_t bytes = 2 * size_t(kBuf) + 128;  // + alignment slack
+  static_assert(kMerge <= kSdStages * kBuf, "merge area fits in the tile buffers");
+  static constexpr size_t bytes = kSdStages * size_t(kBuf) + 128;  // + alignment slack
 };
 
 template <int D>
@@ -285,9 +313,9 @@ __global__ void __launch_bounds__(kSdAttnWarps * 32) sd_attn_kernel(const SdPara
                          : 0u;
       }
   }
-  auto issue = [&](int e) {  // K and V of chosen block e into buffer e & 1
+  auto issue = [&](int e) {  // K and V of chosen block e into ring slot (e - sb0) % S
     const int j = __ldg(ir + e);
-    const uint32_t kb = smem_u32(smem + (e & 1) * L::kBuf), vb = kb + L::kTile;
+    const uint32_t kb = smem_u32(smem + ((e - sb0) % kSdStages) * L::kBuf), vb = kb + L::kTile;
     const __nv_bfloat16* ks = p.k + b * p.sk.b + (int64_t)j * kSdBlk * p.sk.t + hk * p.sk.h;
     const __nv_bfloat16* vs = p.v + b * p.sv.b + (int64_t)j * kSdBlk * p.sv.t + hk * p.sv.h;
     for (int x = tid; x < kSdBlk * kCh; x += blockDim.x) {
@@ -297,10 +325,11 @@ __global__ void __launch_bounds__(kSdAttnWarps * 32) sd_attn_kernel(const SdPara
       cp_async16(vb + off, vs + (int64_t)r * p.sv.t + cc * 8);
     }
   };
-  issue(sb0);
-  cp_async_commit();
-  if (sb0 + 1 < sb1) issue(sb0 + 1);
-  cp_async_commit();
+#pragma unroll
+  for (int x = 0; x < kSdStages; ++x) {  // one commit group per slot, possibly empty
+    if (sb0 + x < sb1) issue(sb0 + x);
+    cp_async_commit();
+  }
 
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // rows gq, gq+8 (log2 domain)
   float oacc[kNT][4];
@@ -308,10 +337,10 @@ __global__ void __launch_bounds__(kSdAttnWarps * 32) sd_attn_kernel(const SdPara
   for (int nt = 0; nt < kNT; ++nt) oacc[nt][0] = oacc[nt][1] = oacc[nt][2] = oacc[nt][3] = 0.f;
   uint32_t bad = 0;
   for (int e = sb0; e < sb1; ++e) {
-    cp_async_wait<1>();
+    cp_async_wait<kSdStages - 1>();  // block e's group has landed
     __syncthreads();
     const int j = __ldg(ir + e);
-    const uint32_t kb = smem_u32(smem + (e & 1) * L::kBuf), vb = kb + L::kTile;
+    const uint32_t kb = smem_u32(smem + ((e - sb0) % kSdStages) * L::kBuf), vb = kb + L::kTile;
     const bool straddle = j == c && t % kSdBlk != kSdBlk - 1;  // keys past t in this block
     if (straddle) {
       // rows past t may hold anything: zero their V so 0-weights stay 0
@@ -403,8 +432,8 @@ __global__ void __launch_bounds__(kSdAttnWarps * 32) sd_attn_kernel(const SdPara
       mma_f16_16816(oacc[2 * pp], pa, vv[pp][0], vv[pp][1]);
       mma_f16_16816(oacc[2 * pp + 1], pa, vv[pp][2], vv[pp][3]);
     }
-    __syncthreads();  // buffer e & 1 is free again
-    if (e + 2 < sb1) issue(e + 2);
+    __syncthreads();  // block e's slot is free again
+    if (e + kSdStages < sb1) issue(e + kSdStages);  // into block e's slot
     cp_async_commit();
   }
   cp_async_wait<0>();
