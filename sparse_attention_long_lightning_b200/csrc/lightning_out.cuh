@@ -40,16 +40,18 @@ constexpr int kLoIssuer = kLoPrepThreads;  // first CONV thread issues MMAs and 
 // 64-column slabs of 128 rows x 128 bytes with the 128-byte swizzle.
 __device__ __forceinline__ void lo_prep_qk_half(uint8_t* sQ, uint8_t* sK, int r, int hf,
                                                 const TcParams& p, const float2* ang_base) {
+  // shared-space accesses by address (the tiles are in shared memory)
+  const uint32_t q_s = smem_u32(sQ), k_s = smem_u32(sK);
   float ssq = 0.f, ssk = 0.f;
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
     const int j = 4 * hf + (u & 3);
     const uint32_t a = (u >> 2) * kTcSlab + swz128(r, j);
     float f[8];
-    bf16x8_to_f32(*reinterpret_cast<const uint4*>(sK + a), f);
+    bf16x8_to_f32(lds128(k_s + a), f);
 #pragma unroll
     for (int e = 0; e < 8; ++e) ssk = fmaf(f[e], f[e], ssk);
-    bf16x8_to_f32(*reinterpret_cast<const uint4*>(sQ + a), f);
+    bf16x8_to_f32(lds128(q_s + a), f);
 #pragma unroll
     for (int e = 0; e < 8; ++e) ssq = fmaf(f[e], f[e], ssq);
   }
@@ -63,10 +65,10 @@ __device__ __forceinline__ void lo_prep_qk_half(uint8_t* sQ, uint8_t* sK, int r,
     const int j = 4 * hf + jj;
     const uint32_t alo = swz128(r, j), ahi = kTcSlab + swz128(r, j);
     float klo[8], khi[8], qlo[8], qhi[8];
-    bf16x8_to_f32(*reinterpret_cast<const uint4*>(sK + alo), klo);
-    bf16x8_to_f32(*reinterpret_cast<const uint4*>(sK + ahi), khi);
-    bf16x8_to_f32(*reinterpret_cast<const uint4*>(sQ + alo), qlo);
-    bf16x8_to_f32(*reinterpret_cast<const uint4*>(sQ + ahi), qhi);
+    bf16x8_to_f32(lds128(k_s + alo), klo);
+    bf16x8_to_f32(lds128(k_s + ahi), khi);
+    bf16x8_to_f32(lds128(q_s + alo), qlo);
+    bf16x8_to_f32(lds128(q_s + ahi), qhi);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const int i = 8 * j + e;  // rotation pair (i, i + 64)
@@ -85,22 +87,23 @@ __device__ __forceinline__ void lo_prep_qk_half(uint8_t* sQ, uint8_t* sK, int r,
       qlo[e] = q0 * cs - q1 * sn;
       qhi[e] = q1 * cs + q0 * sn;
     }
-    *reinterpret_cast<uint4*>(sK + alo) = f32x8_to_f16(klo);
-    *reinterpret_cast<uint4*>(sK + ahi) = f32x8_to_f16(khi);
-    *reinterpret_cast<uint4*>(sQ + alo) = f32x8_to_f16(qlo);
-    *reinterpret_cast<uint4*>(sQ + ahi) = f32x8_to_f16(qhi);
+    sts128(k_s + alo, f32x8_to_f16(klo));
+    sts128(k_s + ahi, f32x8_to_f16(khi));
+    sts128(q_s + alo, f32x8_to_f16(qlo));
+    sts128(q_s + ahi, f32x8_to_f16(qhi));
   }
 }
 
 // Half of the v row (chunks 8hf..8hf+7: slab hf) to fp16 in place.
 __device__ __forceinline__ void lo_prep_v_half(uint8_t* sV, int r, int hf) {
+  const uint32_t v_s = smem_u32(sV);
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
     const uint32_t a = hf * kTcSlab + swz128(r, u);
-    uint4 x = *reinterpret_cast<const uint4*>(sV + a);
+    uint4 x = lds128(v_s + a);
     x.x = bf16x2_to_f16x2(x.x); x.y = bf16x2_to_f16x2(x.y);
     x.z = bf16x2_to_f16x2(x.z); x.w = bf16x2_to_f16x2(x.w);
-    *reinterpret_cast<uint4*>(sV + a) = x;
+    sts128(v_s + a, x);
   }
 }
 

@@ -97,13 +97,15 @@ __device__ __forceinline__ uint4 f32x8_to_f16(const float* f) {
 // non-finite output or state, which the output pass reports.
 __device__ __forceinline__ void tc_prep_kv_quarter(uint8_t* sK, uint8_t* sV, int r, int qd,
                                                    const TcParams& p, const float2* ang_base) {
+  // shared-space accesses by address (the tiles are in shared memory)
+  const uint32_t k_s = smem_u32(sK), v_s = smem_u32(sV);
   float ssk = 0.f;
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const int j = 2 * qd + (u & 1);
     const uint32_t a = (u >> 1) * kTcSlab + swz128(r, j);
     float f[8];
-    bf16x8_to_f32(*reinterpret_cast<const uint4*>(sK + a), f);
+    bf16x8_to_f32(lds128(k_s + a), f);
 #pragma unroll
     for (int e = 0; e < 8; ++e) ssk = fmaf(f[e], f[e], ssk);
   }
@@ -116,8 +118,8 @@ __device__ __forceinline__ void tc_prep_kv_quarter(uint8_t* sK, uint8_t* sV, int
     const int j = 2 * qd + jj;
     const uint32_t alo = swz128(r, j), ahi = kTcSlab + swz128(r, j);
     float klo[8], khi[8];
-    bf16x8_to_f32(*reinterpret_cast<const uint4*>(sK + alo), klo);
-    bf16x8_to_f32(*reinterpret_cast<const uint4*>(sK + ahi), khi);
+    bf16x8_to_f32(lds128(k_s + alo), klo);
+    bf16x8_to_f32(lds128(k_s + ahi), khi);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const int i = 8 * j + e;  // rotation pair (i, i + 64)
@@ -132,17 +134,17 @@ __device__ __forceinline__ void tc_prep_kv_quarter(uint8_t* sK, uint8_t* sV, int
       klo[e] = k0 * cs - k1 * sn;
       khi[e] = k1 * cs + k0 * sn;
     }
-    *reinterpret_cast<uint4*>(sK + alo) = f32x8_to_f16(klo);
-    *reinterpret_cast<uint4*>(sK + ahi) = f32x8_to_f16(khi);
+    sts128(k_s + alo, f32x8_to_f16(klo));
+    sts128(k_s + ahi, f32x8_to_f16(khi));
   }
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const int cj = 4 * qd + u;
     const uint32_t a = (cj >> 3) * kTcSlab + swz128(r, cj & 7);
-    uint4 x = *reinterpret_cast<const uint4*>(sV + a);
+    uint4 x = lds128(v_s + a);
     x.x = bf16x2_to_f16x2(x.x); x.y = bf16x2_to_f16x2(x.y);
     x.z = bf16x2_to_f16x2(x.z); x.w = bf16x2_to_f16x2(x.w);
-    *reinterpret_cast<uint4*>(sV + a) = x;
+    sts128(v_s + a, x);
   }
 }
 
