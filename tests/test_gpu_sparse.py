@@ -53,6 +53,20 @@ def test_select_exact_ties_take_smaller_blocks():
     assert np.array_equal(idx, ref)
 
 
+def test_select_heavy_tailed_scores():
+    """Ten blocks whose keys are a large constant vector: every row's scores are far from
+    normal (ten extreme values on one side), the case a distribution-based shortcut
+    would get wrong; the selection must still match the oracle."""
+    T, Hq, Hkv, D, topk = 64 * 600 + 21, 16, 2, 128, 64
+    s = inputs.sparse_inputs(1, T, Hq, Hkv, D, seed=79)
+    k = s.k.clone()
+    k[:, 64 * 5:64 * 15] = 30.0
+    idx = sala.sparse_select(s.q.cuda(), k.cuda(), topk=topk)
+    rows = _sampled_rows(T, n_mid=1500, seed=5)
+    ref, gap = oracle.sparse_select(_np(s.q[:, rows]), _np(k), topk=topk, rows=rows)
+    check_index_sets(idx.cpu().numpy()[:, :, rows], ref, gap)
+
+
 def test_select_batched_strided():
     """B = 2 with q, k as views of a packed tensor (non-contiguous strides)."""
     B, T, Hq, Hkv, D = 2, 64 * 13 + 30, 16, 2, 128
