@@ -330,6 +330,61 @@ def e2e_measure(layers, sala, steps, stream):
     return e0.elapsed_time(e1) / steps / 1e3, h2d, d2h
 
 
+def decode_components(dev, hbm):
+    """One-token decode steps, timed outside the hybrid-prefill region: the Lightning layer
+    (B64 H32 D128, the fp32 state read and written) and the sparse layer (B64 sequences with
+    131072-token KV caches, 32q/2kv D128).  Both move far more than L2 per step."""
+    import sparse_attention_long_lightning_b200 as sala
+    from sparse_attention_long_lightning_b200 import inputs
+
+    def timed(fn, iters=50, warmup=5):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(iters):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / iters  # ms
+
+    out = {}
+    Bd = 64
+    S = inputs.decode_state(Bd, H, D, seed=1003, device=dev)
+    q, k, v, g = inputs.decode_tokens(Bd, H, D, seed=1003, step=0, device=dev)
+    pos = torch.full((Bd,), 131072, dtype=torch.int32, device=dev)
+    o = torch.empty_like(q)
+    ms = timed(lambda: sala.lightning_decode(q, k, v, g, S, pos, out=o))
+    nbytes = Bd * H * (2 * D * D * 4 + 5 * D * 2)
+    out["lightning_decode_b64"] = {"us": ms * 1e3, "GB/s": nbytes / ms / 1e6,
+                                   "frac_hbm": nbytes / ms / 1e6 / hbm}
+    del S, q, k, v, g, o
+    Tc = 131072
+    gen = inputs.generator(1006, dev)
+    kc = inputs.randn((Bd, Tc, HKV, D), gen, device=dev)
+    vc = inputs.randn((Bd, Tc, HKV, D), gen, device=dev)
+    qd = inputs.randn((Bd, H, D), gen, device=dev)
+    gd = inputs.randn((Bd, H, D), gen, device=dev)
+    kbar = sala.sparse_block_means(kc)
+    p_l = [Tc - 1 - 13 * b for b in range(Bd)]
+    posd = torch.tensor(p_l, dtype=torch.int32, device=dev)
+    n_sel = N_INIT + TOPK + N_LOCAL
+    ws = torch.empty(sala.sparse_decode_workspace(Bd, Tc, H, HKV, D, n_sel), dtype=torch.uint8,
+                     device=dev)
+    od = torch.empty_like(qd)
+    ms = timed(lambda: sala.sparse_decode(qd, kc, vc, kbar, posd, gd, topk=TOPK, n_init=N_INIT,
+                                          n_local=N_LOCAL, out=od, workspace=ws))
+    cand = sum(max(0, p // BLOCK - N_LOCAL - N_INIT + 1) for p in p_l)
+    nbytes = cand * HKV * D * 4 + Bd * HKV * n_sel * BLOCK * D * 2 * 2 + 3 * Bd * H * D * 2
+    out["sparse_decode_b64_128k"] = {"us": ms * 1e3, "GB/s": nbytes / ms / 1e6,
+                                     "frac_hbm": nbytes / ms / 1e6 / hbm}
+    err = sala.get_device_error()
+    if err:
+        raise RuntimeError(f"device error in the decode components: {sala.status_string(err)}")
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -409,7 +464,7 @@ def main():
     # ncu capture of this command at T=131072 with the current kernels (the sparse
     # kernel's own launch; Lightning = state pass + scan + output pass; selection =
     # block means + fused kernel).  Re-measure whenever one of those kernels changes.
-    ncu_traffic = {"attn": 9.09e9, "sel": 1.17e9} if T == 131072 else {}
+    ncu_traffic = {"attn": 9.16e9, "sel": 1.17e9} if T == 131072 else {}
     share = {k: n_ops[k] * op_ms[k] for k in op_ms}
     dom = max(share, key=share.get)
     if dom == "attn":
@@ -450,6 +505,7 @@ def main():
         line["e2e"] = {"value": weak_scaling_value(world, T, e2e_sec), "unit": "tokens/s",
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                        "ms_per_step": e2e_sec * 1e3}
+        line["components"].update(decode_components(dev, hbm))
         if rank == 0 and world == 1:
             tps, info = cpu_baseline(T)
             line["cpu_baseline"] = dict(info, value=tps, unit="tokens/s")
