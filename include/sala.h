@@ -126,6 +126,32 @@ sala_status sala_lightning_decode(const void *q, const void *k, const void *v, c
                                   sala_dtype dt, void *stream);
 
 /*
+ * Lightning state of a token segment, without outputs: the exchange step of a sequence
+ * split across devices (each device holds a contiguous segment; the recurrence is a sum,
+ * so a segment's start state is the initial state plus the contributions of the
+ * segments before it).
+ *   state = (init_zero ? 0 : state) + sum_t kh_t v_t^T over the T tokens,
+ *   kh_t = RoPE_{pos0+t}(RMSNorm(k_t) * k_norm_w)  (as in sala_lightning_prefill)
+ * Arguments, layouts, dtypes and limits as sala_lightning_prefill (k, v, state, k_norm_w,
+ * the strides of k and v); the workspace is sala_lightning_prefill_workspace(B, T, H, D,
+ * chunk) bytes.  Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
+ */
+sala_status sala_lightning_state(const void *k, const void *v, float *state,
+                                 const float *k_norm_w, int B, int T, int H, int D,
+                                 sala_strides sk, sala_strides sv, int chunk, int64_t pos0,
+                                 float rope_base, float eps, int init_zero, void *workspace,
+                                 size_t workspace_bytes, sala_dtype dt, void *stream);
+
+/*
+ * Sum of `count` fp32 arrays: dst[e] = (accumulate ? dst[e] : 0) + sum_{i < count}
+ * src[i * stride + e] for e < n (device pointers; stride >= n when count > 1).  Forms a
+ * segment's start state from the gathered states of the segments before it.
+ * Errors: INVALID_ARG, CUDA.
+ */
+sala_status sala_state_prefix_sum(const float *src, size_t n, int count, size_t stride,
+                                  float *dst, int accumulate, void *stream);
+
+/*
  * Block selection (InfLLM-v2 style, NoPE).
  * For each (b, kv head hk, query row t), c = floor(t / block):
  *   Kbar_j  = mean of the `block` keys of complete block j (fp32)

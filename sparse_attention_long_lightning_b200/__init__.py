@@ -21,7 +21,8 @@ __all__ = [
     "lightning_decode", "sparse_select", "sparse_select_workspace", "sparse_attn",
     "sparse_attn_workspace",
     "get_device_error", "selftest_wait_timeout", "sparse_decode", "sparse_decode_workspace",
-    "sparse_block_means", "status_string", "version", "LIB_PATH",
+    "sparse_block_means", "lightning_state", "state_prefix_sum", "status_string", "version",
+    "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsala.so")
@@ -66,6 +67,11 @@ def load_library(path: Optional[str] = None):
     lib.sala_lightning_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, S, S, S, S,
                                           S, f, f, i, vp]
     lib.sala_lightning_decode.restype = i
+    lib.sala_lightning_state.argtypes = [vp, vp, vp, vp, i, i, i, i, S, S, i, i64, f, f, i, vp, sz,
+                                         i, vp]
+    lib.sala_lightning_state.restype = i
+    lib.sala_state_prefix_sum.argtypes = [vp, sz, i, sz, vp, i, vp]
+    lib.sala_state_prefix_sum.restype = i
     lib.sala_sparse_select_workspace.argtypes = [i, i, i, i, i, i, i]
     lib.sala_sparse_select_workspace.restype = sz
     lib.sala_sparse_select.argtypes = [vp, vp, i, i, i, i, i, S, S, i, i, i, i, vp, vp, sz, i, vp]
@@ -213,6 +219,42 @@ def lightning_decode(q, k, v, g, state, pos, q_norm_w=None, k_norm_w=None, *, ro
         D, _s3(q), _s3(k), _s3(v), _s3(g), _s3(out), float(rope_base), float(eps), _dt(q),
         _stream(stream))
     _check("sala_lightning_decode", st)
+    return out
+
+
+def lightning_state(k, v, state=None, k_norm_w=None, *, chunk=128, pos0=0, rope_base=10000.0,
+                    eps=1e-6, workspace=None, stream=None):
+    """Segment state sum_t kh_t v_t^T of k, v [B,T,H,D] (added to `state` [B,H,D,D] fp32
+    when given, else from zero).  Returns the state."""
+    lib = load_library()
+    _cuda(k, v, state, k_norm_w, workspace)
+    B, T, H, D = k.shape
+    init_zero = state is None
+    if state is None:
+        state = torch.empty((B, H, D, D), dtype=torch.float32, device=k.device)
+    need = lightning_prefill_workspace(B, T, H, D, chunk) if k.dtype == torch.bfloat16 else 0
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=k.device)
+    wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib.sala_lightning_state(_p(k), _p(v), _p(state), _p(k_norm_w), B, T, H, D, _s4(k),
+                                  _s4(v), int(chunk), int(pos0), float(rope_base), float(eps),
+                                  int(init_zero), _p(workspace), wsb, _dt(k), _stream(stream))
+    _check("sala_lightning_state", st)
+    return state
+
+
+def state_prefix_sum(gathered, count, out, accumulate=True, stream=None):
+    """out (+)= sum of gathered[0..count-1] (fp32 tensors of out's size)."""
+    lib = load_library()
+    _cuda(gathered, out)
+    n = out.numel()
+    if gathered.dtype != torch.float32 or out.dtype != torch.float32:
+        raise TypeError("float32 states expected")
+    if not gathered.is_contiguous() or not out.is_contiguous() or gathered[0].numel() != n:
+        raise ValueError("gathered must be [count, *out.shape] contiguous")
+    st = lib.sala_state_prefix_sum(_p(gathered), n, int(count), n, _p(out), int(accumulate),
+                                   _stream(stream))
+    _check("sala_state_prefix_sum", st)
     return out
 
 

@@ -58,7 +58,8 @@ lightning_prefill_cc_kernel(const T* __restrict__ q, const T* __restrict__ k,
   const T* kb = k + b * sk.b + h * sk.h;
   const T* vb = v + b * sv.b + h * sv.h;
   const T* gb = g ? g + b * sg.b + h * sg.h : nullptr;
-  T* ob = o + b * so.b + h * so.h;
+  const bool write_o = o != nullptr;
+  T* ob = write_o ? o + b * so.b + h * so.h : nullptr;
   constexpr int kPer = D / 32;  // elements per lane in a row
 
   for (int t0 = 0; t0 < T_len; t0 += kCT) {
@@ -111,63 +112,65 @@ lightning_prefill_cc_kernel(const T* __restrict__ q, const T* __restrict__ k,
       }
     }
     __syncthreads();
-    // ---- A = Qh Kh^T, lower-triangular inclusive ----
-    {
-      const int r = tid >> 2;
+    if (write_o) {  // o == nullptr: the state update alone
+      // ---- A = Qh Kh^T, lower-triangular inclusive ----
+      {
+        const int r = tid >> 2;
 #pragma unroll 4
-      for (int m = 0; m < kCT / 4; ++m) {
-        const int s = (tid & 3) + 4 * m;
-        float a = 0.0f;
-        if (s <= r) {
+        for (int m = 0; m < kCT / 4; ++m) {
+          const int s = (tid & 3) + 4 * m;
+          float a = 0.0f;
+          if (s <= r) {
 #pragma unroll 8
-          for (int i = 0; i < D; ++i) a = fmaf(Qs[r * kLd + i], Ks[s * kLd + i], a);
+            for (int i = 0; i < D; ++i) a = fmaf(Qs[r * kLd + i], Ks[s * kLd + i], a);
+          }
+          As[r * (kCT + 1) + s] = a;
         }
-        As[r * (kCT + 1) + s] = a;
       }
-    }
-    __syncthreads();
-    // ---- O = A V + Qh S, gate, store ----
-    {
-      const int rr = tid >> 5, jj = tid & 31;
-      constexpr int kNJ = D / 32;
-      float acc[8][kNJ];
+      __syncthreads();
+      // ---- O = A V + Qh S, gate, store ----
+      {
+        const int rr = tid >> 5, jj = tid & 31;
+        constexpr int kNJ = D / 32;
+        float acc[8][kNJ];
 #pragma unroll
-      for (int m = 0; m < 8; ++m)
+        for (int m = 0; m < 8; ++m)
 #pragma unroll
-        for (int nj = 0; nj < kNJ; ++nj) acc[m][nj] = 0.0f;
-      for (int s = 0; s < kCT; ++s) {
-        float vv[kNJ];
+          for (int nj = 0; nj < kNJ; ++nj) acc[m][nj] = 0.0f;
+        for (int s = 0; s < kCT; ++s) {
+          float vv[kNJ];
 #pragma unroll
-        for (int nj = 0; nj < kNJ; ++nj) vv[nj] = Vs[s * kLd + jj + 32 * nj];
+          for (int nj = 0; nj < kNJ; ++nj) vv[nj] = Vs[s * kLd + jj + 32 * nj];
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const float a = As[(rr + 8 * m) * (kCT + 1) + s];
+#pragma unroll
+            for (int nj = 0; nj < kNJ; ++nj) acc[m][nj] = fmaf(a, vv[nj], acc[m][nj]);
+          }
+        }
+        for (int i = 0; i < D; ++i) {
+          float sv_[kNJ];
+#pragma unroll
+          for (int nj = 0; nj < kNJ; ++nj) sv_[nj] = S[i * D + jj + 32 * nj];
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const float qi = Qs[(rr + 8 * m) * kLd + i];
+#pragma unroll
+            for (int nj = 0; nj < kNJ; ++nj) acc[m][nj] = fmaf(qi, sv_[nj], acc[m][nj]);
+          }
+        }
 #pragma unroll
         for (int m = 0; m < 8; ++m) {
-          const float a = As[(rr + 8 * m) * (kCT + 1) + s];
+          const int r = rr + 8 * m;
+          if (r < n) {
+            const int64_t t = t0 + r;
 #pragma unroll
-          for (int nj = 0; nj < kNJ; ++nj) acc[m][nj] = fmaf(a, vv[nj], acc[m][nj]);
-        }
-      }
-      for (int i = 0; i < D; ++i) {
-        float sv_[kNJ];
-#pragma unroll
-        for (int nj = 0; nj < kNJ; ++nj) sv_[nj] = S[i * D + jj + 32 * nj];
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          const float qi = Qs[(rr + 8 * m) * kLd + i];
-#pragma unroll
-          for (int nj = 0; nj < kNJ; ++nj) acc[m][nj] = fmaf(qi, sv_[nj], acc[m][nj]);
-        }
-      }
-#pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const int r = rr + 8 * m;
-        if (r < n) {
-          const int64_t t = t0 + r;
-#pragma unroll
-          for (int nj = 0; nj < kNJ; ++nj) {
-            const int j = jj + 32 * nj;
-            float y = acc[m][nj];
-            if (gb) y *= sigmoidf_(ld(gb + t * sg.t + j));
-            st(ob + t * so.t + j, y);
+            for (int nj = 0; nj < kNJ; ++nj) {
+              const int j = jj + 32 * nj;
+              float y = acc[m][nj];
+              if (gb) y *= sigmoidf_(ld(gb + t * sg.t + j));
+              st(ob + t * so.t + j, y);
+            }
           }
         }
       }

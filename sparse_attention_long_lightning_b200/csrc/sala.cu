@@ -88,6 +88,18 @@ bool make_tmap_bhtd(CUtensorMap* map, const void* base, int B, int T, int H, int
   return r == CUDA_SUCCESS;
 }
 
+// dst = (accumulate ? dst : 0) + sum over i < count of src[i * stride + e], e < n.
+__global__ void __launch_bounds__(256)
+state_prefix_sum_kernel(const float* __restrict__ src, size_t n, int count, size_t stride,
+                        float* __restrict__ dst, int accumulate) {
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+       e += (size_t)gridDim.x * blockDim.x) {
+    float acc = accumulate ? dst[e] : 0.0f;
+    for (int i = 0; i < count; ++i) acc += src[(size_t)i * stride + e];
+    dst[e] = acc;
+  }
+}
+
 template <typename KernelT>
 bool set_smem(KernelT* k, size_t bytes) {
   return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) ==
@@ -249,6 +261,104 @@ sala_status sala_lightning_decode(const void* q, const void* k, const void* v, c
     if (D == 128) SALA_DEC(float, 128); else SALA_DEC(float, 64);
   }
 #undef SALA_DEC
+  SALA_CHECK_LAUNCH();
+  return SALA_OK;
+}
+
+// ------------------------------------------------------------------ sequence-split Lightning
+// A segment's state contribution (no outputs): the state pass and scan of the tensor-core
+// path, or the CUDA-core kernel with its output half skipped.
+sala_status sala_lightning_state(const void* k, const void* v, float* state, const float* k_norm_w,
+                                 int B, int T, int H, int D, sala_strides sk, sala_strides sv,
+                                 int chunk, int64_t pos0, float rope_base, float eps,
+                                 int init_zero, void* workspace, size_t workspace_bytes,
+                                 sala_dtype dt, void* stream) {
+  if (!state || (T > 0 && (!k || !v))) return SALA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || T < 0 || pos0 < 0 || !(rope_base > 1.0f) || !(eps >= 0.0f))
+    return SALA_ERR_INVALID_ARG;
+  if (dt != SALA_BF16 && dt != SALA_F32) return SALA_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128) return SALA_ERR_UNSUPPORTED;
+  if (chunk != 64 && chunk != 128) return SALA_ERR_UNSUPPORTED;
+  const size_t es = esize_of(dt);
+  if (!aligned16(k) || !aligned16(v) || !aligned16(state)) return SALA_ERR_INVALID_ARG;
+  if (!strides_ok(sk, es) || !strides_ok(sv, es)) return SALA_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  const double log2_base = std::log2((double)rope_base);
+  if (T == 0) {
+    if (init_zero && cudaMemsetAsync(state, 0, sizeof(float) * (size_t)B * H * D * D, st) !=
+                         cudaSuccess)
+      return SALA_ERR_CUDA;
+    return SALA_OK;
+  }
+  if (dt == SALA_BF16 && D == 128 && chunk == kTcC) {
+    const int nsm = num_sms();
+    const size_t need = lightning_tc_workspace(B, T, H, chunk, nsm);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return SALA_ERR_WORKSPACE;
+    CUtensorMap tk, tv;
+    if (!make_tmap_bhtd(&tk, k, B, T, H, D, sk, kTcC) || !make_tmap_bhtd(&tv, v, B, T, H, D, sv, kTcC))
+      return SALA_ERR_CUDA;
+    TcParams p{};
+    p.kw = k_norm_w;
+    p.ws = (float*)workspace;
+    p.B = B; p.T = T; p.H = H;
+    p.G = lightning_tc_segments(B, H, T, nsm);
+    p.NC = (T + kTcC - 1) / kTcC;
+    p.pos0 = pos0;
+    p.log2_base = log2_base;
+    p.eps = eps;
+    auto ka = lightning_state_kernel;
+    if (!set_smem(ka, TcSmem<true>::bytes)) return SALA_ERR_CUDA;
+    ka<<<(unsigned)(B * H * p.G), kTcThreads, TcSmem<true>::bytes, st>>>(tk, tv, p);
+    SALA_CHECK_LAUNCH();
+    lightning_scan_kernel<<<dim3(B * H, 16), 256, 0, st>>>(p.ws, state, p.G, init_zero);
+    SALA_CHECK_LAUNCH();
+    return SALA_OK;
+  }
+  // CUDA-core kernel with o == nullptr: q is read but unused, so k stands in for it
+  const sala_strides none{0, 0, 0};
+  const int grid = B * H;
+  if (dt == SALA_F32) {
+    if (D == 64) {
+      auto kern = lightning_prefill_cc_kernel<float, 64>;
+      if (!set_smem(kern, CCSmem<64>::bytes)) return SALA_ERR_CUDA;
+      kern<<<grid, kCCThreads, CCSmem<64>::bytes, st>>>(
+          (const float*)k, (const float*)k, (const float*)v, nullptr, nullptr, state, nullptr,
+          k_norm_w, H, T, sk, sk, sv, none, none, pos0, log2_base, eps, init_zero);
+    } else {
+      auto kern = lightning_prefill_cc_kernel<float, 128>;
+      if (!set_smem(kern, CCSmem<128>::bytes)) return SALA_ERR_CUDA;
+      kern<<<grid, kCCThreads, CCSmem<128>::bytes, st>>>(
+          (const float*)k, (const float*)k, (const float*)v, nullptr, nullptr, state, nullptr,
+          k_norm_w, H, T, sk, sk, sv, none, none, pos0, log2_base, eps, init_zero);
+    }
+  } else if (D == 64) {
+    auto kern = lightning_prefill_cc_kernel<__nv_bfloat16, 64>;
+    if (!set_smem(kern, CCSmem<64>::bytes)) return SALA_ERR_CUDA;
+    kern<<<grid, kCCThreads, CCSmem<64>::bytes, st>>>(
+        (const __nv_bfloat16*)k, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, nullptr,
+        nullptr, state, nullptr, k_norm_w, H, T, sk, sk, sv, none, none, pos0, log2_base, eps,
+        init_zero);
+  } else {
+    auto kern = lightning_prefill_cc_kernel<__nv_bfloat16, 128>;
+    if (!set_smem(kern, CCSmem<128>::bytes)) return SALA_ERR_CUDA;
+    kern<<<grid, kCCThreads, CCSmem<128>::bytes, st>>>(
+        (const __nv_bfloat16*)k, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, nullptr,
+        nullptr, state, nullptr, k_norm_w, H, T, sk, sk, sv, none, none, pos0, log2_base, eps,
+        init_zero);
+  }
+  SALA_CHECK_LAUNCH();
+  return SALA_OK;
+}
+
+sala_status sala_state_prefix_sum(const float* src, size_t n, int count, size_t stride,
+                                  float* dst, int accumulate, void* stream) {
+  if (!dst || (count > 0 && !src) || count < 0 || (count > 1 && stride < n))
+    return SALA_ERR_INVALID_ARG;
+  if (n == 0 || (count == 0 && accumulate)) return SALA_OK;  // nothing to add
+  const int64_t want = 4 * (int64_t)num_sms();
+  const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(want, ((int64_t)n + 255) / 256));
+  state_prefix_sum_kernel<<<grid, 256, 0, as_stream(stream)>>>(src, n, count, stride, dst,
+                                                               accumulate);
   SALA_CHECK_LAUNCH();
   return SALA_OK;
 }

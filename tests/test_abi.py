@@ -125,6 +125,22 @@ def test_sparse_decode_rejects_bad_arguments(lib):
     assert lib.sala_sparse_block_means(p, 1, 4096, 2, 96, sk, p, 64, 1, None) == 2
 
 
+def test_lightning_state_and_prefix_reject_bad_arguments(lib):
+    p = ctypes.c_void_p(16)
+    st = sala.SalaStrides(64 * 4 * 128, 4 * 128, 128)
+    assert lib.sala_lightning_state(p, p, None, None, 1, 64, 4, 128, st, st, 128, 0, 10000.0,
+                                    1e-6, 1, p, 1 << 24, 1, None) == 1  # null state
+    assert lib.sala_lightning_state(p, p, p, None, 1, 64, 4, 48, st, st, 128, 0, 10000.0, 1e-6,
+                                    1, p, 1 << 24, 1, None) == 2        # head_dim
+    assert lib.sala_lightning_state(p, p, p, None, 1, 64, 4, 128, st, st, 128, -1, 10000.0,
+                                    1e-6, 1, p, 1 << 24, 1, None) == 1  # negative position
+    assert lib.sala_lightning_state(p, p, p, None, 1, 64, 4, 128, st, st, 128, 0, 10000.0, 1e-6,
+                                    1, p, 16, 1, None) == 5             # workspace
+    assert lib.sala_state_prefix_sum(p, 1024, 2, 512, p, 1, None) == 1  # overlapping sources
+    assert lib.sala_state_prefix_sum(None, 1024, 2, 1024, p, 1, None) == 1
+    assert lib.sala_state_prefix_sum(None, 1024, 0, 0, p, 1, None) == 0  # nothing to add
+
+
 def test_sparse_decode_workspace_query():
     up = lambda x: (x + 255) // 256 * 256
     n = sala.sparse_decode_workspace(64, 131072, 32, 2, 128, 67)

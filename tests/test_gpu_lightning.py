@@ -201,3 +201,85 @@ def test_lightning_flags_fp16_range():
     sala.lightning_prefill(x.q.cuda(), x.k.cuda(), v.cuda(), x.g.cuda(), chunk=128)
     assert sala.get_device_error() == 6
     assert sala.get_device_error() == 0
+
+
+# ---------------------------------------------------------------------------------------
+# Sequence split across devices: segment states (sala_lightning_state), their prefix
+# (sala_state_prefix_sum) and the segment prefills, run here rank after rank on one GPU.
+# ---------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("D,dtype,chunk", [(128, torch.bfloat16, 128), (64, torch.float32, 64),
+                                           (128, torch.bfloat16, 64)])
+def test_lightning_state_matches_prefill_final_state(D, dtype, chunk):
+    """The state-only call gives the prefill's final state (zero start and a given start)."""
+    B, T, H = 1, 64 * 21 + 5, 4
+    x = inputs.lightning_inputs(B, T, H, D, seed=61, dtype=dtype, device=DEV)
+    _, S_pf = sala.lightning_prefill(x.q, x.k, x.v, x.g, None, chunk=chunk, pos0=7)
+    S = sala.lightning_state(x.k, x.v, None, chunk=chunk, pos0=7)
+    tol = TOL_F32 if dtype == torch.float32 else 1e-6
+    assert raw_rel_err(S.cpu().numpy(), S_pf.cpu().numpy()) <= tol
+    S0 = torch.randn((B, H, D, D), generator=torch.Generator(device=DEV).manual_seed(3),
+                     device=DEV) * 0.05
+    _, S_pf0 = sala.lightning_prefill(x.q, x.k, x.v, x.g, S0.clone(), chunk=chunk, pos0=7)
+    S1 = sala.lightning_state(x.k, x.v, S0.clone(), chunk=chunk, pos0=7)
+    assert raw_rel_err(S1.cpu().numpy(), S_pf0.cpu().numpy()) <= tol
+    _, S_or = oracle.lightning_recurrent(_np(x.k), _np(x.k), _np(x.v), pos0=7)
+    assert raw_rel_err(S.cpu().numpy(), S_or) <= (TOL_F32 if dtype == torch.float32 else TOL_BF16)
+
+
+def test_lightning_sequence_split_three_segments():
+    """Three uneven segments processed as three ranks would: states, prefix, segment
+    prefills.  Outputs and final state agree with one prefill of the whole sequence and
+    with the oracle."""
+    B, H, D = 1, 8, 128
+    lens = [1000, 1024 + 77, 930]
+    T = sum(lens)
+    x = inputs.lightning_inputs(B, T, H, D, seed=62, device=DEV)
+    S_init = torch.randn((B, H, D, D), generator=torch.Generator(device=DEV).manual_seed(4),
+                         device=DEV) * 0.02
+    y_full, S_full = sala.lightning_prefill(x.q, x.k, x.v, x.g, S_init.clone(), pos0=11)
+    offs = [0, lens[0], lens[0] + lens[1]]
+    seg = lambda t, r: t[:, offs[r]:offs[r] + lens[r]]
+    dS = torch.stack([sala.lightning_state(seg(x.k, r), seg(x.v, r), None, pos0=11 + offs[r])
+                      for r in range(3)])
+    ys = []
+    for r in range(3):
+        S0 = sala.state_prefix_sum(dS, r, S_init.clone(), accumulate=True)
+        y, S_end = sala.lightning_prefill(seg(x.q, r), seg(x.k, r), seg(x.v, r), seg(x.g, r), S0,
+                                          pos0=11 + offs[r])
+        ys.append(y)
+    y_split = torch.cat(ys, dim=1)
+    assert sala.get_device_error() == 0
+    from tests._parity import rel_err_bf16_pair
+    assert rel_err_bf16_pair(_np(y_split), _np(y_full)) <= TOL_BF16
+    # segments start off the 128-token chunk grid, so a token's RoPE angle is formed from a
+    # different chunk base (and rounds differently before the fp16 operand cast): the two
+    # final states agree to ~1e-4, both within the oracle tolerance checked below
+    assert raw_rel_err(S_end.cpu().numpy(), S_full.cpu().numpy()) <= 1e-3
+    y_or, S_or = oracle.lightning_recurrent(_np(x.q), _np(x.k), _np(x.v), _np(x.g),
+                                            S_init.double().cpu().numpy(), pos0=11)
+    assert rel_err(_np(y_split), y_or, bf16_out=True) <= TOL_BF16
+    assert raw_rel_err(S_end.cpu().numpy(), S_or) <= TOL_BF16
+
+
+def test_lightning_seqpar_single_rank_group():
+    """The public sequence-parallel call on a one-rank NCCL group is the plain prefill."""
+    import os
+    import socket
+
+    import torch.distributed as dist
+
+    from sparse_attention_long_lightning_b200.seqpar import lightning_prefill_seqpar
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    os.environ["MASTER_ADDR"], os.environ["MASTER_PORT"] = "127.0.0.1", str(port)
+    dist.init_process_group("nccl", rank=0, world_size=1)
+    try:
+        x = inputs.lightning_inputs(1, 777, 4, 128, seed=63, device=DEV)
+        y, S = lightning_prefill_seqpar(x.q, x.k, x.v, x.g, pos0=3)
+        y_ref, S_ref = sala.lightning_prefill(x.q, x.k, x.v, x.g, None, pos0=3)
+        assert torch.equal(y, y_ref)
+        assert raw_rel_err(S.cpu().numpy(), S_ref.cpu().numpy()) <= 1e-6
+    finally:
+        dist.destroy_process_group()
