@@ -53,6 +53,24 @@ def test_select_exact_ties_take_smaller_blocks():
     assert np.array_equal(idx, ref)
 
 
+@pytest.mark.parametrize("n_init,n_local", [(1, 8), (2, 5)])
+def test_select_and_attn_wider_windows(n_init, n_local):
+    """A larger local window and more init blocks (the selection rule's window sizes are
+    parameters): selection and attention against the oracle."""
+    T, Hq, Hkv, D, topk = 64 * 150 + 40, 16, 2, 128, 16
+    s = inputs.sparse_inputs(1, T, Hq, Hkv, D, seed=80 + n_local, gate=True)
+    q, k, v, g = (t.cuda() for t in (s.q, s.k, s.v, s.g))
+    idx = sala.sparse_select(q, k, topk=topk, n_init=n_init, n_local=n_local)
+    rows = _sampled_rows(T, n_mid=600, seed=6)
+    ref, gap = oracle.sparse_select(_np(s.q[:, rows]), _np(s.k), topk=topk, n_init=n_init,
+                                    n_local=n_local, rows=rows)
+    check_index_sets(idx.cpu().numpy()[:, :, rows], ref, gap)
+    y = sala.sparse_attn(q, k, v, idx, g)
+    want = oracle.attention(_np(s.q[:, rows]), _np(s.k), _np(s.v), _np(s.g[:, rows]),
+                            idx=idx.cpu().numpy()[:, :, rows], rows=rows)
+    assert rel_err(_np(y[:, rows]), want, bf16_out=True) <= TOL_BF16
+
+
 def test_select_heavy_tailed_scores():
     """Ten blocks whose keys are a large constant vector: every row's scores are far from
     normal (ten extreme values on one side), the case a distribution-based shortcut

@@ -75,6 +75,21 @@ def test_decode_positions(Hq, Hkv, D, gate):
             assert torch.equal(kbar[b, p // 64], full[b, p // 64])
 
 
+def test_decode_wider_windows():
+    """n_init = 2, n_local = 6, topk = 20: selection and output against the oracle."""
+    Tmax, Hq, Hkv, D = 64 * 64, 32, 2, 128
+    pos_l = [64 * 3, 64 * 9 + 63, 64 * 40 + 5, Tmax - 1]
+    B = len(pos_l)
+    q, g, k, v = _data(B, Tmax, Hq, Hkv, D, seed=409)
+    q, g, k, v = q.to(DEV), g.to(DEV), k.to(DEV), v.to(DEV)
+    kbar = sala.sparse_block_means(k)
+    pos = torch.tensor(pos_l, dtype=torch.int32, device=DEV)
+    idx = torch.empty((B, Hkv, 28), dtype=torch.int32, device=DEV)
+    y = sala.sparse_decode(q, k, v, kbar, pos, g, topk=20, n_init=2, n_local=6, idx_out=idx)
+    assert sala.get_device_error() == 0
+    _check_step(q, g, k, v, pos_l, y, idx, topk=20, n_init=2, n_local=6)
+
+
 def test_decode_steps_continue_a_prefilled_cache():
     """70 consecutive steps after a 1970-token prefill, crossing two block ends: every
     step against the oracle, then the block-mean cache against the oracle's means."""
