@@ -13,11 +13,12 @@
 //   producers (warps 4-7): thread p sums the group's queries of row p in fp32, splits
 //     the sum into bf16 high / low parts and stores them to its TMEM lane: the A
 //     operand of the NEXT item (two A buffers), so the query reads overlap the scan;
-//   issuer (warp 8, one thread): streams 32-candidate tiles of the block means (bf16
-//     high / low, written by block_means_kernel) through a 3-stage shared-memory ring
-//     by TMA and issues S = qs_lo.Kb_hi + qs_hi.Kb_lo + qs_hi.Kb_hi into one of 8 fp32
-//     TMEM score buffers;
-//   consumers (warps 0-3): thread r reads its row's 32 scores of a tile, releases the
+//   issuer (warp 8, one thread): streams 64-candidate tiles of the block means (bf16
+//     high / low, written by block_means_kernel) through a 2-stage shared-memory ring
+//     by TMA and issues S = qs_lo.Kb_hi + qs_hi.Kb_lo + qs_hi.Kb_hi (24 MMAs of N = 64:
+//     the MMA issue, not the data, paces the pipeline) into one of 4 fp32 TMEM score
+//     buffers;
+//   consumers (warps 0-3): thread r reads its row's 64 scores of a tile, releases the
 //     score buffer (per-warp arrival, so the warps run decoupled) and appends the
 //     scores above its row threshold to a per-row buffer (shared memory, block order).
 // When a buffer could overflow on the next tile, the rows of that warp compact their
@@ -34,17 +35,18 @@
 namespace sala {
 
 constexpr int kStcRows = 128;   // query rows per item (= TMEM lanes = consumer threads)
-constexpr int kStcN = 32;       // candidates per tile
-constexpr int kStcCap = 214;    // buffered candidates per row
+constexpr int kStcN = 64;       // candidates per tile (per MMA: fewer, wider MMAs per candidate)
+constexpr int kStcSub = 32;     // candidates appended between buffer checks
+constexpr int kStcCap = 194;    // buffered candidates per row
 constexpr int kStcBins = 64;    // histogram bins per compaction pass
-constexpr int kStcStages = 3;   // block-mean tile ring
-constexpr int kStcAcc = 8;      // TMEM score buffers
+constexpr int kStcStages = 2;   // block-mean tile ring
+constexpr int kStcAcc = 4;      // TMEM score buffers
 constexpr int kStcCoarse = 150;  // entries a compaction during the scan may keep
 constexpr int kStcThreads = 2 * kStcRows + 32;  // consumers, producers, issuer
 
 template <int D>
 struct StcSmem {
-  static constexpr int kHalfB = kStcN * 128;                 // 32 rows x 64 dims bf16: 4 KB
+  static constexpr int kHalfB = kStcN * 128;                 // kStcN rows x 64 dims bf16
   static constexpr int kTileB = (D / 64) * kHalfB;           // one hi or lo tile
   static constexpr int kStage = 2 * kTileB;                  // hi then lo
   static constexpr size_t kB = 0;                                     // [stages]
@@ -388,8 +390,10 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constan
         if (it.ntiles == 0) continue;
         const int buf = u & 1;
         const uint32_t tA = tmem + buf * 2 * kAcols;
-        ok = !*abort_flag && issue_tma(it, 0, g) && (it.ntiles < 2 || issue_tma(it, 1, g + 1)) &&
-             mbar_wait(&a_full[buf], (u >> 1) & 1);
+        ok = !*abort_flag;
+        // the first S - 1 tiles; tile i + S - 1 follows the MMAs of tile i below
+        for (int x = 0; x < kStcStages - 1 && x < it.ntiles && ok; ++x) ok = issue_tma(it, x, g + x);
+        ok = ok && mbar_wait(&a_full[buf], (u >> 1) & 1);
         tc_fence_after();
         for (int i = 0; i < it.ntiles && ok; ++i) {
           const int gg = g + i, st = gg % kStcStages, ab = gg % kStcAcc;
@@ -408,7 +412,9 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constan
           for (int kk = 0; kk < kK; ++kk) tc_mma_ts(d, tA + 8 * kk, desc_b(bh, kk), kId, 1u);
           tc_commit(&mma_done[ab]);
           tc_commit(&stage_free[st]);
-          if (i + 2 < it.ntiles) ok = issue_tma(it, i + 2, gg + 2);
+          // into the stage of tile gg - 1, whose MMAs were issued one tile ago
+          if (i + kStcStages - 1 < it.ntiles)
+            ok = issue_tma(it, i + kStcStages - 1, gg + kStcStages - 1);
         }
         if (!ok) break;
         tc_commit(&a_free[buf]);  // the item's queries are free once its MMAs complete
@@ -452,36 +458,42 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constan
           break;
         }
         tc_fence_after();
-        uint32_t sv[kStcN];
-        tc_ld32(tD + kStcN * ab + lane_off, sv);
+        uint32_t sv[kStcN / kStcSub][kStcSub];
+#pragma unroll
+        for (int sub = 0; sub < kStcN / kStcSub; ++sub)
+          tc_ld32(tD + kStcN * ab + kStcSub * sub + lane_off, sv[sub]);
         tc_wait_ld();
         tc_fence_before();
         __syncwarp();
         if ((tid & 31) == 0) mbar_arrive(&acc_free[ab]);  // this warp is done with it
-        if (buffered) {
-          // scores compared as raw dot products: the 1/sqrt(D) factor preserves the order
-          const int j0 = n_init + i * kStcN;
-          auto append = [&](int cc, bool in_range) {  // predicated, no branch
-            const float sc = __uint_as_float(sv[cc]);
-            const bool p = in_range & (sc > thr);
-            sts_f32_if(p, sA + cnt * (kStcRows * 4), sc);
-            sts_u16_if(p, jA + cnt * (kStcRows * 2), (uint32_t)(j0 + cc));
-            cnt += p ? 1 : 0;
-            smin = p ? fminf(smin, sc) : smin;
-            smax = p ? fmaxf(smax, sc) : smax;
-          };
-          if (j0 + kStcN - 1 <= jmax) {
 #pragma unroll
-            for (int cc = 0; cc < kStcN; ++cc) append(cc, true);
-          } else {
+        for (int sub = 0; sub < kStcN / kStcSub; ++sub) {
+          if (buffered) {
+            // scores compared as raw dot products: the 1/sqrt(D) factor preserves the order
+            const int j0 = n_init + i * kStcN + kStcSub * sub;
+            auto append = [&](int cc, bool in_range) {  // predicated, no branch
+              const float sc = __uint_as_float(sv[sub][cc]);
+              const bool p = in_range & (sc > thr);
+              sts_f32_if(p, sA + cnt * (kStcRows * 4), sc);
+              sts_u16_if(p, jA + cnt * (kStcRows * 2), (uint32_t)(j0 + cc));
+              cnt += p ? 1 : 0;
+              smin = p ? fminf(smin, sc) : smin;
+              smax = p ? fmaxf(smax, sc) : smax;
+            };
+            if (j0 + kStcSub - 1 <= jmax) {
 #pragma unroll
-            for (int cc = 0; cc < kStcN; ++cc) append(cc, j0 + cc <= jmax);
+              for (int cc = 0; cc < kStcSub; ++cc) append(cc, true);
+            } else {
+#pragma unroll
+              for (int cc = 0; cc < kStcSub; ++cc) append(cc, j0 + cc <= jmax);
+            }
           }
-        }
-        if (__any_sync(0xffffffffu, cnt > kStcCap - kStcN) && cnt > topk) {
-          // a cut that keeps at most kStcCoarse entries (all of the topk best)
-          cnt = stc_compact(sA, jA, hA, sh16, cnt, topk, smin, smax, max(kStcCoarse, topk), &thr);
-          smin = thr;
+          if (__any_sync(0xffffffffu, cnt > kStcCap - kStcSub) && cnt > topk) {
+            // a cut that keeps at most kStcCoarse entries (all of the topk best)
+            cnt = stc_compact(sA, jA, hA, sh16, cnt, topk, smin, smax, max(kStcCoarse, topk),
+                              &thr);
+            smin = thr;
+          }
         }
       }
       if (dead) {
