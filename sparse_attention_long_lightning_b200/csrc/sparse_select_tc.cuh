@@ -42,7 +42,8 @@ constexpr int kStcBins = 64;    // histogram bins per compaction pass
 constexpr int kStcStages = 2;   // block-mean tile ring
 constexpr int kStcAcc = 4;      // TMEM score buffers
 constexpr int kStcCoarse = 150;  // entries a compaction during the scan may keep
-constexpr int kStcThreads = 2 * kStcRows + 32;  // consumers, producers, issuer
+constexpr int kStcIssuers = 2;  // threads issuing score MMAs (alternate tiles)
+constexpr int kStcThreads = 2 * kStcRows + 32 * kStcIssuers;  // consumers, producers, issuers
 
 template <int D>
 struct StcSmem {
@@ -282,9 +283,9 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constan
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&a_full[i], kStcRows);
-      mbar_init(&a_free[i], 1);
+      mbar_init(&a_free[i], kStcIssuers);
     }
-    mbar_init(drain, 1);
+    mbar_init(drain, kStcIssuers);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -355,11 +356,15 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constan
       mbar_arrive(&a_full[buf]);
       ++u;
     }
-  } else if (warp == 8) {
-    // ================= issuer: block-mean tiles by TMA, score MMAs
+  } else if (warp >= 8) {
+    // ================= issuers: block-mean tiles by TMA (issuer 0), score MMAs (issuer
+    // iss takes the tiles gg with gg % kStcIssuers == iss: its own stages and buffers)
+    const int iss = warp - 8;
     if ((tid & 31) == 0) {
-      prefetch_tmap(&tm_hi);
-      prefetch_tmap(&tm_lo);
+      if (iss == 0) {
+        prefetch_tmap(&tm_hi);
+        prefetch_tmap(&tm_lo);
+      }
       int g = 0, u = 0, n_issued = 0;
       bool ok = true;
       // tile i of `it` as global tile gg, into stage gg % S once that stage's previous
@@ -392,11 +397,18 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constan
         const uint32_t tA = tmem + buf * 2 * kAcols;
         ok = !*abort_flag;
         // the first S - 1 tiles; tile i + S - 1 follows the MMAs of tile i below
-        for (int x = 0; x < kStcStages - 1 && x < it.ntiles && ok; ++x) ok = issue_tma(it, x, g + x);
+        for (int x = 0; iss == 0 && x < kStcStages - 1 && x < it.ntiles && ok; ++x)
+          ok = issue_tma(it, x, g + x);
         ok = ok && mbar_wait(&a_full[buf], (u >> 1) & 1);
         tc_fence_after();
         for (int i = 0; i < it.ntiles && ok; ++i) {
           const int gg = g + i, st = gg % kStcStages, ab = gg % kStcAcc;
+          if (gg % kStcIssuers != iss) {
+            // another issuer's tile; issuer 0 still refills the stage of tile gg - 1
+            if (iss == 0 && i + kStcStages - 1 < it.ntiles)
+              ok = issue_tma(it, i + kStcStages - 1, gg + kStcStages - 1);
+            continue;
+          }
           ok = mbar_wait(&full[st], (gg / kStcStages) & 1) &&
                (gg < kStcAcc || mbar_wait(&acc_free[ab], ((gg / kStcAcc) + 1) & 1));
           if (!ok) break;
@@ -413,7 +425,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constan
           tc_commit(&mma_done[ab]);
           tc_commit(&stage_free[st]);
           // into the stage of tile gg - 1, whose MMAs were issued one tile ago
-          if (i + kStcStages - 1 < it.ntiles)
+          if (iss == 0 && i + kStcStages - 1 < it.ntiles)
             ok = issue_tma(it, i + kStcStages - 1, gg + kStcStages - 1);
         }
         if (!ok) break;
@@ -424,9 +436,11 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constan
       if (!ok) *abort_flag = 1;
       // wind down: every MMA complete and every copy landed before resources are released
       tc_commit(drain);
-      mbar_wait(drain, 0);
-      for (int x = n_issued > kStcStages ? n_issued - kStcStages : 0; x < n_issued; ++x)
-        mbar_wait(&full[x % kStcStages], (x / kStcStages) & 1);
+      if (iss == 0) {
+        mbar_wait(drain, 0);
+        for (int x = n_issued > kStcStages ? n_issued - kStcStages : 0; x < n_issued; ++x)
+          mbar_wait(&full[x % kStcStages], (x / kStcStages) & 1);
+      }
     }
   } else if (warp < 4) {
     // ================= consumers: scores, per-row buffers, output
