@@ -41,7 +41,8 @@ constexpr int kLoIssuer = kLoPrepThreads;  // first CONV thread issues MMAs and 
 __device__ __forceinline__ void lo_prep_qk_half(uint8_t* sQ, uint8_t* sK, int r, int hf,
                                                 const TcParams& p, const float2* ang_base) {
   // shared-space accesses by address (the tiles are in shared memory)
-  const uint32_t q_s = smem_u32(sQ), k_s = smem_u32(sK);
+  const uint32_t q_s = smem_u32(sQ), k_s = smem_u32(sK), ang_s = smem_u32(ang_base);
+  uint4 bfx;
   float ssq = 0.f, ssk = 0.f;
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
@@ -72,8 +73,11 @@ __device__ __forceinline__ void lo_prep_qk_half(uint8_t* sQ, uint8_t* sK, int r,
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const int i = 8 * j + e;  // rotation pair (i, i + 64)
+      // (base angle, inv_freq) of pairs i, i + 1: one shared 16-byte load per two pairs
+      if ((e & 1) == 0) bfx = lds128(ang_s + 8 * i);
+      const float2 bf = (e & 1) ? make_float2(__uint_as_float(bfx.z), __uint_as_float(bfx.w))
+                                : make_float2(__uint_as_float(bfx.x), __uint_as_float(bfx.y));
       // angle = (chunk base angle, reduced in fp64) + r * inv_freq_i, re-reduced in fp32
-      const float2 bf = ang_base[i];
       float ang = fmaf((float)r, bf.y, bf.x);
       ang = fmaf(-rintf(ang * inv_two_pi), two_pi, ang);
       float sn, cs;

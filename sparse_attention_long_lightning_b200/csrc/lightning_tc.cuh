@@ -89,17 +89,42 @@ __device__ __forceinline__ uint4 f32x8_to_f16(const float* f) {
                     pack_f16x2(f[6], f[7]));
 }
 
+// cos and sin of r * inv_freq_i for the 16 rotation pairs that a state-pass prep thread
+// owns (its row r never changes; pair i = 16 qd + 8 jj + e).  The angle of pair i at
+// token r of a chunk is (chunk base angle B_i) + r * inv_freq_i, so with the chunk's
+// (cos B_i, sin B_i) from shared memory its cos and sin follow by angle addition -- four
+// multiply-adds, no special-function unit work in the per-chunk loop.
+struct TcRowRot {
+  float c[16], s[16];
+};
+
+__device__ __forceinline__ void tc_row_rot_init(TcRowRot& rr, int r, int qd, const double* inv_freq) {
+  const double two_pi = 6.283185307179586476925286766559;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const double a = (double)r * inv_freq[16 * qd + k];
+    const float red = (float)(a - rint(a * (1.0 / two_pi)) * two_pi);
+    sincosf(red, &rr.s[k], &rr.c[k]);
+  }
+}
+
 // Normalise + rotate a quarter of raw bf16 row r of the k tile and convert it, and a
 // quarter of the v row, to fp16 in place.  Four consecutive lanes share a row: quarter
 // qd owns rotation pairs i in [16 qd, 16 qd + 16) (chunks 2qd, 2qd+1 of both 64-column
 // slabs) and v chunks 4qd..4qd+3.  Tiles are two 64-column slabs of 128 rows x 128
-// bytes with the 128-byte swizzle.  An fp16 overflow here shows up downstream as a
+// bytes with the 128-byte swizzle.  `cs_tab` (a static shared array, read with ordinary
+// loads the compiler can schedule) holds the chunk's (cos B_i, sin B_i, cos B_i+1,
+// sin B_i+1) for even i at item (i mod 16) / 2 * 4 + i / 16, so the four quarters of a
+// row read adjacent 16-byte words.  An fp16 overflow here shows up downstream as a
 // non-finite output or state, which the output pass reports.
+__device__ __forceinline__ int tc_ang_item(int i) { return ((i & 15) >> 1) * 4 + (i >> 4); }
+
 __device__ __forceinline__ void tc_prep_kv_quarter(uint8_t* sK, uint8_t* sV, int r, int qd,
-                                                   const TcParams& p, const float2* ang_base) {
+                                                   const TcParams& p, const float4* cs_tab,
+                                                   const TcRowRot& rr) {
   // shared-space accesses by address (the tiles are in shared memory)
   const uint32_t k_s = smem_u32(sK), v_s = smem_u32(sV);
-  float ssk = 0.f;
+  float ss[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const int j = 2 * qd + (u & 1);
@@ -107,12 +132,12 @@ __device__ __forceinline__ void tc_prep_kv_quarter(uint8_t* sK, uint8_t* sV, int
     float f[8];
     bf16x8_to_f32(lds128(k_s + a), f);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) ssk = fmaf(f[e], f[e], ssk);
+    for (int e = 0; e < 8; ++e) ss[u] = fmaf(f[e], f[e], ss[u]);
   }
+  float ssk = (ss[0] + ss[1]) + (ss[2] + ss[3]);
   ssk += __shfl_xor_sync(0xffffffffu, ssk, 1);
   ssk += __shfl_xor_sync(0xffffffffu, ssk, 2);
   const float rk = rsqrtf(ssk * (1.0f / 128.0f) + p.eps);
-  const float two_pi = 6.28318530717958647692f, inv_two_pi = 0.15915494309189533577f;
 #pragma unroll
   for (int jj = 0; jj < 2; ++jj) {
     const int j = 2 * qd + jj;
@@ -120,19 +145,25 @@ __device__ __forceinline__ void tc_prep_kv_quarter(uint8_t* sK, uint8_t* sV, int
     float klo[8], khi[8];
     bf16x8_to_f32(lds128(k_s + alo), klo);
     bf16x8_to_f32(lds128(k_s + ahi), khi);
+    float4 cb;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const int i = 8 * j + e;  // rotation pair (i, i + 64)
-      // angle = (chunk base angle, reduced in fp64) + r * inv_freq_i, re-reduced in fp32
-      const float2 bf = ang_base[i];
-      float ang = fmaf((float)r, bf.y, bf.x);
-      ang = fmaf(-rintf(ang * inv_two_pi), two_pi, ang);
-      float sn, cs;
-      __sincosf(ang, &sn, &cs);
-      const float wk0 = p.kw ? __ldg(p.kw + i) : 1.f, wk1 = p.kw ? __ldg(p.kw + i + 64) : 1.f;
-      const float k0 = klo[e] * rk * wk0, k1 = khi[e] * rk * wk1;
-      klo[e] = k0 * cs - k1 * sn;
-      khi[e] = k1 * cs + k0 * sn;
+      const int k = 8 * jj + e;
+      // (cos B, sin B) of pairs i, i + 1: one shared 16-byte load per two pairs
+      if ((e & 1) == 0) cb = cs_tab[tc_ang_item(i)];
+      const float cB = (e & 1) ? cb.z : cb.x;
+      const float sB = (e & 1) ? cb.w : cb.y;
+      // cos, sin of B + r inv_freq_i, times the row's RMS scale
+      const float cs = fmaf(cB, rr.c[k], -sB * rr.s[k]) * rk;
+      const float sn = fmaf(sB, rr.c[k], cB * rr.s[k]) * rk;
+      float k0 = klo[e], k1 = khi[e];
+      if (p.kw) {
+        k0 *= __ldg(p.kw + i);
+        k1 *= __ldg(p.kw + i + 64);
+      }
+      klo[e] = fmaf(k0, cs, -k1 * sn);
+      khi[e] = fmaf(k1, cs, k0 * sn);
     }
     sts128(k_s + alo, f32x8_to_f16(klo));
     sts128(k_s + ahi, f32x8_to_f16(khi));
@@ -158,28 +189,41 @@ __device__ __forceinline__ uint64_t tc_desc_mn(const uint8_t* base, int kk) {
 }
 
 // State pass: per segment, dS = sum over its chunks of Kh_c^T V_c (TMEM accumulator),
-// written to the workspace as fp32.  Per chunk u (one CTA, 16 warps):
-//   A  wait TMA(u); prep k and v of chunk u in place    [tensor core: state MMA of u-1]
-//   B  wait the state MMA of u-1; TMA(u+2) into its stage; issue the state MMA of u.
+// written to the workspace as fp32.
+//   warps 0-15 (512 threads), per chunk u: wait TMA(u); prep k and v of chunk u in place
+//     (4 lanes per row); each warp then arrives on prepped[u % S];
+//   warp 16 runs the pipeline: once the MMA of u - 1 is done, that stage is refilled with
+//     chunk u - 1 + S; once all 16 warps have prepped chunk u it issues the state MMA of u
+//     (committing to mma_done[u % S]).  Before each copy it writes the chunk's table of
+//     (cos, sin) of the RoPE base angles into an 8-slot ring; the copy's mbarrier orders
+//     those writes before the prep warps' reads.  No CTA-wide barrier in the loop.
 // TMEM: S in columns [0,128).
-__global__ void __launch_bounds__(kTcThreads, 1)
+constexpr int kStThreads = kTcThreads + 32;
+constexpr int kStAngRing = 8;  // > the largest lag (4 chunks) between producer and prep warps
+
+__global__ void __launch_bounds__(kStThreads, 1)
 lightning_state_kernel(const __grid_constant__ CUtensorMap tmk,
                        const __grid_constant__ CUtensorMap tmv, const TcParams p) {
   using L = TcSmem<true>;
+  constexpr int S = L::kStages;
   constexpr uint32_t kIdState = umma_idesc_f16(128, 128, true, true);
+  constexpr int kPrepWarps = kTcThreads / 32;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* stages = smem;
-  uint8_t* misc = stages + L::kStages * L::kStageBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(misc);      // [kStages]
-  uint64_t* mma1_bar = full + 3;                           // state MMA done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(full + 5);
+  uint8_t* misc = stages + S * L::kStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(misc);      // [S]: the stage's chunk landed
+  uint64_t* mma_done = full + S;                           // [S]: its state MMA completed
+  uint64_t* prepped = full + 2 * S;                        // [S]: all prep warps done with it
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 96);
   double* inv_freq = reinterpret_cast<double*>(misc + 128);  // [64]
-  float2* ang_tab = reinterpret_cast<float2*>(misc + 640);   // [2][64]: (base angle, inv_freq)
+  // [kStAngRing][32] items of two pairs' (cos, sin) of the chunk's base angles
+  __shared__ float4 ang_ring[kStAngRing * 32];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool producer = warp == kPrepWarps;
   const int prow = 8 * warp + (lane >> 2), pqd = lane & 3;  // prep: 4 lanes per row
   const int lq = warp & 3, cg = warp >> 2;                  // TMEM: lanes 32lq.., cols 32cg..
   const int trow = 32 * lq + lane;
@@ -194,8 +238,11 @@ lightning_state_kernel(const __grid_constant__ CUtensorMap tmk,
   const int nchunks = c_end - c_begin;
 
   if (tid == 0) {
-    for (int i = 0; i < L::kStages; ++i) mbar_init(&full[i], 1);
-    mbar_init(mma1_bar, 1);
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&mma_done[i], 1);
+      mbar_init(&prepped[i], kPrepWarps);
+    }
     fence_mbar_init();
   }
   if (warp == 0) tc_alloc(tmem_slot, L::kTmemCols);
@@ -205,88 +252,106 @@ lightning_state_kernel(const __grid_constant__ CUtensorMap tmk,
   tc_fence_after();
   const uint32_t t_s = *tmem_slot;
   const uint32_t lane_off = (uint32_t)(32 * lq) << 16;
-
-  // base angle of each rotation pair at the first token of chunk u (fp64 reduction)
-  auto fill_angles = [&](int u) {
-    if (tid < 64) {
-      const double a = (double)(p.pos0 + (int64_t)(c_begin + u) * kTcC) * inv_freq[tid];
-      const double two_pi = 6.283185307179586476925286766559;
-      const double red_a = a - rint(a * (1.0 / two_pi)) * two_pi;
-      ang_tab[(u & 1) * 64 + tid] = make_float2((float)red_a, (float)inv_freq[tid]);
-    }
-  };
-  auto issue = [&](int u) {
-    const int si = u % L::kStages;
-    uint8_t* dk = stages + si * L::kStageBytes;
-    uint8_t* dv = dk + kTcTile;
-    const int t0 = (c_begin + u) * kTcC;
-    mbar_arrive_expect_tx(&full[si], L::kStageBytes);
-    tma_load_4d(dk, &tmk, &full[si], 0, h, t0, b);
-    tma_load_4d(dk + kTcSlab, &tmk, &full[si], 64, h, t0, b);
-    tma_load_4d(dv, &tmv, &full[si], 0, h, t0, b);
-    tma_load_4d(dv + kTcSlab, &tmv, &full[si], 64, h, t0, b);
-  };
-  int issued = 0;
-  if (tid == 0) {
-    prefetch_tmap(&tmk);
-    prefetch_tmap(&tmv);
-    for (; issued < L::kStages && issued < nchunks; ++issued) issue(issued);
-  }
-  __syncthreads();  // inv_freq visible
-  fill_angles(0);
-  __syncthreads();  // angle table for chunk 0 visible
-
-  uint32_t ph1 = 0;  // completed phases of mma1_bar
   bool ok = true;
-  for (int u = 0; u < nchunks; ++u) {
-    const int s = u % L::kStages;
-    uint8_t* sK = stages + s * L::kStageBytes;
-    uint8_t* sV = sK + kTcTile;
-    // ---- A: prep(u) while the tensor core runs the state MMA of u-1
-    ok = ok && mbar_wait(&full[s], (u / L::kStages) & 1);
-    if (ok) tc_prep_kv_quarter(sK, sV, prow, pqd, p, ang_tab + (u & 1) * 64);
-    fence_proxy_async_smem();
-    // angles of chunk u+1 (other parity; prep(u-1), the last reader, is behind a barrier)
-    if (u + 1 < nchunks) fill_angles(u + 1);
-    // ---- B: wait for the previous state MMA, refill its stage, issue this chunk's
-    if (u > 0) {
-      ok = ok && mbar_wait(mma1_bar, ph1 & 1);
-      ++ph1;
-    }
-    tc_fence_before();
-    ok = __syncthreads_and(ok);
-    if (!ok) break;
-    tc_fence_after();
-    if (tid == 0) {
-      if (u > 0 && issued < nchunks) issue(issued++);  // stage of chunk u-1 is free
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        tc_mma_ss(t_s, tc_desc_mn(sK, kk), tc_desc_mn(sV, kk), kIdState,
-                  (u == 0 && kk == 0) ? 0u : 1u);
-      tc_commit(mma1_bar);
-    }
-  }
 
-  // drain: the last state MMA, then the segment sum
-  if (ok && nchunks > 0) {
-    ok = mbar_wait(mma1_bar, ph1 & 1);
-    tc_fence_after();
-    if (ok) {
-      float* dst = p.ws + ((size_t)bh * p.G + seg) * (128 * 128) + (size_t)trow * 128 + 32 * cg;
-      uint32_t r[32];
-      tc_ld32(t_s + lane_off + 32 * cg, r);
-      tc_wait_ld();
+  if (producer) {
+    // (cos, sin) of each rotation pair's angle at the first token of chunk n (fp64
+    // reduction), written by the 32 lanes, then chunk n's copy (lane 0)
+    auto fill_and_issue = [&](int n) {
+      const double two_pi = 6.283185307179586476925286766559;
+      const double t0 = (double)(p.pos0 + (int64_t)(c_begin + n) * kTcC);
+      float cs[2], sn[2];
 #pragma unroll
-      for (int v4 = 0; v4 < 8; ++v4)
-        *reinterpret_cast<float4*>(dst + 4 * v4) =
-            make_float4(__uint_as_float(r[4 * v4]), __uint_as_float(r[4 * v4 + 1]),
-                        __uint_as_float(r[4 * v4 + 2]), __uint_as_float(r[4 * v4 + 3]));
+      for (int k = 0; k < 2; ++k) {  // pairs 2 lane, 2 lane + 1
+        const double a = t0 * inv_freq[2 * lane + k];
+        const float red = (float)(a - rint(a * (1.0 / two_pi)) * two_pi);
+        sincosf(red, &sn[k], &cs[k]);
+      }
+      ang_ring[(n % kStAngRing) * 32 + tc_ang_item(2 * lane)] =
+          make_float4(cs[0], sn[0], cs[1], sn[1]);
+      __syncwarp();
+      if (lane == 0) {
+        const int si = n % S;
+        uint8_t* dk = stages + si * L::kStageBytes;
+        uint8_t* dv = dk + kTcTile;
+        const int tok = (c_begin + n) * kTcC;
+        mbar_arrive_expect_tx(&full[si], L::kStageBytes);  // release: orders the table writes
+        tma_load_4d(dk, &tmk, &full[si], 0, h, tok, b);
+        tma_load_4d(dk + kTcSlab, &tmk, &full[si], 64, h, tok, b);
+        tma_load_4d(dv, &tmv, &full[si], 0, h, tok, b);
+        tma_load_4d(dv + kTcSlab, &tmv, &full[si], 64, h, tok, b);
+      }
+      __syncwarp();
+    };
+    if (lane == 0) {
+      prefetch_tmap(&tmk);
+      prefetch_tmap(&tmv);
+    }
+    int issued = 0;
+    for (; issued < S && issued < nchunks; ++issued) fill_and_issue(issued);
+    int mmas = 0;  // state MMAs issued (chunks 0 .. mmas-1)
+    for (int u = 0; u < nchunks; ++u) {
+      const int s = u % S;
+      // refill the stage of chunk u - 1 as soon as its MMA has read it (early in prep(u))
+      if (u >= 1 && issued < nchunks) {
+        if (lane == 0) ok = mbar_wait(&mma_done[(u - 1) % S], ((u - 1) / S) & 1);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        fill_and_issue(issued++);
+      }
+      if (lane == 0) {
+        ok = mbar_wait(&prepped[s], (u / S) & 1);
+        if (ok) {
+          tc_fence_after();
+          uint8_t* sK = stages + s * L::kStageBytes;
+          uint8_t* sV = sK + kTcTile;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            tc_mma_ss(t_s, tc_desc_mn(sK, kk), tc_desc_mn(sV, kk), kIdState,
+                      (u == 0 && kk == 0) ? 0u : 1u);
+          tc_commit(&mma_done[s]);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      mmas = u + 1;
+    }
+    if (lane == 0) {
+      // the last MMA issued completes before TMEM is read or released
+      if (mmas > 0 && !mbar_wait(&mma_done[(mmas - 1) % S], ((mmas - 1) / S) & 1)) ok = false;
+      // every copy issued lands before the CTA's shared memory goes away (on the normal
+      // path the prep warps have consumed them all already)
+      for (int n = issued > S ? issued - S : 0; n < issued; ++n)
+        mbar_wait(&full[n % S], (n / S) & 1);
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+  } else {
+    TcRowRot rr;
+    tc_row_rot_init(rr, prow, pqd, inv_freq);
+    for (int u = 0; u < nchunks; ++u) {
+      const int s = u % S;
+      uint8_t* sK = stages + s * L::kStageBytes;
+      uint8_t* sV = sK + kTcTile;
+      ok = mbar_wait(&full[s], (u / S) & 1);
+      if (ok) tc_prep_kv_quarter(sK, sV, prow, pqd, p, ang_ring + (u % kStAngRing) * 32, rr);
+      fence_proxy_async_smem();
+      // a warp whose wait failed stops arriving; the producer's wait then runs out too
+      if (!__all_sync(0xffffffffu, ok)) break;
+      if (lane == 0) mbar_arrive(&prepped[s]);
     }
   }
-  if (!ok && tid == 0) {
-    // wind down: let the last issued copies land before the CTA's shared memory goes away
-    for (int u = issued > L::kStages ? issued - L::kStages : 0; u < issued; ++u)
-      mbar_wait(&full[u % L::kStages], (u / L::kStages) & 1);
+  ok = __syncthreads_and(ok);
+  tc_fence_after();
+  if (!producer && ok && nchunks > 0) {
+    float* dst = p.ws + ((size_t)bh * p.G + seg) * (128 * 128) + (size_t)trow * 128 + 32 * cg;
+    uint32_t r[32];
+    tc_ld32(t_s + lane_off + 32 * cg, r);
+    tc_wait_ld();
+#pragma unroll
+    for (int v4 = 0; v4 < 8; ++v4)
+      *reinterpret_cast<float4*>(dst + 4 * v4) =
+          make_float4(__uint_as_float(r[4 * v4]), __uint_as_float(r[4 * v4 + 1]),
+                      __uint_as_float(r[4 * v4 + 2]), __uint_as_float(r[4 * v4 + 3]));
   }
   tc_fence_before();
   __syncthreads();

@@ -185,7 +185,7 @@ sala_status sala_lightning_prefill(const void* q, const void* k, const void* v, 
     auto ka = lightning_state_kernel;
     auto kc = lightning_out_kernel;
     if (!set_smem(ka, TcSmem<true>::bytes) || !set_smem(kc, TcSmem<false>::bytes)) return SALA_ERR_CUDA;
-    ka<<<grid, kTcThreads, TcSmem<true>::bytes, st>>>(tk, tv, p);
+    ka<<<grid, kStThreads, TcSmem<true>::bytes, st>>>(tk, tv, p);
     SALA_CHECK_LAUNCH();
     lightning_scan_kernel<<<dim3(B * H, 16), 256, 0, st>>>(p.ws, state, p.G, init_zero);
     SALA_CHECK_LAUNCH();
@@ -308,7 +308,7 @@ sala_status sala_lightning_state(const void* k, const void* v, float* state, con
     p.eps = eps;
     auto ka = lightning_state_kernel;
     if (!set_smem(ka, TcSmem<true>::bytes)) return SALA_ERR_CUDA;
-    ka<<<(unsigned)(B * H * p.G), kTcThreads, TcSmem<true>::bytes, st>>>(tk, tv, p);
+    ka<<<(unsigned)(B * H * p.G), kStThreads, TcSmem<true>::bytes, st>>>(tk, tv, p);
     SALA_CHECK_LAUNCH();
     lightning_scan_kernel<<<dim3(B * H, 16), 256, 0, st>>>(p.ws, state, p.G, init_zero);
     SALA_CHECK_LAUNCH();
@@ -767,7 +767,7 @@ sala_status sala_lightning_prefill_noalloc(const void* q, const void* k, const v
   auto ka = lightning_state_kernel;
   auto kc = lightning_out_kernel;
   if (!set_smem(ka, TcSmem<true>::bytes) || !set_smem(kc, TcSmem<false>::bytes)) return SALA_ERR_CUDA;
-  ka<<<grid, kTcThreads, TcSmem<true>::bytes, st>>>(tk, tv, p);
+  ka<<<grid, kStThreads, TcSmem<true>::bytes, st>>>(tk, tv, p);
   SALA_CHECK_LAUNCH();
   lightning_scan_kernel<<<dim3(B * H, 16), 256, 0, st>>>(p.ws, state, p.G, init_zero);
   SALA_CHECK_LAUNCH();
