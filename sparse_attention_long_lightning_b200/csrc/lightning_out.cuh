@@ -34,54 +34,63 @@ constexpr int kLoPrepThreads = 256;   // warps 0-7
 constexpr int kLoConvThreads = 256;   // warps 8-15
 constexpr int kLoIssuer = kLoPrepThreads;  // first CONV thread issues MMAs and copies
 
+// Item of the per-chunk angle table that holds rotation pairs i and i + 1 (i even): the
+// two halves of a row read adjacent 16-byte words.
+__device__ __forceinline__ int lo_ang_item(int i) { return ((i & 31) >> 1) * 2 + (i >> 5); }
+
 // Normalise + rotate half of raw bf16 row r of the q and k tiles and convert it to fp16
 // in place.  Two consecutive lanes share a row: half hf owns rotation pairs i in
 // [32 hf, 32 hf + 32) (chunks 4hf..4hf+3 of both 64-column slabs).  Tiles are two
-// 64-column slabs of 128 rows x 128 bytes with the 128-byte swizzle.
+// 64-column slabs of 128 rows x 128 bytes with the 128-byte swizzle.  `ang` holds
+// (base angle, inv_freq) of pairs i, i + 1 at item lo_ang_item(i).  The tiles and the
+// table are in the kernel's __shared__ arrays: ordinary accesses, which the compiler
+// is free to schedule.
 __device__ __forceinline__ void lo_prep_qk_half(uint8_t* sQ, uint8_t* sK, int r, int hf,
-                                                const TcParams& p, const float2* ang_base) {
-  // shared-space accesses by address (the tiles are in shared memory)
-  const uint32_t q_s = smem_u32(sQ), k_s = smem_u32(sK), ang_s = smem_u32(ang_base);
-  uint4 bfx;
-  float ssq = 0.f, ssk = 0.f;
+                                                const TcParams& p, const float4* ang) {
+  auto ld = [](const uint8_t* base, uint32_t off) {
+    return *reinterpret_cast<const uint4*>(base + off);
+  };
+  auto st = [](uint8_t* base, uint32_t off, uint4 v) {
+    *reinterpret_cast<uint4*>(base + off) = v;
+  };
+  float ssq[2] = {0.f, 0.f}, ssk[2] = {0.f, 0.f};
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
     const int j = 4 * hf + (u & 3);
     const uint32_t a = (u >> 2) * kTcSlab + swz128(r, j);
     float f[8];
-    bf16x8_to_f32(lds128(k_s + a), f);
+    bf16x8_to_f32(ld(sK, a), f);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) ssk = fmaf(f[e], f[e], ssk);
-    bf16x8_to_f32(lds128(q_s + a), f);
+    for (int e = 0; e < 8; ++e) ssk[u & 1] = fmaf(f[e], f[e], ssk[u & 1]);
+    bf16x8_to_f32(ld(sQ, a), f);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) ssq = fmaf(f[e], f[e], ssq);
+    for (int e = 0; e < 8; ++e) ssq[u & 1] = fmaf(f[e], f[e], ssq[u & 1]);
   }
-  ssk += __shfl_xor_sync(0xffffffffu, ssk, 1);
-  ssq += __shfl_xor_sync(0xffffffffu, ssq, 1);
-  const float rk = rsqrtf(ssk * (1.0f / 128.0f) + p.eps);
-  const float rq = rsqrtf(ssq * (1.0f / 128.0f) + p.eps);
+  float sk = ssk[0] + ssk[1], sq = ssq[0] + ssq[1];
+  sk += __shfl_xor_sync(0xffffffffu, sk, 1);
+  sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+  const float rk = rsqrtf(sk * (1.0f / 128.0f) + p.eps);
+  const float rq = rsqrtf(sq * (1.0f / 128.0f) + p.eps);
   const float two_pi = 6.28318530717958647692f, inv_two_pi = 0.15915494309189533577f;
 #pragma unroll
   for (int jj = 0; jj < 4; ++jj) {
     const int j = 4 * hf + jj;
     const uint32_t alo = swz128(r, j), ahi = kTcSlab + swz128(r, j);
     float klo[8], khi[8], qlo[8], qhi[8];
-    bf16x8_to_f32(lds128(k_s + alo), klo);
-    bf16x8_to_f32(lds128(k_s + ahi), khi);
-    bf16x8_to_f32(lds128(q_s + alo), qlo);
-    bf16x8_to_f32(lds128(q_s + ahi), qhi);
+    bf16x8_to_f32(ld(sK, alo), klo);
+    bf16x8_to_f32(ld(sK, ahi), khi);
+    bf16x8_to_f32(ld(sQ, alo), qlo);
+    bf16x8_to_f32(ld(sQ, ahi), qhi);
+    float4 bb;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const int i = 8 * j + e;  // rotation pair (i, i + 64)
-      // (base angle, inv_freq) of pairs i, i + 1: one shared 16-byte load per two pairs
-      if ((e & 1) == 0) bfx = lds128(ang_s + 8 * i);
-      const float2 bf = (e & 1) ? make_float2(__uint_as_float(bfx.z), __uint_as_float(bfx.w))
-                                : make_float2(__uint_as_float(bfx.x), __uint_as_float(bfx.y));
+      if ((e & 1) == 0) bb = ang[lo_ang_item(i)];
       // angle = (chunk base angle, reduced in fp64) + r * inv_freq_i, re-reduced in fp32
-      float ang = fmaf((float)r, bf.y, bf.x);
-      ang = fmaf(-rintf(ang * inv_two_pi), two_pi, ang);
+      float ang_i = (e & 1) ? fmaf((float)r, bb.w, bb.z) : fmaf((float)r, bb.y, bb.x);
+      ang_i = fmaf(-rintf(ang_i * inv_two_pi), two_pi, ang_i);
       float sn, cs;
-      __sincosf(ang, &sn, &cs);
+      __sincosf(ang_i, &sn, &cs);
       const float wk0 = p.kw ? __ldg(p.kw + i) : 1.f, wk1 = p.kw ? __ldg(p.kw + i + 64) : 1.f;
       const float wq0 = p.qw ? __ldg(p.qw + i) : 1.f, wq1 = p.qw ? __ldg(p.qw + i + 64) : 1.f;
       const float k0 = klo[e] * rk * wk0, k1 = khi[e] * rk * wk1;
@@ -91,23 +100,22 @@ __device__ __forceinline__ void lo_prep_qk_half(uint8_t* sQ, uint8_t* sK, int r,
       qlo[e] = q0 * cs - q1 * sn;
       qhi[e] = q1 * cs + q0 * sn;
     }
-    sts128(k_s + alo, f32x8_to_f16(klo));
-    sts128(k_s + ahi, f32x8_to_f16(khi));
-    sts128(q_s + alo, f32x8_to_f16(qlo));
-    sts128(q_s + ahi, f32x8_to_f16(qhi));
+    st(sK, alo, f32x8_to_f16(klo));
+    st(sK, ahi, f32x8_to_f16(khi));
+    st(sQ, alo, f32x8_to_f16(qlo));
+    st(sQ, ahi, f32x8_to_f16(qhi));
   }
 }
 
 // Half of the v row (chunks 8hf..8hf+7: slab hf) to fp16 in place.
 __device__ __forceinline__ void lo_prep_v_half(uint8_t* sV, int r, int hf) {
-  const uint32_t v_s = smem_u32(sV);
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
-    const uint32_t a = hf * kTcSlab + swz128(r, u);
-    uint4 x = lds128(v_s + a);
+    uint4* a = reinterpret_cast<uint4*>(sV + hf * kTcSlab + swz128(r, u));
+    uint4 x = *a;
     x.x = bf16x2_to_f16x2(x.x); x.y = bf16x2_to_f16x2(x.y);
     x.z = bf16x2_to_f16x2(x.z); x.w = bf16x2_to_f16x2(x.w);
-    sts128(v_s + a, x);
+    *a = x;
   }
 }
 
@@ -151,8 +159,8 @@ lightning_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
   constexpr uint32_t kIdPV = umma_idesc_f16(128, 128, false, true);
 
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  // 1024-byte aligned, derived from the __shared__ array so it stays a shared pointer
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* stages = smem;
   uint8_t* sop = smem + 2 * L::kStageBytes;
   uint8_t* misc = sop + L::kSop;
@@ -168,8 +176,8 @@ lightning_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
   volatile int* conv_abort = reinterpret_cast<volatile int*>(misc + 108);
   float* red = reinterpret_cast<float*>(misc + 112);           // [16]
   double* inv_freq = reinterpret_cast<double*>(misc + 192);    // [64]
-  float2* ang_tab = reinterpret_cast<float2*>(misc + 704);     // [2][64]: (base angle, inv_freq)
-  static_assert(704 + 2 * 64 * 8 <= L::kMisc, "misc area");
+  // [2][32]: (base angle, inv_freq) of rotation pairs i, i + 1 at item lo_ang_item(i)
+  __shared__ float4 ang_tab[2 * 32];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool is_prep = tid < kLoPrepThreads;
@@ -208,11 +216,14 @@ lightning_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
 
   // base angle of each rotation pair at the first token of chunk u (fp64 reduction)
   auto fill_angles = [&](int u) {
-    if (tid < 64) {
-      const double a = (double)(p.pos0 + (int64_t)(c_begin + u) * kTcC) * inv_freq[tid];
+    if (tid < 32) {  // pairs 2 tid, 2 tid + 1
+      const double t0 = (double)(p.pos0 + (int64_t)(c_begin + u) * kTcC);
       const double two_pi = 6.283185307179586476925286766559;
-      const double red_a = a - rint(a * (1.0 / two_pi)) * two_pi;
-      ang_tab[(u & 1) * 64 + tid] = make_float2((float)red_a, (float)inv_freq[tid]);
+      const double a0 = t0 * inv_freq[2 * tid], a1 = t0 * inv_freq[2 * tid + 1];
+      const double r0 = a0 - rint(a0 * (1.0 / two_pi)) * two_pi;
+      const double r1 = a1 - rint(a1 * (1.0 / two_pi)) * two_pi;
+      ang_tab[(u & 1) * 32 + lo_ang_item(2 * tid)] =
+          make_float4((float)r0, (float)inv_freq[2 * tid], (float)r1, (float)inv_freq[2 * tid + 1]);
     }
   };
   // q/k of chunk u (free once the score/inter/state MMAs of chunk u-2 are done) and v of
@@ -300,7 +311,7 @@ lightning_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
       const int s = u & 1;
       uint8_t* st = stages + s * L::kStageBytes;
       fail |= !mbar_wait(&full_qk[s], (u >> 1) & 1);
-      if (!fail) lo_prep_qk_half(st, st + kTcTile, prow, phf, p, ang_tab + s * 64);
+      if (!fail) lo_prep_qk_half(st, st + kTcTile, prow, phf, p, ang_tab + s * 32);
       fail |= !mbar_wait(&full_v[s], (u >> 1) & 1);
       if (!fail) lo_prep_v_half(st + 2 * kTcTile, prow, phf);
       fence_proxy_async_smem();

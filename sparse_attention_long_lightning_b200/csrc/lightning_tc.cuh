@@ -40,8 +40,12 @@ struct TcSmem {
   static constexpr int kStages = kStateOnly ? 3 : 2;
   static constexpr int kStageBytes = (kStateOnly ? 2 : 3) * kTcTile;
   static constexpr int kSop = kStateOnly ? 0 : kTcTile;
-  static constexpr int kMisc = 2048;
+  // barriers, TMEM slot, inv_freq and scratch (< 704 bytes used).  The per-chunk angle
+  // tables are static __shared__ arrays of the kernels (4 KiB state pass, 1 KiB output
+  // pass) and count against the same 232448-byte per-block limit.
+  static constexpr int kMisc = 1024;
   static constexpr size_t bytes = 1024 /*alignment slack*/ + size_t(kStages) * kStageBytes + kSop + kMisc;
+  static_assert(bytes + (kStateOnly ? 4096 : 1024) <= 232448, "shared memory per block");
   static constexpr uint32_t kTmemCols = kStateOnly ? 128 : 512;
 };
 
@@ -122,15 +126,20 @@ __device__ __forceinline__ int tc_ang_item(int i) { return ((i & 15) >> 1) * 4 +
 __device__ __forceinline__ void tc_prep_kv_quarter(uint8_t* sK, uint8_t* sV, int r, int qd,
                                                    const TcParams& p, const float4* cs_tab,
                                                    const TcRowRot& rr) {
-  // shared-space accesses by address (the tiles are in shared memory)
-  const uint32_t k_s = smem_u32(sK), v_s = smem_u32(sV);
+  // ordinary 16-byte accesses: sK and sV point into the kernel's __shared__ array, so these
+  // are shared-memory instructions the compiler is free to schedule
+  auto ld = [](const uint8_t* base, uint32_t off) {
+    return *reinterpret_cast<const uint4*>(base + off);
+  };
+  auto st = [](uint8_t* base, uint32_t off, uint4 v) {
+    *reinterpret_cast<uint4*>(base + off) = v;
+  };
   float ss[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const int j = 2 * qd + (u & 1);
-    const uint32_t a = (u >> 1) * kTcSlab + swz128(r, j);
     float f[8];
-    bf16x8_to_f32(lds128(k_s + a), f);
+    bf16x8_to_f32(ld(sK, (u >> 1) * kTcSlab + swz128(r, j)), f);
 #pragma unroll
     for (int e = 0; e < 8; ++e) ss[u] = fmaf(f[e], f[e], ss[u]);
   }
@@ -143,8 +152,8 @@ __device__ __forceinline__ void tc_prep_kv_quarter(uint8_t* sK, uint8_t* sV, int
     const int j = 2 * qd + jj;
     const uint32_t alo = swz128(r, j), ahi = kTcSlab + swz128(r, j);
     float klo[8], khi[8];
-    bf16x8_to_f32(lds128(k_s + alo), klo);
-    bf16x8_to_f32(lds128(k_s + ahi), khi);
+    bf16x8_to_f32(ld(sK, alo), klo);
+    bf16x8_to_f32(ld(sK, ahi), khi);
     float4 cb;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
@@ -165,17 +174,17 @@ __device__ __forceinline__ void tc_prep_kv_quarter(uint8_t* sK, uint8_t* sV, int
       klo[e] = fmaf(k0, cs, -k1 * sn);
       khi[e] = fmaf(k1, cs, k0 * sn);
     }
-    sts128(k_s + alo, f32x8_to_f16(klo));
-    sts128(k_s + ahi, f32x8_to_f16(khi));
+    st(sK, alo, f32x8_to_f16(klo));
+    st(sK, ahi, f32x8_to_f16(khi));
   }
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const int cj = 4 * qd + u;
     const uint32_t a = (cj >> 3) * kTcSlab + swz128(r, cj & 7);
-    uint4 x = lds128(v_s + a);
+    uint4 x = ld(sV, a);
     x.x = bf16x2_to_f16x2(x.x); x.y = bf16x2_to_f16x2(x.y);
     x.z = bf16x2_to_f16x2(x.z); x.w = bf16x2_to_f16x2(x.w);
-    sts128(v_s + a, x);
+    st(sV, a, x);
   }
 }
 
@@ -210,8 +219,8 @@ lightning_state_kernel(const __grid_constant__ CUtensorMap tmk,
   constexpr int kPrepWarps = kTcThreads / 32;
 
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  // 1024-byte aligned, derived from the __shared__ array so it stays a shared pointer
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* stages = smem;
   uint8_t* misc = stages + S * L::kStageBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(misc);      // [S]: the stage's chunk landed
