@@ -76,34 +76,39 @@ __device__ __forceinline__ void lo_prep_qk_half(uint8_t* sQ, uint8_t* sK, int r,
   for (int jj = 0; jj < 4; ++jj) {
     const int j = 4 * hf + jj;
     const uint32_t alo = swz128(r, j), ahi = kTcSlab + swz128(r, j);
-    float klo[8], khi[8], qlo[8], qhi[8];
-    bf16x8_to_f32(ld(sK, alo), klo);
-    bf16x8_to_f32(ld(sK, ahi), khi);
-    bf16x8_to_f32(ld(sQ, alo), qlo);
-    bf16x8_to_f32(ld(sQ, ahi), qhi);
-    float4 bb;
+    // cos, sin of the 8 pairs' angles first (shared by q and k), then k, then q: fewer
+    // values live at once
+    float cs[8], sn[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int i = 8 * j + e;  // rotation pair (i, i + 64)
-      if ((e & 1) == 0) bb = ang[lo_ang_item(i)];
-      // angle = (chunk base angle, reduced in fp64) + r * inv_freq_i, re-reduced in fp32
-      float ang_i = (e & 1) ? fmaf((float)r, bb.w, bb.z) : fmaf((float)r, bb.y, bb.x);
-      ang_i = fmaf(-rintf(ang_i * inv_two_pi), two_pi, ang_i);
-      float sn, cs;
-      __sincosf(ang_i, &sn, &cs);
-      const float wk0 = p.kw ? __ldg(p.kw + i) : 1.f, wk1 = p.kw ? __ldg(p.kw + i + 64) : 1.f;
-      const float wq0 = p.qw ? __ldg(p.qw + i) : 1.f, wq1 = p.qw ? __ldg(p.qw + i + 64) : 1.f;
-      const float k0 = klo[e] * rk * wk0, k1 = khi[e] * rk * wk1;
-      const float q0 = qlo[e] * rq * wq0, q1 = qhi[e] * rq * wq1;
-      klo[e] = k0 * cs - k1 * sn;
-      khi[e] = k1 * cs + k0 * sn;
-      qlo[e] = q0 * cs - q1 * sn;
-      qhi[e] = q1 * cs + q0 * sn;
+    for (int e2 = 0; e2 < 4; ++e2) {
+      const float4 bb = ang[lo_ang_item(8 * j + 2 * e2)];
+#pragma unroll
+      for (int o = 0; o < 2; ++o) {
+        // angle = (chunk base angle, reduced in fp64) + r * inv_freq_i, re-reduced in fp32
+        float a = o ? fmaf((float)r, bb.w, bb.z) : fmaf((float)r, bb.y, bb.x);
+        a = fmaf(-rintf(a * inv_two_pi), two_pi, a);
+        __sincosf(a, &sn[2 * e2 + o], &cs[2 * e2 + o]);
+      }
     }
-    st(sK, alo, f32x8_to_f16(klo));
-    st(sK, ahi, f32x8_to_f16(khi));
-    st(sQ, alo, f32x8_to_f16(qlo));
-    st(sQ, ahi, f32x8_to_f16(qhi));
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {  // t = 0: k, t = 1: q
+      uint8_t* base = t ? sQ : sK;
+      const float rs = t ? rq : rk;
+      const float* w = t ? p.qw : p.kw;
+      float xlo[8], xhi[8];
+      bf16x8_to_f32(ld(base, alo), xlo);
+      bf16x8_to_f32(ld(base, ahi), xhi);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int i = 8 * j + e;  // rotation pair (i, i + 64)
+        const float w0 = w ? __ldg(w + i) : 1.f, w1 = w ? __ldg(w + i + 64) : 1.f;
+        const float x0 = xlo[e] * rs * w0, x1 = xhi[e] * rs * w1;
+        xlo[e] = x0 * cs[e] - x1 * sn[e];
+        xhi[e] = x1 * cs[e] + x0 * sn[e];
+      }
+      st(base, alo, f32x8_to_f16(xlo));
+      st(base, ahi, f32x8_to_f16(xhi));
+    }
   }
 }
 
