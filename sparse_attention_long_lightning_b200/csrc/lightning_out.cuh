@@ -112,11 +112,12 @@ __device__ __forceinline__ void lo_prep_qk_half(uint8_t* sQ, uint8_t* sK, int r,
   }
 }
 
-// Half of the v row (chunks 8hf..8hf+7: slab hf) to fp16 in place.
+// Half of the v row (slab hf) to fp16 in place; half 1 runs four chunks out of step so
+// the two lanes of a row hit different bank groups.
 __device__ __forceinline__ void lo_prep_v_half(uint8_t* sV, int r, int hf) {
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
-    uint4* a = reinterpret_cast<uint4*>(sV + hf * kTcSlab + swz128(r, u));
+    uint4* a = reinterpret_cast<uint4*>(sV + hf * kTcSlab + swz128(r, (u + 4 * hf) & 7));
     uint4 x = *a;
     x.x = bf16x2_to_f16x2(x.x); x.y = bf16x2_to_f16x2(x.y);
     x.z = bf16x2_to_f16x2(x.z); x.w = bf16x2_to_f16x2(x.w);

@@ -115,7 +115,7 @@ __device__ __forceinline__ void tc_row_rot_init(TcRowRot& rr, int r, int qd, con
 // Normalise + rotate a quarter of raw bf16 row r of the k tile and convert it, and a
 // quarter of the v row, to fp16 in place.  Four consecutive lanes share a row: quarter
 // qd owns rotation pairs i in [16 qd, 16 qd + 16) (chunks 2qd, 2qd+1 of both 64-column
-// slabs) and v chunks 4qd..4qd+3.  Tiles are two 64-column slabs of 128 rows x 128
+// slabs) and four v chunks.  Tiles are two 64-column slabs of 128 rows x 128
 // bytes with the 128-byte swizzle.  `cs_tab` (a static shared array, read with ordinary
 // loads the compiler can schedule) holds the chunk's (cos B_i, sin B_i, cos B_i+1,
 // sin B_i+1) for even i at item (i mod 16) / 2 * 4 + i / 16, so the four quarters of a
@@ -177,10 +177,12 @@ __device__ __forceinline__ void tc_prep_kv_quarter(uint8_t* sK, uint8_t* sV, int
     st(sK, alo, f32x8_to_f16(klo));
     st(sK, ahi, f32x8_to_f16(khi));
   }
+  // v: quarter qd converts chunks 4 (qd & 1) .. +3 of slab qd >> 1, the slab-1 quarters
+  // two chunks out of step, so the 8 lanes of a quarter-warp hit 8 different bank groups
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
-    const int cj = 4 * qd + u;
-    const uint32_t a = (cj >> 3) * kTcSlab + swz128(r, cj & 7);
+    const int c = 4 * (qd & 1) + ((u + 2 * (qd >> 1)) & 3);
+    const uint32_t a = (qd >> 1) * kTcSlab + swz128(r, c);
     uint4 x = ld(sV, a);
     x.x = bf16x2_to_f16x2(x.x); x.y = bf16x2_to_f16x2(x.y);
     x.z = bf16x2_to_f16x2(x.z); x.w = bf16x2_to_f16x2(x.w);
