@@ -431,8 +431,8 @@ def main():
     dev = torch.device("cuda", torch.cuda.current_device())
     hbm, tf_burst, tf_sust, peak_src = _peaks()
     T = args.T
-    share = args.share_buffers or T > 131072
-    layers = make_layers(T, dev, seed=1005 + 1000 * rank, share=share)
+    shared_bufs = args.share_buffers or T > 131072
+    layers = make_layers(T, dev, seed=1005 + 1000 * rank, share=shared_bufs)
     gb = resident_bytes(layers) / 1e9
     stream = torch.cuda.current_stream()
 
@@ -492,7 +492,7 @@ def main():
     # ncu capture of this command at T=131072 with the current kernels (the sparse
     # kernel's own launch; Lightning = state pass + scan + output pass; selection =
     # block means + fused kernel).  Re-measure whenever one of those kernels changes.
-    ncu_traffic = {"attn": 9.16e9, "sel": 1.17e9} if T == 131072 else {}
+    ncu_traffic = {"attn": 8.91e9, "sel": 1.17e9} if T == 131072 else {}
     share = {k: n_ops[k] * op_ms[k] for k in op_ms}
     dom = max(share, key=share.get)
     if dom == "attn":
@@ -523,7 +523,7 @@ def main():
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": f"inputs (~{gb:.0f} GB resident) far exceed L2; no flush",
                        "buffers": ("one set per layer type, shared by the layers of that type"
-                                   if share else "fresh seeded inputs per layer"),
+                                   if shared_bufs else "fresh seeded inputs per layer"),
                        "chunk": CHUNK, "block": BLOCK, "topk": TOPK, "n_init": N_INIT,
                        "n_local": N_LOCAL},
             "roofline": roof, "components": comps, "clocks": clk.summary()}
