@@ -101,10 +101,15 @@ __device__ __forceinline__ void lo_prep_qk_half(uint8_t* sQ, uint8_t* sK, int r,
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const int i = 8 * j + e;  // rotation pair (i, i + 64)
-        const float w0 = w ? __ldg(w + i) : 1.f, w1 = w ? __ldg(w + i + 64) : 1.f;
-        const float x0 = xlo[e] * rs * w0, x1 = xhi[e] * rs * w1;
-        xlo[e] = x0 * cs[e] - x1 * sn[e];
-        xhi[e] = x1 * cs[e] + x0 * sn[e];
+        // the row's RMS scale rides on cos/sin; the optional weights on the elements
+        const float c = cs[e] * rs, sg = sn[e] * rs;
+        float x0 = xlo[e], x1 = xhi[e];
+        if (w) {
+          x0 *= __ldg(w + i);
+          x1 *= __ldg(w + i + 64);
+        }
+        xlo[e] = fmaf(x0, c, -x1 * sg);
+        xhi[e] = fmaf(x1, c, x0 * sg);
       }
       st(base, alo, f32x8_to_f16(xlo));
       st(base, ahi, f32x8_to_f16(xhi));
