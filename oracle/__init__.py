@@ -60,11 +60,13 @@ def _load():
         lib.oracle_block_means.argtypes = [_dp, i, i, i, i, i, _dp]
         lib.oracle_sparse_select.argtypes = [
             _dp, _dp, i, i, i, i, i, i, i, i, i, _i64p, i, _i32p, _dp, _dp, i]
+        lib.oracle_sparse_select_mode.argtypes = [
+            _dp, _dp, i, i, i, i, i, i, i, i, i, _i64p, i, _i32p, _dp, _dp, i, i]
         lib.oracle_attention.argtypes = [
             _dp, _dp, _dp, _dp, _i32p, i, i, i, i, i, i, i, d, _i64p, i, _dp]
         for f in ("oracle_qk_prep", "oracle_lightning_recurrent", "oracle_lightning_quadratic",
                   "oracle_lightning_chunked", "oracle_lightning_decode", "oracle_block_means",
-                  "oracle_sparse_select", "oracle_attention"):
+                  "oracle_sparse_select", "oracle_sparse_select_mode", "oracle_attention"):
             getattr(lib, f).restype = None
         _lib = lib
     return _lib
@@ -165,11 +167,19 @@ def block_means(k, blk=64):
     return out
 
 
+SCORE_MODES = {"group_sum": 0, "head_softmax": 1}
+
+
 def sparse_select(q, k, *, blk=64, topk=64, n_init=1, n_local=2, rows=None, T=None,
-                  want_scores=False):
+                  want_scores=False, score="group_sum"):
     """Block selection.  q: [B, nrows, Hq, D] (rows listed in `rows`, else all T);
     k: [B, T, Hkv, D].  Returns (idx [B,Hkv,nrows,n_sel] int32, gap [B,Hkv,nrows])
-    and, with want_scores, candidate scores [B,Hkv,nrows,max_cand] (NaN = none)."""
+    and, with want_scores, candidate scores [B,Hkv,nrows,max_cand] (NaN = none).
+    score="group_sum": (1/sqrt(D)) sum over the group's heads of q_h . Kbar_j;
+    score="head_softmax": each head's scaled dot products softmax-normalised over the
+    row's candidates, then summed over the group's heads."""
+    if score not in SCORE_MODES:
+        raise ValueError(f"score must be one of {sorted(SCORE_MODES)}")
     lib = _load()
     B, nr, Hq, D = np.shape(q)
     _, Tk, Hkv, _ = np.shape(k)
@@ -183,9 +193,10 @@ def sparse_select(q, k, *, blk=64, topk=64, n_init=1, n_local=2, rows=None, T=No
     gap = np.zeros((B, Hkv, nrows))
     max_cand = max(1, T // blk)
     sc = np.zeros((B, Hkv, nrows, max_cand)) if want_scores else None
-    lib.oracle_sparse_select(qp, kp, B, T, Hq, Hkv, D, blk, topk, n_init, n_local, rp, nrows,
-                             idx.ctypes.data_as(_i32p), gap.ctypes.data_as(_dp),
-                             sc.ctypes.data_as(_dp) if sc is not None else None, max_cand)
+    lib.oracle_sparse_select_mode(qp, kp, B, T, Hq, Hkv, D, blk, topk, n_init, n_local, rp,
+                                  nrows, idx.ctypes.data_as(_i32p), gap.ctypes.data_as(_dp),
+                                  sc.ctypes.data_as(_dp) if sc is not None else None, max_cand,
+                                  SCORE_MODES[score])
     return (idx, gap, sc) if want_scores else (idx, gap)
 
 

@@ -355,6 +355,46 @@ static int block_scores(const double *q_row, const double *kbar_b, int nb, int H
 }
 
 /*
+ * Per-head softmax-normalised block scores (the selection variant that scores a
+ * block by how much of each head's attention it would draw): for each query head h
+ * of the group, s_{h,j} = (1/sqrt(D)) q[t, h] . kbar[j, hk] over the same candidate
+ * set as block_scores, p_{h,j} = exp(s_{h,j}) / sum_{j'} exp(s_{h,j'}) (softmax over
+ * the candidates, computed with the per-head maximum subtracted), and
+ *   score_j = sum_{h in group(hk)} p_{h,j}.
+ * Each head's p sums to 1, so a row's scores sum to the group size.
+ */
+static int block_scores_head_softmax(const double *q_row, const double *kbar_b, int nb, int Hq,
+                                     int Hkv, int D, int blk, int n_init, int n_local, int64_t t,
+                                     int hk, cand_t *out)
+{
+    int grp = Hq / Hkv;
+    int64_t c = t / blk;
+    int64_t lo = n_init, hi = c - n_local;
+    if (hi > nb - 1) hi = nb - 1; /* only complete blocks have a representative */
+    int n = hi >= lo ? (int)(hi - lo + 1) : 0;
+    double scale = 1.0 / sqrt((double)D);
+    double *s = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+    for (int e = 0; e < n; ++e) {
+        out[e].j = (int)(lo + e);
+        out[e].score = 0.0;
+    }
+    for (int h = hk * grp; h < (hk + 1) * grp; ++h) {
+        double m = -INFINITY, l = 0.0;
+        for (int e = 0; e < n; ++e) {
+            double acc = 0.0;
+            for (int d = 0; d < D; ++d)
+                acc += q_row[(int64_t)h * D + d] * kbar_b[((int64_t)(lo + e) * Hkv + hk) * D + d];
+            s[e] = acc * scale;
+            if (s[e] > m) m = s[e];
+        }
+        for (int e = 0; e < n; ++e) l += exp(s[e] - m);
+        for (int e = 0; e < n; ++e) out[e].score += exp(s[e] - m) / l;
+    }
+    free(s);
+    return n;
+}
+
+/*
  * Block selection for query rows: top-`topk` candidates by score (ties -> smaller
  * block index), united with the init blocks {0..n_init-1} and the local window
  * {c-n_local+1..c} (clipped to [0, c]), sorted ascending, padded with -1 to
@@ -367,10 +407,26 @@ static int block_scores(const double *q_row, const double *kbar_b, int nb, int H
  * scores_out: [B, Hkv, nrows, max_cand] or NULL -- candidate scores by block
  * index offset (entry j - n_init), NaN where not a candidate.
  */
+void oracle_sparse_select_mode(const double *q, const double *k, int B, int T, int Hq, int Hkv,
+                               int D, int blk, int topk, int n_init, int n_local,
+                               const int64_t *rows, int nrows, int32_t *idx, double *gap,
+                               double *scores_out, int max_cand, int mode);
+
 void oracle_sparse_select(const double *q, const double *k, int B, int T, int Hq, int Hkv,
                           int D, int blk, int topk, int n_init, int n_local,
                           const int64_t *rows, int nrows, int32_t *idx, double *gap,
                           double *scores_out, int max_cand)
+{
+    oracle_sparse_select_mode(q, k, B, T, Hq, Hkv, D, blk, topk, n_init, n_local, rows, nrows,
+                              idx, gap, scores_out, max_cand, 0);
+}
+
+/* mode 0: group-summed scores (block_scores); mode 1: per-head softmax-normalised
+ * scores summed over the group (block_scores_head_softmax). */
+void oracle_sparse_select_mode(const double *q, const double *k, int B, int T, int Hq, int Hkv,
+                               int D, int blk, int topk, int n_init, int n_local,
+                               const int64_t *rows, int nrows, int32_t *idx, double *gap,
+                               double *scores_out, int max_cand, int mode)
 {
     int nb = T / blk;
     int n_sel = n_init + topk + n_local;
@@ -384,9 +440,13 @@ void oracle_sparse_select(const double *q, const double *k, int B, int T, int Hq
                 int64_t c = t / blk;
                 cand_t *cands = (cand_t *)malloc(sizeof(cand_t) * (size_t)(c + 1));
                 int *sel = (int *)malloc(sizeof(int) * (size_t)(n_sel + 1));
-                int n = block_scores(q + IDX4(b, r, 0, 0, nrows, Hq, D),
-                                     kbar + (int64_t)b * nb * Hkv * D, nb, Hq, Hkv, D, blk,
-                                     n_init, n_local, t, hk, cands);
+                int n = mode == 1
+                            ? block_scores_head_softmax(q + IDX4(b, r, 0, 0, nrows, Hq, D),
+                                                        kbar + (int64_t)b * nb * Hkv * D, nb, Hq,
+                                                        Hkv, D, blk, n_init, n_local, t, hk, cands)
+                            : block_scores(q + IDX4(b, r, 0, 0, nrows, Hq, D),
+                                           kbar + (int64_t)b * nb * Hkv * D, nb, Hq, Hkv, D, blk,
+                                           n_init, n_local, t, hk, cands);
                 if (scores_out) {
                     double *so = scores_out + (((int64_t)b * Hkv + hk) * nrows + r) * max_cand;
                     for (int e = 0; e < max_cand; ++e) so[e] = NAN;

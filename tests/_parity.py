@@ -44,14 +44,15 @@ def raw_rel_err(out, ref) -> float:
     return float(np.abs(out - ref).max() / max(np.sqrt(np.mean(ref * ref)), 1e-300))
 
 
-def check_index_sets(idx_gpu, idx_ref, gap):
+def check_index_sets(idx_gpu, idx_ref, gap, tie_band=None):
     """Bit-exact per row, except rows whose oracle gap between the topk-th and
-    (topk+1)-th candidate score is < 1e-4: there the chosen sets may differ only
-    by near-tied members (same size, same forced blocks, every row sorted)."""
+    (topk+1)-th candidate score is below the tie band (1e-4, or `tie_band`, a scalar
+    or per-row array): there the chosen sets may differ only by near-tied members
+    (same size, same forced blocks, every row sorted)."""
     idx_gpu = np.asarray(idx_gpu)
     idx_ref = np.asarray(idx_ref)
     same = (idx_gpu == idx_ref).all(axis=-1)
-    tie = gap < GAP_TIE
+    tie = gap < (GAP_TIE if tie_band is None else tie_band)
     bad = ~same & ~tie
     assert not bad.any(), f"{int(bad.sum())} rows differ without a near-tie"
     # structural validity of the tied rows

@@ -500,3 +500,72 @@ def test_decode_selection_bruteforce():
                           set(range(max(n_init, c - n_local + 1), c + 1)))
             got = idx[b, hk][idx[b, hk] >= 0].tolist()
             assert got == want, (b, hk)
+
+
+# ---------------------------------------------------------------- per-head softmax selection
+def test_head_softmax_scores_sum_to_group_size():
+    """Each head's softmax over a row's candidates sums to 1, so a row's scores sum to
+    the number of heads in the group (a wrong normalisation axis breaks this)."""
+    rng = np.random.default_rng(21)
+    blk, D, Hq, Hkv = 8, 16, 8, 2
+    T = blk * 40 + 5
+    q, k = rng.standard_normal((1, T, Hq, D)), rng.standard_normal((1, T, Hkv, D))
+    rows = [blk * 5, blk * 17 + 3, T - 1]
+    _, _, sc = oracle.sparse_select(q[:, rows], k, blk=blk, topk=4, rows=rows, want_scores=True,
+                                    score="head_softmax")
+    for r in range(len(rows)):
+        for hk in range(Hkv):
+            assert np.isclose(np.nansum(sc[0, hk, r]), Hq // Hkv, rtol=1e-12)
+
+
+def test_head_softmax_one_head_is_softmax_of_group_scores():
+    """With one query head per KV head the score is the softmax (scipy) of the
+    group-sum score over the row's candidates, and the choice is the same."""
+    from scipy.special import softmax
+
+    rng = np.random.default_rng(22)
+    blk, D, H = 8, 16, 3
+    T = blk * 30 + 7
+    q, k = rng.standard_normal((1, T, H, D)), rng.standard_normal((1, T, H, D))
+    rows = list(range(blk * 3, T, 13))
+    i0, _, s0 = oracle.sparse_select(q[:, rows], k, blk=blk, topk=5, rows=rows, want_scores=True)
+    i1, _, s1 = oracle.sparse_select(q[:, rows], k, blk=blk, topk=5, rows=rows, want_scores=True,
+                                     score="head_softmax")
+    for hk in range(H):
+        for r in range(len(rows)):
+            m = ~np.isnan(s0[0, hk, r])
+            if m.any():
+                assert np.allclose(s1[0, hk, r][m], softmax(s0[0, hk, r][m]), rtol=1e-12,
+                                   atol=1e-15)
+    assert np.array_equal(i0, i1)
+
+
+def test_head_softmax_planted_closed_form():
+    """Every candidate block's keys are zero except block J, whose keys all equal u, and
+    query head h is alpha_h * u: s_{h,J} = a_h = alpha_h |u|^2 / sqrt(D), 0 elsewhere, so
+    score_J = sum_h e^{a_h} / (e^{a_h} + n - 1) and every other candidate scores
+    sum_h 1 / (e^{a_h} + n - 1) (n candidates)."""
+    blk, D, Hq = 8, 8, 4
+    nb = 14
+    T = blk * nb
+    u = RNG.standard_normal(D) * 0.5
+    alpha = np.array([0.3, -0.7, 1.1, 0.05])
+    J = 6
+    k = np.zeros((1, T, 1, D))
+    k[0, J * blk:(J + 1) * blk, 0] = u
+    q = np.zeros((1, T, Hq, D))
+    for h in range(Hq):
+        q[0, :, h] = alpha[h] * u
+    t = T - 1
+    _, _, sc = oracle.sparse_select(q[:, [t]], k, blk=blk, topk=3, rows=[t], want_scores=True,
+                                    score="head_softmax")
+    c = t // blk
+    n = c - 2  # candidates 1 .. c - 2
+    a = alpha * (u @ u) / math.sqrt(D)
+    want_J = np.sum(np.exp(a) / (np.exp(a) + n - 1))
+    want_other = np.sum(1.0 / (np.exp(a) + n - 1))
+    row = sc[0, 0, 0]
+    assert np.isclose(row[J - 1], want_J, rtol=1e-12)
+    for j in range(1, c - 1):
+        if j != J:
+            assert np.isclose(row[j - 1], want_other, rtol=1e-12)
