@@ -185,6 +185,34 @@ sala_status sala_sparse_select(const void *q, const void *k, int B, int T, int H
                                sala_dtype dt, void *stream);
 
 /*
+ * Block selection, per-head softmax-normalised variant.  The pages leave the
+ * selection score open; this variant scores a candidate block by the attention
+ * share each query head of the group would give its representative key:
+ *   s_{h,j}  = (1/sqrt(D)) q_{t,h} . Kbar_j           (h in group(hk))
+ *   p_{h,j}  = exp(s_{h,j}) / sum_{j'} exp(s_{h,j'})   (softmax over the row's
+ *              candidates n_init <= j' <= c - n_local, complete blocks only)
+ *   score_j  = sum_{h in group(hk)} p_{h,j}
+ * Everything else (candidates, top `topk` with ties -> smaller j, init blocks,
+ * local window, sorted, -1 padded) is as in sala_sparse_select.  Each head's p sums
+ * to 1, so a row's scores sum to G; with G = 1 the choice equals sala_sparse_select's.
+ * fp32 arithmetic (expf, IEEE division): a decision between two scores closer than
+ * about 1e-5 of their size may differ from exact arithmetic.
+ *
+ *   arguments, layouts and ownership as sala_sparse_select; ws of
+ *   >= sala_sparse_select_head_softmax_workspace() bytes (block means and a score
+ *   scratch of at most 1 GiB); G = Hq / Hkv must be 1, 2, 4, 8, 16 or 32.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
+ */
+size_t sala_sparse_select_head_softmax_workspace(int B, int T, int Hq, int Hkv, int D,
+                                                 int block);
+
+sala_status sala_sparse_select_head_softmax(const void *q, const void *k, int B, int T, int Hq,
+                                            int Hkv, int D, sala_strides sq, sala_strides sk,
+                                            int block, int topk, int n_init, int n_local,
+                                            int32_t *idx, void *ws, size_t ws_bytes,
+                                            sala_dtype dt, void *stream);
+
+/*
  * Block-sparse softmax attention (NoPE, causal).
  * For each (b, query head h, row t), hk = h / (Hq / Hkv):
  *   keys = union of blocks [j*block, (j+1)*block) over the entries j >= 0 of

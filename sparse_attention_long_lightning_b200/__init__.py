@@ -18,7 +18,7 @@ import torch
 __all__ = [
     "SalaError", "load_library", "lightning_prefill", "lightning_prefill_workspace",
     "lightning_prefill_noalloc",
-    "lightning_decode", "sparse_select", "sparse_select_workspace", "sparse_attn",
+    "lightning_decode", "sparse_select", "sparse_select_workspace", "sparse_select_head_softmax_workspace", "sparse_attn",
     "sparse_attn_workspace",
     "get_device_error", "selftest_wait_timeout", "sparse_decode", "sparse_decode_workspace",
     "sparse_block_means", "lightning_state", "state_prefix_sum", "status_string", "version",
@@ -76,6 +76,11 @@ def load_library(path: Optional[str] = None):
     lib.sala_sparse_select_workspace.restype = sz
     lib.sala_sparse_select.argtypes = [vp, vp, i, i, i, i, i, S, S, i, i, i, i, vp, vp, sz, i, vp]
     lib.sala_sparse_select.restype = i
+    lib.sala_sparse_select_head_softmax_workspace.argtypes = [i, i, i, i, i, i]
+    lib.sala_sparse_select_head_softmax_workspace.restype = sz
+    lib.sala_sparse_select_head_softmax.argtypes = [vp, vp, i, i, i, i, i, S, S, i, i, i, i, vp,
+                                                    vp, sz, i, vp]
+    lib.sala_sparse_select_head_softmax.restype = i
     lib.sala_sparse_decode_workspace.argtypes = [i, i, i, i, i, i]
     lib.sala_sparse_decode_workspace.restype = sz
     lib.sala_sparse_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, S, S, S, S, S,
@@ -262,9 +267,16 @@ def sparse_select_workspace(B, T, Hq, Hkv, D, block=64, topk=64) -> int:
     return int(load_library().sala_sparse_select_workspace(B, T, Hq, Hkv, D, block, topk))
 
 
+def sparse_select_head_softmax_workspace(B, T, Hq, Hkv, D, block=64) -> int:
+    return int(load_library().sala_sparse_select_head_softmax_workspace(B, T, Hq, Hkv, D, block))
+
+
 def sparse_select(q, k, *, topk=64, n_init=1, n_local=2, block=64, out=None, workspace=None,
-                  stream=None):
-    """Block selection.  q [B,T,Hq,D], k [B,T,Hkv,D] -> idx [B,Hkv,T,n_init+topk+n_local] int32."""
+                  stream=None, score="group_sum"):
+    """Block selection.  q [B,T,Hq,D], k [B,T,Hkv,D] -> idx [B,Hkv,T,n_init+topk+n_local] int32.
+    score="group_sum" (sala_sparse_select) or "head_softmax" (sala_sparse_select_head_softmax)."""
+    if score not in ("group_sum", "head_softmax"):
+        raise ValueError("score must be 'group_sum' or 'head_softmax'")
     lib = load_library()
     _cuda(q, k, out, workspace)
     B, T, Hq, D = q.shape
@@ -272,14 +284,16 @@ def sparse_select(q, k, *, topk=64, n_init=1, n_local=2, block=64, out=None, wor
     n_sel = n_init + topk + n_local
     if out is None:
         out = torch.empty((B, Hkv, T, n_sel), dtype=torch.int32, device=q.device)
-    need = sparse_select_workspace(B, T, Hq, Hkv, D, block, topk)
+    hsm = score == "head_softmax"
+    need = (sparse_select_head_softmax_workspace(B, T, Hq, Hkv, D, block) if hsm
+            else sparse_select_workspace(B, T, Hq, Hkv, D, block, topk))
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    st = lib.sala_sparse_select(_p(q), _p(k), B, T, Hq, Hkv, D, _s4(q), _s4(k), int(block),
-                                int(topk), int(n_init), int(n_local), _p(out), _p(workspace), wsb,
-                                _dt(q), _stream(stream))
-    _check("sala_sparse_select", st)
+    fn = lib.sala_sparse_select_head_softmax if hsm else lib.sala_sparse_select
+    st = fn(_p(q), _p(k), B, T, Hq, Hkv, D, _s4(q), _s4(k), int(block), int(topk), int(n_init),
+            int(n_local), _p(out), _p(workspace), wsb, _dt(q), _stream(stream))
+    _check("sala_sparse_select_head_softmax" if hsm else "sala_sparse_select", st)
     return out
 
 

@@ -108,6 +108,37 @@ bool set_smem(KernelT* k, size_t bytes) {
 
 }  // namespace
 
+namespace sala {
+
+// Head-softmax scoring kernel for group size G (a power of two up to 32).
+template <int D, int G>
+static bool launch_hsm(dim3 grid, cudaStream_t st, const __nv_bfloat16* q, const float* kbar,
+                       float* scores, int nb, int Hkv, sala_strides sq, int r0, int r1,
+                       int rows_pass, int n_init, int n_local, float inv_sqrt_d) {
+  auto kern = block_scores_hsm_kernel<D, G>;
+  if (!set_smem(kern, hsm_smem_bytes<D>())) return false;
+  grid.x = (unsigned)((r1 - r0 + kHsmRows / G - 1) / (kHsmRows / G));
+  kern<<<grid, 256, hsm_smem_bytes<D>(), st>>>(q, kbar, scores, nb, Hkv, sq, r0, r1, rows_pass,
+                                               n_init, n_local, inv_sqrt_d);
+  return true;
+}
+template <int D>
+static bool launch_hsm_g(int G, dim3 grid, cudaStream_t st, const __nv_bfloat16* q,
+                         const float* kbar, float* scores, int nb, int Hkv, sala_strides sq,
+                         int r0, int r1, int rows_pass, int n_init, int n_local, float isd) {
+  switch (G) {
+    case 1: return launch_hsm<D, 1>(grid, st, q, kbar, scores, nb, Hkv, sq, r0, r1, rows_pass, n_init, n_local, isd);
+    case 2: return launch_hsm<D, 2>(grid, st, q, kbar, scores, nb, Hkv, sq, r0, r1, rows_pass, n_init, n_local, isd);
+    case 4: return launch_hsm<D, 4>(grid, st, q, kbar, scores, nb, Hkv, sq, r0, r1, rows_pass, n_init, n_local, isd);
+    case 8: return launch_hsm<D, 8>(grid, st, q, kbar, scores, nb, Hkv, sq, r0, r1, rows_pass, n_init, n_local, isd);
+    case 16: return launch_hsm<D, 16>(grid, st, q, kbar, scores, nb, Hkv, sq, r0, r1, rows_pass, n_init, n_local, isd);
+    case 32: return launch_hsm<D, 32>(grid, st, q, kbar, scores, nb, Hkv, sq, r0, r1, rows_pass, n_init, n_local, isd);
+    default: return false;
+  }
+}
+
+}  // namespace sala
+
 extern "C" {
 
 const char* sala_status_string(sala_status s) {
@@ -377,21 +408,32 @@ size_t sala_sparse_select_workspace(int B, int T, int Hq, int Hkv, int D, int bl
   return sel_fused(T, topk) ? L.total_fused : L.total;
 }
 
-sala_status sala_sparse_select(const void* q, const void* k, int B, int T, int Hq, int Hkv,
-                               int D, sala_strides sq, sala_strides sk, int block, int topk,
-                               int n_init, int n_local, int32_t* idx, void* ws, size_t ws_bytes,
-                               sala_dtype dt, void* stream) {
+size_t sala_sparse_select_head_softmax_workspace(int B, int T, int Hq, int Hkv, int D,
+                                                 int block) {
+  (void)Hq;
+  if (B <= 0 || T <= 0 || Hkv <= 0 || D <= 0 || block != kSelBlk) return 0;
+  return sel_layout(B, T, Hkv, D).total;
+}
+
+// mode 0: group-summed scores (fused tensor-core path for topk <= 64, else the score
+// scratch); mode 1: per-head softmax-normalised scores (score scratch).
+static sala_status sparse_select_impl(const void* q, const void* k, int B, int T, int Hq,
+                                      int Hkv, int D, sala_strides sq, sala_strides sk,
+                                      int block, int topk, int n_init, int n_local, int32_t* idx,
+                                      void* ws, size_t ws_bytes, sala_dtype dt, void* stream,
+                                      int mode) {
   if (T > 0 && (!q || !k || !idx)) return SALA_ERR_INVALID_ARG;
   if (B <= 0 || T < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return SALA_ERR_INVALID_ARG;
   if (topk < 1 || n_init < 0 || n_local < 1) return SALA_ERR_INVALID_ARG;
   if (dt != SALA_BF16) return SALA_ERR_UNSUPPORTED;
   if (block != kSelBlk || (D != 64 && D != 128) || topk > 256 || Hq / Hkv > 32)
     return SALA_ERR_UNSUPPORTED;
+  if (mode == 1 && ((Hq / Hkv) & (Hq / Hkv - 1)) != 0) return SALA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !strides_ok(sq, 2) || !strides_ok(sk, 2))
     return SALA_ERR_INVALID_ARG;
   if (T == 0) return SALA_OK;
   const SelLayout L = sel_layout(B, T, Hkv, D);
-  const bool fused = sel_fused(T, topk);
+  const bool fused = mode == 0 && sel_fused(T, topk);
   if (!ws || ws_bytes < (fused ? L.total_fused : L.total)) return SALA_ERR_WORKSPACE;
   cudaStream_t st = as_stream(stream);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
@@ -439,7 +481,17 @@ sala_status sala_sparse_select(const void* q, const void* k, int B, int T, int H
   }
   for (int r0 = 0; r0 < T; r0 += L.rows_pass) {
     const int r1 = std::min(T, r0 + L.rows_pass);
-    if (L.nb > 0) {
+    if (L.nb > 0 && mode == 1) {
+      const bool ok =
+          D == 128 ? launch_hsm_g<128>(G, dim3(1, Hkv, B), st, (const __nv_bfloat16*)q, kbar,
+                                       scores, L.nb, Hkv, sq, r0, r1, L.rows_pass, n_init,
+                                       n_local, inv_sqrt_d)
+                   : launch_hsm_g<64>(G, dim3(1, Hkv, B), st, (const __nv_bfloat16*)q, kbar,
+                                      scores, L.nb, Hkv, sq, r0, r1, L.rows_pass, n_init,
+                                      n_local, inv_sqrt_d);
+      if (!ok) return SALA_ERR_CUDA;
+      SALA_CHECK_LAUNCH();
+    } else if (L.nb > 0) {
       dim3 gs((r1 - r0 + kScTile - 1) / kScTile, Hkv, B);
       if (D == 128) {
         auto kern = block_scores_kernel<128>;
@@ -463,6 +515,23 @@ sala_status sala_sparse_select(const void* q, const void* k, int B, int T, int H
     SALA_CHECK_LAUNCH();
   }
   return SALA_OK;
+}
+
+sala_status sala_sparse_select(const void* q, const void* k, int B, int T, int Hq, int Hkv,
+                               int D, sala_strides sq, sala_strides sk, int block, int topk,
+                               int n_init, int n_local, int32_t* idx, void* ws, size_t ws_bytes,
+                               sala_dtype dt, void* stream) {
+  return sparse_select_impl(q, k, B, T, Hq, Hkv, D, sq, sk, block, topk, n_init, n_local, idx,
+                            ws, ws_bytes, dt, stream, 0);
+}
+
+sala_status sala_sparse_select_head_softmax(const void* q, const void* k, int B, int T, int Hq,
+                                            int Hkv, int D, sala_strides sq, sala_strides sk,
+                                            int block, int topk, int n_init, int n_local,
+                                            int32_t* idx, void* ws, size_t ws_bytes,
+                                            sala_dtype dt, void* stream) {
+  return sparse_select_impl(q, k, B, T, Hq, Hkv, D, sq, sk, block, topk, n_init, n_local, idx,
+                            ws, ws_bytes, dt, stream, 1);
 }
 
 // ------------------------------------------------------------------ sparse attention

@@ -20,7 +20,7 @@ from sparse_attention_long_lightning_b200 import inputs
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--op", required=True, choices=["lightning", "decode", "select", "attn",
-                                                       "sparse_decode"])
+                                                       "sparse_decode", "select_hsm"])
     ap.add_argument("--T", type=int, default=16384)
     ap.add_argument("--B", type=int, default=64, help="batch for decode")
     ap.add_argument("--iters", type=int, default=3)
@@ -68,6 +68,14 @@ def main():
         o = torch.empty_like(s.q)
         if a.op == "select":
             fn = lambda: sala.sparse_select(s.q, s.k, out=idx, workspace=ws)
+        elif a.op == "select_hsm":
+            wsh = torch.empty(sala.sparse_select_head_softmax_workspace(1, a.T, 32, 2, 128),
+                              dtype=torch.uint8, device=dev)
+            fn = lambda: sala.sparse_select(s.q, s.k, out=idx, workspace=wsh, score="head_softmax")
+            # per-head scores: 2 passes x (query heads x candidate pairs) x D multiply-adds
+            pairs = sum(max(0, t // 64 - 2) for t in range(a.T)) * 32
+            print(f"select_hsm: {pairs * 128 * 2 / 1e12:.3f} T multiply-adds per call "
+                  f"(two passes over {pairs / 1e9:.2f} G query-head x candidate pairs)")
         else:
             fn = lambda: sala.sparse_attn(s.q, s.k, s.v, idx, s.g, out=o, workspace=ws)
     for _ in range(a.warmup):

@@ -161,3 +161,27 @@ def test_workspace_queries(lib):
     assert sala.sparse_select_workspace(1, 1 << 20, 32, 2, 128, 64, 200) <= (1 << 30) + (1 << 26)
     assert sala.sparse_attn_workspace(1, 131072, 2, 128) == 131072 * 2 * 128 * 2
     assert sala.sparse_attn_workspace(1, 0, 2, 128) == 0
+
+
+def test_head_softmax_select_rejects_bad_arguments(lib):
+    p = ctypes.c_void_p(16)
+    st = sala.SalaStrides(64 * 6 * 128, 6 * 128, 128)
+    # group of 3 heads: not a power of two
+    assert lib.sala_sparse_select_head_softmax(p, p, 1, 640, 6, 2, 128, st, st, 64, 4, 1, 2, p,
+                                               p, 1 << 30, 1, None) == 2
+    # Hq not a multiple of Hkv
+    assert lib.sala_sparse_select_head_softmax(p, p, 1, 640, 3, 2, 128, st, st, 64, 4, 1, 2, p,
+                                               p, 1 << 30, 1, None) == 1
+    # workspace too small (the score scratch is always needed)
+    need = sala.sparse_select_head_softmax_workspace(1, 640, 4, 2, 128)
+    assert lib.sala_sparse_select_head_softmax(p, p, 1, 640, 4, 2, 128, st, st, 64, 4, 1, 2, p,
+                                               p, need - 1, 1, None) == 5
+
+
+def test_head_softmax_workspace_has_score_scratch():
+    nb = 131072 // 64
+    means = nb * 2 * 128 * (4 + 2 + 2)
+    n = sala.sparse_select_head_softmax_workspace(1, 131072, 32, 2, 128)
+    assert means + (1 << 29) <= n <= means + (1 << 30) + 4096
+    assert n == sala.sparse_select_workspace(1, 131072, 32, 2, 128, 64, 100)
+    assert sala.sparse_select_head_softmax_workspace(1, 0, 32, 2, 128) == 0
