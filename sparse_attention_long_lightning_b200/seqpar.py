@@ -79,3 +79,67 @@ def lightning_prefill_seqpar(q, k, v, g=None, state=None, q_norm_w=None, k_norm_
     return seqpar_prefill(q, k, v, g, S_init, rank=rank, offsets=offsets, pos0=pos0,
                           gather_states=gather_states, state_fn=state_fn, prefix_fn=prefix_fn,
                           prefill_fn=prefill_fn)
+
+
+# ---------------------------------------------------------------------------------------
+# KV-head-parallel sparse layer.  Block selection and block-sparse attention of KV head
+# hk touch only hk's keys/values and the query heads of its group (the GQA group shares
+# the selection), so ranks that each own a contiguous range of KV heads (with their
+# query groups) need no exchange; the only collective is the optional all-gather of the
+# outputs along the head axis.  It scales to at most Hkv ranks (2 for 32q/2kv).
+# ---------------------------------------------------------------------------------------
+
+def kvhead_range(Hkv: int, rank: int, world: int):
+    """KV heads [lo, hi) owned by `rank` of `world` (contiguous, sizes differ by <= 1)."""
+    if not 0 <= rank < world or world > Hkv:
+        raise ValueError("need 0 <= rank < world <= Hkv")
+    return rank * Hkv // world, (rank + 1) * Hkv // world
+
+
+def sparse_layer_headpar(q, k, v, g=None, *, rank: int, world: int, select_fn: Callable,
+                         attn_fn: Callable, gather_fn: Optional[Callable] = None):
+    """This rank's share of a sparse layer: q, g [B,T,Hq,D] and k, v [B,T,Hkv,D] hold all
+    heads (or views of them); the rank computes
+      idx = select_fn(q_r, k_r), o_r = attn_fn(q_r, k_r, v_r, idx, g_r)
+    on its KV heads and their query groups (views, no copies) and returns o_r, or the
+    full [B,T,Hq,D] output when `gather_fn(o_r) -> list of every rank's o in rank order`
+    is given."""
+    Hq, Hkv = q.shape[2], k.shape[2]
+    grp = Hq // Hkv
+    lo, hi = kvhead_range(Hkv, rank, world)
+    q_r, g_r = q[:, :, lo * grp:hi * grp], (None if g is None else g[:, :, lo * grp:hi * grp])
+    k_r, v_r = k[:, :, lo:hi], v[:, :, lo:hi]
+    idx = select_fn(q_r, k_r)
+    o_r = attn_fn(q_r, k_r, v_r, idx, g_r)
+    if gather_fn is None:
+        return o_r
+    return torch.cat(list(gather_fn(o_r)), dim=2)
+
+
+def sparse_layer_kvhead_parallel(q, k, v, g=None, *, group=None, topk=64, n_init=1, n_local=2,
+                                 block=64, gather=True):
+    """KV-head-parallel sparse layer on this rank's GPU (one process per GPU, NCCL):
+    libsala selection and attention on the rank's KV heads; with gather=True the outputs
+    of all ranks are all-gathered (every rank's share has the same shape when Hkv is a
+    multiple of the world size)."""
+    import torch.distributed as dist
+
+    import sparse_attention_long_lightning_b200 as sala
+
+    rank, world = dist.get_rank(group), dist.get_world_size(group)
+    if k.shape[2] % world:
+        raise ValueError("Hkv must be a multiple of the world size")
+
+    def select_fn(qq, kk):
+        return sala.sparse_select(qq, kk, topk=topk, n_init=n_init, n_local=n_local, block=block)
+
+    def attn_fn(qq, kk, vv, idx, gg):
+        return sala.sparse_attn(qq, kk, vv, idx, gg, block=block)
+
+    def gather_fn(o_r):
+        parts = [torch.empty_like(o_r) for _ in range(world)]
+        dist.all_gather(parts, o_r.contiguous(), group=group)
+        return parts
+
+    return sparse_layer_headpar(q, k, v, g, rank=rank, world=world, select_fn=select_fn,
+                                attn_fn=attn_fn, gather_fn=gather_fn if gather else None)

@@ -110,3 +110,70 @@ def test_seqpar_host_logic_two_ranks(lens):
     for rank in range(world):
         dy, dS, scale = out[rank]
         assert dy <= 1e-10 and dS <= 1e-10 * max(1.0, scale)
+
+
+# ---------------------------------------------------------------------------------------
+# KV-head-parallel sparse layer: each rank selects and attends on its own KV heads and
+# their query groups; the all-gathered output must equal the full layer exactly (the
+# per-KV-head computations are independent).  fp64 oracle standing in for the kernels.
+# ---------------------------------------------------------------------------------------
+
+def _headpar_worker(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    from datetime import timedelta
+
+    import numpy as np
+
+    import oracle
+    from sparse_attention_long_lightning_b200.seqpar import sparse_layer_headpar
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        rng = np.random.default_rng(123)
+        T, Hq, Hkv, D, topk = 64 * 12 + 5, 8, 4, 16, 3
+        q, g = (torch.from_numpy(rng.standard_normal((1, T, Hq, D))) for _ in range(2))
+        k, v = (torch.from_numpy(rng.standard_normal((1, T, Hkv, D))) for _ in range(2))
+
+        def select_fn(qq, kk):
+            return oracle.sparse_select(qq.numpy(), kk.numpy(), topk=topk)[0]
+
+        def attn_fn(qq, kk, vv, idx, gg):
+            return torch.from_numpy(oracle.attention(qq.numpy(), kk.numpy(), vv.numpy(),
+                                                     gg.numpy(), idx=idx))
+
+        def gather_fn(o_r):
+            parts = [torch.empty_like(o_r) for _ in range(world)]
+            dist.all_gather(parts, o_r.contiguous())
+            return parts
+
+        y = sparse_layer_headpar(q, k, v, g, rank=rank, world=world, select_fn=select_fn,
+                                 attn_fn=attn_fn, gather_fn=gather_fn)
+        idx_full = select_fn(q, k)
+        y_full = attn_fn(q, k, v, idx_full, g)
+        out[rank] = (tuple(y.shape), float((y - y_full).abs().max()))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sparse_kvhead_parallel_two_ranks():
+    world = 2
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.spawn(_headpar_worker, args=(world, _free_port(), out), nprocs=world, join=True)
+    for rank in range(world):
+        shape, err = out[rank]
+        assert shape == (1, 64 * 12 + 5, 8, 16)
+        assert err == 0.0
+
+
+def test_kvhead_ranges_cover_all_heads():
+    from sparse_attention_long_lightning_b200.seqpar import kvhead_range
+    for Hkv in (1, 2, 3, 8):
+        for world in range(1, Hkv + 1):
+            spans = [kvhead_range(Hkv, r, world) for r in range(world)]
+            assert spans[0][0] == 0 and spans[-1][1] == Hkv
+            assert all(a[1] == b[0] for a, b in zip(spans, spans[1:]))
+            assert all(hi > lo for lo, hi in spans)
+    with pytest.raises(ValueError):
+        kvhead_range(2, 0, 3)

@@ -212,3 +212,36 @@ def test_bounded_wait_reports_timeout():
     o = sala.sparse_attn(s.q.cuda(), s.k.cuda(), s.v.cuda(), idx)
     ref = oracle.attention(_np(s.q), _np(s.k), _np(s.v), idx=idx.cpu().numpy())
     assert rel_err(_np(o), ref, True) <= TOL_BF16
+
+
+def test_sparse_kvhead_parallel_single_rank_group():
+    """The public KV-head-parallel call on a one-rank NCCL group (all heads on this rank,
+    outputs all-gathered) is the plain selection + attention, bit for bit; and a rank's
+    share computed on head views equals the same heads of the full layer."""
+    import os
+    import socket
+
+    import torch.distributed as dist
+
+    from sparse_attention_long_lightning_b200.seqpar import (sparse_layer_headpar,
+                                                              sparse_layer_kvhead_parallel)
+    T, Hq, Hkv, D = 64 * 30 + 11, 32, 2, 128
+    s = inputs.sparse_inputs(1, T, Hq, Hkv, D, seed=818, device=DEV, gate=True)
+    y_ref = sala.sparse_attn(s.q, s.k, s.v, sala.sparse_select(s.q, s.k, topk=16), s.g)
+    # rank 1 of 2 computed locally: KV head 1 and query heads 16..31, from views
+    y1 = sparse_layer_headpar(s.q, s.k, s.v, s.g, rank=1, world=2,
+                              select_fn=lambda qq, kk: sala.sparse_select(qq, kk, topk=16),
+                              attn_fn=lambda qq, kk, vv, idx, gg: sala.sparse_attn(qq, kk, vv,
+                                                                                   idx, gg))
+    assert torch.equal(y1, y_ref[:, :, 16:])
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    os.environ["MASTER_ADDR"], os.environ["MASTER_PORT"] = "127.0.0.1", str(port)
+    dist.init_process_group("nccl", rank=0, world_size=1)
+    try:
+        y = sparse_layer_kvhead_parallel(s.q, s.k, s.v, s.g, topk=16)
+        assert torch.equal(y, y_ref)
+    finally:
+        dist.destroy_process_group()
+    assert sala.get_device_error() == 0
