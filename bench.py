@@ -492,7 +492,7 @@ def main():
     # ncu capture of this command at T=131072 with the current kernels (the sparse
     # kernel's own launch; Lightning = state pass + scan + output pass; selection =
     # block means + fused kernel).  Re-measure whenever one of those kernels changes.
-    ncu_traffic = {"attn": 8.91e9, "sel": 1.17e9} if T == 131072 else {}
+    ncu_traffic = {"attn": 9.64e9, "sel": 1.16e9} if T == 131072 else {}
     share = {k: n_ops[k] * op_ms[k] for k in op_ms}
     dom = max(share, key=share.get)
     if dom == "attn":
