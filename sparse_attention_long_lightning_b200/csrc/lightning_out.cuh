@@ -86,7 +86,10 @@ __device__ __forceinline__ void lo_prep_qk_half(uint8_t* sQ, uint8_t* sK, int r,
       for (int o = 0; o < 2; ++o) {
         // angle = (chunk base angle, reduced in fp64) + r * inv_freq_i, re-reduced in fp32
         float a = o ? fmaf((float)r, bb.w, bb.z) : fmaf((float)r, bb.y, bb.x);
-        a = fmaf(-rintf(a * inv_two_pi), two_pi, a);
+        // nearest multiple of 2 pi by adding and removing 1.5 * 2^23 (exact rounding to
+        // nearest for |a / 2 pi| < 2^22; plain adds instead of a rounding instruction)
+        const float turns = (a * inv_two_pi + 12582912.0f) - 12582912.0f;
+        a = fmaf(-turns, two_pi, a);
         __sincosf(a, &sn[2 * e2 + o], &cs[2 * e2 + o]);
       }
     }
