@@ -21,8 +21,9 @@
 // two 64-column slabs each) into shared memory; threads normalise/rotate q and k and
 // convert q, k, v to fp16 IN PLACE (same swizzled layout), so a tile is directly a
 // tcgen05 operand.  fp16 (10-bit mantissa) keeps the rounding of the normalised,
-// rotated operands well inside the 1e-2 tolerance, where bf16 would not.  One thread
-// issues the MMAs, fp32 accumulation in tensor memory.
+// rotated operands well inside the 1e-2 tolerance, where bf16 would not.  A single
+// thread issues each kernel's MMAs (in the state pass, the producer warp's), fp32
+// accumulation in tensor memory.
 #pragma once
 
 #include "lightning_cc.cuh"
