@@ -41,6 +41,23 @@ SPARSE_LAYERS = (2, 6)
 NUM_LAYERS = 8
 
 
+def source_digest() -> str:
+    """First 12 hex digits of the sha256 of the CUDA sources and the C header the library
+    is built from (the GPU host gets no git history, so this identifies the build)."""
+    import glob
+    import hashlib
+    root = os.path.dirname(os.path.abspath(__file__))
+    files = sorted(glob.glob(os.path.join(root, "sparse_attention_long_lightning_b200", "csrc",
+                                          "*.cu*")))
+    files.append(os.path.join(root, "include", "sala.h"))
+    h = hashlib.sha256()
+    for f in files:
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
 def _peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -526,7 +543,8 @@ def main():
                                    if shared_bufs else "fresh seeded inputs per layer"),
                        "chunk": CHUNK, "block": BLOCK, "topk": TOPK, "n_init": N_INIT,
                        "n_local": N_LOCAL},
-            "roofline": roof, "components": comps, "clocks": clk.summary()}
+            "roofline": roof, "components": comps, "clocks": clk.summary(),
+            "build": {"sources_sha256": source_digest(), "library": sala.version()}}
 
     if not args.no_extras:
         line["gpu_launches"] = count_launches(layers, sala) * args.steps

@@ -22,6 +22,7 @@ __all__ = [
     "sparse_attn_workspace",
     "get_device_error", "selftest_wait_timeout", "sparse_decode", "sparse_decode_workspace",
     "sparse_block_means", "lightning_state", "state_prefix_sum", "status_string", "version",
+    "set_tracing",
     "LIB_PATH",
 ]
 
@@ -34,6 +35,40 @@ class SalaError(RuntimeError):
     def __init__(self, fn: str, status: int, text: str):
         super().__init__(f"{fn} failed: {text} ({status})")
         self.status = status
+
+
+_TRACE = os.environ.get("SALA_NVTX", "") not in ("", "0")
+
+
+def set_tracing(on: bool = True) -> None:
+    """Wrap every compute call of the library in an NVTX range named after its C entry
+    point, for profiler timelines (SALA_NVTX=1 at import does the same).  Off by
+    default: the calls are then made directly."""
+    global _TRACE
+    _TRACE = bool(on)
+
+
+class _Lib:
+    """The loaded libsala: attribute access goes to the C library; with tracing on, the
+    compute entry points come back wrapped in NVTX ranges (workspace queries and the
+    status helpers never are)."""
+
+    _PLAIN = ("sala_status_string", "sala_version")
+
+    def __init__(self, cdll):
+        self._cdll = cdll
+
+    def __getattr__(self, name):
+        fn = getattr(self._cdll, name)
+        if (not _TRACE or not name.startswith("sala_") or name.endswith("_workspace")
+                or name in self._PLAIN):
+            return fn
+
+        def traced(*args):
+            with torch.cuda.nvtx.range(name):
+                return fn(*args)
+
+        return traced
 
 
 class SalaStrides(ctypes.Structure):
@@ -97,8 +132,8 @@ def load_library(path: Optional[str] = None):
     lib.sala_get_device_error.restype = i
     lib.sala_selftest_wait_timeout.argtypes = [ctypes.c_longlong, vp]
     lib.sala_selftest_wait_timeout.restype = i
-    _lib = lib
-    return lib
+    _lib = _Lib(lib)
+    return _lib
 
 
 def status_string(status: int) -> str:

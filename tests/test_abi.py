@@ -185,3 +185,21 @@ def test_head_softmax_workspace_has_score_scratch():
     assert means + (1 << 29) <= n <= means + (1 << 30) + 4096
     assert n == sala.sparse_select_workspace(1, 131072, 32, 2, 128, 64, 100)
     assert sala.sparse_select_head_softmax_workspace(1, 0, 32, 2, 128) == 0
+
+
+def test_tracing_wraps_compute_calls_only(lib):
+    """With tracing on, compute entry points go through an NVTX range (and still return
+    the library's status); workspace queries and status helpers are the bare calls."""
+    raw = lib._cdll
+    sala.set_tracing(True)
+    try:
+        traced = lib.sala_sparse_select
+        assert traced is not raw.sala_sparse_select
+        p = ctypes.c_void_p(16)
+        st = sala.SalaStrides(64 * 2 * 128, 2 * 128, 128)
+        assert traced(p, p, 1, 64, 3, 2, 128, st, st, 64, 4, 1, 2, p, p, 1 << 20, 1, None) == 1
+        assert lib.sala_sparse_select_workspace is raw.sala_sparse_select_workspace
+        assert lib.sala_status_string is raw.sala_status_string
+    finally:
+        sala.set_tracing(False)
+    assert lib.sala_sparse_select is raw.sala_sparse_select

@@ -48,6 +48,12 @@ def test_single_process_passthrough():
     assert bench.weak_scaling_value(1, 1000, 0.5) == 2000
 
 
+def test_bench_build_digest_is_stable():
+    import bench
+    a, b = bench.source_digest(), bench.source_digest()
+    assert a == b and len(a) == 12 and int(a, 16) >= 0
+
+
 # ---------------------------------------------------------------------------------------
 # Sequence-parallel Lightning prefill: the multi-rank host logic (segment offsets, the
 # all-gather of segment states in rank order, the prefix) on CPU ranks, with the fp64
