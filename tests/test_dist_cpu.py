@@ -107,9 +107,9 @@ def _seqpar_worker(rank, world, port, lens, out):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("lens", [(100, 157), (64, 64)])
-def test_seqpar_host_logic_two_ranks(lens):
-    world = 2
+@pytest.mark.parametrize("lens", [(100, 157), (64, 64), (37, 128, 90)])
+def test_seqpar_host_logic_multi_rank(lens):
+    world = len(lens)
     mgr = mp.Manager()
     out = mgr.dict()
     mp.spawn(_seqpar_worker, args=(world, _free_port(), list(lens), out), nprocs=world, join=True)
