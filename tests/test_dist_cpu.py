@@ -162,8 +162,8 @@ def _headpar_worker(rank, world, port, out):
         dist.destroy_process_group()
 
 
-def test_sparse_kvhead_parallel_two_ranks():
-    world = 2
+@pytest.mark.parametrize("world", [2, 4])
+def test_sparse_kvhead_parallel_ranks(world):
     mgr = mp.Manager()
     out = mgr.dict()
     mp.spawn(_headpar_worker, args=(world, _free_port(), out), nprocs=world, join=True)
