@@ -64,9 +64,16 @@ def _load():
             _dp, _dp, i, i, i, i, i, i, i, i, i, _i64p, i, _i32p, _dp, _dp, i, i]
         lib.oracle_attention.argtypes = [
             _dp, _dp, _dp, _dp, _i32p, i, i, i, i, i, i, i, d, _i64p, i, _dp]
+        lib.oracle_lightning_recurrent_prepared.argtypes = [
+            _dp, _dp, _dp, _dp, _dp, i, i, i, i, _dp, _dp]
+        lib.oracle_matmul_nt.argtypes = [_dp, _dp, i64, i, i, _dp]
+        lib.oracle_lightning_projection.argtypes = [
+            _dp, _dp, _dp, _dp, i, i, i, i, i, i64, d, d, _dp, _dp, _dp, _dp]
         for f in ("oracle_qk_prep", "oracle_lightning_recurrent", "oracle_lightning_quadratic",
                   "oracle_lightning_chunked", "oracle_lightning_decode", "oracle_block_means",
-                  "oracle_sparse_select", "oracle_sparse_select_mode", "oracle_attention"):
+                  "oracle_sparse_select", "oracle_sparse_select_mode", "oracle_attention",
+                  "oracle_lightning_recurrent_prepared", "oracle_matmul_nt",
+                  "oracle_lightning_projection"):
             getattr(lib, f).restype = None
         _lib = lib
     return _lib
@@ -115,6 +122,47 @@ def lightning_recurrent(q, k, v, g=None, S0=None, qw=None, kw=None, *, pos0=0,
     return y, S
 
 
+def lightning_recurrent_prepared(qh, kh, v, gate=None, S0=None):
+    """Recurrent Lightning attention on prepared operands: qh, kh already normalised and
+    rotated, `gate` the output multiplier (sigmoid already applied) or None.
+    qh, kh, v, gate: [B,T,H,D].  Returns (y [B,T,H,D], S_final)."""
+    lib = _load()
+    B, T, H, D = np.shape(qh)
+    (qh, qp), (kh, kp), (v, vp), (gate, gp), (S0, sp) = _d(qh), _d(kh), _d(v), _d(gate), _d(S0)
+    y = np.zeros((B, T, H, D))
+    S = np.zeros((B, H, D, D))
+    lib.oracle_lightning_recurrent_prepared(qp, kp, vp, gp, sp, B, T, H, D,
+                                            y.ctypes.data_as(_dp), S.ctypes.data_as(_dp))
+    return y, S
+
+
+def matmul_nt(x, w):
+    """y = x W^T for x [M, K], W [N, K] (plain fp64 loops)."""
+    lib = _load()
+    (x, xp), (w, wp) = _d(x), _d(w)
+    M, K = x.shape
+    N = w.shape[0]
+    y = np.zeros((M, N))
+    lib.oracle_matmul_nt(xp, wp, M, K, N, y.ctypes.data_as(_dp))
+    return y
+
+
+def lightning_projection(x, w, qw=None, kw=None, *, H, D, pos0=0, base=10000.0, eps=1e-6):
+    """Lightning-layer inputs from hidden states x [B,T,hidden] and the projection weight
+    W [4 H D, hidden] (rows: q heads, then k, v, g heads).  Returns (qh, kh, v, gate),
+    each [B,T,H,D]: q, k normalised and rotated at pos0 + t, v as projected, gate =
+    sigmoid(g)."""
+    lib = _load()
+    B, T, hidden = np.shape(x)
+    (x, xp), (w, wp), (qw, qwp), (kw, kwp) = _d(x), _d(w), _d(qw), _d(kw)
+    if w.shape != (4 * H * D, hidden):
+        raise ValueError("W must be [4 H D, hidden]")
+    outs = [np.zeros((B, T, H, D)) for _ in range(4)]
+    lib.oracle_lightning_projection(xp, wp, qwp, kwp, B, T, hidden, H, D, int(pos0), base, eps,
+                                    *(o.ctypes.data_as(_dp) for o in outs))
+    return tuple(outs)
+
+
 def lightning_quadratic(q, k, v, g=None, S0=None, qw=None, kw=None, *, pos0=0,
                         base=10000.0, eps=1e-6):
     """Quadratic masked form of the same attention; returns y [B,T,H,D]."""
@@ -142,14 +190,18 @@ def lightning_chunked(q, k, v, g=None, S0=None, qw=None, kw=None, *, chunk, pos0
     return y, S
 
 
-def lightning_decode(q, k, v, g, S, pos, qw=None, kw=None, *, base=10000.0, eps=1e-6):
+def lightning_decode(q, k, v, g, S, pos, qw=None, kw=None, *, base=10000.0, eps=1e-6,
+                     inplace=False):
     """One decode step.  q,k,v,g: [B,H,D]; S: [B,H,D,D]; pos: [B].
-    Returns (y [B,H,D], S_new)."""
+    Returns (y [B,H,D], S_new).  With inplace=True and S a C-contiguous float64 array,
+    S itself is updated (and returned) instead of a copy."""
     lib = _load()
     B, H, D = np.shape(q)
     (q, qp), (k, kp), (v, vp), (g, gp) = _d(q), _d(k), _d(v), _d(g)
     (qw, qwp), (kw, kwp) = _d(qw), _d(kw)
-    S = np.array(S, dtype=np.float64, copy=True, order="C")
+    if not (inplace and isinstance(S, np.ndarray) and S.dtype == np.float64
+            and S.flags.c_contiguous):
+        S = np.array(S, dtype=np.float64, copy=True, order="C")
     p = np.ascontiguousarray(np.asarray(pos, dtype=np.int64))
     y = np.zeros((B, H, D))
     lib.oracle_lightning_decode(qp, kp, vp, gp, S.ctypes.data_as(_dp), qwp, kwp,
@@ -224,11 +276,12 @@ def attention(q, k, v, g=None, idx=None, *, blk=64, scale=None, rows=None):
 
 
 def sparse_decode(q, k_cache, v_cache, pos, g=None, *, blk=64, topk=64, n_init=1, n_local=2,
-                  scale=None):
+                  scale=None, want_scores=False):
     """Sparse-layer decode step: for each sequence b, row p = pos[b] of the prefill
     computation (sparse_select then attention) over cache rows 0..p only.
     q, g: [B, Hq, D]; k_cache, v_cache: [B, Tmax, Hkv, D]; pos: [B] ints.
-    Returns (y [B, Hq, D], idx [B, Hkv, n_sel] int32, gap [B, Hkv])."""
+    Returns (y [B, Hq, D], idx [B, Hkv, n_sel] int32, gap [B, Hkv]) and, with
+    want_scores, the candidate scores [B, Hkv, Tmax // blk] (NaN = not a candidate)."""
     q = np.asarray(q, dtype=np.float64)
     B, Hq, D = q.shape
     Hkv = np.shape(k_cache)[2]
@@ -236,15 +289,18 @@ def sparse_decode(q, k_cache, v_cache, pos, g=None, *, blk=64, topk=64, n_init=1
     y = np.zeros((B, Hq, D))
     idx = np.zeros((B, Hkv, n_sel), dtype=np.int32)
     gap = np.zeros((B, Hkv))
+    ncap = max(1, np.shape(k_cache)[1] // blk)
+    sc = np.full((B, Hkv, ncap), np.nan)
     for b in range(B):
         p = int(pos[b])
         kk = np.asarray(k_cache[b:b + 1, :p + 1], dtype=np.float64)
         vv = np.asarray(v_cache[b:b + 1, :p + 1], dtype=np.float64)
         qr = q[b][None, None]
         gr = None if g is None else np.asarray(g[b], dtype=np.float64)[None, None]
-        ib, gb = sparse_select(qr, kk, blk=blk, topk=topk, n_init=n_init, n_local=n_local,
-                               rows=[p], T=p + 1)
+        ib, gb, sb = sparse_select(qr, kk, blk=blk, topk=topk, n_init=n_init, n_local=n_local,
+                                   rows=[p], T=p + 1, want_scores=True)
         y[b] = attention(qr, kk, vv, gr, idx=ib, blk=blk, scale=scale, rows=[p])[0, 0]
         idx[b] = ib[0, :, 0]
         gap[b] = gb[0, :, 0]
-    return y, idx, gap
+        sc[b, :, :sb.shape[-1]] = sb[0, :, 0]
+    return (y, idx, gap, sc) if want_scores else (y, idx, gap)

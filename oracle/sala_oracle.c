@@ -140,6 +140,41 @@ void oracle_lightning_recurrent(const double *q, const double *k, const double *
 }
 
 /*
+ * The same recurrence on operands that are already prepared: qh, kh normalised and
+ * rotated, and the gate given as its multiplier (sigmoid(g) already applied):
+ *   S_t = S_{t-1} + kh_t v_t^T,   y_t = gate_t * (qh_t^T S_t)   (gate NULL: y_t = o_t).
+ * qh, kh, v, gate: [B, T, H, D]; S0 as above (NULL = zero); y: [B, T, H, D];
+ * S_out: [B, H, D, D] or NULL.
+ */
+void oracle_lightning_recurrent_prepared(const double *qh, const double *kh, const double *v,
+                                         const double *gate, const double *S0, int B, int T,
+                                         int H, int D, double *y, double *S_out)
+{
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < H; ++h) {
+            double *S = (double *)malloc(sizeof(double) * D * D);
+            if (S0)
+                memcpy(S, S0 + ((int64_t)b * H + h) * D * D, sizeof(double) * D * D);
+            else
+                memset(S, 0, sizeof(double) * D * D);
+            for (int t = 0; t < T; ++t) {
+                int64_t at = IDX4(b, t, h, 0, T, H, D);
+                for (int i = 0; i < D; ++i)
+                    for (int j = 0; j < D; ++j) S[i * D + j] += kh[at + i] * v[at + j];
+                for (int j = 0; j < D; ++j) {
+                    double o = 0.0;
+                    for (int i = 0; i < D; ++i) o += qh[at + i] * S[i * D + j];
+                    y[at + j] = gate ? gate[at + j] * o : o;
+                }
+            }
+            if (S_out) memcpy(S_out + ((int64_t)b * H + h) * D * D, S, sizeof(double) * D * D);
+            free(S);
+        }
+    }
+}
+
+/*
  * Quadratic (parallel) form of the same recurrence: unrolling
  * S_t = S0 + sum_{s<=t} k_s v_s^T gives
  *   o_t = q_t^T S0 + sum_{s<=t} (q_t . k_s) v_s,
@@ -543,4 +578,60 @@ void oracle_attention(const double *q, const double *k, const double *v, const d
                 }
                 free(mark);
             }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Input projection of a Lightning layer with its preparation fused in.      */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Plain matrix product y = x W^T: x [M, K] (rows = tokens), W [N, K] (rows =
+ * output features, the layout of a linear layer's weight), y [M, N].
+ */
+void oracle_matmul_nt(const double *x, const double *w, int64_t M, int K, int N, double *y)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int k = 0; k < K; ++k) acc += x[m * K + k] * w[(int64_t)n * K + k];
+            y[m * N + n] = acc;
+        }
+}
+
+/*
+ * Lightning-layer inputs from hidden states x [B, T, hidden] (tech-report mirror,
+ * section 02 (3): QK-normalisation and an output gate in the linear layers; section
+ * 02 (4): RoPE in the linear layers):
+ *   [q | k | v | g] = x W^T, W [4 H D, hidden] with the q rows first, then k, v, g
+ *   (head h of a section = its rows h D .. h D + D - 1);
+ *   qh = RoPE(RMSNorm(q) * qw), kh = RoPE(RMSNorm(k) * kw) at position pos0 + t;
+ *   v unchanged; gate = sigmoid(g), the output gate's multiplier.
+ * qw, kw: [D] or NULL (weight 1).  Outputs qh, kh, v, gate: [B, T, H, D].
+ */
+void oracle_lightning_projection(const double *x, const double *w, const double *qw,
+                                 const double *kw, int B, int T, int hidden, int H, int D,
+                                 int64_t pos0, double base, double eps, double *qh, double *kh,
+                                 double *v, double *gate)
+{
+    int N = 4 * H * D;
+    int64_t M = (int64_t)B * T;
+    double *y = (double *)malloc(sizeof(double) * (size_t)(M > 0 ? M : 1) * N);
+    oracle_matmul_nt(x, w, M, hidden, N, y);
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int h = 0; h < H; ++h) {
+            int64_t t = m % T;
+            const double *row = y + m * N;
+            int64_t o = (m * H + h) * D;
+            oracle_qk_prep(row + (int64_t)(0 * H + h) * D, qw, D, eps, (double)(pos0 + t), base,
+                           qh + o);
+            oracle_qk_prep(row + (int64_t)(1 * H + h) * D, kw, D, eps, (double)(pos0 + t), base,
+                           kh + o);
+            for (int d = 0; d < D; ++d) {
+                v[o + d] = row[(int64_t)(2 * H + h) * D + d];
+                gate[o + d] = sigmoid(row[(int64_t)(3 * H + h) * D + d]);
+            }
+        }
+    free(y);
 }

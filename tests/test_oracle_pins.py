@@ -569,3 +569,107 @@ def test_head_softmax_planted_closed_form():
     for j in range(1, c - 1):
         if j != J:
             assert np.isclose(row[j - 1], want_other, rtol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# Input projection of a Lightning layer with its preparation, and the recurrence on
+# prepared operands (the fused hybrid-layer epilogue)
+# ----------------------------------------------------------------------------
+
+def test_matmul_nt_matches_numpy():
+    """y = x W^T against numpy's matrix product (a transposed operand would fail)."""
+    rng = np.random.default_rng(71)
+    x, w = rng.standard_normal((37, 96)), rng.standard_normal((80, 96))
+    np.testing.assert_allclose(oracle.matmul_nt(x, w), x @ w.T, rtol=1e-12, atol=1e-12)
+
+
+def _proj_case(B=2, T=9, hidden=48, H=3, D=8, seed=72):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((B, T, hidden))
+    w = rng.standard_normal((4 * H * D, hidden)) / math.sqrt(hidden)
+    return x, w
+
+
+def test_projection_sections_v_and_gate():
+    """v is the third block of W's rows applied to x, gate = expit(fourth block)
+    (scipy's logistic function), each head taking D consecutive rows."""
+    from scipy.special import expit
+    B, T, hidden, H, D = 2, 9, 48, 3, 8
+    x, w = _proj_case(B, T, hidden, H, D)
+    qh, kh, v, gate = oracle.lightning_projection(x, w, H=H, D=D, pos0=5)
+    y = (x.reshape(-1, hidden) @ w.T).reshape(B, T, 4, H, D)
+    np.testing.assert_allclose(v, y[:, :, 2], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(gate, expit(y[:, :, 3]), rtol=1e-12, atol=1e-15)
+
+
+def test_projection_qk_at_position_zero_is_rmsnorm():
+    """At position 0 (pos0 = 0, token 0) the rotation is the identity: qh, kh are the
+    projected q, k divided by their RMS (times the norm weight)."""
+    B, T, hidden, H, D = 1, 4, 48, 3, 8
+    x, w = _proj_case(B, T, hidden, H, D, seed=73)
+    rng = np.random.default_rng(74)
+    qw, kw = 1 + 0.1 * rng.standard_normal(D), 1 + 0.1 * rng.standard_normal(D)
+    qh, kh, _, _ = oracle.lightning_projection(x, w, qw, kw, H=H, D=D, pos0=0, eps=1e-6)
+    y = (x.reshape(-1, hidden) @ w.T).reshape(B, T, 4, H, D)
+    for sec, out, wt in ((0, qh, qw), (1, kh, kw)):
+        raw = y[0, 0, sec]
+        want = raw / np.sqrt(np.mean(raw * raw, axis=-1, keepdims=True) + 1e-6) * wt
+        np.testing.assert_allclose(out[0, 0], want, rtol=1e-12)
+
+
+def test_projection_rope_relative_and_norm_preserving():
+    """For the same hidden state placed at two positions, qh has the same norm (RoPE is
+    a rotation) and qh(m) . kh(n) depends only on m - n."""
+    B, T, hidden, H, D = 1, 1, 48, 1, 8
+    x, w = _proj_case(B, T, hidden, H, D, seed=75)
+    prep = {p: oracle.lightning_projection(x, w, H=H, D=D, pos0=p) for p in (3, 10, 103, 110)}
+    q3, k10 = prep[3][0][0, 0, 0], prep[10][1][0, 0, 0]
+    q103, k110 = prep[103][0][0, 0, 0], prep[110][1][0, 0, 0]
+    assert np.isclose(q3 @ k10, q103 @ k110, rtol=1e-10)
+    assert np.isclose(np.linalg.norm(q3), np.linalg.norm(q103), rtol=1e-12)
+    assert not np.isclose(q3 @ k10, prep[3][0][0, 0, 0] @ prep[103][1][0, 0, 0], rtol=1e-3)
+
+
+def test_projection_positions_follow_the_token_index():
+    """Token t of each sequence sits at pos0 + t (the batch index does not shift it)."""
+    B, T, hidden, H, D = 2, 5, 48, 2, 8
+    x, w = _proj_case(B, T, hidden, H, D, seed=76)
+    x[1] = x[0]
+    qh, kh, _, _ = oracle.lightning_projection(x, w, H=H, D=D, pos0=7)
+    np.testing.assert_allclose(qh[1], qh[0], rtol=1e-13)
+    one, _, _, _ = oracle.lightning_projection(x[:, 3:4], w, H=H, D=D, pos0=10)
+    np.testing.assert_allclose(one[:, 0], qh[:, 3], rtol=1e-12)
+
+
+def test_prepared_recurrence_equals_raw_recurrence():
+    """Fed the prepared operands of the raw q, k (qk_prep at each position) and
+    sigmoid(g), the prepared recurrence gives the raw recurrence's outputs and state."""
+    rng = np.random.default_rng(77)
+    B, T, H, D = 2, 11, 2, 8
+    q, k, v, g = (rng.standard_normal((B, T, H, D)) for _ in range(4))
+    S0 = 0.1 * rng.standard_normal((B, H, D, D))
+    y_raw, S_raw = oracle.lightning_recurrent(q, k, v, g, S0, pos0=4)
+    qh = np.empty_like(q)
+    kh = np.empty_like(k)
+    for b in range(B):
+        for t in range(T):
+            for h in range(H):
+                qh[b, t, h] = oracle.qk_prep(q[b, t, h], pos=4 + t)
+                kh[b, t, h] = oracle.qk_prep(k[b, t, h], pos=4 + t)
+    y, S = oracle.lightning_recurrent_prepared(qh, kh, v, 1 / (1 + np.exp(-g)), S0)
+    np.testing.assert_allclose(y, y_raw, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(S, S_raw, rtol=1e-12, atol=1e-12)
+
+
+def test_prepared_recurrence_quadratic_form():
+    """Unrolled: y_t = gate_t * (qh_t^T S0 + sum_{s<=t} (qh_t . kh_s) v_s), by numpy."""
+    rng = np.random.default_rng(78)
+    B, T, H, D = 1, 13, 2, 8
+    qh, kh, v, gate = (rng.standard_normal((B, T, H, D)) for _ in range(4))
+    S0 = rng.standard_normal((B, H, D, D))
+    y, S = oracle.lightning_recurrent_prepared(qh, kh, v, gate, S0)
+    for h in range(H):
+        P = np.tril(qh[0, :, h] @ kh[0, :, h].T)
+        want = (P @ v[0, :, h] + qh[0, :, h] @ S0[0, h]) * gate[0, :, h]
+        np.testing.assert_allclose(y[0, :, h], want, rtol=1e-11, atol=1e-11)
+        np.testing.assert_allclose(S[0, h], S0[0, h] + kh[0, :, h].T @ v[0, :, h], rtol=1e-12)
