@@ -11,11 +11,13 @@ Inputs are synthetic N(0,1) per layer (seed 1005 + layer), all resident in HBM
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Multi-GPU: one process per GPU (torchrun); every rank runs its own independent
-sequence (weak scaling, no data-path collective); the step time is the max over
-ranks; value = tokens processed by all ranks / that time.
+Multi-GPU: one process per GPU.  Run as is with ``--gpus N`` (N > 1), bench.py
+starts the N ranks itself through torch.distributed.run; under torchrun, WORLD_SIZE
+must equal N.  Every rank runs its own independent sequence (weak scaling, no
+data-path collective); the step time is the max over ranks; value = tokens processed
+by all ranks / that time.
 ``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
-workload (rank 0 only).
+workload (rank 0 only) and reports the whole-step throughput extrapolated from it.
 """
 from __future__ import annotations
 
@@ -35,6 +37,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "Hybrid-attn prefill tokens/s at 128K (lightning+sparse); % of roofline"
+# DRAM read + write bytes per launch of a kernel, by T (see the comment where it is used)
+NCU_TRAFFIC = {131072: {}}
 B, H, HKV, D = 1, 32, 2, 128
 CHUNK, BLOCK, TOPK, N_INIT, N_LOCAL = 128, 64, 64, 1, 2
 SPARSE_LAYERS = (2, 6)
@@ -255,56 +259,93 @@ def count_launches(layers, sala):
     return n
 
 
-def cpu_baseline(T, small=False):
-    """Time the fp64 oracle on a bounded, stratified sample of the same workload and
-    scale it to tokens/s of the whole 8-layer stack.  Returns (tok/s, info)."""
-    import oracle
-    from sparse_attention_long_lightning_b200 import inputs
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    # Lightning: 16 heads x nt tokens (all cores busy), per token-head cost.
-    nh, nt = 16, (256 if small else 1024)
-    x = inputs.lightning_inputs(1, nt, nh, D, seed=1005)
-    arr = [t.double().numpy() for t in (x.q, x.k, x.v, x.g)]
-    t0 = time.perf_counter()
-    oracle.lightning_recurrent(*arr)
-    light_s_per_tokhead = (time.perf_counter() - t0) / (nh * nt)
-    # Sparse: selection + attention for rows spread evenly over [0, T), both KV heads.
-    s = inputs.sparse_inputs(1, T, H, HKV, D, seed=1007, gate=True)
-    k64, v64 = s.k.double().numpy(), s.v.double().numpy()
-    nrows = 32 if small else 128
-    rows = np.unique(np.linspace(0, T - 1, nrows).astype(np.int64))
-    q_rows, g_rows = s.q[:, rows].double().numpy(), s.g[:, rows].double().numpy()
-    t0 = time.perf_counter()
-    idx, _ = oracle.sparse_select(q_rows, k64, rows=rows, T=T)
-    oracle.attention(q_rows, k64, v64, g_rows, idx=idx, rows=rows)
-    sparse_s_per_row = (time.perf_counter() - t0) / len(rows)
-    per_token = 6 * H * light_s_per_tokhead + 2 * sparse_s_per_row
-    info = {"kind": "oracle", "cores": cores,
-            "sample": f"Lightning: {nh} heads x {nt} tokens; sparse: {len(rows)} rows evenly "
-                      f"spaced over T={T} (select+attention, 2 KV heads); scaled to 6 Lightning "
-                      f"+ 2 sparse layers x {T} tokens"}
-    return 1.0 / per_token, info
+ORACLE_SAMPLE = {"light_heads": 16, "light_tokens": 1024, "sparse_rows": 128}
+
+
+class OracleSample:
+    """A bounded, stratified sample of one step for the fp64 oracle on the host cores:
+    Lightning over `light_heads` heads x `light_tokens` tokens, and selection + attention
+    of the sparse layer for `sparse_rows` rows evenly spaced over [0, T) (both KV heads).
+    The inputs are drawn once; time() runs the oracle on the sample and scales each
+    part by its share of the full step (6 Lightning layers x 32 heads x T tokens, 2 sparse
+    layers x T rows).  The in-bench cpu_baseline and `--impl reference` use this same
+    sample."""
+
+    def __init__(self, T):
+        from sparse_attention_long_lightning_b200 import inputs
+        self.T = T
+        nh, nt, nr = (ORACLE_SAMPLE[k] for k in ("light_heads", "light_tokens", "sparse_rows"))
+        x = inputs.lightning_inputs(1, nt, nh, D, seed=1005)
+        self.light = [t.double().numpy() for t in (x.q, x.k, x.v, x.g)]
+        s = inputs.sparse_inputs(1, T, H, HKV, D, seed=1007, gate=True)
+        self.k64, self.v64 = s.k.double().numpy(), s.v.double().numpy()
+        self.rows = np.unique(np.linspace(0, T - 1, nr).astype(np.int64))
+        self.q_rows = s.q[:, self.rows].double().numpy()
+        self.g_rows = s.g[:, self.rows].double().numpy()
+        self.light_units = nh * nt                  # token-heads in the sample
+        self.sparse_units = len(self.rows)          # rows in the sample
+        self.light_factor = 6 * H * T / self.light_units
+        self.sparse_factor = 2 * T / self.sparse_units
+        self.cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+        self.description = (f"Lightning: {nh} heads x {nt} tokens (x{self.light_factor:.0f} to "
+                            f"6 layers x {H} heads x {T} tokens); sparse: {len(self.rows)} rows "
+                            f"evenly spaced over T={T}, select+attention, 2 KV heads "
+                            f"(x{self.sparse_factor:.0f} to 2 layers x {T} rows)")
+
+    def time(self):
+        """(seconds the sample took, extrapolated seconds of one full step)."""
+        import oracle
+        t0 = time.perf_counter()
+        oracle.lightning_recurrent(*self.light)
+        t1 = time.perf_counter()
+        idx, _ = oracle.sparse_select(self.q_rows, self.k64, rows=self.rows, T=self.T)
+        oracle.attention(self.q_rows, self.k64, self.v64, self.g_rows, idx=idx, rows=self.rows)
+        t2 = time.perf_counter()
+        full = (t1 - t0) * self.light_factor + (t2 - t1) * self.sparse_factor
+        return t2 - t0, full
+
+    def info(self):
+        return {"kind": "oracle", "cores": self.cores, "sample": self.description,
+                "extrapolated": True,
+                "factor": {"lightning": self.light_factor, "sparse": self.sparse_factor}}
+
+
+def cpu_baseline(T):
+    """Time the fp64 oracle once on the bounded sample and scale it to tokens/s of the
+    whole 8-layer stack.  Returns (tok/s, info)."""
+    smp = OracleSample(T)
+    _, full = smp.time()
+    return T / full, smp.info()
 
 
 def run_reference(args):
-    """--impl reference: the fp64 CPU oracle on a bounded sample of the workload."""
+    """--impl reference: the fp64 CPU oracle, as it stands, on the bounded sample of the
+    workload (rank 0 only; other ranks exit without work).  Each step times the sample
+    once; `steps` counts the samples timed and `ms_per_step` is their measured time.  The
+    value is the whole-step throughput extrapolated from the sample (marked as such)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     T = args.T
-    times = []
-    info = None
+    smp = OracleSample(T)
+    sample_s, full_s = [], []
     for i in range(args.warmup + args.steps):
-        t0 = time.perf_counter()
-        tps, info = cpu_baseline(T, small=True)
+        a, b = smp.time()
         if i >= args.warmup:
-            times.append(T / tps)
-    sec = float(np.mean(times))
-    value = T / sec
+            sample_s.append(a)
+            full_s.append(b)
+    full = float(np.mean(full_s))
+    value = T / full
+    info = smp.info()
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": float(np.mean(sample_s)) * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
+            "extrapolated": {"value_from": "sample", "sample": info["sample"],
+                             "factor": info["factor"],
+                             "full_step_ms_estimate": full * 1e3,
+                             "ms_per_step_is": "measured time of one sample"},
             "config": {"workload": f"SALA hybrid attention prefill, 8 layers (Lightning 0,1,3,4,5,7;"
                                    f" sparse 2,6), B1 T{T} H32 Hkv2 D128",
                        "global_batch": B, "seq_len": T, "parallelism": "cpu"},
@@ -313,6 +354,28 @@ def run_reference(args):
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
     return 0
+
+
+def launch_ranks(args):
+    """`--gpus N` with N > 1 outside torchrun: start N ranks on this node through
+    torch.distributed.run (one process per GPU, rendezvous on 127.0.0.1) and return its
+    exit status.  Inside torchrun, WORLD_SIZE must equal N."""
+    ws = os.environ.get("WORLD_SIZE")
+    if ws is not None:
+        if int(ws) != args.gpus:
+            sys.stderr.write(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={ws}\n")
+            return 2
+        return None
+    if args.gpus <= 1:
+        return None
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={args.gpus}", "--master-addr", "127.0.0.1",
+           "--master-port", str(port), os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
 
 
 def e2e_measure(layers, sala, steps, stream):
@@ -426,6 +489,58 @@ def decode_components(dev, hbm):
     return out
 
 
+def projection_components(dev, hbm, tf_burst):
+    """The fused projection GEMM of a Lightning layer (x [16384, 4096] times W [16384,
+    4096]^T, QK-norm / RoPE / sigmoid epilogue) against the bf16 tensor peak, and the
+    Lightning prefill on prepared operands at T=131072 against HBM (same bytes as the raw
+    prefill: qh, kh, gate (fp16) and v read, o written).  Timed alone, outside the hybrid
+    step."""
+    import sparse_attention_long_lightning_b200 as sala
+    from sparse_attention_long_lightning_b200 import inputs
+
+    def timed(fn, iters=10, warmup=3):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(iters):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / iters  # ms
+
+    out = {}
+    Tp, hidden = 16384, 4096
+    gen = inputs.generator(1008, dev)
+    x = inputs.randn((1, Tp, hidden), gen, device=dev)
+    w = inputs.randn((4 * H * D, hidden), gen, device=dev, scale=hidden ** -0.5)
+    outs = sala.lightning_projection(x, w, heads=H, head_dim=D)
+    ms = timed(lambda: sala.lightning_projection(x, w, heads=H, head_dim=D, out=outs))
+    flops = 2.0 * Tp * hidden * 4 * H * D
+    out["lightning_projection_t16k"] = {"ms": ms, "TFLOP/s": flops / ms / 1e9,
+                                        "frac_tensor": flops / ms / 1e9 / tf_burst,
+                                        "peak": "bf16_tflops (burst, timed alone)"}
+    del x, w, outs
+    T = 131072
+    qh = inputs.randn((1, T, H, D), gen, torch.float16, dev)
+    kh = inputs.randn((1, T, H, D), gen, torch.float16, dev)
+    v = inputs.randn((1, T, H, D), gen, device=dev)
+    gate = inputs.randn((1, T, H, D), gen, device=dev).sigmoid().to(torch.float16)
+    o = torch.empty_like(v)
+    ws = torch.empty(sala.lightning_prefill_workspace(1, T, H, D, CHUNK), dtype=torch.uint8,
+                     device=dev)
+    ms = timed(lambda: sala.lightning_prefill_prepared(qh, kh, v, gate, None, out=o,
+                                                       workspace=ws))
+    nbytes = 5 * T * H * D * 2 + H * D * D * 4
+    out["lightning_prefill_prepared"] = {"ms": ms, "GB/s": nbytes / ms / 1e6,
+                                         "frac_hbm": nbytes / ms / 1e6 / hbm}
+    err = sala.get_device_error()
+    if err:
+        raise RuntimeError(f"device error in the projection components: {sala.status_string(err)}")
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -439,6 +554,9 @@ def main():
     ap.add_argument("--share-buffers", action="store_true",
                     help="one input/output set per layer type (implied for T > 131072)")
     args = ap.parse_args()
+    rc = launch_ranks(args)
+    if rc is not None:
+        return rc
     if args.impl == "reference":
         return run_reference(args)
 
@@ -505,11 +623,11 @@ def main():
         "sparse_attn": {"ms": op_ms["attn"], "TFLOP/s": attn_flops / op_ms["attn"] / 1e9,
                         "frac_tensor": attn_flops / op_ms["attn"] / 1e9 / tf_sust},
     }
-    # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch, from one
-    # ncu capture of this command at T=131072 with the current kernels (the sparse
-    # kernel's own launch; Lightning = state pass + scan + output pass; selection =
-    # block means + fused kernel).  Re-measure whenever one of those kernels changes.
-    ncu_traffic = {"attn": 9.64e9, "sel": 1.16e9} if T == 131072 else {}
+    # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
+    # dominant kernels, each from a capture of that one kernel alone (profile_case.py,
+    # `-k` one kernel, `-c` a few launches, a few GB on the device), summarised under
+    # profiles/.  Set to None when a kernel changes until it is captured again.
+    ncu_traffic = NCU_TRAFFIC.get(T, {})
     share = {k: n_ops[k] * op_ms[k] for k in op_ms}
     dom = max(share, key=share.get)
     if dom == "attn":
@@ -554,6 +672,7 @@ def main():
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                        "ms_per_step": e2e_sec * 1e3}
         line["components"].update(decode_components(dev, hbm))
+        line["components"].update(projection_components(dev, hbm, tf_burst))
         if rank == 0 and world == 1:
             tps, info = cpu_baseline(T)
             line["cpu_baseline"] = dict(info, value=tps, unit="tokens/s")

@@ -50,7 +50,8 @@ typedef enum {
     SALA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
     SALA_ERR_TIMEOUT = 4,      /* a device-side bounded wait ran out */
     SALA_ERR_WORKSPACE = 5,    /* workspace missing or smaller than required */
-    SALA_ERR_RANGE = 6         /* a value left the fp16 operand range on the device */
+    SALA_ERR_RANGE = 6         /* a non-finite value reached a result on the device, or a
+                                  decode position lies outside the cache */
 } sala_status;
 
 typedef enum { SALA_F32 = 0, SALA_BF16 = 1 } sala_dtype;
@@ -90,10 +91,15 @@ const char *sala_version(void);
  *   pos0        position of token 0 (RoPE), >= 0
  *   workspace   device scratch of at least sala_lightning_prefill_workspace()
  *               bytes (may be NULL when that returns 0); contents are scratch
+ *               (per-segment states and each segment's largest |v|)
  *   dt          SALA_BF16 (D = 64 or 128) or SALA_F32 (D = 64 or 128)
+ * Values: any finite bf16 v.  The tensor-core path multiplies v in fp16 after a
+ *   power-of-two scale chosen per token segment from the segment's largest |v| (a
+ *   segment whose values fp16 does not hold is recomputed with that scale), and
+ *   undoes the scale in fp32.
  * Errors: INVALID_ARG (null q/k/v/o/state, bad sizes, strides or alignment),
  *         UNSUPPORTED (other D/chunk/dtype), WORKSPACE, CUDA.  Device: RANGE
- *         when a bf16-path tensor-core operand exceeds the fp16 range.
+ *         when an output or the state is not finite (a non-finite input).
  */
 size_t sala_lightning_prefill_workspace(int B, int T, int H, int D, int chunk, sala_dtype dt);
 
@@ -226,11 +232,14 @@ sala_status sala_sparse_select_head_softmax(const void *q, const void *k, int B,
  *   scale       softmax scale; 0 selects 1/sqrt(D)
  *   ws          device scratch of >= sala_sparse_attn_workspace() bytes, 16-byte
  *               aligned, caller-owned; it receives an fp16 copy of v (the P.V
- *               tensor-core operand) and may be reused once the call has run
+ *               tensor-core operand) times 2^-e, e a power-of-two exponent per
+ *               (sequence, KV head) chosen from the largest |v| so that any finite
+ *               bf16 v keeps its significant bits (the output is multiplied by
+ *               2^e), and may be reused once the call has run
  *   block = 64, D = 64 or 128, 1 <= Hq / Hkv <= 16 (the GQA group fills one
  *   16-row tensor-core tile, padded with zero rows when smaller).
- * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.  Device: RANGE when a v value
- *   does not fit the fp16 tensor-core operand (|v| >= 65536).
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.  Device: RANGE when v holds
+ *   an infinite or NaN value.
  */
 size_t sala_sparse_attn_workspace(int B, int T, int Hkv, int D);
 
@@ -263,9 +272,11 @@ sala_status sala_sparse_attn(const void *q, const void *k, const void *v, const 
  *   ws          device scratch of >= sala_sparse_decode_workspace() bytes, 16-byte
  *               aligned, caller-owned (scores, selection, split partials)
  *   block = 64, Tmax a multiple of 64, D = 64 or 128, 1 <= Hq / Hkv <= 16.
+ * Values: any finite bf16 v (P.V runs as two bf16 products, P's high and low parts,
+ *   on v as stored).
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.  Device: RANGE when a pos[b] lies
- *   outside [0, Tmax) (that sequence is skipped) or a v value does not fit the fp16
- *   tensor-core operand (|v| >= 65536).
+ *   outside [0, Tmax) (that sequence is skipped) or an output is not finite (a
+ *   non-finite input).
  */
 size_t sala_sparse_decode_workspace(int B, int Tmax, int Hq, int Hkv, int D, int n_sel);
 
@@ -288,14 +299,59 @@ sala_status sala_sparse_block_means(const void *k, int B, int T, int Hkv, int D,
                                     float *kbar, int kbar_blocks, sala_dtype dt, void *stream);
 
 /*
+ * Input projection of a Lightning layer with its operand preparation fused into the GEMM
+ * epilogue (tech-report mirror, section 02 (3): QK-normalisation and an output gate in
+ * the linear layers; section 02 (4): RoPE in the linear layers):
+ *   [q | k | v | g] = x W^T;  qh = RoPE(RMSNorm(q) * q_norm_w), kh = RoPE(RMSNorm(k) *
+ *   k_norm_w) at position pos0 + t;  v as projected;  gate = sigmoid(g) (fp16: a value
+ *   in (0, 1)).
+ * The weights are the caller's (the pages publish none; tests use seeded synthetic ones).
+ *
+ *   x        [B, T, hidden] bf16, rows packed: row r = b*T + t at x + r * x_row_stride
+ *            (elements; x_row_stride >= hidden, rows 16-byte aligned)
+ *   w        [4 H D, hidden] bf16 contiguous: rows h*D.. of section s (q, k, v, g) are
+ *            head h's output features
+ *   q_norm_w, k_norm_w  [D] fp32 or NULL (weight 1)
+ *   qh, kh, gate  [B,T,H,D] fp16 outputs;  v  [B,T,H,D] bf16 output (strides sq..sg)
+ *   D = 64 or 128, hidden a multiple of 64, H*D a multiple of 256; dt = SALA_BF16.
+ * tcgen05 GEMM (128 x 256 tiles, fp32 accumulation in tensor memory); no workspace.
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA.
+ */
+sala_status sala_lightning_projection(const void *x, const void *w, const float *q_norm_w,
+                                      const float *k_norm_w, void *qh, void *kh, void *v,
+                                      void *gate, int B, int T, int hidden, int H, int D,
+                                      int64_t x_row_stride, sala_strides sq, sala_strides sk,
+                                      sala_strides sv, sala_strides sg, int64_t pos0,
+                                      float rope_base, float eps, sala_dtype dt, void *stream);
+
+/*
+ * Lightning prefill on prepared operands, the outputs of sala_lightning_projection: the
+ * recurrence of sala_lightning_prefill with q, k already normalised and rotated and the
+ * gate already a multiplier,
+ *   S_t = S_{t-1} + kh_t v_t^T,  y_t = gate_t * (qh_t^T S_t)   (gate NULL: no gate).
+ *   qh, kh, gate  [B,T,H,D] fp16;  v, o  [B,T,H,D] bf16;  state as in
+ *            sala_lightning_prefill (in/out, or zero-initialised with init_zero)
+ *   D = 128, chunk = 128 (tensor-core path); workspace of
+ *   sala_lightning_prefill_workspace(B, T, H, 128, 128, SALA_BF16) bytes.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.  Device: RANGE when an output or
+ *   the state is not finite.
+ */
+sala_status sala_lightning_prefill_prepared(const void *qh, const void *kh, const void *v,
+                                            const void *gate, void *o, float *state, int B, int T,
+                                            int H, int D, sala_strides sq, sala_strides sk,
+                                            sala_strides sv, sala_strides sg, sala_strides so,
+                                            int chunk, int init_zero, void *workspace,
+                                            size_t workspace_bytes, void *stream);
+
+/*
  * Lightning prefill that allocates nothing (no counterpart in the paper: this is
  * a library convenience).  Some callers cannot hand the library a workspace:
  * code embedded in a host framework that owns all device memory and offers its
  * plugins no allocator, or a serving loop whose memory pool is frozen after
  * start-up and must not call cudaMalloc on the hot path.  This entry point takes
  * the same arguments as sala_lightning_prefill minus the workspace and keeps its
- * per-segment state scratch in a fixed 16 MiB array that lives in the library's
- * device image (every GPU that loads the library holds it until exit).
+ * per-segment state scratch in a fixed array of 16 MiB + 64 KiB that lives in the
+ * library's device image (every GPU that loads the library holds it until exit).
  *
  * Limits: the bf16 / head_dim 128 / chunk 128 path needs B*H <= 256 (one 64 KiB
  * state per segment, at least one segment per head); larger B*H returns

@@ -17,7 +17,7 @@ import torch
 
 __all__ = [
     "SalaError", "load_library", "lightning_prefill", "lightning_prefill_workspace",
-    "lightning_prefill_noalloc",
+    "lightning_prefill_noalloc", "lightning_projection", "lightning_prefill_prepared",
     "lightning_decode", "sparse_select", "sparse_select_workspace", "sparse_select_head_softmax_workspace", "sparse_attn",
     "sparse_attn_workspace",
     "get_device_error", "selftest_wait_timeout", "sparse_decode", "sparse_decode_workspace",
@@ -99,6 +99,12 @@ def load_library(path: Optional[str] = None):
     lib.sala_lightning_prefill_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, S,
                                                    S, S, S, S, i, i64, f, f, i, i, vp]
     lib.sala_lightning_prefill_noalloc.restype = i
+    lib.sala_lightning_projection.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i64,
+                                              S, S, S, S, i64, f, f, i, vp]
+    lib.sala_lightning_projection.restype = i
+    lib.sala_lightning_prefill_prepared.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, S, S, S, S,
+                                                    S, i, i, vp, sz, vp]
+    lib.sala_lightning_prefill_prepared.restype = i
     lib.sala_lightning_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, S, S, S, S,
                                           S, f, f, i, vp]
     lib.sala_lightning_decode.restype = i
@@ -240,6 +246,68 @@ def lightning_prefill_noalloc(q, k, v, g, state, out, q_norm_w=None, k_norm_w=No
         _s4(q), _s4(k), _s4(v), _s4(g), _s4(out), int(chunk), int(pos0), float(rope_base),
         float(eps), 1 if init_zero else 0, _dt(q), _stream(stream))
     _check("sala_lightning_prefill_noalloc", st)
+    return out, state
+
+
+def lightning_projection(x, w, q_norm_w=None, k_norm_w=None, *, heads, head_dim=128, pos0=0,
+                         rope_base=10000.0, eps=1e-6, out=None, stream=None):
+    """Input projection of a Lightning layer with its preparation fused in.
+
+    x: [B, T, hidden] bf16 (rows packed: x.stride(0) == T * x.stride(1)); w: [4 H D,
+    hidden] bf16 contiguous (q heads, then k, v, g).  Returns (qh, kh, v, gate), each
+    [B, T, H, D]: qh, kh fp16 (RMSNorm, norm weight, RoPE at pos0 + t), v bf16, gate =
+    sigmoid(g) fp16.  `out` may give the four output tensors."""
+    lib = load_library()
+    _cuda(x, w, q_norm_w, k_norm_w)
+    B, T, hidden = x.shape
+    H, D = int(heads), int(head_dim)
+    if x.dtype != torch.bfloat16 or w.dtype != torch.bfloat16:
+        raise TypeError("x and w must be bf16")
+    if w.shape != (4 * H * D, hidden) or not w.is_contiguous():
+        raise ValueError("w must be a contiguous [4 H D, hidden] tensor")
+    if x.stride(2) != 1 or (B > 1 and x.stride(0) != T * x.stride(1)):
+        raise ValueError("x rows must be packed with unit stride along hidden")
+    if out is None:
+        shape = (B, T, H, D)
+        out = (torch.empty(shape, dtype=torch.float16, device=x.device),
+               torch.empty(shape, dtype=torch.float16, device=x.device),
+               torch.empty(shape, dtype=torch.bfloat16, device=x.device),
+               torch.empty(shape, dtype=torch.float16, device=x.device))
+    qh, kh, v, gate = out
+    _cuda(qh, kh, v, gate)
+    st = lib.sala_lightning_projection(
+        _p(x), _p(w), _p(q_norm_w), _p(k_norm_w), _p(qh), _p(kh), _p(v), _p(gate), B, T, hidden,
+        H, D, x.stride(1), _s4(qh), _s4(kh), _s4(v), _s4(gate), int(pos0), float(rope_base),
+        float(eps), SALA_BF16, _stream(stream))
+    _check("sala_lightning_projection", st)
+    return qh, kh, v, gate
+
+
+def lightning_prefill_prepared(qh, kh, v, gate=None, state=None, *, chunk=128, out=None,
+                               workspace=None, stream=None):
+    """Lightning prefill on prepared operands (lightning_projection's outputs): qh, kh
+    [B,T,H,D] fp16 already normalised and rotated, v bf16, gate fp16 multiplier (or
+    None).  `state` as in lightning_prefill.  Returns (out [B,T,H,D] bf16, state)."""
+    lib = load_library()
+    _cuda(qh, kh, v, gate, state, out)
+    B, T, H, D = qh.shape
+    if qh.dtype != torch.float16 or kh.dtype != torch.float16 or v.dtype != torch.bfloat16:
+        raise TypeError("qh, kh must be fp16 and v bf16")
+    if gate is not None and gate.dtype != torch.float16:
+        raise TypeError("gate must be fp16 (the sigmoid multiplier)")
+    init_zero = 1 if state is None else 0
+    if state is None:
+        state = torch.empty((B, H, D, D), dtype=torch.float32, device=qh.device)
+    if out is None:
+        out = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=qh.device)
+    need = lightning_prefill_workspace(B, T, H, D, chunk, torch.bfloat16)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=qh.device)
+    wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib.sala_lightning_prefill_prepared(
+        _p(qh), _p(kh), _p(v), _p(gate), _p(out), _p(state), B, T, H, D, _s4(qh), _s4(kh),
+        _s4(v), _s4(gate), _s4(out), int(chunk), init_zero, _p(workspace), wsb, _stream(stream))
+    _check("sala_lightning_prefill_prepared", st)
     return out, state
 
 

@@ -30,15 +30,15 @@ struct CCSmem {
   static constexpr size_t bytes = (S + 3 * Q + A) * sizeof(float);
 };
 
+// One head (b, h) = bh through all T_len tokens, starting from S0 ([D][D], or zero when
+// null) and leaving the final state in Sg.
 template <typename T, int D>
-__global__ void __launch_bounds__(kCCThreads)
-lightning_prefill_cc_kernel(const T* __restrict__ q, const T* __restrict__ k,
-                            const T* __restrict__ v, const T* __restrict__ g,
-                            T* __restrict__ o, float* __restrict__ state,
-                            const float* __restrict__ qw, const float* __restrict__ kw,
-                            int H, int T_len, sala_strides sq, sala_strides sk, sala_strides sv,
-                            sala_strides sg, sala_strides so, int64_t pos0, double log2_base,
-                            float eps, int init_zero) {
+__device__ __forceinline__ void lightning_cc_head(
+    int bh, const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+    const T* __restrict__ g, T* __restrict__ o, const float* S0, float* Sg,
+    const float* __restrict__ qw, const float* __restrict__ kw, int H, int T_len,
+    sala_strides sq, sala_strides sk, sala_strides sv, sala_strides sg, sala_strides so,
+    int64_t pos0, double log2_base, float eps) {
   constexpr int kLd = CCSmem<D>::kLd;
   extern __shared__ float smem[];
   float* S = smem;                        // [D][D]
@@ -47,12 +47,10 @@ lightning_prefill_cc_kernel(const T* __restrict__ q, const T* __restrict__ k,
   float* Vs = Ks + CCSmem<D>::Q;
   float* As = Vs + CCSmem<D>::Q;          // [kCT][kCT+1]
 
-  const int bh = blockIdx.x;
   const int b = bh / H, h = bh % H;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  float* Sg = state + (size_t)bh * D * D;
 
-  for (int e = tid; e < D * D; e += kCCThreads) S[e] = init_zero ? 0.0f : Sg[e];
+  for (int e = tid; e < D * D; e += kCCThreads) S[e] = S0 ? S0[e] : 0.0f;
 
   const T* qb = q + b * sq.b + h * sq.h;
   const T* kb = k + b * sk.b + h * sk.h;
@@ -206,6 +204,60 @@ lightning_prefill_cc_kernel(const T* __restrict__ q, const T* __restrict__ k,
   }
   __syncthreads();
   for (int e = tid; e < D * D; e += kCCThreads) Sg[e] = S[e];
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kCCThreads)
+lightning_prefill_cc_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                            const T* __restrict__ v, const T* __restrict__ g,
+                            T* __restrict__ o, float* __restrict__ state,
+                            const float* __restrict__ qw, const float* __restrict__ kw,
+                            int H, int T_len, sala_strides sq, sala_strides sk, sala_strides sv,
+                            sala_strides sg, sala_strides so, int64_t pos0, double log2_base,
+                            float eps, int init_zero) {
+  float* Sg = state + (size_t)blockIdx.x * D * D;
+  lightning_cc_head<T, D>(blockIdx.x, q, k, v, g, o, init_zero ? nullptr : Sg, Sg, qw, kw, H,
+                          T_len, sq, sk, sv, sg, so, pos0, log2_base, eps);
+}
+
+// Largest |v| of a head far above its rms: the tensor-core path's fp16 operands (11
+// significant bits) would leave errors of ~2^-11 of the products with that value, which
+// for a head dominated by a few large values exceeds the 1e-2 bound relative to the
+// output's rms.  Such heads are recomputed in fp32.
+constexpr float kCCOutlierRatio = 16.0f;
+
+// Recomputes, on CUDA cores in fp32, every head (grid B*H) of a tensor-core prefill
+// whose v is outlier-heavy (largest |v| > kCCOutlierRatio x rms(v), from the per-segment
+// statistics the state pass wrote: vmax, vssq [B*H][G]); other heads return at once.
+// The start state comes from ws (segment 0's start state, [B*H][G][D][D]) since the
+// scan has already overwritten `state` with the final state.
+template <int D>
+__global__ void __launch_bounds__(kCCThreads)
+lightning_cc_fixup_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                          const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ g,
+                          __nv_bfloat16* __restrict__ o, float* __restrict__ state,
+                          const float* __restrict__ qw, const float* __restrict__ kw, int H,
+                          int T_len, sala_strides sq, sala_strides sk, sala_strides sv,
+                          sala_strides sg, sala_strides so, int64_t pos0, double log2_base,
+                          float eps, const float* __restrict__ ws, int G,
+                          const float* __restrict__ vmax, const float* __restrict__ vssq) {
+  const int bh = blockIdx.x;
+  __shared__ int s_flag;
+  if (threadIdx.x == 0) {
+    float m = 0.f;
+    double ss = 0.0;
+    for (int s = 0; s < G; ++s) {
+      m = fmaxf(m, vmax[(size_t)bh * G + s]);
+      ss += (double)vssq[(size_t)bh * G + s];
+    }
+    const double rms = sqrt(ss / ((double)T_len * D));
+    s_flag = (m < INFINITY) && (double)m > (double)kCCOutlierRatio * rms;
+  }
+  __syncthreads();
+  if (!s_flag) return;
+  lightning_cc_head<__nv_bfloat16, D>(bh, q, k, v, g, o, ws + (size_t)bh * G * D * D,
+                                      state + (size_t)bh * D * D, qw, kw, H, T_len, sq, sk, sv,
+                                      sg, so, pos0, log2_base, eps);
 }
 
 }  // namespace sala

@@ -122,18 +122,28 @@ __device__ __forceinline__ void lo_prep_qk_half(uint8_t* sQ, uint8_t* sK, int r,
 
 // Half of the v row (slab hf) to fp16 in place; half 1 runs four chunks out of step so
 // the two lanes of a row hit different bank groups.
-__device__ __forceinline__ void lo_prep_v_half(uint8_t* sV, int r, int hf) {
+// v is scaled by vscale (a power of two chosen from the segment's largest |v|; 1 for
+// values that fp16 holds as they are).
+__device__ __forceinline__ void lo_prep_v_half(uint8_t* sV, int r, int hf, float vscale) {
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
     uint4* a = reinterpret_cast<uint4*>(sV + hf * kTcSlab + swz128(r, (u + 4 * hf) & 7));
     uint4 x = *a;
-    x.x = bf16x2_to_f16x2(x.x); x.y = bf16x2_to_f16x2(x.y);
-    x.z = bf16x2_to_f16x2(x.z); x.w = bf16x2_to_f16x2(x.w);
+    if (vscale == 1.0f) {
+      x.x = bf16x2_to_f16x2(x.x); x.y = bf16x2_to_f16x2(x.y);
+      x.z = bf16x2_to_f16x2(x.z); x.w = bf16x2_to_f16x2(x.w);
+    } else {
+      x.x = bf16x2_to_f16x2_scaled(x.x, vscale); x.y = bf16x2_to_f16x2_scaled(x.y, vscale);
+      x.z = bf16x2_to_f16x2_scaled(x.z, vscale); x.w = bf16x2_to_f16x2_scaled(x.w, vscale);
+    }
     *a = x;
   }
 }
 
-// Gated bf16 epilogue of 32 columns: y = O * 2^e * sigmoid(g), stored as 64 bytes.
+// Gated bf16 epilogue of 32 columns: y = O * os * sigmoid(g) (os = 2^e undoes the operand
+// scales), stored as 64 bytes.  kGateMult: the gate tensor already holds the multiplier,
+// as fp16.
+template <bool kGateMult>
 __device__ __forceinline__ void lo_store32(const uint32_t (&r)[32], const uint4* gv, bool gated,
                                            float os, __nv_bfloat16* orow, uint32_t& bad) {
   float chk = 0.f;
@@ -144,9 +154,12 @@ __device__ __forceinline__ void lo_store32(const uint32_t (&r)[32], const uint4*
     for (int e = 0; e < 8; ++e) y[e] = __uint_as_float(r[8 * c8 + e]) * os;
     if (gated) {
       float gf[8];
-      bf16x8_to_f32(gv[c8], gf);
+      if (kGateMult)
+        f16x8_to_f32(gv[c8], gf);
+      else
+        bf16x8_to_f32(gv[c8], gf);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) y[e] *= sigmoidf_(gf[e]);
+      for (int e = 0; e < 8; ++e) y[e] *= kGateMult ? gf[e] : sigmoidf_(gf[e]);
     }
 #pragma unroll
     for (int e = 0; e < 8; ++e) chk += y[e];
@@ -162,6 +175,10 @@ __device__ __forceinline__ void lo_store32(const uint32_t (&r)[32], const uint4*
 
 // TMEM columns: P fp32 [0,128) with its fp16 copy in [0,32) and [64,96), O[2] [128,384),
 // S [384,512).
+// kPrepared: q and k arrive already normalised and rotated as fp16 and the gate tensor
+// holds sigmoid(g) as fp16 (the projection epilogue's outputs), so the PREP warps only
+// convert v.
+template <bool kPrepared>
 __global__ void __launch_bounds__(kTcThreads, 1)
 lightning_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                      const __grid_constant__ CUtensorMap tmv, const TcParams p) {
@@ -201,6 +218,11 @@ lightning_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
   const int c_begin = (int)((int64_t)seg * p.NC / p.G);
   const int c_end = (int)((int64_t)(seg + 1) * p.NC / p.G);
   const int nchunks = c_end - c_begin;
+  // v of this segment enters the MMAs as fp16 times 2^-ev (ev = 0 unless the segment's
+  // largest |v|, recorded by the state pass, lies outside what fp16 holds); the TMEM
+  // state and outputs carry the same factor, undone in the epilogue
+  const int ev = v_operand_exp(__ldg(p.vmax + (size_t)bh * p.G + seg));
+  const float vscale = pow2i(-ev), oscale = pow2i(ev);
   // CONV thread: TMEM lane row trow, columns 64*ch .. 64*ch+63
   const int lq = warp & 3, ch = (warp - 8) >> 2;
   const int trow = 32 * lq + lane;
@@ -281,8 +303,10 @@ lightning_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
       const float* src = wseg + (size_t)trow * 128 + 64 * ch;
 #pragma unroll
       for (int v4 = 0; v4 < 8; ++v4) {
-        const float4 x = *reinterpret_cast<const float4*>(src + 4 * v4);
-        const float4 y = *reinterpret_cast<const float4*>(src + 32 + 4 * v4);
+        float4 x = *reinterpret_cast<const float4*>(src + 4 * v4);
+        float4 y = *reinterpret_cast<const float4*>(src + 32 + 4 * v4);
+        x.x *= vscale; x.y *= vscale; x.z *= vscale; x.w *= vscale;
+        y.x *= vscale; y.y *= vscale; y.z *= vscale; y.w *= vscale;
         r0[4 * v4 + 0] = __float_as_uint(x.x); r0[4 * v4 + 1] = __float_as_uint(x.y);
         r0[4 * v4 + 2] = __float_as_uint(x.z); r0[4 * v4 + 3] = __float_as_uint(x.w);
         r1[4 * v4 + 0] = __float_as_uint(y.x); r1[4 * v4 + 1] = __float_as_uint(y.y);
@@ -325,9 +349,11 @@ lightning_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
       const int s = u & 1;
       uint8_t* st = stages + s * L::kStageBytes;
       fail |= !mbar_wait(&full_qk[s], (u >> 1) & 1);
-      if (!fail) lo_prep_qk_half(st, st + kTcTile, prow, phf, p, ang_tab + s * 32);
+      if constexpr (!kPrepared) {
+        if (!fail) lo_prep_qk_half(st, st + kTcTile, prow, phf, p, ang_tab + s * 32);
+      }
       fail |= !mbar_wait(&full_v[s], (u >> 1) & 1);
-      if (!fail) lo_prep_v_half(st + 2 * kTcTile, prow, phf);
+      if (!fail) lo_prep_v_half(st + 2 * kTcTile, prow, phf, vscale);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&prep_done[s]);
@@ -384,7 +410,8 @@ lightning_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
           uint32_t r[32];
           tc_ld32(t_o + 32 * hh, r);
           tc_wait_ld();
-          if (t < p.T) lo_store32(r, gv + 4 * hh, gated, pow2i(e_prev), orow + 32 * hh, bad);
+          if (t < p.T) lo_store32<kPrepared>(r, gv + 4 * hh, gated, pow2i(e_prev) * oscale, orow + 32 * hh,
+                              bad);
         }
       }
       {
@@ -492,7 +519,8 @@ lightning_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
           uint32_t r[32];
           tc_ld32(t_o + 32 * hh, r);
           tc_wait_ld();
-          if (t < p.T) lo_store32(r, gv + 4 * hh, gated, pow2i(e_prev), orow + 32 * hh, bad);
+          if (t < p.T) lo_store32<kPrepared>(r, gv + 4 * hh, gated, pow2i(e_prev) * oscale, orow + 32 * hh,
+                              bad);
         }
       }
     }

@@ -56,6 +56,8 @@ struct TcParams {
   const float* qw;
   const float* kw;
   float* ws;  // [B*H][G][128][128] fp32: segment sums, turned into segment start states
+  float* vmax;  // [B*H][G]: max |v| over each segment (written by the state pass)
+  float* vssq;  // [B*H][G]: sum of v^2 over each segment (written by the state pass)
   sala_strides sg, so;
   int B, T, H, G, NC;
   int64_t pos0;
@@ -79,14 +81,21 @@ __device__ __forceinline__ int tc_block_scale_exp(float m, float* red) {
   return x > 15 ? x - 15 : 0;
 }
 
-__device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
-
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* f) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     f[2 * i] = __uint_as_float(w[i] << 16);
     f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+__device__ __forceinline__ void f16x8_to_f32(const uint4& u, float* f) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+    f[2 * i] = h.x;
+    f[2 * i + 1] = h.y;
   }
 }
 __device__ __forceinline__ uint4 f32x8_to_f16(const float* f) {
@@ -113,20 +122,56 @@ __device__ __forceinline__ void tc_row_rot_init(TcRowRot& rr, int r, int qd, con
   }
 }
 
+// A quarter of raw bf16 row r of the v tile to fp16 in place, times vscale (a power of
+// two); its largest |v| goes into vmax and its sum of squares into vss.
+__device__ __forceinline__ void tc_prep_v_quarter(uint8_t* sV, int r, int qd, float vscale,
+                                                  float& vmax, float& vss) {
+  auto ld = [](const uint8_t* base, uint32_t off) {
+    return *reinterpret_cast<const uint4*>(base + off);
+  };
+  auto st = [](uint8_t* base, uint32_t off, uint4 v) {
+    *reinterpret_cast<uint4*>(base + off) = v;
+  };
+  // v: quarter qd converts chunks 4 (qd & 1) .. +3 of slab qd >> 1, the slab-1 quarters
+  // two chunks out of step, so the 8 lanes of a quarter-warp hit 8 different bank groups
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int c = 4 * (qd & 1) + ((u + 2 * (qd >> 1)) & 3);
+    const uint32_t a = (qd >> 1) * kTcSlab + swz128(r, c);
+    uint4 x = ld(sV, a);
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xffff0000u);
+      vmax = fmaxf(vmax, fmaxf(fabsf(lo), fabsf(hi)));
+      vss = fmaf(lo, lo, fmaf(hi, hi, vss));
+    }
+    if (vscale == 1.0f) {
+      x.x = bf16x2_to_f16x2(x.x); x.y = bf16x2_to_f16x2(x.y);
+      x.z = bf16x2_to_f16x2(x.z); x.w = bf16x2_to_f16x2(x.w);
+    } else {
+      x.x = bf16x2_to_f16x2_scaled(x.x, vscale); x.y = bf16x2_to_f16x2_scaled(x.y, vscale);
+      x.z = bf16x2_to_f16x2_scaled(x.z, vscale); x.w = bf16x2_to_f16x2_scaled(x.w, vscale);
+    }
+    st(sV, a, x);
+  }
+}
+
 // Normalise + rotate a quarter of raw bf16 row r of the k tile and convert it, and a
-// quarter of the v row, to fp16 in place.  Four consecutive lanes share a row: quarter
+// quarter of the v row (times vscale, a power of two; its largest |v| goes into vmax),
+// to fp16 in place.  Four consecutive lanes share a row: quarter
 // qd owns rotation pairs i in [16 qd, 16 qd + 16) (chunks 2qd, 2qd+1 of both 64-column
 // slabs) and four v chunks.  Tiles are two 64-column slabs of 128 rows x 128
 // bytes with the 128-byte swizzle.  `cs_tab` (a static shared array, read with ordinary
 // loads the compiler can schedule) holds the chunk's (cos B_i, sin B_i, cos B_i+1,
 // sin B_i+1) for even i at item (i mod 16) / 2 * 4 + i / 16, so the four quarters of a
-// row read adjacent 16-byte words.  An fp16 overflow here shows up downstream as a
-// non-finite output or state, which the output pass reports.
+// row read adjacent 16-byte words.
 __device__ __forceinline__ int tc_ang_item(int i) { return ((i & 15) >> 1) * 4 + (i >> 4); }
 
 __device__ __forceinline__ void tc_prep_kv_quarter(uint8_t* sK, uint8_t* sV, int r, int qd,
                                                    const TcParams& p, const float4* cs_tab,
-                                                   const TcRowRot& rr) {
+                                                   const TcRowRot& rr, float vscale,
+                                                   float& vmax, float& vss) {
   // ordinary 16-byte accesses: sK and sV point into the kernel's __shared__ array, so these
   // are shared-memory instructions the compiler is free to schedule
   auto ld = [](const uint8_t* base, uint32_t off) {
@@ -178,17 +223,7 @@ __device__ __forceinline__ void tc_prep_kv_quarter(uint8_t* sK, uint8_t* sV, int
     st(sK, alo, f32x8_to_f16(klo));
     st(sK, ahi, f32x8_to_f16(khi));
   }
-  // v: quarter qd converts chunks 4 (qd & 1) .. +3 of slab qd >> 1, the slab-1 quarters
-  // two chunks out of step, so the 8 lanes of a quarter-warp hit 8 different bank groups
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int c = 4 * (qd & 1) + ((u + 2 * (qd >> 1)) & 3);
-    const uint32_t a = (qd >> 1) * kTcSlab + swz128(r, c);
-    uint4 x = ld(sV, a);
-    x.x = bf16x2_to_f16x2(x.x); x.y = bf16x2_to_f16x2(x.y);
-    x.z = bf16x2_to_f16x2(x.z); x.w = bf16x2_to_f16x2(x.w);
-    st(sV, a, x);
-  }
+  tc_prep_v_quarter(sV, r, qd, vscale, vmax, vss);
 }
 
 // K-major operand (rows = M or N, 128-byte rows along K), k-step kk of 16 elements.
@@ -213,6 +248,9 @@ __device__ __forceinline__ uint64_t tc_desc_mn(const uint8_t* base, int kk) {
 constexpr int kStThreads = kTcThreads + 32;
 constexpr int kStAngRing = 8;  // > the largest lag (4 chunks) between producer and prep warps
 
+// kPrepared: k arrives already normalised and rotated as fp16 (the projection epilogue's
+// output), so the prep warps only convert v.
+template <bool kPrepared>
 __global__ void __launch_bounds__(kStThreads, 1)
 lightning_state_kernel(const __grid_constant__ CUtensorMap tmk,
                        const __grid_constant__ CUtensorMap tmv, const TcParams p) {
@@ -265,105 +303,161 @@ lightning_state_kernel(const __grid_constant__ CUtensorMap tmk,
   const uint32_t t_s = *tmem_slot;
   const uint32_t lane_off = (uint32_t)(32 * lq) << 16;
   bool ok = true;
+  // The first attempt converts v to fp16 as is and records the segment's largest |v|.
+  // If that lies outside what fp16 holds exactly (v_operand_exp != 0), the segment runs
+  // once more with v scaled by 2^-ev and the sum is scaled back by 2^ev when written:
+  // the workspace always holds unscaled fp32 sums.  Stage and phase bookkeeping runs on
+  // chunk counts that continue across the attempts.
+  float vmax = 0.f, vss = 0.f, vss_seg = 0.f;
+  float vscale = 1.0f;
+  int ev = 0;
+  __shared__ uint32_t s_vmax;
+  __shared__ float s_vss;
+  TcRowRot rr;
+  if constexpr (!kPrepared) {
+    if (!producer) tc_row_rot_init(rr, prow, pqd, inv_freq);
+  }
 
-  if (producer) {
-    // (cos, sin) of each rotation pair's angle at the first token of chunk n (fp64
-    // reduction), written by the 32 lanes, then chunk n's copy (lane 0)
-    auto fill_and_issue = [&](int n) {
-      const double two_pi = 6.283185307179586476925286766559;
-      const double t0 = (double)(p.pos0 + (int64_t)(c_begin + n) * kTcC);
-      float cs[2], sn[2];
+  for (int attempt = 0; attempt < 2; ++attempt) {
+    const int base = attempt * nchunks;  // global chunk count before this attempt
+    if (producer) {
+      // (cos, sin) of each rotation pair's angle at the first token of chunk n (fp64
+      // reduction), written by the 32 lanes, then chunk n's copy (lane 0)
+      auto fill_and_issue = [&](int n) {
+        const int gi = base + n;
+        if constexpr (!kPrepared) {
+          const double two_pi = 6.283185307179586476925286766559;
+          const double t0 = (double)(p.pos0 + (int64_t)(c_begin + n) * kTcC);
+          float cs[2], sn[2];
 #pragma unroll
-      for (int k = 0; k < 2; ++k) {  // pairs 2 lane, 2 lane + 1
-        const double a = t0 * inv_freq[2 * lane + k];
-        const float red = (float)(a - rint(a * (1.0 / two_pi)) * two_pi);
-        sincosf(red, &sn[k], &cs[k]);
+          for (int k = 0; k < 2; ++k) {  // pairs 2 lane, 2 lane + 1
+            const double a = t0 * inv_freq[2 * lane + k];
+            const float red = (float)(a - rint(a * (1.0 / two_pi)) * two_pi);
+            sincosf(red, &sn[k], &cs[k]);
+          }
+          ang_ring[(gi % kStAngRing) * 32 + tc_ang_item(2 * lane)] =
+              make_float4(cs[0], sn[0], cs[1], sn[1]);
+        }
+        __syncwarp();
+        if (lane == 0) {
+          const int si = gi % S;
+          uint8_t* dk = stages + si * L::kStageBytes;
+          uint8_t* dv = dk + kTcTile;
+          const int tok = (c_begin + n) * kTcC;
+          mbar_arrive_expect_tx(&full[si], L::kStageBytes);  // release: orders the table writes
+          tma_load_4d(dk, &tmk, &full[si], 0, h, tok, b);
+          tma_load_4d(dk + kTcSlab, &tmk, &full[si], 64, h, tok, b);
+          tma_load_4d(dv, &tmv, &full[si], 0, h, tok, b);
+          tma_load_4d(dv + kTcSlab, &tmv, &full[si], 64, h, tok, b);
+        }
+        __syncwarp();
+      };
+      if (lane == 0 && attempt == 0) {
+        prefetch_tmap(&tmk);
+        prefetch_tmap(&tmv);
       }
-      ang_ring[(n % kStAngRing) * 32 + tc_ang_item(2 * lane)] =
-          make_float4(cs[0], sn[0], cs[1], sn[1]);
-      __syncwarp();
-      if (lane == 0) {
-        const int si = n % S;
-        uint8_t* dk = stages + si * L::kStageBytes;
-        uint8_t* dv = dk + kTcTile;
-        const int tok = (c_begin + n) * kTcC;
-        mbar_arrive_expect_tx(&full[si], L::kStageBytes);  // release: orders the table writes
-        tma_load_4d(dk, &tmk, &full[si], 0, h, tok, b);
-        tma_load_4d(dk + kTcSlab, &tmk, &full[si], 64, h, tok, b);
-        tma_load_4d(dv, &tmv, &full[si], 0, h, tok, b);
-        tma_load_4d(dv + kTcSlab, &tmv, &full[si], 64, h, tok, b);
-      }
-      __syncwarp();
-    };
-    if (lane == 0) {
-      prefetch_tmap(&tmk);
-      prefetch_tmap(&tmv);
-    }
-    int issued = 0;
-    for (; issued < S && issued < nchunks; ++issued) fill_and_issue(issued);
-    int mmas = 0;  // state MMAs issued (chunks 0 .. mmas-1)
-    for (int u = 0; u < nchunks; ++u) {
-      const int s = u % S;
-      // refill the stage of chunk u - 1 as soon as its MMA has read it (early in prep(u))
-      if (u >= 1 && issued < nchunks) {
-        if (lane == 0) ok = mbar_wait(&mma_done[(u - 1) % S], ((u - 1) / S) & 1);
+      int issued = 0;
+      for (; issued < S && issued < nchunks; ++issued) fill_and_issue(issued);
+      int mmas = 0;  // state MMAs issued in this attempt (chunks 0 .. mmas-1)
+      for (int u = 0; u < nchunks; ++u) {
+        const int gu = base + u;
+        const int s = gu % S;
+        // refill the stage of chunk u - 1 as soon as its MMA has read it (early in prep(u))
+        if (u >= 1 && issued < nchunks) {
+          if (lane == 0) ok = mbar_wait(&mma_done[(gu - 1) % S], ((gu - 1) / S) & 1);
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+          fill_and_issue(issued++);
+        }
+        if (lane == 0) {
+          ok = mbar_wait(&prepped[s], (gu / S) & 1);
+          if (ok) {
+            tc_fence_after();
+            uint8_t* sK = stages + s * L::kStageBytes;
+            uint8_t* sV = sK + kTcTile;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              tc_mma_ss(t_s, tc_desc_mn(sK, kk), tc_desc_mn(sV, kk), kIdState,
+                        (u == 0 && kk == 0) ? 0u : 1u);
+            tc_commit(&mma_done[s]);
+          }
+        }
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
-        fill_and_issue(issued++);
+        mmas = u + 1;
       }
       if (lane == 0) {
-        ok = mbar_wait(&prepped[s], (u / S) & 1);
-        if (ok) {
-          tc_fence_after();
-          uint8_t* sK = stages + s * L::kStageBytes;
-          uint8_t* sV = sK + kTcTile;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            tc_mma_ss(t_s, tc_desc_mn(sK, kk), tc_desc_mn(sV, kk), kIdState,
-                      (u == 0 && kk == 0) ? 0u : 1u);
-          tc_commit(&mma_done[s]);
-        }
+        // the last MMA issued completes before TMEM is read, re-initialised or released
+        if (mmas > 0 &&
+            !mbar_wait(&mma_done[(base + mmas - 1) % S], ((base + mmas - 1) / S) & 1))
+          ok = false;
+        // every copy issued lands before the CTA's shared memory goes away (on the normal
+        // path the prep warps have consumed them all already)
+        for (int n = issued > S ? issued - S : 0; n < issued; ++n)
+          mbar_wait(&full[(base + n) % S], ((base + n) / S) & 1);
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
-      mmas = u + 1;
+    } else {
+      for (int u = 0; u < nchunks; ++u) {
+        const int gu = base + u;
+        const int s = gu % S;
+        uint8_t* sK = stages + s * L::kStageBytes;
+        uint8_t* sV = sK + kTcTile;
+        ok = mbar_wait(&full[s], (gu / S) & 1);
+        if (ok) {
+          if constexpr (kPrepared)
+            tc_prep_v_quarter(sV, prow, pqd, vscale, vmax, vss);
+          else
+            tc_prep_kv_quarter(sK, sV, prow, pqd, p, ang_ring + (gu % kStAngRing) * 32, rr,
+                               vscale, vmax, vss);
+        }
+        fence_proxy_async_smem();
+        // a warp whose wait failed stops arriving; the producer's wait then runs out too
+        if (!__all_sync(0xffffffffu, ok)) break;
+        if (lane == 0) mbar_arrive(&prepped[s]);
+      }
     }
-    if (lane == 0) {
-      // the last MMA issued completes before TMEM is read or released
-      if (mmas > 0 && !mbar_wait(&mma_done[(mmas - 1) % S], ((mmas - 1) / S) & 1)) ok = false;
-      // every copy issued lands before the CTA's shared memory goes away (on the normal
-      // path the prep warps have consumed them all already)
-      for (int n = issued > S ? issued - S : 0; n < issued; ++n)
-        mbar_wait(&full[n % S], (n / S) & 1);
+    if (tid == 0) {
+      s_vmax = 0u;
+      s_vss = 0.f;
     }
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-  } else {
-    TcRowRot rr;
-    tc_row_rot_init(rr, prow, pqd, inv_freq);
-    for (int u = 0; u < nchunks; ++u) {
-      const int s = u % S;
-      uint8_t* sK = stages + s * L::kStageBytes;
-      uint8_t* sV = sK + kTcTile;
-      ok = mbar_wait(&full[s], (u / S) & 1);
-      if (ok) tc_prep_kv_quarter(sK, sV, prow, pqd, p, ang_ring + (u % kStAngRing) * 32, rr);
-      fence_proxy_async_smem();
-      // a warp whose wait failed stops arriving; the producer's wait then runs out too
-      if (!__all_sync(0xffffffffu, ok)) break;
-      if (lane == 0) mbar_arrive(&prepped[s]);
+    ok = __syncthreads_and(ok);
+    if (attempt == 1 || !ok) break;
+    // the segment's largest |v| (non-negative floats order as their bit patterns) and sum
+    // of squares
+    if (!producer) {
+      const uint32_t m = __reduce_max_sync(0xffffffffu, __float_as_uint(vmax));
+      float ss = vss;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      if (lane == 0) {
+        atomicMax(&s_vmax, m);
+        atomicAdd(&s_vss, ss);
+      }
     }
+    __syncthreads();
+    vmax = __uint_as_float(s_vmax);
+    vss_seg = s_vss;
+    ev = v_operand_exp(vmax);
+    if (ev == 0) break;
+    vscale = pow2i(-ev);
   }
-  ok = __syncthreads_and(ok);
+  if (tid == 0 && ok) {
+    p.vmax[(size_t)bh * p.G + seg] = vmax;
+    p.vssq[(size_t)bh * p.G + seg] = vss_seg;
+  }
   tc_fence_after();
   if (!producer && ok && nchunks > 0) {
     float* dst = p.ws + ((size_t)bh * p.G + seg) * (128 * 128) + (size_t)trow * 128 + 32 * cg;
     uint32_t r[32];
     tc_ld32(t_s + lane_off + 32 * cg, r);
     tc_wait_ld();
+    const float us = pow2i(ev);  // undo the v scale of a second attempt (1 otherwise)
 #pragma unroll
     for (int v4 = 0; v4 < 8; ++v4)
       *reinterpret_cast<float4*>(dst + 4 * v4) =
-          make_float4(__uint_as_float(r[4 * v4]), __uint_as_float(r[4 * v4 + 1]),
-                      __uint_as_float(r[4 * v4 + 2]), __uint_as_float(r[4 * v4 + 3]));
+          make_float4(__uint_as_float(r[4 * v4]) * us, __uint_as_float(r[4 * v4 + 1]) * us,
+                      __uint_as_float(r[4 * v4 + 2]) * us, __uint_as_float(r[4 * v4 + 3]) * us);
   }
   tc_fence_before();
   __syncthreads();
@@ -405,9 +499,22 @@ inline int lightning_tc_segments(int B, int H, int T, int nsm) {
   return G;
 }
 
+// Workspace: [B*H][G] segment states (fp32 128x128), then [B*H][G] floats of the
+// segments' largest |v| and [B*H][G] floats of their sums of v^2 (256-byte aligned).
+inline size_t lightning_tc_states_bytes(int B, int H, int G) {
+  return (size_t)B * H * G * 128 * 128 * sizeof(float);
+}
+inline size_t lightning_tc_vmax_bytes(int B, int H, int G) {
+  return ((size_t)B * H * G * sizeof(float) + 255) / 256 * 256;
+}
+// the segments' sums of v^2 follow their maxima
+inline size_t lightning_tc_stats_bytes(int B, int H, int G) {
+  return 2 * lightning_tc_vmax_bytes(B, H, G);
+}
 inline size_t lightning_tc_workspace(int B, int T, int H, int chunk, int nsm) {
   if (chunk != kTcC || T <= 0) return 0;
-  return (size_t)B * H * lightning_tc_segments(B, H, T, nsm) * 128 * 128 * sizeof(float);
+  const int G = lightning_tc_segments(B, H, T, nsm);
+  return lightning_tc_states_bytes(B, H, G) + lightning_tc_stats_bytes(B, H, G);
 }
 
 }  // namespace sala

@@ -181,12 +181,47 @@ __device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
 }
+// bf16 pair (lo in the low half) from two floats, round to nearest even.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+// a, b -> packed bf16x2 of their round-to-nearest values (low half = a); `lo` gets the
+// packed bf16x2 of the rounding residuals, so hi + lo carries ~16 significant bits.
+__device__ __forceinline__ uint32_t pack_bf16x2_hi_lo(float a, float b, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  const float2 hf = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
 // Packed bf16x2 -> packed f16x2 (exact inside the fp16 normal range).
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t x) {
   const float lo = __uint_as_float(x << 16);
   const float hi = __uint_as_float(x & 0xffff0000u);
   return pack_f16x2(lo, hi);
 }
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
+
+// Power-of-two exponent e for the fp16 copy of v over a token range whose largest |v| is
+// m: v * 2^-e stays below 2^15 and its largest value above 2^-4, so the 11 significant
+// bits of fp16 hold every bf16 value that matters to the result (values more than 2^-19
+// below the largest lose low bits as fp16 subnormals, far below the tolerance).  0 when
+// the fp16 range already holds the values, and for a zero or non-finite maximum (a
+// non-finite input is reported downstream as a non-finite output).
+__device__ __forceinline__ int v_operand_exp(float m) {
+  if (!(m > 0.0f) || !(m < INFINITY)) return 0;
+  int x = 0;
+  frexpf(m, &x);  // m < 2^x
+  if (x >= -3 && x <= 15) return 0;
+  return min(max(x - 15, -110), 110);
+}
+
+// Packed bf16x2 -> packed f16x2 of the values times s (a power of two).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_scaled(uint32_t x, float s) {
+  return pack_f16x2(__uint_as_float(x << 16) * s, __uint_as_float(x & 0xffff0000u) * s);
+}
+
 // Non-zero if either half of a packed f16x2 is inf or NaN.
 __device__ __forceinline__ uint32_t f16x2_nonfinite(uint32_t x) {
   return ((x & 0x7c00u) == 0x7c00u) | ((x & 0x7c000000u) == 0x7c000000u);
@@ -310,6 +345,43 @@ __device__ __forceinline__ void tc_st32(uint32_t taddr, const uint32_t (&r)[32])
       "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
       "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
       "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+// 16 lanes x 64 columns of 32-bit data (shape 16x64b, 32 repetitions): thread t of the
+// warp gets TMEM lane (base + 8 (t & 1) + (t >> 2)), columns 2k + ((t >> 1) & 1) for
+// k = 0..31 in r[k].  Partner threads t and t ^ 2 share a lane (even / odd columns).
+__device__ __forceinline__ void tc_ld16x64(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x64b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tc_st16x64_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x64b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+// Same shape, 16 repetitions: thread t writes columns 2k + ((t >> 1) & 1), k = 0..15.
+__device__ __forceinline__ void tc_st16x64_x16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x64b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
       : "memory");
 }
 // Named barrier over `count` threads (a multiple of 32) of this CTA.

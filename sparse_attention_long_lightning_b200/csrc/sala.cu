@@ -18,6 +18,7 @@
 #include "lightning_decode.cuh"
 #include "lightning_tc.cuh"
 #include "lightning_out.cuh"
+#include "proj_gemm.cuh"
 #include "sparse_attn.cuh"
 #include "sparse_decode.cuh"
 #include "sparse_select.cuh"
@@ -86,6 +87,30 @@ bool make_tmap_bhtd(CUtensorMap* map, const void* base, int B, int T, int H, int
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// Per-segment statistics of v that the state pass writes, after the segment states.
+void set_tc_stats(TcParams& p, void* stats_base) {
+  uint8_t* base = static_cast<uint8_t*>(stats_base);
+  p.vmax = reinterpret_cast<float*>(base);
+  p.vssq = reinterpret_cast<float*>(base + lightning_tc_vmax_bytes(p.B, p.H, p.G));
+}
+
+// Heads whose v is outlier-heavy are recomputed in fp32 after a tensor-core prefill (or
+// state-only pass, o == nullptr); all other heads' CTAs return at once.
+bool launch_lightning_fixup(const void* q, const void* k, const void* v, const void* g, void* o,
+                            float* state, const float* qw, const float* kw, sala_strides sq,
+                            sala_strides sk, sala_strides sv, sala_strides sg, sala_strides so,
+                            const TcParams& p, cudaStream_t st) {
+  auto kern = lightning_cc_fixup_kernel<128>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)CCSmem<128>::bytes) != cudaSuccess)
+    return false;
+  kern<<<p.B * p.H, kCCThreads, CCSmem<128>::bytes, st>>>(
+      (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
+      (const __nv_bfloat16*)g, (__nv_bfloat16*)o, state, qw, kw, p.H, p.T, sq, sk, sv, sg, so,
+      p.pos0, p.log2_base, p.eps, p.ws, p.G, p.vmax, p.vssq);
+  return cudaPeekAtLastError() == cudaSuccess;
 }
 
 // dst = (accumulate ? dst : 0) + sum over i < count of src[i * stride + e], e < n.
@@ -208,13 +233,14 @@ sala_status sala_lightning_prefill(const void* q, const void* k, const void* v, 
     p.so = so;
     p.B = B; p.T = T; p.H = H;
     p.G = lightning_tc_segments(B, H, T, nsm);
+    set_tc_stats(p, (uint8_t*)workspace + lightning_tc_states_bytes(B, H, p.G));
     p.NC = (T + kTcC - 1) / kTcC;
     p.pos0 = pos0;
     p.log2_base = log2_base;
     p.eps = eps;
     const unsigned grid = (unsigned)(B * H * p.G);
-    auto ka = lightning_state_kernel;
-    auto kc = lightning_out_kernel;
+    auto ka = lightning_state_kernel<false>;
+    auto kc = lightning_out_kernel<false>;
     if (!set_smem(ka, TcSmem<true>::bytes) || !set_smem(kc, TcSmem<false>::bytes)) return SALA_ERR_CUDA;
     ka<<<grid, kStThreads, TcSmem<true>::bytes, st>>>(tk, tv, p);
     SALA_CHECK_LAUNCH();
@@ -222,6 +248,9 @@ sala_status sala_lightning_prefill(const void* q, const void* k, const void* v, 
     SALA_CHECK_LAUNCH();
     kc<<<grid, kTcThreads, TcSmem<false>::bytes, st>>>(tq, tk, tv, p);
     SALA_CHECK_LAUNCH();
+    if (!launch_lightning_fixup(q, k, v, g, o, state, q_norm_w, k_norm_w, sq, sk, sv, sg, so, p,
+                                st))
+      return SALA_ERR_CUDA;
     return SALA_OK;
   }
   const int grid = B * H;
@@ -254,6 +283,65 @@ sala_status sala_lightning_prefill(const void* q, const void* k, const void* v, 
         (const __nv_bfloat16*)g, (__nv_bfloat16*)o, state, q_norm_w, k_norm_w, H, T, sq, sk, sv,
         sg, so, pos0, log2_base, eps, init_zero);
   }
+  SALA_CHECK_LAUNCH();
+  return SALA_OK;
+}
+
+// Lightning prefill on prepared operands (the outputs of sala_lightning_projection):
+// fp16 q and k already normalised and rotated, bf16 v, fp16 gate multiplier.
+sala_status sala_lightning_prefill_prepared(const void* qh, const void* kh, const void* v,
+                                            const void* gate, void* o, float* state, int B,
+                                            int T, int H, int D, sala_strides sq,
+                                            sala_strides sk, sala_strides sv, sala_strides sg,
+                                            sala_strides so, int chunk, int init_zero,
+                                            void* workspace, size_t workspace_bytes,
+                                            void* stream) {
+  if (!state || (T > 0 && (!qh || !kh || !v || !o))) return SALA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || T < 0) return SALA_ERR_INVALID_ARG;
+  if (D != 128 || chunk != kTcC) return SALA_ERR_UNSUPPORTED;
+  if (!aligned16(qh) || !aligned16(kh) || !aligned16(v) || !aligned16(o) || !aligned16(state) ||
+      (gate && !aligned16(gate)))
+    return SALA_ERR_INVALID_ARG;
+  if (!strides_ok(sq, 2) || !strides_ok(sk, 2) || !strides_ok(sv, 2) || !strides_ok(so, 2) ||
+      (gate && !strides_ok(sg, 2)))
+    return SALA_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  if (T == 0) {
+    if (init_zero && cudaMemsetAsync(state, 0, sizeof(float) * (size_t)B * H * D * D, st) !=
+                         cudaSuccess)
+      return SALA_ERR_CUDA;
+    return SALA_OK;
+  }
+  const int nsm = num_sms();
+  const size_t need = lightning_tc_workspace(B, T, H, chunk, nsm);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return SALA_ERR_WORKSPACE;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_bhtd(&tq, qh, B, T, H, D, sq, kTcC, 1, true) ||
+      !make_tmap_bhtd(&tk, kh, B, T, H, D, sk, kTcC, 1, true) ||
+      !make_tmap_bhtd(&tv, v, B, T, H, D, sv, kTcC))
+    return SALA_ERR_CUDA;
+  TcParams p{};
+  p.g = (const __nv_bfloat16*)gate;
+  p.o = (__nv_bfloat16*)o;
+  p.ws = (float*)workspace;
+  p.sg = sg;
+  p.so = so;
+  p.B = B; p.T = T; p.H = H;
+  p.G = lightning_tc_segments(B, H, T, nsm);
+  set_tc_stats(p, (uint8_t*)workspace + lightning_tc_states_bytes(B, H, p.G));
+  p.NC = (T + kTcC - 1) / kTcC;
+  p.pos0 = 0;
+  p.log2_base = std::log2(10000.0);  // unused: the operands are already rotated
+  p.eps = 0.f;
+  const unsigned grid = (unsigned)(B * H * p.G);
+  auto ka = lightning_state_kernel<true>;
+  auto kc = lightning_out_kernel<true>;
+  if (!set_smem(ka, TcSmem<true>::bytes) || !set_smem(kc, TcSmem<false>::bytes)) return SALA_ERR_CUDA;
+  ka<<<grid, kStThreads, TcSmem<true>::bytes, st>>>(tk, tv, p);
+  SALA_CHECK_LAUNCH();
+  lightning_scan_kernel<<<dim3(B * H, 16), 256, 0, st>>>(p.ws, state, p.G, init_zero);
+  SALA_CHECK_LAUNCH();
+  kc<<<grid, kTcThreads, TcSmem<false>::bytes, st>>>(tq, tk, tv, p);
   SALA_CHECK_LAUNCH();
   return SALA_OK;
 }
@@ -296,6 +384,83 @@ sala_status sala_lightning_decode(const void* q, const void* k, const void* v, c
   return SALA_OK;
 }
 
+// ------------------------------------------------------------------ Lightning input projection
+namespace {
+// 2-D bf16 tensor map over `rows` rows of `cols` elements (row stride in elements) with a
+// (64, box_rows) box and 128-byte swizzle.
+bool make_tmap_2d(CUtensorMap* map, const void* base, int64_t rows, int cols, int64_t row_stride,
+                  int box_rows) {
+  auto enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_stride * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+}  // namespace
+
+sala_status sala_lightning_projection(const void* x, const void* w, const float* q_norm_w,
+                                      const float* k_norm_w, void* qh, void* kh, void* v,
+                                      void* gate, int B, int T, int hidden, int H, int D,
+                                      int64_t x_row_stride, sala_strides sq, sala_strides sk,
+                                      sala_strides sv, sala_strides sg, int64_t pos0,
+                                      float rope_base, float eps, sala_dtype dt, void* stream) {
+  if (B <= 0 || T < 0 || H <= 0 || hidden <= 0 || pos0 < 0 || !(rope_base > 1.0f) ||
+      !(eps >= 0.0f))
+    return SALA_ERR_INVALID_ARG;
+  if (T > 0 && (!x || !w || !qh || !kh || !v || !gate)) return SALA_ERR_INVALID_ARG;
+  if (dt != SALA_BF16) return SALA_ERR_UNSUPPORTED;
+  if ((D != 64 && D != 128) || hidden % kPjBK != 0 || (H * D) % kPjBN != 0)
+    return SALA_ERR_UNSUPPORTED;
+  if (x_row_stride < hidden || (x_row_stride * 2) % 16 != 0) return SALA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(qh) || !aligned16(kh) || !aligned16(v) ||
+      !aligned16(gate))
+    return SALA_ERR_INVALID_ARG;
+  if (!strides_ok(sq, 2) || !strides_ok(sk, 2) || !strides_ok(sv, 2) || !strides_ok(sg, 2))
+    return SALA_ERR_INVALID_ARG;
+  if (T == 0) return SALA_OK;
+  const int64_t M = (int64_t)B * T;
+  const int64_t N = 4 * (int64_t)H * D;
+  if (M > (int64_t)INT32_MAX || N > (int64_t)INT32_MAX) return SALA_ERR_UNSUPPORTED;
+  CUtensorMap tx, tw;
+  if (!make_tmap_2d(&tx, x, M, hidden, x_row_stride, kPjBM) ||
+      !make_tmap_2d(&tw, w, N, hidden, hidden, kPjBN))
+    return SALA_ERR_CUDA;
+  ProjParams p;
+  p.qh = (__half*)qh;
+  p.kh = (__half*)kh;
+  p.v = (__nv_bfloat16*)v;
+  p.gate = (__half*)gate;
+  p.sq = sq; p.sk = sk; p.sv = sv; p.sg = sg;
+  p.qw = q_norm_w;
+  p.kw = k_norm_w;
+  p.M = M;
+  p.T = T; p.H = H; p.hidden = hidden;
+  p.m_tiles = (int)((M + kPjBM - 1) / kPjBM);
+  p.n_tiles = (int)(N / kPjBN);
+  p.pos0 = pos0;
+  p.log2_base = std::log2((double)rope_base);
+  p.eps = eps;
+  const int64_t ntiles = (int64_t)p.m_tiles * p.n_tiles;
+  if (ntiles > (int64_t)INT32_MAX) return SALA_ERR_UNSUPPORTED;
+  const unsigned grid = (unsigned)std::min<int64_t>(ntiles, num_sms());
+  cudaStream_t st = as_stream(stream);
+  if (D == 128) {
+    auto kern = lightning_proj_kernel<128>;
+    if (!set_smem(kern, kPjSmem)) return SALA_ERR_CUDA;
+    kern<<<grid, kPjThreads, kPjSmem, st>>>(tx, tw, p);
+  } else {
+    auto kern = lightning_proj_kernel<64>;
+    if (!set_smem(kern, kPjSmem)) return SALA_ERR_CUDA;
+    kern<<<grid, kPjThreads, kPjSmem, st>>>(tx, tw, p);
+  }
+  SALA_CHECK_LAUNCH();
+  return SALA_OK;
+}
+
 // ------------------------------------------------------------------ sequence-split Lightning
 // A segment's state contribution (no outputs): the state pass and scan of the tensor-core
 // path, or the CUDA-core kernel with its output half skipped.
@@ -333,16 +498,23 @@ sala_status sala_lightning_state(const void* k, const void* v, float* state, con
     p.ws = (float*)workspace;
     p.B = B; p.T = T; p.H = H;
     p.G = lightning_tc_segments(B, H, T, nsm);
+    set_tc_stats(p, (uint8_t*)workspace + lightning_tc_states_bytes(B, H, p.G));
     p.NC = (T + kTcC - 1) / kTcC;
     p.pos0 = pos0;
     p.log2_base = log2_base;
     p.eps = eps;
-    auto ka = lightning_state_kernel;
+    auto ka = lightning_state_kernel<false>;
     if (!set_smem(ka, TcSmem<true>::bytes)) return SALA_ERR_CUDA;
     ka<<<(unsigned)(B * H * p.G), kStThreads, TcSmem<true>::bytes, st>>>(tk, tv, p);
     SALA_CHECK_LAUNCH();
     lightning_scan_kernel<<<dim3(B * H, 16), 256, 0, st>>>(p.ws, state, p.G, init_zero);
     SALA_CHECK_LAUNCH();
+    {
+      const sala_strides none{0, 0, 0};
+      if (!launch_lightning_fixup(k, k, v, nullptr, nullptr, state, nullptr, k_norm_w, sk, sk, sv,
+                                  none, none, p, st))
+        return SALA_ERR_CUDA;
+    }
     return SALA_OK;
   }
   // CUDA-core kernel with o == nullptr: q is read but unused, so k stands in for it
@@ -535,9 +707,28 @@ sala_status sala_sparse_select_head_softmax(const void* q, const void* k, int B,
 }
 
 // ------------------------------------------------------------------ sparse attention
+// Workspace: the fp16 copy of v [B, T, Hkv, D], the per-chunk largest |v| and sum-of-
+// squares partials [B * Hkv][kVChunks] each, the exponents and the outlier flags
+// [B * Hkv] each, every part 256-byte aligned.
+namespace {
+struct SaLayout {
+  size_t part_off, part_ss_off, vexp_off, vflag_off, total;
+};
+SaLayout sa_layout(int B, int T, int Hkv, int D) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  SaLayout L{};
+  L.part_off = up((size_t)B * T * Hkv * D * 2);
+  L.part_ss_off = L.part_off + up((size_t)B * Hkv * kVChunks * sizeof(float));
+  L.vexp_off = L.part_ss_off + up((size_t)B * Hkv * kVChunks * sizeof(float));
+  L.vflag_off = L.vexp_off + up((size_t)B * Hkv * sizeof(int));
+  L.total = L.vflag_off + up((size_t)B * Hkv * sizeof(int));
+  return L;
+}
+}  // namespace
+
 size_t sala_sparse_attn_workspace(int B, int T, int Hkv, int D) {
   if (B <= 0 || T <= 0 || Hkv <= 0 || D <= 0) return 0;
-  return ((size_t)B * T * Hkv * D * 2 + 255) / 256 * 256;  // fp16 copy of v
+  return sa_layout(B, T, Hkv, D).total;
 }
 
 sala_status sala_sparse_attn(const void* q, const void* k, const void* v, const void* g,
@@ -550,6 +741,7 @@ sala_status sala_sparse_attn(const void* q, const void* k, const void* v, const 
     return SALA_ERR_INVALID_ARG;
   if (dt != SALA_BF16) return SALA_ERR_UNSUPPORTED;
   if (block != kSaBlk || (D != 64 && D != 128) || Hq / Hkv > 16) return SALA_ERR_UNSUPPORTED;
+  if (Hkv > 65535 || B > 65535) return SALA_ERR_UNSUPPORTED;  // grid y / z of the v pre-pass
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (g && !aligned16(g)))
     return SALA_ERR_INVALID_ARG;
   if (!strides_ok(sq, 2) || !strides_ok(sk, 2) || !strides_ok(sv, 2) || !strides_ok(so, 2) ||
@@ -569,6 +761,13 @@ sala_status sala_sparse_attn(const void* q, const void* k, const void* v, const 
   p.g = (const __nv_bfloat16*)g;
   p.o = (__nv_bfloat16*)o;
   p.idx = idx;
+  const SaLayout L = sa_layout(B, T, Hkv, D);
+  float* vpart = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.part_off);
+  float* vpart_ss = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.part_ss_off);
+  int* vexp = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.vexp_off);
+  int* vflag = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.vflag_off);
+  p.vexp = vexp;
+  p.vflag = vflag;
   p.sq = sq; p.sg = sg; p.so = so;
   p.n_sel = n_sel; p.B = B; p.T = T; p.Hq = Hq; p.Hkv = Hkv; p.G = Hq / Hkv;
   const float sc = scale > 0.0f ? scale : 1.0f / std::sqrt((float)D);
@@ -578,23 +777,35 @@ sala_status sala_sparse_attn(const void* q, const void* k, const void* v, const 
   const int64_t want = num_sms();
   const unsigned grid = (unsigned)std::min<int64_t>(want, p.rows);
   {
-    // fp16 copy of v for the P.V MMAs; values that would not survive raise SALA_ERR_RANGE
-    const int64_t n = (int64_t)B * T * Hkv * (D / 8);
-    const unsigned cg = (unsigned)std::min<int64_t>((n + 255) / 256, 4 * want);
-    to_f16_copy_kernel<<<cg, 256, 0, st>>>((const __nv_bfloat16*)v, sv, B, T, Hkv, D,
-                                           (__half*)ws);
+    // fp16 copy of v for the P.V MMAs, scaled by 2^-e per (sequence, KV head) so that
+    // every bf16 value keeps its significant bits; a non-finite v raises SALA_ERR_RANGE
+    const dim3 gv(kVChunks, Hkv, B);
+    v_absmax_kernel<<<gv, 256, 0, st>>>((const __nv_bfloat16*)v, sv, T, Hkv, D, vpart, vpart_ss);
+    SALA_CHECK_LAUNCH();
+    to_f16_copy_kernel<<<gv, 256, 0, st>>>((const __nv_bfloat16*)v, sv, T, Hkv, D, vpart,
+                                           vpart_ss, vexp, vflag, (__half*)ws);
     SALA_CHECK_LAUNCH();
   }
+  // the common variant, then the one for outlier-heavy heads (which returns at once
+  // when there are none)
   if (D == 128) {
     constexpr int NS = 3;
-    auto kern = sparse_attn_kernel<128, NS>;
-    if (!set_smem(kern, SaSmem<128, NS>::bytes)) return SALA_ERR_CUDA;
-    kern<<<grid, kSaThreads, SaSmem<128, NS>::bytes, st>>>(tk, tv, p);
+    auto k0 = sparse_attn_kernel<128, NS, false>;
+    auto k1 = sparse_attn_kernel<128, NS, true>;
+    if (!set_smem(k0, SaSmem<128, NS>::bytes) || !set_smem(k1, SaSmem<128, NS>::bytes))
+      return SALA_ERR_CUDA;
+    k0<<<grid, kSaThreads, SaSmem<128, NS>::bytes, st>>>(tk, tv, p);
+    SALA_CHECK_LAUNCH();
+    k1<<<grid, kSaThreads, SaSmem<128, NS>::bytes, st>>>(tk, tv, p);
   } else {
     constexpr int NS = 6;
-    auto kern = sparse_attn_kernel<64, NS>;
-    if (!set_smem(kern, SaSmem<64, NS>::bytes)) return SALA_ERR_CUDA;
-    kern<<<grid, kSaThreads, SaSmem<64, NS>::bytes, st>>>(tk, tv, p);
+    auto k0 = sparse_attn_kernel<64, NS, false>;
+    auto k1 = sparse_attn_kernel<64, NS, true>;
+    if (!set_smem(k0, SaSmem<64, NS>::bytes) || !set_smem(k1, SaSmem<64, NS>::bytes))
+      return SALA_ERR_CUDA;
+    k0<<<grid, kSaThreads, SaSmem<64, NS>::bytes, st>>>(tk, tv, p);
+    SALA_CHECK_LAUNCH();
+    k1<<<grid, kSaThreads, SaSmem<64, NS>::bytes, st>>>(tk, tv, p);
   }
   SALA_CHECK_LAUNCH();
   return SALA_OK;
@@ -755,9 +966,11 @@ sala_status sala_sparse_block_means(const void* k, int B, int T, int Hkv, int D,
 namespace {
 
 // Fixed scratch for sala_lightning_prefill_noalloc: room for 256 fp32 128x128
-// segment states.  Host code may not use the symbol itself as a device address;
-// the per-device address comes from cudaGetSymbolAddress below.
-constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+// segment states (16 MiB) followed by their 256 largest-|v| words (one 256-byte
+// line is enough; 64 KiB are reserved).  Host code may not use the symbol itself as a
+// device address; the per-device address comes from cudaGetSymbolAddress below.
+constexpr size_t kNoAllocStateBytes = size_t(16) << 20;
+constexpr size_t kNoAllocScratchBytes = kNoAllocStateBytes + (size_t(64) << 10);
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 std::mutex g_noalloc_mu;
@@ -806,7 +1019,7 @@ sala_status sala_lightning_prefill_noalloc(const void* q, const void* k, const v
       (g && !strides_ok(sg, 2)))
     return SALA_ERR_INVALID_ARG;
   constexpr int64_t kStateBytes = 128 * 128 * sizeof(float);
-  const int64_t capacity = (int64_t)(kNoAllocScratchBytes / kStateBytes);  // segment states
+  const int64_t capacity = (int64_t)(kNoAllocStateBytes / kStateBytes);  // segment states
   if ((int64_t)B * H > capacity) return SALA_ERR_WORKSPACE;
   void* scratch = noalloc_scratch_address();
   if (!scratch) return SALA_ERR_CUDA;
@@ -829,12 +1042,13 @@ sala_status sala_lightning_prefill_noalloc(const void* q, const void* k, const v
   const int g_cap = (int)(capacity / ((int64_t)B * H));
   if (G > g_cap) G = g_cap;
   p.G = G;
+  set_tc_stats(p, (uint8_t*)scratch + kNoAllocStateBytes);
   p.pos0 = pos0;
   p.log2_base = std::log2((double)rope_base);
   p.eps = eps;
   const unsigned grid = (unsigned)(B * H * p.G);
-  auto ka = lightning_state_kernel;
-  auto kc = lightning_out_kernel;
+  auto ka = lightning_state_kernel<false>;
+  auto kc = lightning_out_kernel<false>;
   if (!set_smem(ka, TcSmem<true>::bytes) || !set_smem(kc, TcSmem<false>::bytes)) return SALA_ERR_CUDA;
   ka<<<grid, kStThreads, TcSmem<true>::bytes, st>>>(tk, tv, p);
   SALA_CHECK_LAUNCH();
@@ -842,6 +1056,9 @@ sala_status sala_lightning_prefill_noalloc(const void* q, const void* k, const v
   SALA_CHECK_LAUNCH();
   kc<<<grid, kTcThreads, TcSmem<false>::bytes, st>>>(tq, tk, tv, p);
   SALA_CHECK_LAUNCH();
+  if (!launch_lightning_fixup(q, k, v, g, o, state, q_norm_w, k_norm_w, sq, sk, sv, sg, so, p,
+                              st))
+    return SALA_ERR_CUDA;
   return SALA_OK;
 }
 

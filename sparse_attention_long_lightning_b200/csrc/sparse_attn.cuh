@@ -16,9 +16,9 @@
 // warps that split every 64-key block 16 keys apiece: the group's 16 query
 // heads form the M = 16 operand of m16n8k16 tensor-core MMAs (Q K^T in bf16
 // with four independent accumulator chains, P V in fp16 on an fp16 copy of V
-// that a pre-pass writes once and checks for values outside the fp16 range;
-// fp32 accumulation), the online softmax runs per warp in registers with a
-// lazily raised reference maximum (rescaling only when a
+// that a pre-pass writes once, scaled by a power of two per (sequence, KV head)
+// so that any bf16 V fits; fp32 accumulation), the online softmax runs per warp
+// in registers with a lazily raised reference maximum (rescaling only when a
 // score exceeds it by more than 2^8), and the four partial (max, sum, O)
 // triples are merged through shared memory at the end of the row.  All waits
 // are bounded; a wait that runs out raises SALA_ERR_TIMEOUT in the device
@@ -53,6 +53,9 @@ struct SaParams {
   const __nv_bfloat16* g;
   __nv_bfloat16* o;
   const int32_t* idx;
+  const int* vexp;   // [B * Hkv]: exponent e of the fp16 copy of v (values times 2^-e)
+  const int* vflag;  // [B * Hkv]: 1 when v is outlier-heavy (P V then runs on P's fp16
+                     // high and low parts)
   sala_strides sq, sg, so;
   int n_sel, B, T, Hq, Hkv, G;
   float scale_log2;  // softmax scale * log2(e)
@@ -64,7 +67,24 @@ __device__ __forceinline__ bool sa_block_live(int j, int64_t t) {
   return j >= 0 && (int64_t)j * kSaBlk <= t;
 }
 
-template <int D, int NS>
+// The first row >= r, in r's class modulo `stride`, of a (sequence, KV head) that this
+// variant handles: kPrecise rows belong to heads whose v is outlier-heavy (vflag set),
+// the others to the rest.  Whole heads are skipped at once.
+template <bool kPrecise>
+__device__ __forceinline__ int64_t sa_next_row(int64_t r, int64_t stride, const SaParams& p) {
+  while (r < p.rows) {
+    const int64_t head = r / p.T;  // b * Hkv + hk
+    if ((__ldg(p.vflag + head) != 0) == kPrecise) return r;
+    const int64_t next = (head + 1) * p.T;
+    r += (next - r + stride - 1) / stride * stride;
+  }
+  return r;
+}
+
+// kPrecise: the variant for heads whose v is outlier-heavy, where P V also takes P's
+// fp16 rounding residual; the two variants are launched one after the other, each on its
+// own heads, so the common one carries no cost for the other.
+template <int D, int NS, bool kPrecise>
 __global__ void __launch_bounds__(kSaThreads, 1)
 sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_v, const SaParams p) {
@@ -110,8 +130,9 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
       }
       uint32_t it = 0;
       bool ok = true;
-      for (int64_t r = blockIdx.x + (int64_t)grp * gridDim.x; r < p.rows && ok;
-           r += (int64_t)kSaGroups * gridDim.x) {
+      const int64_t rstride = (int64_t)kSaGroups * gridDim.x;
+      for (int64_t r = sa_next_row<kPrecise>(blockIdx.x + (int64_t)grp * gridDim.x, rstride, p);
+           r < p.rows && ok; r = sa_next_row<kPrecise>(r + rstride, rstride, p)) {
         const int64_t t = r % T;
         const int hk = (int)((r / T) % p.Hkv);
         const int b = (int)(r / (T * p.Hkv));
@@ -157,8 +178,9 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
   uint32_t it = 0, nmrg = 0;
   float* myML = mergeML + wq * 32;
   const int ct = wq * 32 + lane;            // 0..127 within the group
-  for (int64_t r = blockIdx.x + (int64_t)grp * gridDim.x; r < p.rows;
-       r += (int64_t)kSaGroups * gridDim.x) {
+  const int64_t rstride = (int64_t)kSaGroups * gridDim.x;
+  for (int64_t r = sa_next_row<kPrecise>(blockIdx.x + (int64_t)grp * gridDim.x, rstride, p);
+       r < p.rows; r = sa_next_row<kPrecise>(r + rstride, rstride, p)) {
     const int64_t t = r % T;
     const int hk = (int)((r / T) % p.Hkv);
     const int b = (int)(r / (T * p.Hkv));
@@ -194,6 +216,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
 #pragma unroll
     for (int nt = 0; nt < kNT; ++nt) oacc[nt][0] = oacc[nt][1] = oacc[nt][2] = oacc[nt][3] = 0.f;
     bool ok = !*abort_flag;
+    constexpr bool precise = kPrecise;
     int s_last = 0;
 
     for (int e = 0; e < nblk && ok; ++e) {
@@ -282,8 +305,9 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
         }
       }
       const float mu0 = m0 == -INFINITY ? 0.f : m0, mu1 = m1 == -INFINITY ? 0.f : m1;
-      // P in fp16 (10-bit mantissa), V is the fp16 copy
-      uint32_t pa[4];
+      // P in fp16 (10-bit mantissa), V is the fp16 copy; for outlier-heavy v also P's
+      // fp16 rounding residual
+      uint32_t pa[4], pl[4];
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
         const float p0 = exp2f(sc[nt][0] - mu0), p1 = exp2f(sc[nt][1] - mu0);
@@ -292,12 +316,25 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
         l1 += p2 + p3;
         pa[nt * 2 + 0] = pack_f16x2(p0, p1);
         pa[nt * 2 + 1] = pack_f16x2(p2, p3);
+        if constexpr (precise) {
+          const float2 h0 = __half22float2(*reinterpret_cast<const __half2*>(&pa[nt * 2]));
+          const float2 h1 = __half22float2(*reinterpret_cast<const __half2*>(&pa[nt * 2 + 1]));
+          pl[nt * 2 + 0] = pack_f16x2(p0 - h0.x, p1 - h0.y);
+          pl[nt * 2 + 1] = pack_f16x2(p2 - h1.x, p3 - h1.y);
+        }
       }
       // ---- O += P V
 #pragma unroll
       for (int pp = 0; pp < kNT / 2; ++pp) {
         mma_f16_16816(oacc[2 * pp], pa, vv[pp][0], vv[pp][1]);
         mma_f16_16816(oacc[2 * pp + 1], pa, vv[pp][2], vv[pp][3]);
+      }
+      if constexpr (precise) {
+#pragma unroll
+        for (int pp = 0; pp < kNT / 2; ++pp) {
+          mma_f16_16816(oacc[2 * pp], pl, vv[pp][0], vv[pp][1]);
+          mma_f16_16816(oacc[2 * pp + 1], pl, vv[pp][2], vv[pp][3]);
+        }
       }
       ++it;
     }
@@ -355,7 +392,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
         wgt[w] = (M == -INFINITY) ? 0.f : exp2f(mw - M);
         Lsum += wgt[w] * mergeML[w * 32 + 16 + row];
       }
-      const float inv = Lsum > 0.f ? 1.0f / Lsum : 0.f;
+      // 1 / sum, times 2^e to undo the scale of the fp16 copy of v
+      const float inv = Lsum > 0.f ? pow2i(__ldg(p.vexp + b * p.Hkv + hk)) / Lsum : 0.f;
       const __nv_bfloat16* gr = p.g ? p.g + b * p.sg.b + t * p.sg.t + (int64_t)h * p.sg.h : nullptr;
       __nv_bfloat16* orow = p.o + b * p.so.b + t * p.so.t + (int64_t)h * p.so.h;
 #pragma unroll
@@ -383,35 +421,135 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
   }
 }
 
-// Writes the fp16 copy of a bf16 [B, T, H, D] tensor (contiguous [B, T, H, D]
-// output) that the P.V MMAs read.  bf16 -> fp16 is exact for normal values
-// below 65504 (8 significant bits fit in 11); values that would not survive
-// (|x| >= 65536 in bf16, inf or NaN) raise SALA_ERR_RANGE.  Tiny values become
-// fp16 subnormals (absolute error below 2^-25).
+// The fp16 copy of v that the P.V MMAs read, written once per call in two launches
+// over grid (kVChunks, Hkv, B), each CTA covering rows [x T / kVChunks, (x + 1) T /
+// kVChunks) of one (sequence, KV head):
+//   v_absmax_kernel    the largest |v| of those rows -> part[(b Hkv + hk) kVChunks + x],
+//                      their sum of v^2 -> part_ss[...];
+//   to_f16_copy_kernel the (sequence, KV head)'s largest |v| from the partials, its
+//                      exponent e (v_operand_exp: v 2^-e below 2^15, the largest above
+//                      2^-4, e = 0 whenever fp16 holds the values as they are), the rows
+//                      times 2^-e into the contiguous [B, T, Hkv, D] copy, and e itself
+//                      (CTA x = 0) into vexp[b Hkv + hk], and vflag[b Hkv + hk] = 1 when
+//                      the largest |v| exceeds kSaOutlierRatio x rms(v).  The attention
+//                      epilogue multiplies by 2^e.  A non-finite v raises SALA_ERR_RANGE.
+constexpr int kVChunks = 128;
+
+__device__ __forceinline__ float bf16x8_absmax(const uint4& u, float m) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    m = fmaxf(m, fmaxf(fabsf(__uint_as_float(w[k] << 16)),
+                       fabsf(__uint_as_float(w[k] & 0xffff0000u))));
+  return m;
+}
+
+// Largest of `n` non-negative partial maxima (every thread of the CTA gets it); a NaN or
+// infinite partial makes the result infinite.  Non-negative floats, +inf included, order
+// as their bit patterns.
+__device__ __forceinline__ float cta_max_of(const float* part, int n, float* red) {
+  float m = 0.f;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const float x = part[i];
+    m = x < INFINITY ? fmaxf(m, x) : INFINITY;
+  }
+  const uint32_t mb = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = __uint_as_float(mb);
+  __syncthreads();
+  float r = 0.f;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r = fmaxf(r, red[w]);
+  __syncthreads();
+  return r;
+}
+
 __global__ void __launch_bounds__(256)
-to_f16_copy_kernel(const __nv_bfloat16* __restrict__ x, sala_strides s, int B, int T, int H,
-                   int D, __half* __restrict__ y) {
-  const int64_t rows = (int64_t)B * T * H;
+v_absmax_kernel(const __nv_bfloat16* __restrict__ x, sala_strides s, int T, int Hkv, int D,
+                float* __restrict__ part, float* __restrict__ part_ss) {
+  const int hk = blockIdx.y, b = blockIdx.z;
+  const int64_t r0 = (int64_t)blockIdx.x * T / kVChunks, r1 = (int64_t)(blockIdx.x + 1) * T / kVChunks;
   const int per_row = D / 8;
-  uint32_t bad = 0;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < rows * per_row;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t row = i / per_row;
+  float m = 0.f, ss = 0.f;
+  bool nonfinite = false;
+  for (int64_t i = r0 * per_row + threadIdx.x; i < r1 * per_row; i += blockDim.x) {
+    const int64_t t = i / per_row;
     const int c = (int)(i % per_row);
-    const int h = (int)(row % H);
-    const int64_t t = (row / H) % T;
-    const int b = (int)(row / ((int64_t)H * T));
-    const uint4 u = *reinterpret_cast<const uint4*>(x + b * s.b + t * s.t + h * s.h + 8 * c);
+    const uint4 u = *reinterpret_cast<const uint4*>(x + b * s.b + t * s.t + hk * s.h + 8 * c);
+    m = bf16x8_absmax(u, m);
+    float f[8];
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-    uint32_t hv[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      bad |= ((w[k] & 0x7fffu) >= 0x4780u) | (((w[k] >> 16) & 0x7fffu) >= 0x4780u);
-      hv[k] = bf16x2_to_f16x2(w[k]);
+      f[2 * k] = __uint_as_float(w[k] << 16);
+      f[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
     }
-    *reinterpret_cast<uint4*>(y + i * 8) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) ss = fmaf(f[k], f[k], ss);
+    // inf or NaN: exponent field all ones in either half of any word
+    nonfinite |= ((u.x & 0x7f80u) == 0x7f80u) | ((u.x & 0x7f800000u) == 0x7f800000u) |
+                 ((u.y & 0x7f80u) == 0x7f80u) | ((u.y & 0x7f800000u) == 0x7f800000u) |
+                 ((u.z & 0x7f80u) == 0x7f80u) | ((u.z & 0x7f800000u) == 0x7f800000u) |
+                 ((u.w & 0x7f80u) == 0x7f80u) | ((u.w & 0x7f800000u) == 0x7f800000u);
   }
-  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) raise_device_error(SALA_ERR_RANGE);
+  __shared__ float red[8], red_ss[8];
+  uint32_t mb = __reduce_max_sync(0xffffffffu, __float_as_uint(nonfinite ? INFINITY : m));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  if ((threadIdx.x & 31) == 0) {
+    red[threadIdx.x >> 5] = __uint_as_float(mb);
+    red_ss[threadIdx.x >> 5] = ss;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float r = 0.f, rs = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+      r = fmaxf(r, red[w]);
+      rs += red_ss[w];
+    }
+    part[((int64_t)b * Hkv + hk) * kVChunks + blockIdx.x] = r;
+    part_ss[((int64_t)b * Hkv + hk) * kVChunks + blockIdx.x] = rs;
+  }
+}
+
+// v of a (sequence, KV head) is outlier-heavy when its largest |v| exceeds this many times
+// its rms: P's fp16 rounding (2^-11) times such a value can exceed 1e-2 of the output's
+// rms, so P V also takes P's low part.
+constexpr float kSaOutlierRatio = 16.0f;
+
+__global__ void __launch_bounds__(256)
+to_f16_copy_kernel(const __nv_bfloat16* __restrict__ x, sala_strides s, int T, int Hkv, int D,
+                   const float* __restrict__ part, const float* __restrict__ part_ss,
+                   int* __restrict__ vexp, int* __restrict__ vflag, __half* __restrict__ y) {
+  const int hk = blockIdx.y, b = blockIdx.z;
+  __shared__ float red[8];
+  const float m = cta_max_of(part + ((int64_t)b * Hkv + hk) * kVChunks, kVChunks, red);
+  if (!(m < INFINITY)) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) raise_device_error(SALA_ERR_RANGE);
+  }
+  const int e = v_operand_exp(m);
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    vexp[(int64_t)b * Hkv + hk] = e;
+    double ss = 0.0;
+    for (int i = 0; i < kVChunks; ++i) ss += (double)part_ss[((int64_t)b * Hkv + hk) * kVChunks + i];
+    const double rms = sqrt(ss / ((double)T * D));
+    vflag[(int64_t)b * Hkv + hk] = (m < INFINITY) && (double)m > (double)kSaOutlierRatio * rms;
+  }
+  const float sc = pow2i(-e);
+  const int64_t r0 = (int64_t)blockIdx.x * T / kVChunks, r1 = (int64_t)(blockIdx.x + 1) * T / kVChunks;
+  const int per_row = D / 8;
+  for (int64_t i = r0 * per_row + threadIdx.x; i < r1 * per_row; i += blockDim.x) {
+    const int64_t t = i / per_row;
+    const int c = (int)(i % per_row);
+    const uint4 u = *reinterpret_cast<const uint4*>(x + b * s.b + t * s.t + hk * s.h + 8 * c);
+    uint4 o;
+    if (e == 0) {
+      o = make_uint4(bf16x2_to_f16x2(u.x), bf16x2_to_f16x2(u.y), bf16x2_to_f16x2(u.z),
+                     bf16x2_to_f16x2(u.w));
+    } else {
+      o = make_uint4(bf16x2_to_f16x2_scaled(u.x, sc), bf16x2_to_f16x2_scaled(u.y, sc),
+                     bf16x2_to_f16x2_scaled(u.z, sc), bf16x2_to_f16x2_scaled(u.w, sc));
+    }
+    *reinterpret_cast<uint4*>(y + (((int64_t)b * T + t) * Hkv + hk) * D + 8 * c) = o;
+  }
 }
 
 }  // namespace sala

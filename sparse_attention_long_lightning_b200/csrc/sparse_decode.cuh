@@ -22,7 +22,8 @@
 //   sd_attn_kernel    one CTA per (split, KV head, sequence): the split's share of the
 //                     chosen blocks, a cp.async ring of K/V tiles, the group's query
 //                     heads as the M = 16 operand of m16n8k16 tensor-core MMAs (Q K^T in
-//                     bf16; P in fp16 on V converted to fp16 in registers), online softmax
+//                     bf16; P V as two bf16 MMAs, P's high and low parts, on V as stored,
+//                     so any bf16 V is exact), online softmax
 //                     per warp, the four warps merged into one partial (max, sum, O)
 //   sd_combine_kernel one CTA per (query head, sequence): merges the splits, applies the
 //                     gate, writes bf16.
@@ -335,7 +336,6 @@ __global__ void __launch_bounds__(kSdAttnWarps * 32) sd_attn_kernel(const SdPara
   float oacc[kNT][4];
 #pragma unroll
   for (int nt = 0; nt < kNT; ++nt) oacc[nt][0] = oacc[nt][1] = oacc[nt][2] = oacc[nt][3] = 0.f;
-  uint32_t bad = 0;
   for (int e = sb0; e < sb1; ++e) {
     cp_async_wait<kSdStages - 1>();  // block e's group has landed
     __syncthreads();
@@ -368,7 +368,7 @@ __global__ void __launch_bounds__(kSdAttnWarps * 32) sd_attn_kernel(const SdPara
         mma_bf16_16816(sc[1], qa[kk], b2, b3);
       }
     }
-    // ---- V fragments (bf16 -> fp16, range-checked)
+    // ---- V fragments, bf16 as stored (no range limit)
     uint32_t vv[kNT / 2][4];
     {
       const int mat = lane >> 3, rin = lane & 7;
@@ -378,12 +378,6 @@ __global__ void __launch_bounds__(kSdAttnWarps * 32) sd_attn_kernel(const SdPara
         const uint32_t chunk = 2 * pp + (mat >> 1);
         ldsm_x4_t(vb + (chunk >> 3) * L::kHalf + swz128(vrow, chunk & 7), vv[pp][0], vv[pp][1],
                   vv[pp][2], vv[pp][3]);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint32_t w = vv[pp][i];
-          bad |= ((w & 0x7fffu) >= 0x4780u) | (((w >> 16) & 0x7fffu) >= 0x4780u);
-          vv[pp][i] = bf16x2_to_f16x2(w);
-        }
       }
     }
     // ---- scale, causal mask, online softmax
@@ -417,27 +411,30 @@ __global__ void __launch_bounds__(kSdAttnWarps * 32) sd_attn_kernel(const SdPara
       oacc[nt][2] *= al1; oacc[nt][3] *= al1;
     }
     const float mu0 = m0 == -INFINITY ? 0.f : m0, mu1 = m1 == -INFINITY ? 0.f : m1;
-    uint32_t pa[4];
+    // P as a bf16 high part plus a bf16 low part (the rounding residual): with V in bf16
+    // the two P V products carry ~16 significant bits of P and any bf16 V exactly
+    uint32_t pa[4], pl[4];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
       const float p0 = exp2f(sc[nt][0] - mu0), p1 = exp2f(sc[nt][1] - mu0);
       const float p2 = exp2f(sc[nt][2] - mu1), p3 = exp2f(sc[nt][3] - mu1);
       l0 += p0 + p1;
       l1 += p2 + p3;
-      pa[nt * 2 + 0] = pack_f16x2(p0, p1);
-      pa[nt * 2 + 1] = pack_f16x2(p2, p3);
+      pa[nt * 2 + 0] = pack_bf16x2_hi_lo(p0, p1, pl[nt * 2 + 0]);
+      pa[nt * 2 + 1] = pack_bf16x2_hi_lo(p2, p3, pl[nt * 2 + 1]);
     }
 #pragma unroll
     for (int pp = 0; pp < kNT / 2; ++pp) {
-      mma_f16_16816(oacc[2 * pp], pa, vv[pp][0], vv[pp][1]);
-      mma_f16_16816(oacc[2 * pp + 1], pa, vv[pp][2], vv[pp][3]);
+      mma_bf16_16816(oacc[2 * pp], pa, vv[pp][0], vv[pp][1]);
+      mma_bf16_16816(oacc[2 * pp + 1], pa, vv[pp][2], vv[pp][3]);
+      mma_bf16_16816(oacc[2 * pp], pl, vv[pp][0], vv[pp][1]);
+      mma_bf16_16816(oacc[2 * pp + 1], pl, vv[pp][2], vv[pp][3]);
     }
     __syncthreads();  // block e's slot is free again
     if (e + kSdStages < sb1) issue(e + kSdStages);  // into block e's slot
     cp_async_commit();
   }
   cp_async_wait<0>();
-  if (__any_sync(0xffffffffu, bad) && lane == 0) raise_device_error(SALA_ERR_RANGE);
 
   // ---- merge the four warps' partial states into the split's partial
   l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
@@ -510,6 +507,7 @@ __global__ void __launch_bounds__(D) sd_combine_kernel(const SdParams p) {
   }
   float y = Ls > 0.f ? acc / Ls : 0.f;
   if (p.g) y *= sigmoidf_(__bfloat162float(p.g[b * p.sg.b + (int64_t)h * p.sg.h + d]));
+  if (!(fabsf(y) < INFINITY)) raise_device_error(SALA_ERR_RANGE);  // non-finite input
   p.o[b * p.so.b + (int64_t)h * p.so.h + d] = __float2bfloat16_rn(y);
 }
 

@@ -252,12 +252,6 @@ topk_select_kernel(const float* __restrict__ scores, int32_t* __restrict__ idx, 
   for (int e = pos + lane; e < n_sel; e += 32) out[e] = -1;
 }
 
-// bf16 pair (lo in the low half) from two floats, round to nearest even.
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-
 }  // namespace sala
 
 namespace sala {

@@ -2,7 +2,9 @@
 
     python -m sparse_attention_long_lightning_b200.profile_case --op attn --T 16384 --iters 3
 
-Ops: lightning (prefill, B1 H32 D128 bf16 chunk 128), decode (B64 H32 D128 bf16),
+Ops: lightning (prefill, B1 H32 D128 bf16 chunk 128), lightning_prepared (the same on
+prepared fp16 q/k operands), proj (the fused input projection of a Lightning layer, T
+tokens x hidden -> 4 x 32 heads of 128), decode (B64 H32 D128 bf16),
 select / attn (B1 Hq32 Hkv2 D128 bf16, top-64 + 1 + 2), sparse_decode (B sequences,
 Hq32 Hkv2 D128 bf16, KV caches of T tokens, one step at positions near the end).
 Prints the mean CUDA-event time per call.
@@ -20,7 +22,9 @@ from sparse_attention_long_lightning_b200 import inputs
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--op", required=True, choices=["lightning", "decode", "select", "attn",
-                                                       "sparse_decode", "select_hsm"])
+                                                       "sparse_decode", "select_hsm", "proj",
+                                                       "lightning_prepared"])
+    ap.add_argument("--hidden", type=int, default=4096, help="hidden size for proj")
     ap.add_argument("--T", type=int, default=16384)
     ap.add_argument("--B", type=int, default=64, help="batch for decode")
     ap.add_argument("--iters", type=int, default=3)
@@ -35,6 +39,23 @@ def main():
                          dtype=torch.uint8, device=dev)
         fn = lambda: sala.lightning_prefill(x.q, x.k, x.v, x.g, None, chunk=128, out=o,
                                             workspace=ws)
+    elif a.op == "lightning_prepared":
+        gen = inputs.generator(1002, dev)
+        qh = inputs.randn((1, a.T, 32, 128), gen, torch.float16, dev)
+        kh = inputs.randn((1, a.T, 32, 128), gen, torch.float16, dev)
+        v = inputs.randn((1, a.T, 32, 128), gen, device=dev)
+        gate = inputs.randn((1, a.T, 32, 128), gen, device=dev).sigmoid().to(torch.float16)
+        o = torch.empty_like(v)
+        ws = torch.empty(max(1, sala.lightning_prefill_workspace(1, a.T, 32, 128, 128)),
+                         dtype=torch.uint8, device=dev)
+        fn = lambda: sala.lightning_prefill_prepared(qh, kh, v, gate, None, out=o, workspace=ws)
+    elif a.op == "proj":
+        gen = inputs.generator(1008, dev)
+        x = inputs.randn((1, a.T, a.hidden), gen, device=dev)
+        w = inputs.randn((4 * 32 * 128, a.hidden), gen, device=dev, scale=a.hidden ** -0.5)
+        outs = sala.lightning_projection(x, w, heads=32, head_dim=128)
+        fn = lambda: sala.lightning_projection(x, w, heads=32, head_dim=128, out=outs)
+        print(f"proj: {2.0 * a.T * a.hidden * 4 * 32 * 128 / 1e12:.3f} TFLOP per call")
     elif a.op == "decode":
         S = inputs.decode_state(a.B, 32, 128, seed=1003, device=dev)
         q, k, v, g = inputs.decode_tokens(a.B, 32, 128, seed=1003, step=0, device=dev)

@@ -159,8 +159,14 @@ def test_workspace_queries(lib):
     n = sala.sparse_select_workspace(1, 131072, 32, 2, 128, 64, 100)
     assert means + (1 << 29) <= n <= means + (1 << 30) + 4096
     assert sala.sparse_select_workspace(1, 1 << 20, 32, 2, 128, 64, 200) <= (1 << 30) + (1 << 26)
-    assert sala.sparse_attn_workspace(1, 131072, 2, 128) == 131072 * 2 * 128 * 2
+    # fp16 copy of v, then 128 partial maxima and 128 partial sums of squares, one
+    # exponent and one outlier flag per (sequence, KV head), each part 256-byte aligned
+    assert sala.sparse_attn_workspace(1, 131072, 2, 128) == 131072 * 2 * 128 * 2 + 2 * 1024 + 2 * 256
     assert sala.sparse_attn_workspace(1, 0, 2, 128) == 0
+    # Lightning (bf16, D128, chunk 128): segment states plus the segments' largest |v|
+    n = sala.lightning_prefill_workspace(1, 131072, 32, 128, 128)
+    G = n // (32 * 128 * 128 * 4)
+    assert G >= 1 and n == 32 * G * 128 * 128 * 4 + 2 * ((32 * G * 4 + 255) // 256 * 256)
 
 
 def test_head_softmax_select_rejects_bad_arguments(lib):

@@ -48,6 +48,42 @@ def test_single_process_passthrough():
     assert bench.weak_scaling_value(1, 1000, 0.5) == 2000
 
 
+def test_bench_gpus_flag_launches_ranks(monkeypatch):
+    """`--gpus N` outside torchrun starts N ranks through torch.distributed.run on
+    127.0.0.1; inside torchrun a WORLD_SIZE that differs from N is an error; N = 1 runs
+    in this process."""
+    import argparse
+
+    import bench
+    calls = []
+    monkeypatch.setattr(bench.subprocess, "call", lambda cmd: calls.append(cmd) or 0)
+    monkeypatch.setattr(bench.sys, "argv", ["bench.py", "--gpus", "4", "--steps", "3"])
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    assert bench.launch_ranks(argparse.Namespace(gpus=4)) == 0
+    cmd = calls[0]
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node=4" in cmd and "127.0.0.1" in cmd
+    assert cmd[-4:] == ["--gpus", "4", "--steps", "3"]
+    assert bench.launch_ranks(argparse.Namespace(gpus=1)) is None
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    assert bench.launch_ranks(argparse.Namespace(gpus=4)) == 2
+    assert bench.launch_ranks(argparse.Namespace(gpus=2)) is None
+
+
+def test_bench_reference_sample_is_labelled(monkeypatch):
+    """The oracle sample used by both CPU legs states its scale factors."""
+    import bench
+    monkeypatch.setitem(bench.ORACLE_SAMPLE, "light_tokens", 64)
+    monkeypatch.setitem(bench.ORACLE_SAMPLE, "sparse_rows", 4)
+    smp = bench.OracleSample(4096)
+    info = smp.info()
+    assert info["extrapolated"] is True and info["kind"] == "oracle"
+    assert info["factor"]["lightning"] == 6 * 32 * 4096 / (16 * 64)
+    assert info["factor"]["sparse"] == 2 * 4096 / 4
+    sample_s, full_s = smp.time()
+    assert 0 < sample_s < full_s
+
+
 def test_bench_build_digest_is_stable():
     import bench
     a, b = bench.source_digest(), bench.source_digest()

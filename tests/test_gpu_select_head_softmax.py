@@ -38,7 +38,9 @@ def _check(idx_gpu, q, k, topk, rows=None, **kw):
     ref, gap, sc = oracle.sparse_select(qn, _np(k), topk=topk, rows=rows, want_scores=True,
                                         score="head_softmax", **kw)
     got = idx_gpu if rows is None else idx_gpu[:, :, rows]
-    return check_index_sets(got, ref, gap, tie_band=_band(sc, topk))
+    t = np.arange(q.shape[1]) if rows is None else np.asarray(rows)
+    win = {key: kw[key] for key in ("n_init", "n_local") if key in kw}
+    return check_index_sets(got, ref, gap, sc, t, topk=topk, tie_band=_band(sc, topk), **win)
 
 
 @pytest.mark.parametrize("T,Hq,Hkv,D,topk", [

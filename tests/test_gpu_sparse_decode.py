@@ -37,10 +37,12 @@ def _check_step(q, g, k, v, pos, y, idx, topk=64, n_init=1, n_local=2):
     """Selection vs the oracle's, output vs the oracle's attention over the GPU selection."""
     qn, kn, vn = _np(q), _np(k), _np(v)
     gn = None if g is None else _np(g)
-    _, ref_idx, gap = oracle.sparse_decode(qn, kn, vn, pos, gn, topk=topk, n_init=n_init,
-                                           n_local=n_local)
+    _, ref_idx, gap, sc = oracle.sparse_decode(qn, kn, vn, pos, gn, topk=topk, n_init=n_init,
+                                               n_local=n_local, want_scores=True)
     gi = idx.cpu().numpy()
-    check_index_sets(gi[:, :, None, :], ref_idx[:, :, None, :], gap[:, :, None])
+    check_index_sets(gi[:, :, None, :], ref_idx[:, :, None, :], gap[:, :, None],
+                     sc[:, :, None, :], np.asarray(pos)[:, None, None], topk=topk,
+                     n_init=n_init, n_local=n_local)
     for b, p in enumerate(pos):
         want = oracle.attention(qn[b][None, None], kn[b:b + 1, :p + 1], vn[b:b + 1, :p + 1],
                                 None if gn is None else gn[b][None, None],
@@ -131,13 +133,15 @@ def test_decode_matches_prefill_rows():
     k[:, :T], v[:, :T] = s.k, s.v
     kbar = sala.sparse_block_means(k[:, :T], kbar_blocks=Tmax // 64)
     rows = [5, 64 * 3 + 2, 64 * 17 + 63, 64 * 30 + 40, T - 1]
-    _, gap = oracle.sparse_select(_np(s.q[:, rows]), _np(s.k), rows=rows)
+    _, gap, sc = oracle.sparse_select(_np(s.q[:, rows]), _np(s.k), rows=rows, want_scores=True)
     idx = torch.empty((1, Hkv, 67), dtype=torch.int32, device=DEV)
     for r, p in enumerate(rows):
         pos = torch.tensor([p], dtype=torch.int32, device=DEV)
         y = sala.sparse_decode(s.q[:, p], k, v, kbar.clone(), pos, s.g[:, p], idx_out=idx)
+        # the prefill's selection stands in for the oracle's here: both sides are the GPU's,
+        # so the oracle's gap and scores decide which rows may differ and how
         check_index_sets(idx.cpu().numpy()[:, :, None], idx_pf[:, :, p:p + 1].cpu().numpy(),
-                         gap[:, :, r:r + 1])
+                         gap[:, :, r:r + 1], sc[:, :, r:r + 1], p, topk=64)
         if torch.equal(idx[0], idx_pf[0, :, p]):
             assert rel_err_bf16_pair(_np(y[0]), _np(y_pf[0, p])) <= TOL_BF16
 
