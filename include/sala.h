@@ -250,6 +250,47 @@ sala_status sala_sparse_attn(const void *q, const void *k, const void *v, const 
                              void *ws, size_t ws_bytes, sala_dtype dt, void *stream);
 
 /*
+ * Block selection and block-sparse attention for a window of query rows: the
+ * operations of sala_sparse_select / sala_sparse_select_head_softmax and
+ * sala_sparse_attn (same definitions, MiniCPM-SALA tech-report mirror, section
+ * 02 (2)) for the Tq query rows at positions qpos0 .. qpos0 + Tq - 1 of a sequence
+ * whose keys and values cover positions 0 .. Tk - 1.  Row t of q, g, o and idx is
+ * position qpos0 + t: its block c = floor((qpos0 + t) / block) sets its candidates,
+ * local window and causal mask.  The result for each row equals that row of the
+ * whole-sequence call (bit for bit when k and v are the whole sequence's, Tk = T:
+ * the attention's per-(sequence, KV head) v scale is then the same), so a sequence
+ * can be split over devices by query rows after gathering k and v on each.
+ *
+ *   q, g, o     [B,Tq,Hq,D] (g may be NULL), k, v [B,Tk,Hkv,D] (bf16), strided
+ *   idx         [B,Hkv,Tq,n_sel] int32, contiguous (output of the selection, input
+ *               of the attention)
+ *   score       0: group-summed scores (sala_sparse_select), 1: per-head
+ *               softmax-normalised scores (sala_sparse_select_head_softmax)
+ *   ws          selection: >= sala_sparse_select_rows_workspace() bytes (block means
+ *               of the Tk keys, plus the score scratch when score = 1 or topk > 64);
+ *               attention: >= sala_sparse_attn_workspace(B, Tk, Hkv, D) bytes (the
+ *               fp16 copy of the Tk values); caller-owned, reusable after the call
+ *   0 <= qpos0, qpos0 + Tq <= Tk; every other limit as in the whole-sequence calls.
+ * Errors: INVALID_ARG (also for a window outside [0, Tk)), UNSUPPORTED, WORKSPACE,
+ *   CUDA.  Device (attention): RANGE when v holds an infinite or NaN value.
+ */
+size_t sala_sparse_select_rows_workspace(int B, int Tq, int Tk, int Hq, int Hkv, int D,
+                                         int block, int topk, int score);
+
+sala_status sala_sparse_select_rows(const void *q, const void *k, int B, int Tq, int qpos0,
+                                    int Tk, int Hq, int Hkv, int D, sala_strides sq,
+                                    sala_strides sk, int block, int topk, int n_init,
+                                    int n_local, int score, int32_t *idx, void *ws,
+                                    size_t ws_bytes, sala_dtype dt, void *stream);
+
+sala_status sala_sparse_attn_rows(const void *q, const void *k, const void *v, const void *g,
+                                  const int32_t *idx, int n_sel, void *o, int B, int Tq,
+                                  int qpos0, int Tk, int Hq, int Hkv, int D, sala_strides sq,
+                                  sala_strides sk, sala_strides sv, sala_strides sg,
+                                  sala_strides so, int block, float scale, void *ws,
+                                  size_t ws_bytes, sala_dtype dt, void *stream);
+
+/*
  * Sparse-layer decode (InfLLM-v2 style, NoPE): one new query per sequence.
  * For sequence b at position p = pos[b], whose cache already holds the new token's key
  * and value at row p, the step computes row t = p of the prefill pair

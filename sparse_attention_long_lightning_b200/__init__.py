@@ -134,6 +134,14 @@ def load_library(path: Optional[str] = None):
     lib.sala_sparse_attn.argtypes = [vp, vp, vp, vp, vp, i, vp, i, i, i, i, i, S, S, S, S, S, i, f,
                                      vp, sz, i, vp]
     lib.sala_sparse_attn.restype = i
+    lib.sala_sparse_select_rows_workspace.argtypes = [i, i, i, i, i, i, i, i, i]
+    lib.sala_sparse_select_rows_workspace.restype = sz
+    lib.sala_sparse_select_rows.argtypes = [vp, vp, i, i, i, i, i, i, i, S, S, i, i, i, i, i, vp,
+                                            vp, sz, i, vp]
+    lib.sala_sparse_select_rows.restype = i
+    lib.sala_sparse_attn_rows.argtypes = [vp, vp, vp, vp, vp, i, vp, i, i, i, i, i, i, i, S, S, S,
+                                          S, S, i, f, vp, sz, i, vp]
+    lib.sala_sparse_attn_rows.restype = i
     lib.sala_get_device_error.argtypes = [vp]
     lib.sala_get_device_error.restype = i
     lib.sala_selftest_wait_timeout.argtypes = [ctypes.c_longlong, vp]
@@ -374,10 +382,32 @@ def sparse_select_head_softmax_workspace(B, T, Hq, Hkv, D, block=64) -> int:
     return int(load_library().sala_sparse_select_head_softmax_workspace(B, T, Hq, Hkv, D, block))
 
 
+def sparse_select_rows_workspace(B, Tq, Tk, Hq, Hkv, D, block=64, topk=64,
+                                 score="group_sum") -> int:
+    mode = 1 if score == "head_softmax" else 0
+    return int(load_library().sala_sparse_select_rows_workspace(B, Tq, Tk, Hq, Hkv, D, block,
+                                                                topk, mode))
+
+
+def _q_window(q, k, q_pos0):
+    """(Tq, qpos0, Tk) of a call whose q rows may be a window of k's positions; None when
+    q covers all of k's positions from 0 (the whole-sequence entry points)."""
+    Tq, Tk = q.shape[1], k.shape[1]
+    if q_pos0 is None:
+        if Tq != Tk:
+            raise ValueError("q and k differ in length: pass q_pos0, the position of q's row 0")
+        return None
+    if not 0 <= int(q_pos0) <= Tk - Tq:
+        raise ValueError("the q rows must lie inside k's positions")
+    return Tq, int(q_pos0), Tk
+
+
 def sparse_select(q, k, *, topk=64, n_init=1, n_local=2, block=64, out=None, workspace=None,
-                  stream=None, score="group_sum"):
+                  stream=None, score="group_sum", q_pos0=None):
     """Block selection.  q [B,T,Hq,D], k [B,T,Hkv,D] -> idx [B,Hkv,T,n_init+topk+n_local] int32.
-    score="group_sum" (sala_sparse_select) or "head_softmax" (sala_sparse_select_head_softmax)."""
+    score="group_sum" (sala_sparse_select) or "head_softmax" (sala_sparse_select_head_softmax).
+    With q_pos0, q holds Tq rows at positions q_pos0 .. q_pos0 + Tq - 1 of a sequence whose
+    keys k [B,Tk,Hkv,D] cover 0 .. Tk - 1 (sala_sparse_select_rows); idx is [B,Hkv,Tq,n_sel]."""
     if score not in ("group_sum", "head_softmax"):
         raise ValueError("score must be 'group_sum' or 'head_softmax'")
     lib = load_library()
@@ -388,6 +418,19 @@ def sparse_select(q, k, *, topk=64, n_init=1, n_local=2, block=64, out=None, wor
     if out is None:
         out = torch.empty((B, Hkv, T, n_sel), dtype=torch.int32, device=q.device)
     hsm = score == "head_softmax"
+    win = _q_window(q, k, q_pos0)
+    if win is not None:
+        Tq, qp, Tk = win
+        need = sparse_select_rows_workspace(B, Tq, Tk, Hq, Hkv, D, block, topk, score)
+        if workspace is None and need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
+        st = lib.sala_sparse_select_rows(_p(q), _p(k), B, Tq, qp, Tk, Hq, Hkv, D, _s4(q), _s4(k),
+                                         int(block), int(topk), int(n_init), int(n_local),
+                                         1 if hsm else 0, _p(out), _p(workspace), wsb, _dt(q),
+                                         _stream(stream))
+        _check("sala_sparse_select_rows", st)
+        return out
     need = (sparse_select_head_softmax_workspace(B, T, Hq, Hkv, D, block) if hsm
             else sparse_select_workspace(B, T, Hq, Hkv, D, block, topk))
     if workspace is None and need:
@@ -405,8 +448,10 @@ def sparse_attn_workspace(B, T, Hkv, D) -> int:
 
 
 def sparse_attn(q, k, v, idx, g=None, *, block=64, scale=0.0, out=None, workspace=None,
-                stream=None):
-    """Block-sparse attention.  q,g [B,T,Hq,D]; k,v [B,T,Hkv,D]; idx [B,Hkv,T,n_sel] int32."""
+                stream=None, q_pos0=None):
+    """Block-sparse attention.  q,g [B,T,Hq,D]; k,v [B,T,Hkv,D]; idx [B,Hkv,T,n_sel] int32.
+    With q_pos0, q, g, idx and the output hold Tq rows at positions q_pos0 .. q_pos0 + Tq - 1
+    of a sequence whose k, v [B,Tk,Hkv,D] cover 0 .. Tk - 1 (sala_sparse_attn_rows)."""
     lib = load_library()
     _cuda(q, k, v, idx, g, out, workspace)
     B, T, Hq, D = q.shape
@@ -415,6 +460,19 @@ def sparse_attn(q, k, v, idx, g=None, *, block=64, scale=0.0, out=None, workspac
         raise ValueError("idx must be a contiguous int32 tensor")
     if out is None:
         out = torch.empty_like(q, memory_format=torch.contiguous_format)
+    win = _q_window(q, k, q_pos0)
+    if win is not None:
+        Tq, qp, Tk = win
+        need = sparse_attn_workspace(B, Tk, Hkv, D)
+        if workspace is None and need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
+        st = lib.sala_sparse_attn_rows(_p(q), _p(k), _p(v), _p(g), _p(idx), int(idx.shape[-1]),
+                                       _p(out), B, Tq, qp, Tk, Hq, Hkv, D, _s4(q), _s4(k), _s4(v),
+                                       _s4(g), _s4(out), int(block), float(scale), _p(workspace),
+                                       wsb, _dt(q), _stream(stream))
+        _check("sala_sparse_attn_rows", st)
+        return out
     need = sparse_attn_workspace(B, T, Hkv, D)
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)

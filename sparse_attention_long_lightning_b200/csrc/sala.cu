@@ -138,26 +138,27 @@ namespace sala {
 // Head-softmax scoring kernel for group size G (a power of two up to 32).
 template <int D, int G>
 static bool launch_hsm(dim3 grid, cudaStream_t st, const __nv_bfloat16* q, const float* kbar,
-                       float* scores, int nb, int Hkv, sala_strides sq, int r0, int r1,
-                       int rows_pass, int n_init, int n_local, float inv_sqrt_d) {
+                       float* scores, int nb, int Hkv, sala_strides sq, int qpos0, int r0,
+                       int r1, int rows_pass, int n_init, int n_local, float inv_sqrt_d) {
   auto kern = block_scores_hsm_kernel<D, G>;
   if (!set_smem(kern, hsm_smem_bytes<D>())) return false;
   grid.x = (unsigned)((r1 - r0 + kHsmRows / G - 1) / (kHsmRows / G));
-  kern<<<grid, 256, hsm_smem_bytes<D>(), st>>>(q, kbar, scores, nb, Hkv, sq, r0, r1, rows_pass,
-                                               n_init, n_local, inv_sqrt_d);
+  kern<<<grid, 256, hsm_smem_bytes<D>(), st>>>(q, kbar, scores, nb, Hkv, sq, qpos0, r0, r1,
+                                               rows_pass, n_init, n_local, inv_sqrt_d);
   return true;
 }
 template <int D>
 static bool launch_hsm_g(int G, dim3 grid, cudaStream_t st, const __nv_bfloat16* q,
                          const float* kbar, float* scores, int nb, int Hkv, sala_strides sq,
-                         int r0, int r1, int rows_pass, int n_init, int n_local, float isd) {
+                         int qp, int r0, int r1, int rows_pass, int n_init, int n_local,
+                         float isd) {
   switch (G) {
-    case 1: return launch_hsm<D, 1>(grid, st, q, kbar, scores, nb, Hkv, sq, r0, r1, rows_pass, n_init, n_local, isd);
-    case 2: return launch_hsm<D, 2>(grid, st, q, kbar, scores, nb, Hkv, sq, r0, r1, rows_pass, n_init, n_local, isd);
-    case 4: return launch_hsm<D, 4>(grid, st, q, kbar, scores, nb, Hkv, sq, r0, r1, rows_pass, n_init, n_local, isd);
-    case 8: return launch_hsm<D, 8>(grid, st, q, kbar, scores, nb, Hkv, sq, r0, r1, rows_pass, n_init, n_local, isd);
-    case 16: return launch_hsm<D, 16>(grid, st, q, kbar, scores, nb, Hkv, sq, r0, r1, rows_pass, n_init, n_local, isd);
-    case 32: return launch_hsm<D, 32>(grid, st, q, kbar, scores, nb, Hkv, sq, r0, r1, rows_pass, n_init, n_local, isd);
+    case 1: return launch_hsm<D, 1>(grid, st, q, kbar, scores, nb, Hkv, sq, qp, r0, r1, rows_pass, n_init, n_local, isd);
+    case 2: return launch_hsm<D, 2>(grid, st, q, kbar, scores, nb, Hkv, sq, qp, r0, r1, rows_pass, n_init, n_local, isd);
+    case 4: return launch_hsm<D, 4>(grid, st, q, kbar, scores, nb, Hkv, sq, qp, r0, r1, rows_pass, n_init, n_local, isd);
+    case 8: return launch_hsm<D, 8>(grid, st, q, kbar, scores, nb, Hkv, sq, qp, r0, r1, rows_pass, n_init, n_local, isd);
+    case 16: return launch_hsm<D, 16>(grid, st, q, kbar, scores, nb, Hkv, sq, qp, r0, r1, rows_pass, n_init, n_local, isd);
+    case 32: return launch_hsm<D, 32>(grid, st, q, kbar, scores, nb, Hkv, sq, qp, r0, r1, rows_pass, n_init, n_local, isd);
     default: return false;
   }
 }
@@ -572,30 +573,38 @@ sala_status sala_state_prefix_sum(const float* src, size_t n, int count, size_t 
 // bounded scratch.
 static bool sel_fused(int T, int topk) { return topk <= kSelFusedMaxK && T / kSelBlk <= 65535; }
 
-size_t sala_sparse_select_workspace(int B, int T, int Hq, int Hkv, int D, int block, int topk) {
+size_t sala_sparse_select_rows_workspace(int B, int Tq, int Tk, int Hq, int Hkv, int D,
+                                         int block, int topk, int score) {
   (void)Hq;
-  if (B <= 0 || T <= 0 || Hkv <= 0 || block != kSelBlk || (D != 64 && D != 128) || topk < 1)
+  if (B <= 0 || Tq <= 0 || Tk <= 0 || Hkv <= 0 || block != kSelBlk || (D != 64 && D != 128) ||
+      topk < 1 || (score != 0 && score != 1))
     return 0;
-  const SelLayout L = sel_layout(B, T, Hkv, D);
-  return sel_fused(T, topk) ? L.total_fused : L.total;
+  const SelLayout L = sel_layout(B, Tq, Tk, Hkv, D);
+  return score == 0 && sel_fused(Tk, topk) ? L.total_fused : L.total;
+}
+
+size_t sala_sparse_select_workspace(int B, int T, int Hq, int Hkv, int D, int block, int topk) {
+  return sala_sparse_select_rows_workspace(B, T, T, Hq, Hkv, D, block, topk, 0);
 }
 
 size_t sala_sparse_select_head_softmax_workspace(int B, int T, int Hq, int Hkv, int D,
                                                  int block) {
   (void)Hq;
   if (B <= 0 || T <= 0 || Hkv <= 0 || D <= 0 || block != kSelBlk) return 0;
-  return sel_layout(B, T, Hkv, D).total;
+  return sel_layout(B, T, T, Hkv, D).total;
 }
 
 // mode 0: group-summed scores (fused tensor-core path for topk <= 64, else the score
-// scratch); mode 1: per-head softmax-normalised scores (score scratch).
-static sala_status sparse_select_impl(const void* q, const void* k, int B, int T, int Hq,
-                                      int Hkv, int D, sala_strides sq, sala_strides sk,
-                                      int block, int topk, int n_init, int n_local, int32_t* idx,
-                                      void* ws, size_t ws_bytes, sala_dtype dt, void* stream,
-                                      int mode) {
+// scratch); mode 1: per-head softmax-normalised scores (score scratch).  The T query rows
+// are positions qpos0 .. qpos0 + T - 1 of a sequence whose keys cover 0 .. Tk - 1.
+static sala_status sparse_select_impl(const void* q, const void* k, int B, int T, int qpos0,
+                                      int Tk, int Hq, int Hkv, int D, sala_strides sq,
+                                      sala_strides sk, int block, int topk, int n_init,
+                                      int n_local, int32_t* idx, void* ws, size_t ws_bytes,
+                                      sala_dtype dt, void* stream, int mode) {
   if (T > 0 && (!q || !k || !idx)) return SALA_ERR_INVALID_ARG;
   if (B <= 0 || T < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return SALA_ERR_INVALID_ARG;
+  if (qpos0 < 0 || Tk < 0 || (int64_t)qpos0 + T > (int64_t)Tk) return SALA_ERR_INVALID_ARG;
   if (topk < 1 || n_init < 0 || n_local < 1) return SALA_ERR_INVALID_ARG;
   if (dt != SALA_BF16) return SALA_ERR_UNSUPPORTED;
   if (block != kSelBlk || (D != 64 && D != 128) || topk > 256 || Hq / Hkv > 32)
@@ -604,8 +613,8 @@ static sala_status sparse_select_impl(const void* q, const void* k, int B, int T
   if (!aligned16(q) || !aligned16(k) || !strides_ok(sq, 2) || !strides_ok(sk, 2))
     return SALA_ERR_INVALID_ARG;
   if (T == 0) return SALA_OK;
-  const SelLayout L = sel_layout(B, T, Hkv, D);
-  const bool fused = mode == 0 && sel_fused(T, topk);
+  const SelLayout L = sel_layout(B, T, Tk, Hkv, D);
+  const bool fused = mode == 0 && sel_fused(Tk, topk);
   if (!ws || ws_bytes < (fused ? L.total_fused : L.total)) return SALA_ERR_WORKSPACE;
   cudaStream_t st = as_stream(stream);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
@@ -639,14 +648,14 @@ static sala_status sparse_select_impl(const void* q, const void* k, int B, int T
       auto kern = select_tc_kernel<128>;
       if (!set_smem(kern, StcSmem<128>::bytes)) return SALA_ERR_CUDA;
       kern<<<grid, kStcThreads, StcSmem<128>::bytes, st>>>(th, tl, (const __nv_bfloat16*)q, idx,
-                                                          T, L.nb, Hkv, B, G, sq, topk, n_init,
-                                                          n_local);
+                                                          T, qpos0, L.nb, Hkv, B, G, sq, topk,
+                                                          n_init, n_local);
     } else {
       auto kern = select_tc_kernel<64>;
       if (!set_smem(kern, StcSmem<64>::bytes)) return SALA_ERR_CUDA;
       kern<<<grid, kStcThreads, StcSmem<64>::bytes, st>>>(th, tl, (const __nv_bfloat16*)q, idx,
-                                                         T, L.nb, Hkv, B, G, sq, topk, n_init,
-                                                         n_local);
+                                                         T, qpos0, L.nb, Hkv, B, G, sq, topk,
+                                                         n_init, n_local);
     }
     SALA_CHECK_LAUNCH();
     return SALA_OK;
@@ -656,11 +665,11 @@ static sala_status sparse_select_impl(const void* q, const void* k, int B, int T
     if (L.nb > 0 && mode == 1) {
       const bool ok =
           D == 128 ? launch_hsm_g<128>(G, dim3(1, Hkv, B), st, (const __nv_bfloat16*)q, kbar,
-                                       scores, L.nb, Hkv, sq, r0, r1, L.rows_pass, n_init,
-                                       n_local, inv_sqrt_d)
+                                       scores, L.nb, Hkv, sq, qpos0, r0, r1, L.rows_pass,
+                                       n_init, n_local, inv_sqrt_d)
                    : launch_hsm_g<64>(G, dim3(1, Hkv, B), st, (const __nv_bfloat16*)q, kbar,
-                                      scores, L.nb, Hkv, sq, r0, r1, L.rows_pass, n_init,
-                                      n_local, inv_sqrt_d);
+                                      scores, L.nb, Hkv, sq, qpos0, r0, r1, L.rows_pass,
+                                      n_init, n_local, inv_sqrt_d);
       if (!ok) return SALA_ERR_CUDA;
       SALA_CHECK_LAUNCH();
     } else if (L.nb > 0) {
@@ -669,21 +678,22 @@ static sala_status sparse_select_impl(const void* q, const void* k, int B, int T
         auto kern = block_scores_kernel<128>;
         if (!set_smem(kern, score_smem_bytes<128>())) return SALA_ERR_CUDA;
         kern<<<gs, 256, score_smem_bytes<128>(), st>>>((const __nv_bfloat16*)q, kbar, scores,
-                                                        L.nb, Hkv, G, sq, r0, r1, L.rows_pass,
-                                                        n_init, n_local, inv_sqrt_d);
+                                                        L.nb, Hkv, G, sq, qpos0, r0, r1,
+                                                        L.rows_pass, n_init, n_local, inv_sqrt_d);
       } else {
         auto kern = block_scores_kernel<64>;
         if (!set_smem(kern, score_smem_bytes<64>())) return SALA_ERR_CUDA;
         kern<<<gs, 256, score_smem_bytes<64>(), st>>>((const __nv_bfloat16*)q, kbar, scores,
-                                                       L.nb, Hkv, G, sq, r0, r1, L.rows_pass,
-                                                       n_init, n_local, inv_sqrt_d);
+                                                       L.nb, Hkv, G, sq, qpos0, r0, r1,
+                                                       L.rows_pass, n_init, n_local, inv_sqrt_d);
       }
       SALA_CHECK_LAUNCH();
     }
     const int64_t nwarps = (int64_t)B * Hkv * (r1 - r0);
     const int64_t nblk = (nwarps + kTopkWarps - 1) / kTopkWarps;
     topk_select_kernel<<<(unsigned)nblk, kTopkWarps * 32, 0, st>>>(
-        scores, idx, B, T, Hkv, L.nb > 0 ? L.nb : 1, r0, r1, L.rows_pass, topk, n_init, n_local);
+        scores, idx, B, T, qpos0, Hkv, L.nb > 0 ? L.nb : 1, r0, r1, L.rows_pass, topk, n_init,
+        n_local);
     SALA_CHECK_LAUNCH();
   }
   return SALA_OK;
@@ -693,8 +703,8 @@ sala_status sala_sparse_select(const void* q, const void* k, int B, int T, int H
                                int D, sala_strides sq, sala_strides sk, int block, int topk,
                                int n_init, int n_local, int32_t* idx, void* ws, size_t ws_bytes,
                                sala_dtype dt, void* stream) {
-  return sparse_select_impl(q, k, B, T, Hq, Hkv, D, sq, sk, block, topk, n_init, n_local, idx,
-                            ws, ws_bytes, dt, stream, 0);
+  return sparse_select_impl(q, k, B, T, 0, T, Hq, Hkv, D, sq, sk, block, topk, n_init, n_local,
+                            idx, ws, ws_bytes, dt, stream, 0);
 }
 
 sala_status sala_sparse_select_head_softmax(const void* q, const void* k, int B, int T, int Hq,
@@ -702,8 +712,18 @@ sala_status sala_sparse_select_head_softmax(const void* q, const void* k, int B,
                                             int block, int topk, int n_init, int n_local,
                                             int32_t* idx, void* ws, size_t ws_bytes,
                                             sala_dtype dt, void* stream) {
-  return sparse_select_impl(q, k, B, T, Hq, Hkv, D, sq, sk, block, topk, n_init, n_local, idx,
-                            ws, ws_bytes, dt, stream, 1);
+  return sparse_select_impl(q, k, B, T, 0, T, Hq, Hkv, D, sq, sk, block, topk, n_init, n_local,
+                            idx, ws, ws_bytes, dt, stream, 1);
+}
+
+sala_status sala_sparse_select_rows(const void* q, const void* k, int B, int Tq, int qpos0,
+                                    int Tk, int Hq, int Hkv, int D, sala_strides sq,
+                                    sala_strides sk, int block, int topk, int n_init,
+                                    int n_local, int score, int32_t* idx, void* ws,
+                                    size_t ws_bytes, sala_dtype dt, void* stream) {
+  if (score != 0 && score != 1) return SALA_ERR_INVALID_ARG;
+  return sparse_select_impl(q, k, B, Tq, qpos0, Tk, Hq, Hkv, D, sq, sk, block, topk, n_init,
+                            n_local, idx, ws, ws_bytes, dt, stream, score);
 }
 
 // ------------------------------------------------------------------ sparse attention
@@ -731,14 +751,18 @@ size_t sala_sparse_attn_workspace(int B, int T, int Hkv, int D) {
   return sa_layout(B, T, Hkv, D).total;
 }
 
-sala_status sala_sparse_attn(const void* q, const void* k, const void* v, const void* g,
-                             const int32_t* idx, int n_sel, void* o, int B, int T, int Hq,
-                             int Hkv, int D, sala_strides sq, sala_strides sk, sala_strides sv,
-                             sala_strides sg, sala_strides so, int block, float scale,
-                             void* ws, size_t ws_bytes, sala_dtype dt, void* stream) {
+// The T query rows (q, g, o, idx) are positions qpos0 .. qpos0 + T - 1; k and v hold
+// positions 0 .. Tk - 1.
+static sala_status sparse_attn_impl(const void* q, const void* k, const void* v, const void* g,
+                                    const int32_t* idx, int n_sel, void* o, int B, int T,
+                                    int qpos0, int Tk, int Hq, int Hkv, int D, sala_strides sq,
+                                    sala_strides sk, sala_strides sv, sala_strides sg,
+                                    sala_strides so, int block, float scale, void* ws,
+                                    size_t ws_bytes, sala_dtype dt, void* stream) {
   if (T > 0 && (!q || !k || !v || !o || !idx)) return SALA_ERR_INVALID_ARG;
   if (B <= 0 || T < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || n_sel <= 0 || !(scale >= 0.0f))
     return SALA_ERR_INVALID_ARG;
+  if (qpos0 < 0 || Tk < 0 || (int64_t)qpos0 + T > (int64_t)Tk) return SALA_ERR_INVALID_ARG;
   if (dt != SALA_BF16) return SALA_ERR_UNSUPPORTED;
   if (block != kSaBlk || (D != 64 && D != 128) || Hq / Hkv > 16) return SALA_ERR_UNSUPPORTED;
   if (Hkv > 65535 || B > 65535) return SALA_ERR_UNSUPPORTED;  // grid y / z of the v pre-pass
@@ -748,20 +772,20 @@ sala_status sala_sparse_attn(const void* q, const void* k, const void* v, const 
       (g && !strides_ok(sg, 2)))
     return SALA_ERR_INVALID_ARG;
   if (T == 0) return SALA_OK;
-  if (!ws || !aligned16(ws) || ws_bytes < sala_sparse_attn_workspace(B, T, Hkv, D))
+  if (!ws || !aligned16(ws) || ws_bytes < sala_sparse_attn_workspace(B, Tk, Hkv, D))
     return SALA_ERR_WORKSPACE;
-  // the fp16 copy of v: contiguous [B, T, Hkv, D]
-  const sala_strides sv16 = {(int64_t)T * Hkv * D, (int64_t)Hkv * D, (int64_t)D};
+  // the fp16 copy of v: contiguous [B, Tk, Hkv, D]
+  const sala_strides sv16 = {(int64_t)Tk * Hkv * D, (int64_t)Hkv * D, (int64_t)D};
   CUtensorMap tk, tv;
-  if (!make_tmap_bhtd(&tk, k, B, T, Hkv, D, sk, kSaBlk) ||
-      !make_tmap_bhtd(&tv, ws, B, T, Hkv, D, sv16, kSaBlk, 1, true))
+  if (!make_tmap_bhtd(&tk, k, B, Tk, Hkv, D, sk, kSaBlk) ||
+      !make_tmap_bhtd(&tv, ws, B, Tk, Hkv, D, sv16, kSaBlk, 1, true))
     return SALA_ERR_CUDA;
   SaParams p;
   p.q = (const __nv_bfloat16*)q;
   p.g = (const __nv_bfloat16*)g;
   p.o = (__nv_bfloat16*)o;
   p.idx = idx;
-  const SaLayout L = sa_layout(B, T, Hkv, D);
+  const SaLayout L = sa_layout(B, Tk, Hkv, D);
   float* vpart = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.part_off);
   float* vpart_ss = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.part_ss_off);
   int* vexp = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.vexp_off);
@@ -773,6 +797,7 @@ sala_status sala_sparse_attn(const void* q, const void* k, const void* v, const 
   const float sc = scale > 0.0f ? scale : 1.0f / std::sqrt((float)D);
   p.scale_log2 = sc * 1.4426950408889634f;
   p.rows = (int64_t)B * Hkv * T;
+  p.qpos0 = qpos0;
   cudaStream_t st = as_stream(stream);
   const int64_t want = num_sms();
   const unsigned grid = (unsigned)std::min<int64_t>(want, p.rows);
@@ -780,9 +805,10 @@ sala_status sala_sparse_attn(const void* q, const void* k, const void* v, const 
     // fp16 copy of v for the P.V MMAs, scaled by 2^-e per (sequence, KV head) so that
     // every bf16 value keeps its significant bits; a non-finite v raises SALA_ERR_RANGE
     const dim3 gv(kVChunks, Hkv, B);
-    v_absmax_kernel<<<gv, 256, 0, st>>>((const __nv_bfloat16*)v, sv, T, Hkv, D, vpart, vpart_ss);
+    v_absmax_kernel<<<gv, 256, 0, st>>>((const __nv_bfloat16*)v, sv, Tk, Hkv, D, vpart,
+                                        vpart_ss);
     SALA_CHECK_LAUNCH();
-    to_f16_copy_kernel<<<gv, 256, 0, st>>>((const __nv_bfloat16*)v, sv, T, Hkv, D, vpart,
+    to_f16_copy_kernel<<<gv, 256, 0, st>>>((const __nv_bfloat16*)v, sv, Tk, Hkv, D, vpart,
                                            vpart_ss, vexp, vflag, (__half*)ws);
     SALA_CHECK_LAUNCH();
   }
@@ -809,6 +835,25 @@ sala_status sala_sparse_attn(const void* q, const void* k, const void* v, const 
   }
   SALA_CHECK_LAUNCH();
   return SALA_OK;
+}
+
+sala_status sala_sparse_attn(const void* q, const void* k, const void* v, const void* g,
+                             const int32_t* idx, int n_sel, void* o, int B, int T, int Hq,
+                             int Hkv, int D, sala_strides sq, sala_strides sk, sala_strides sv,
+                             sala_strides sg, sala_strides so, int block, float scale,
+                             void* ws, size_t ws_bytes, sala_dtype dt, void* stream) {
+  return sparse_attn_impl(q, k, v, g, idx, n_sel, o, B, T, 0, T, Hq, Hkv, D, sq, sk, sv, sg, so,
+                          block, scale, ws, ws_bytes, dt, stream);
+}
+
+sala_status sala_sparse_attn_rows(const void* q, const void* k, const void* v, const void* g,
+                                  const int32_t* idx, int n_sel, void* o, int B, int Tq,
+                                  int qpos0, int Tk, int Hq, int Hkv, int D, sala_strides sq,
+                                  sala_strides sk, sala_strides sv, sala_strides sg,
+                                  sala_strides so, int block, float scale, void* ws,
+                                  size_t ws_bytes, sala_dtype dt, void* stream) {
+  return sparse_attn_impl(q, k, v, g, idx, n_sel, o, B, Tq, qpos0, Tk, Hq, Hkv, D, sq, sk, sv,
+                          sg, so, block, scale, ws, ws_bytes, dt, stream);
 }
 
 // ------------------------------------------------------------------ sparse-layer decode

@@ -57,9 +57,10 @@ struct SaParams {
   const int* vflag;  // [B * Hkv]: 1 when v is outlier-heavy (P V then runs on P's fp16
                      // high and low parts)
   sala_strides sq, sg, so;
-  int n_sel, B, T, Hq, Hkv, G;
+  int n_sel, B, T, Hq, Hkv, G;  // T: query rows (q, g, o, idx); keys come by TMA
   float scale_log2;  // softmax scale * log2(e)
   int64_t rows;      // B * Hkv * T
+  int64_t qpos0;     // sequence position of query row 0 (row t is position qpos0 + t)
 };
 
 // A selected block j takes part in row t iff j >= 0 and its first key is <= t.
@@ -134,12 +135,13 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
       for (int64_t r = sa_next_row<kPrecise>(blockIdx.x + (int64_t)grp * gridDim.x, rstride, p);
            r < p.rows && ok; r = sa_next_row<kPrecise>(r + rstride, rstride, p)) {
         const int64_t t = r % T;
+        const int64_t tp = p.qpos0 + t;  // the row's position
         const int hk = (int)((r / T) % p.Hkv);
         const int b = (int)(r / (T * p.Hkv));
         const int32_t* ir = p.idx + r * p.n_sel;
         for (int e = 0; e < p.n_sel; ++e) {
           const int j = __ldg(ir + e);
-          if (!sa_block_live(j, t)) continue;
+          if (!sa_block_live(j, tp)) continue;
           const int s = it % NS;
           if (*abort_flag || !mbar_wait(&empty[s], ((it / NS) & 1) ^ 1)) { ok = false; break; }
           uint8_t* st = stages + size_t(s) * L::kStage;
@@ -182,6 +184,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
   for (int64_t r = sa_next_row<kPrecise>(blockIdx.x + (int64_t)grp * gridDim.x, rstride, p);
        r < p.rows; r = sa_next_row<kPrecise>(r + rstride, rstride, p)) {
     const int64_t t = r % T;
+    const int64_t tp = p.qpos0 + t;  // the row's position
     const int hk = (int)((r / T) % p.Hkv);
     const int b = (int)(r / (T * p.Hkv));
 
@@ -191,7 +194,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
       const int32_t* ir = p.idx + r * p.n_sel;
       for (int e0 = 0; e0 < p.n_sel; e0 += 32) {
         const int e = e0 + lane;
-        const bool live = e < p.n_sel && sa_block_live(__ldg(ir + e), t);
+        const bool live = e < p.n_sel && sa_block_live(__ldg(ir + e), tp);
         nblk += __popc(__ballot_sync(0xffffffffu, live));
       }
     }
@@ -270,8 +273,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
       } else {
         s_last = s;
       }
-      // ---- scale; causal mask only where the block reaches past t
-      const bool straddle = (int64_t)j * kSaBlk + kSaBlk - 1 > t;
+      // ---- scale; causal mask only where the block reaches past the row's position
+      const bool straddle = (int64_t)j * kSaBlk + kSaBlk - 1 > tp;
       const int64_t key0 = (int64_t)j * kSaBlk + wq * 16 + tq * 2;
       float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
@@ -279,7 +282,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           float x = sc[nt][c] * p.scale_log2;
-          if (straddle && key0 + nt * 8 + (c & 1) > t) x = -INFINITY;
+          if (straddle && key0 + nt * 8 + (c & 1) > tp) x = -INFINITY;
           sc[nt][c] = x;
         }
         mx0 = fmaxf(mx0, fmaxf(sc[nt][0], sc[nt][1]));

@@ -11,6 +11,9 @@
 // Scores are fp32 (inputs are bf16, so the products are exact and only the
 // fp32 sums round).  Rows are processed in passes so the score scratch stays
 // bounded (at most 1 GiB) at any sequence length.
+// The query rows may be a window of the sequence (a shard of it): row t of q and
+// idx is position qpos0 + t, which sets its block c and so its candidates; the
+// keys (and their block means) cover positions 0 .. Tk - 1.
 #pragma once
 
 #include <climits>
@@ -35,9 +38,10 @@ struct SelLayout {
   size_t total_fused, total;
 };
 
-inline SelLayout sel_layout(int B, int T, int Hkv, int D) {
+// T: query rows, Tk: key positions.
+inline SelLayout sel_layout(int B, int T, int Tk, int Hkv, int D) {
   SelLayout L{};
-  L.nb = T / kSelBlk;
+  L.nb = Tk / kSelBlk;
   const size_t per_row = (size_t)B * Hkv * (size_t)(L.nb > 0 ? L.nb : 1) * 4;
   size_t rp = kSelScoreCap / per_row;
   rp = rp / kSelBlk * kSelBlk;
@@ -88,7 +92,7 @@ template <int D>
 __global__ void __launch_bounds__(256)
 block_scores_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ kbar,
                     float* __restrict__ scores, int nb, int Hkv, int G, sala_strides sq,
-                    int r_begin, int r_end, int rows_pass, int n_init, int n_local,
+                    int qpos0, int r_begin, int r_end, int rows_pass, int n_init, int n_local,
                     float inv_sqrt_d) {
   extern __shared__ float sc_smem[];
   float (*qsT)[kScLd] = reinterpret_cast<float (*)[kScLd]>(sc_smem);            // [D][kScLd]
@@ -98,7 +102,7 @@ block_scores_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict
   const int hk = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int t0 = r_begin + tile * kScTile;
   const int t_last = min(t0 + kScTile, r_end) - 1;
-  const int j_hi = min(t_last / kSelBlk - n_local, nb - 1);  // last candidate of the tile
+  const int j_hi = min((qpos0 + t_last) / kSelBlk - n_local, nb - 1);  // the tile's last candidate
   if (j_hi < n_init) return;
 
   // group-summed queries, transposed: qsT[d][r]
@@ -137,7 +141,7 @@ block_scores_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict
     for (int u = 0; u < 4; ++u) {
       const int t = t0 + ty * 4 + u;
       if (t > t_last) continue;
-      const int jmax = t / kSelBlk - n_local;  // candidates of row t end here
+      const int jmax = (qpos0 + t) / kSelBlk - n_local;  // candidates of row t end here
       float* srow = srow_base + (int64_t)(t - r_begin) * nb;
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
@@ -158,8 +162,8 @@ constexpr int kTopkWarps = 8;
 
 __global__ void __launch_bounds__(kTopkWarps * 32)
 topk_select_kernel(const float* __restrict__ scores, int32_t* __restrict__ idx, int B, int T,
-                   int Hkv, int nb, int r_begin, int r_end, int rows_pass, int topk, int n_init,
-                   int n_local) {
+                   int qpos0, int Hkv, int nb, int r_begin, int r_end, int rows_pass, int topk,
+                   int n_init, int n_local) {
   __shared__ uint32_t hist_all[kTopkWarps][256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rows_here = r_end - r_begin;
@@ -169,7 +173,7 @@ topk_select_kernel(const float* __restrict__ scores, int32_t* __restrict__ idx, 
   const int hk = (int)((gw / rows_here) % Hkv);
   const int b = (int)(gw / ((int64_t)rows_here * Hkv));
   const int t = r_begin + tr;
-  const int c = t / kSelBlk;
+  const int c = (qpos0 + t) / kSelBlk;  // the row's block
   const int n_sel = n_init + topk + n_local;
   int32_t* out = idx + (((int64_t)b * Hkv + hk) * T + t) * n_sel;
   const float* srow = scores + (((int64_t)b * Hkv + hk) * rows_pass + tr) * (int64_t)nb;
@@ -279,8 +283,8 @@ template <int D, int G>
 __global__ void __launch_bounds__(256)
 block_scores_hsm_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ kbar,
                         float* __restrict__ scores, int nb, int Hkv, sala_strides sq,
-                        int r_begin, int r_end, int rows_pass, int n_init, int n_local,
-                        float inv_sqrt_d) {
+                        int qpos0, int r_begin, int r_end, int rows_pass, int n_init,
+                        int n_local, float inv_sqrt_d) {
   static_assert(G >= 1 && G <= 32 && (G & (G - 1)) == 0, "group of 1..32 heads, power of 2");
   constexpr int R = kHsmRows / G;  // query rows per tile
   constexpr int GIN = G < 8 ? G : 8;  // heads of one query row inside a thread
@@ -292,7 +296,7 @@ block_scores_hsm_kernel(const __nv_bfloat16* __restrict__ q, const float* __rest
   const int hk = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int t0 = r_begin + tile * R;
   const int t_last = min(t0 + R, r_end) - 1;
-  const int j_hi = min(t_last / kSelBlk - n_local, nb - 1);  // last candidate of the tile
+  const int j_hi = min((qpos0 + t_last) / kSelBlk - n_local, nb - 1);  // the tile's last candidate
   if (j_hi < n_init) return;
 
   for (int e = tid; e < kHsmRows * D; e += 256) {
@@ -308,7 +312,7 @@ block_scores_hsm_kernel(const __nv_bfloat16* __restrict__ q, const float* __rest
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
     const int t = t0 + (8 * qr + u) / G;
-    jmax[u] = t <= t_last ? min(t / kSelBlk - n_local, nb - 1) : n_init - 1;
+    jmax[u] = t <= t_last ? min((qpos0 + t) / kSelBlk - n_local, nb - 1) : n_init - 1;
   }
 
   float acc[8][8];

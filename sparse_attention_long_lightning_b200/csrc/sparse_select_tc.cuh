@@ -225,8 +225,9 @@ __device__ __noinline__ int stc_compact(uint32_t sA, uint32_t jA, uint32_t hA, i
 template <int D>
 __global__ void __launch_bounds__(kStcThreads, 1)
 select_tc_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constant__ CUtensorMap tm_lo,
-                 const __nv_bfloat16* __restrict__ q, int32_t* __restrict__ idx, int T, int nb,
-                 int Hkv, int B, int G, sala_strides sq, int topk, int n_init, int n_local) {
+                 const __nv_bfloat16* __restrict__ q, int32_t* __restrict__ idx, int T, int qpos0,
+                 int nb, int Hkv, int B, int G, sala_strides sq, int topk, int n_init,
+                 int n_local) {
   using L = StcSmem<D>;
   constexpr int kK = D / 16;     // k-steps
   constexpr int kAcols = D / 2;  // TMEM columns of one A operand (bf16 pairs)
@@ -265,7 +266,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constan
     it.t0 = (nq2 - 1 - x) * kStcRows;
     it.hk = rem % Hkv;
     it.b = rem / Hkv;
-    const int t_last = min(it.t0 + kStcRows - 1, T - 1);
+    const int t_last = qpos0 + min(it.t0 + kStcRows - 1, T - 1);  // the item's last position
     const int jhi = min(t_last / kSelBlk - n_local, nb - 1);  // last candidate of the item
     const int n_item = jhi >= n_init ? jhi - n_init + 1 : 0;
     it.ntiles = n_item > topk ? (n_item + kStcN - 1) / kStcN : 0;  // 0: nothing to score
@@ -457,7 +458,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constan
       const Item it = info(k);
       const int t = it.t0 + row;
       const bool live = t < T;
-      const int c = t / kSelBlk;
+      const int c = (qpos0 + t) / kSelBlk;  // the row's block
       const int jmax = min(c - n_local, nb - 1);  // last candidate of this row
       const int n_row = jmax >= n_init ? jmax - n_init + 1 : 0;
       const bool buffered = live && n_row > topk;

@@ -143,3 +143,106 @@ def sparse_layer_kvhead_parallel(q, k, v, g=None, *, group=None, topk=64, n_init
 
     return sparse_layer_headpar(q, k, v, g, rank=rank, world=world, select_fn=select_fn,
                                 attn_fn=attn_fn, gather_fn=gather_fn if gather else None)
+
+
+# ---------------------------------------------------------------------------------------
+# Query-range-parallel sparse layer.  One sequence split into contiguous token segments,
+# one per rank (as for the sequence-parallel Lightning prefill).  A query row's selection
+# and attention read the keys/values of every earlier position, so each rank first
+# gathers the whole sequence's k and v (one all-gather each, into its own HBM: no kernel
+# reads a peer's memory) and then computes the selection and attention of its own query
+# rows only, at their positions in the sequence (sala_sparse_select_rows,
+# sala_sparse_attn_rows).  The rows are independent, so the result equals the single-
+# device layer row for row; it scales with the number of ranks (not bounded by Hkv like
+# the KV-head split), at the cost of every rank holding all of k and v (1 GiB at 1M tokens,
+# 2 KV heads, D128, bf16).
+# ---------------------------------------------------------------------------------------
+
+def segment_offsets(lens: Sequence[int]):
+    """First token of each rank's segment, from the segment lengths in rank order."""
+    out, acc = [], 0
+    for n in lens:
+        if n < 0:
+            raise ValueError("segment lengths must be >= 0")
+        out.append(acc)
+        acc += int(n)
+    return out
+
+
+def gather_token_segments(x, lens: Sequence[int], group=None):
+    """Join every rank's contiguous token segment x [B, T_r, ...] (rank order) along the
+    token axis into [B, sum(lens), ...] with one all-gather.  Equal segments of a single
+    sequence (B = 1) land in place; otherwise the segments are padded to the longest for
+    the collective and joined after it."""
+    import torch.distributed as dist
+
+    world = len(lens)
+    Tm, B, rest = max(lens), x.shape[0], tuple(x.shape[2:])
+    if x.shape[1] != lens[dist.get_rank(group)]:
+        raise ValueError("x does not hold this rank's segment length")
+    if B == 1 and all(n == Tm for n in lens):
+        out = torch.empty((1, world * Tm) + rest, dtype=x.dtype, device=x.device)
+        dist.all_gather_into_tensor(out.view((world * Tm,) + rest), x[0].contiguous(),
+                                    group=group)
+        return out
+    xp = torch.zeros((B, Tm) + rest, dtype=x.dtype, device=x.device)
+    xp[:, :x.shape[1]] = x
+    buf = torch.empty((world * B, Tm) + rest, dtype=x.dtype, device=x.device)
+    dist.all_gather_into_tensor(buf, xp, group=group)
+    buf = buf.view((world, B, Tm) + rest)
+    return torch.cat([buf[r, :, :lens[r]] for r in range(world)], dim=1)
+
+
+def sparse_layer_qrange(q, k, v, g=None, *, rank: int, offsets: Sequence[int],
+                        gather_kv: Callable, select_fn: Callable, attn_fn: Callable,
+                        gather_fn: Optional[Callable] = None):
+    """This rank's share of a sparse layer split over query ranges.  q, g [B,T_r,Hq,D] and
+    k, v [B,T_r,Hkv,D] are the rank's token segment, which starts at position
+    offsets[rank].  With the compute and the collectives passed in:
+      K, V = gather_kv(k, v)            the whole sequence's keys / values [B,T,Hkv,D]
+      idx  = select_fn(q, K, p)         [B,Hkv,T_r,n_sel], q's rows at positions p ..
+      o    = attn_fn(q, K, V, idx, g, p) [B,T_r,Hq,D]
+    returns o, or the whole [B,T,Hq,D] when `gather_fn(o) -> [B,T,Hq,D]` is given."""
+    p = int(offsets[rank])
+    K, V = gather_kv(k, v)
+    if K.shape[1] < p + q.shape[1]:
+        raise ValueError("the gathered keys do not reach this rank's rows")
+    idx = select_fn(q, K, p)
+    o = attn_fn(q, K, V, idx, g, p)
+    return o if gather_fn is None else gather_fn(o)
+
+
+def sparse_layer_query_parallel(q, k, v, g=None, *, group=None, topk=64, n_init=1, n_local=2,
+                                block=64, score="group_sum", gather=True):
+    """Query-range-parallel sparse layer on this rank's GPU (one process per GPU, NCCL).
+    q, g [B,T_r,Hq,D] and k, v [B,T_r,Hkv,D]: this rank's contiguous token segment of the
+    sequence (rank order; lengths may differ).  k and v are all-gathered into this GPU's
+    memory, then libsala selects and attends for the rank's rows at their positions.
+    Returns the rank's output rows, or with gather=True the whole sequence's output."""
+    import torch.distributed as dist
+
+    import sparse_attention_long_lightning_b200 as sala
+
+    rank, world = dist.get_rank(group), dist.get_world_size(group)
+    lens_t = torch.zeros(world, dtype=torch.int64, device=q.device)
+    dist.all_gather_into_tensor(lens_t, torch.tensor([q.shape[1]], dtype=torch.int64,
+                                                     device=q.device), group=group)
+    lens = [int(n) for n in lens_t.tolist()]
+    offsets = segment_offsets(lens)
+
+    def gather_kv(kk, vv):
+        return gather_token_segments(kk, lens, group), gather_token_segments(vv, lens, group)
+
+    def select_fn(qq, K, p):
+        return sala.sparse_select(qq, K, topk=topk, n_init=n_init, n_local=n_local, block=block,
+                                  score=score, q_pos0=p)
+
+    def attn_fn(qq, K, V, idx, gg, p):
+        return sala.sparse_attn(qq, K, V, idx, gg, block=block, q_pos0=p)
+
+    def gather_fn(o):
+        return gather_token_segments(o, lens, group)
+
+    return sparse_layer_qrange(q, k, v, g, rank=rank, offsets=offsets, gather_kv=gather_kv,
+                               select_fn=select_fn, attn_fn=attn_fn,
+                               gather_fn=gather_fn if gather else None)

@@ -193,6 +193,40 @@ def test_head_softmax_workspace_has_score_scratch():
     assert sala.sparse_select_head_softmax_workspace(1, 0, 32, 2, 128) == 0
 
 
+def test_row_window_calls_reject_bad_windows(lib):
+    p = ctypes.c_void_p(16)
+    st = sala.SalaStrides(64 * 2 * 128, 2 * 128, 128)
+    ws = 1 << 30
+    sel = lambda Tq, q0, Tk, score=0: lib.sala_sparse_select_rows(
+        p, p, 1, Tq, q0, Tk, 2, 2, 128, st, st, 64, 4, 1, 2, score, p, p, ws, 1, None)
+    att = lambda Tq, q0, Tk: lib.sala_sparse_attn_rows(
+        p, p, p, None, p, 7, p, 1, Tq, q0, Tk, 2, 2, 128, st, st, st, Z, st, 64, 0.0, p, ws, 1,
+        None)
+    for fn in (sel, att):
+        assert fn(64, 1, 64) == 1        # window runs past the keys
+        assert fn(64, -1, 640) == 1      # negative first position
+        assert fn(64, 0, 32) == 1        # fewer keys than query rows
+        assert fn(0, 640, 640) == 0      # an empty window at the end is a no-op
+    assert sel(64, 0, 640, score=2) == 1  # unknown score rule
+    # the whole-sequence calls keep their own checks
+    assert lib.sala_sparse_select_rows(p, p, 1, 64, 0, 64, 3, 2, 128, st, st, 64, 4, 1, 2, 0, p,
+                                       p, ws, 1, None) == 1
+
+
+def test_row_window_workspace_queries():
+    nb = 131072 // 64
+    means = nb * 2 * 128 * (4 + 2 + 2)
+    # block means of all Tk keys; the score scratch (head softmax) sized by the Tq rows
+    n = sala.sparse_select_rows_workspace(1, 16384, 131072, 32, 2, 128)
+    assert n == sala.sparse_select_workspace(1, 131072, 32, 2, 128, 64, 64)
+    assert means <= n <= means + 1024
+    hs = sala.sparse_select_rows_workspace(1, 64, 131072, 32, 2, 128, score="head_softmax")
+    assert hs == means + 2 * 64 * nb * 4
+    full = sala.sparse_select_rows_workspace(1, 131072, 131072, 32, 2, 128, score="head_softmax")
+    assert full == sala.sparse_select_head_softmax_workspace(1, 131072, 32, 2, 128)
+    assert sala.sparse_select_rows_workspace(1, 64, 0, 32, 2, 128) == 0
+
+
 def test_tracing_wraps_compute_calls_only(lib):
     """With tracing on, compute entry points go through an NVTX range (and still return
     the library's status); workspace queries and status helpers are the bare calls."""

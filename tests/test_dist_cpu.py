@@ -219,3 +219,80 @@ def test_kvhead_ranges_cover_all_heads():
             assert all(hi > lo for lo, hi in spans)
     with pytest.raises(ValueError):
         kvhead_range(2, 0, 3)
+
+
+# ---------------------------------------------------------------------------------------
+# Query-range-parallel sparse layer: each rank holds a contiguous token segment, gathers
+# the whole sequence's k and v, and selects / attends for its own rows at their positions.
+# fp64 oracle (row windows) standing in for the kernels; the gathered output must equal
+# the whole-sequence layer exactly (rows are independent).
+# ---------------------------------------------------------------------------------------
+
+def _qrange_worker(rank, world, port, lens, B, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    from datetime import timedelta
+
+    import numpy as np
+
+    import oracle
+    from sparse_attention_long_lightning_b200.seqpar import (gather_token_segments,
+                                                             segment_offsets,
+                                                             sparse_layer_qrange)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        rng = np.random.default_rng(321)
+        T, Hq, Hkv, D, topk = sum(lens), 4, 2, 16, 3
+        q, g = (torch.from_numpy(rng.standard_normal((B, T, Hq, D))) for _ in range(2))
+        k, v = (torch.from_numpy(rng.standard_normal((B, T, Hkv, D))) for _ in range(2))
+        offs = segment_offsets(lens)
+        lo, hi = offs[rank], offs[rank] + lens[rank]
+        seg = lambda x: x[:, lo:hi].contiguous()  # this rank's tokens
+
+        def gather_kv(kk, vv):
+            return gather_token_segments(kk, lens), gather_token_segments(vv, lens)
+
+        def select_fn(qq, K, p):
+            rows = list(range(p, p + qq.shape[1]))
+            return oracle.sparse_select(qq.numpy(), K.numpy(), topk=topk, rows=rows, T=K.shape[1])[0]
+
+        def attn_fn(qq, K, V, idx, gg, p):
+            rows = list(range(p, p + qq.shape[1]))
+            return torch.from_numpy(oracle.attention(qq.numpy(), K.numpy(), V.numpy(), gg.numpy(),
+                                                     idx=idx, rows=rows))
+
+        y = sparse_layer_qrange(seg(q), seg(k), seg(v), seg(g), rank=rank, offsets=offs,
+                                gather_kv=gather_kv, select_fn=select_fn, attn_fn=attn_fn,
+                                gather_fn=lambda o: gather_token_segments(o, lens))
+        idx_full = oracle.sparse_select(q.numpy(), k.numpy(), topk=topk)[0]
+        y_full = torch.from_numpy(oracle.attention(q.numpy(), k.numpy(), v.numpy(), g.numpy(),
+                                                   idx=idx_full))
+        out[rank] = (tuple(y.shape), float((y - y_full).abs().max()))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("lens,B", [
+    ((400, 400), 1),             # equal segments: the in-place all-gather
+    ((300, 517, 40), 1),         # three uneven segments, one shorter than a block
+    ((64 * 5 + 3, 64 * 4), 2),   # two sequences per rank
+])
+def test_sparse_query_parallel_ranks(lens, B):
+    world = len(lens)
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.spawn(_qrange_worker, args=(world, _free_port(), list(lens), B, out), nprocs=world,
+             join=True)
+    for rank in range(world):
+        shape, err = out[rank]
+        assert shape == (B, sum(lens), 4, 16)
+        assert err == 0.0
+
+
+def test_segment_offsets():
+    from sparse_attention_long_lightning_b200.seqpar import segment_offsets
+    assert segment_offsets([3, 0, 5]) == [0, 3, 3]
+    assert segment_offsets([]) == []
+    with pytest.raises(ValueError):
+        segment_offsets([2, -1])
