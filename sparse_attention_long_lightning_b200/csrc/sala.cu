@@ -23,6 +23,7 @@
 #include "sparse_decode.cuh"
 #include "sparse_select.cuh"
 #include "sparse_select_tc.cuh"
+#include "sparse_select_hsm_tc.cuh"
 
 using namespace sala;
 
@@ -135,30 +136,33 @@ bool set_smem(KernelT* k, size_t bytes) {
 
 namespace sala {
 
-// Head-softmax scoring kernel for group size G (a power of two up to 32).
+// Per-head softmax-normalised scores on tcgen05 for group size G (a power of two up to
+// 32): one persistent CTA per SM over the rows [geo.r0, geo.r1) of a score pass.
 template <int D, int G>
-static bool launch_hsm(dim3 grid, cudaStream_t st, const __nv_bfloat16* q, const float* kbar,
-                       float* scores, int nb, int Hkv, sala_strides sq, int qpos0, int r0,
-                       int r1, int rows_pass, int n_init, int n_local, float inv_sqrt_d) {
-  auto kern = block_scores_hsm_kernel<D, G>;
-  if (!set_smem(kern, hsm_smem_bytes<D>())) return false;
-  grid.x = (unsigned)((r1 - r0 + kHsmRows / G - 1) / (kHsmRows / G));
-  kern<<<grid, 256, hsm_smem_bytes<D>(), st>>>(q, kbar, scores, nb, Hkv, sq, qpos0, r0, r1,
-                                               rows_pass, n_init, n_local, inv_sqrt_d);
+static bool launch_hsm_tc(cudaStream_t st, const CUtensorMap& tq, const CUtensorMap& th,
+                          const CUtensorMap& tm, const CUtensorMap& tl, float* scores, HtGeom geo,
+                          int rows_pass, float scale_log2) {
+  auto kern = select_hsm_tc_kernel<D, G>;
+  if (!set_smem(kern, HtSmem<D>::bytes)) return false;
+  geo.R = kHtLanes / G;
+  geo.nitems = (geo.r1 - geo.r0 + geo.R - 1) / geo.R * geo.hb;
+  const int grid = std::max(1, std::min(geo.nitems, num_sms()));
+  geo.nrounds = (geo.nitems + grid - 1) / grid;
+  kern<<<grid, kHtThreads, HtSmem<D>::bytes, st>>>(tq, th, tm, tl, scores, geo, rows_pass,
+                                                   scale_log2);
   return true;
 }
 template <int D>
-static bool launch_hsm_g(int G, dim3 grid, cudaStream_t st, const __nv_bfloat16* q,
-                         const float* kbar, float* scores, int nb, int Hkv, sala_strides sq,
-                         int qp, int r0, int r1, int rows_pass, int n_init, int n_local,
-                         float isd) {
+static bool launch_hsm_tc_g(int G, cudaStream_t st, const CUtensorMap& tq, const CUtensorMap& th,
+                            const CUtensorMap& tm, const CUtensorMap& tl, float* scores,
+                            const HtGeom& geo, int rows_pass, float sl) {
   switch (G) {
-    case 1: return launch_hsm<D, 1>(grid, st, q, kbar, scores, nb, Hkv, sq, qp, r0, r1, rows_pass, n_init, n_local, isd);
-    case 2: return launch_hsm<D, 2>(grid, st, q, kbar, scores, nb, Hkv, sq, qp, r0, r1, rows_pass, n_init, n_local, isd);
-    case 4: return launch_hsm<D, 4>(grid, st, q, kbar, scores, nb, Hkv, sq, qp, r0, r1, rows_pass, n_init, n_local, isd);
-    case 8: return launch_hsm<D, 8>(grid, st, q, kbar, scores, nb, Hkv, sq, qp, r0, r1, rows_pass, n_init, n_local, isd);
-    case 16: return launch_hsm<D, 16>(grid, st, q, kbar, scores, nb, Hkv, sq, qp, r0, r1, rows_pass, n_init, n_local, isd);
-    case 32: return launch_hsm<D, 32>(grid, st, q, kbar, scores, nb, Hkv, sq, qp, r0, r1, rows_pass, n_init, n_local, isd);
+    case 1: return launch_hsm_tc<D, 1>(st, tq, th, tm, tl, scores, geo, rows_pass, sl);
+    case 2: return launch_hsm_tc<D, 2>(st, tq, th, tm, tl, scores, geo, rows_pass, sl);
+    case 4: return launch_hsm_tc<D, 4>(st, tq, th, tm, tl, scores, geo, rows_pass, sl);
+    case 8: return launch_hsm_tc<D, 8>(st, tq, th, tm, tl, scores, geo, rows_pass, sl);
+    case 16: return launch_hsm_tc<D, 16>(st, tq, th, tm, tl, scores, geo, rows_pass, sl);
+    case 32: return launch_hsm_tc<D, 32>(st, tq, th, tm, tl, scores, geo, rows_pass, sl);
     default: return false;
   }
 }
@@ -621,18 +625,29 @@ static sala_status sparse_select_impl(const void* q, const void* k, int B, int T
   float* kbar = reinterpret_cast<float*>(wsb + L.kbar_off);
   __nv_bfloat16* khi = reinterpret_cast<__nv_bfloat16*>(wsb + L.khi_off);
   __nv_bfloat16* klo = reinterpret_cast<__nv_bfloat16*>(wsb + L.klo_off);
+  // the third part of the means: per-head softmax scores only (workspace `total`)
+  __nv_bfloat16* klo2 = mode == 1 ? reinterpret_cast<__nv_bfloat16*>(wsb + L.klo2_off) : nullptr;
   float* scores = reinterpret_cast<float*>(wsb + L.score_off);
   const int G = Hq / Hkv;
   const float inv_sqrt_d = 1.0f / std::sqrt((float)D);
   if (L.nb > 0) {
     dim3 gm(L.nb, Hkv, B);
     if (D == 128)
-      block_means_kernel<128><<<gm, 128, 0, st>>>((const __nv_bfloat16*)k, kbar, khi, klo, L.nb,
-                                                   Hkv, sk);
+      block_means_kernel<128><<<gm, 128, 0, st>>>((const __nv_bfloat16*)k, kbar, khi, klo, klo2,
+                                                   L.nb, Hkv, sk);
     else
-      block_means_kernel<64><<<gm, 64, 0, st>>>((const __nv_bfloat16*)k, kbar, khi, klo, L.nb,
-                                                 Hkv, sk);
+      block_means_kernel<64><<<gm, 64, 0, st>>>((const __nv_bfloat16*)k, kbar, khi, klo, klo2,
+                                                 L.nb, Hkv, sk);
     SALA_CHECK_LAUNCH();
+  }
+  CUtensorMap hq, hh, hm, hl;  // per-head softmax path: q, and the means' three bf16 parts
+  if (mode == 1 && L.nb > 0) {
+    const sala_strides skb{(int64_t)L.nb * Hkv * D, (int64_t)Hkv * D, (int64_t)D};
+    if (!make_tmap_bhtd(&hq, q, B, T, Hq, D, sq, kHtLanes / G, G) ||
+        !make_tmap_bhtd(&hh, khi, B, L.nb, Hkv, D, skb, kHtN) ||
+        !make_tmap_bhtd(&hm, klo, B, L.nb, Hkv, D, skb, kHtN) ||
+        !make_tmap_bhtd(&hl, klo2, B, L.nb, Hkv, D, skb, kHtN))
+      return SALA_ERR_CUDA;
   }
   if (fused) {
     // block means (bf16 hi / lo) as a [B, nb, Hkv, D] tensor, 32-candidate boxes
@@ -663,13 +678,20 @@ static sala_status sparse_select_impl(const void* q, const void* k, int B, int T
   for (int r0 = 0; r0 < T; r0 += L.rows_pass) {
     const int r1 = std::min(T, r0 + L.rows_pass);
     if (L.nb > 0 && mode == 1) {
-      const bool ok =
-          D == 128 ? launch_hsm_g<128>(G, dim3(1, Hkv, B), st, (const __nv_bfloat16*)q, kbar,
-                                       scores, L.nb, Hkv, sq, qpos0, r0, r1, L.rows_pass,
-                                       n_init, n_local, inv_sqrt_d)
-                   : launch_hsm_g<64>(G, dim3(1, Hkv, B), st, (const __nv_bfloat16*)q, kbar,
-                                      scores, L.nb, Hkv, sq, qpos0, r0, r1, L.rows_pass,
-                                      n_init, n_local, inv_sqrt_d);
+      HtGeom geo{};
+      geo.r0 = r0;
+      geo.r1 = r1;
+      geo.qpos0 = qpos0;
+      geo.nb = L.nb;
+      geo.Hkv = Hkv;
+      geo.hb = Hkv * B;
+      geo.n_init = n_init;
+      geo.n_local = n_local;
+      const float sl = inv_sqrt_d * 1.4426950408889634f;
+      const bool ok = D == 128 ? launch_hsm_tc_g<128>(G, st, hq, hh, hm, hl, scores, geo,
+                                                      L.rows_pass, sl)
+                               : launch_hsm_tc_g<64>(G, st, hq, hh, hm, hl, scores, geo,
+                                                     L.rows_pass, sl);
       if (!ok) return SALA_ERR_CUDA;
       SALA_CHECK_LAUNCH();
     } else if (L.nb > 0) {

@@ -35,6 +35,7 @@ struct SelLayout {
   size_t kbar_off, kbar_bytes;   // block means, fp32
   size_t khi_off, klo_off;       // block means as bf16 high / low parts
   size_t score_off, score_bytes; // score scratch (topk > kSelFusedMaxK only)
+  size_t klo2_off;               // third bf16 part of the means (score-scratch layout only)
   size_t total_fused, total;
 };
 
@@ -57,18 +58,21 @@ inline SelLayout sel_layout(int B, int T, int Tk, int Hkv, int D) {
   L.score_off = L.klo_off + up(nelem * 2);
   L.total_fused = L.score_off;
   L.score_bytes = per_row * (size_t)L.rows_pass;
-  L.total = L.score_off + L.score_bytes;
+  L.klo2_off = L.score_off + up(L.score_bytes);
+  L.total = L.klo2_off + up(nelem * 2);
   return L;
 }
 
 // ---- kernel 1: block means.  grid (nb, Hkv, B), block D threads.
 // Writes the fp32 mean and its split into bf16 high and low parts (hi + lo
-// carries 16 significant bits: the tensor-core scoring operand).
+// carries 16 significant bits: the tensor-core scoring operand); with klo2, also
+// the third part lo2 = mean - hi - lo, so that hi + lo + lo2 is the fp32 mean exactly
+// (each remainder is exact in fp32 and has at most 8 significant bits left at the end).
 template <int D>
 __global__ void __launch_bounds__(D)
 block_means_kernel(const __nv_bfloat16* __restrict__ k, float* __restrict__ kbar,
-                   __nv_bfloat16* __restrict__ khi, __nv_bfloat16* __restrict__ klo, int nb,
-                   int Hkv, sala_strides sk) {
+                   __nv_bfloat16* __restrict__ khi, __nv_bfloat16* __restrict__ klo,
+                   __nv_bfloat16* __restrict__ klo2, int nb, int Hkv, sala_strides sk) {
   const int j = blockIdx.x, hk = blockIdx.y, b = blockIdx.z, d = threadIdx.x;
   const __nv_bfloat16* src = k + b * sk.b + (int64_t)j * kSelBlk * sk.t + hk * sk.h + d;
   float acc = 0.f;
@@ -79,7 +83,10 @@ block_means_kernel(const __nv_bfloat16* __restrict__ k, float* __restrict__ kbar
   kbar[o] = m;
   const __nv_bfloat16 h = __float2bfloat16_rn(m);
   khi[o] = h;
-  klo[o] = __float2bfloat16_rn(m - __bfloat162float(h));
+  const float r1 = m - __bfloat162float(h);
+  const __nv_bfloat16 lo = __float2bfloat16_rn(r1);
+  klo[o] = lo;
+  if (klo2) klo2[o] = __float2bfloat16_rn(r1 - __bfloat162float(lo));
 }
 
 // ---- kernel 2: block scores for a 64-row tile.  grid (row tiles, Hkv, B), 256 threads.
@@ -254,157 +261,6 @@ topk_select_kernel(const float* __restrict__ scores, int32_t* __restrict__ idx, 
   for (int j = lo + lane; j <= c; j += 32) out[pos + (j - lo)] = j;
   pos += (c >= lo) ? c - lo + 1 : 0;
   for (int e = pos + lane; e < n_sel; e += 32) out[e] = -1;
-}
-
-}  // namespace sala
-
-namespace sala {
-
-// ---- selection variant: per-head softmax-normalised scores summed over the group.
-//   s_{h,j} = (1/sqrt(D)) q_{t,h} . Kbar_j  for the same candidates as kernel 2,
-//   score_j = sum_{h in group(hk)} exp(s_{h,j} - m_h) / sum_{j'} exp(s_{h,j'} - m_h),
-// m_h the row's maximum for head h.  Written into the same score scratch, so the
-// top-k kernel above selects from it unchanged.  fp32 throughout (exact products of
-// bf16 q and fp32 means, expf, IEEE division).
-//
-// grid (row tiles, Hkv, B), 256 threads.  A tile is R = 256 / G query rows times the
-// G heads of the group: 256 query-head rows f = (t - t0) * G + h.  Thread (qr, tc)
-// owns rows f = 8 qr .. 8 qr + 7 and candidates 8 tc .. 8 tc + 7 of each 64-candidate
-// tile (qr = 4 warp + lane / 8, tc = lane % 8), so the 8 lanes sharing rows are one
-// lane group and a query row's G heads are in one thread (G <= 8) or in lanes 8 or
-// 16 apart (G = 16, 32).  Pass 1 keeps each query-head row's running maximum and sum
-// of exponentials; pass 2 recomputes the scores and writes the sums.
-constexpr int kHsmRows = 256;
-constexpr int kHsmLd = kHsmRows + 4;
-template <int D>
-constexpr size_t hsm_smem_bytes() { return size_t(D) * (kHsmLd + kScLd) * sizeof(float); }
-
-template <int D, int G>
-__global__ void __launch_bounds__(256)
-block_scores_hsm_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ kbar,
-                        float* __restrict__ scores, int nb, int Hkv, sala_strides sq,
-                        int qpos0, int r_begin, int r_end, int rows_pass, int n_init,
-                        int n_local, float inv_sqrt_d) {
-  static_assert(G >= 1 && G <= 32 && (G & (G - 1)) == 0, "group of 1..32 heads, power of 2");
-  constexpr int R = kHsmRows / G;  // query rows per tile
-  constexpr int GIN = G < 8 ? G : 8;  // heads of one query row inside a thread
-  extern __shared__ float hs_smem[];
-  float (*qT)[kHsmLd] = reinterpret_cast<float (*)[kHsmLd]>(hs_smem);           // [D][kHsmLd]
-  float (*kT)[kScLd] = reinterpret_cast<float (*)[kScLd]>(hs_smem + D * kHsmLd);  // [D][kScLd]
-  const int ntiles = (r_end - r_begin + R - 1) / R;
-  const int tile = ntiles - 1 - blockIdx.x;  // long (late) rows first
-  const int hk = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
-  const int t0 = r_begin + tile * R;
-  const int t_last = min(t0 + R, r_end) - 1;
-  const int j_hi = min((qpos0 + t_last) / kSelBlk - n_local, nb - 1);  // the tile's last candidate
-  if (j_hi < n_init) return;
-
-  for (int e = tid; e < kHsmRows * D; e += 256) {
-    const int f = e / D, d = e % D;
-    const int t = t0 + f / G, h = hk * G + f % G;
-    qT[d][f] = t <= t_last
-                   ? __bfloat162float(q[b * sq.b + (int64_t)t * sq.t + (int64_t)h * sq.h + d])
-                   : 0.f;
-  }
-  const int warp = tid >> 5, lane = tid & 31;
-  const int qr = 4 * warp + (lane >> 3), tc = lane & 7;
-  int jmax[8];  // last candidate of each of this thread's rows (n_init - 1: none)
-#pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    const int t = t0 + (8 * qr + u) / G;
-    jmax[u] = t <= t_last ? min((qpos0 + t) / kSelBlk - n_local, nb - 1) : n_init - 1;
-  }
-
-  float acc[8][8];
-  auto tile_scores = [&](int jt0) {
-    __syncthreads();  // qT written / previous kT consumed
-    for (int e = tid; e < kScTile * D; e += 256) {
-      const int jj = e / D, d = e % D;
-      const int j = jt0 + jj;
-      kT[d][jj] = j <= j_hi ? kbar[(((int64_t)b * nb + j) * Hkv + hk) * D + d] : 0.f;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int u = 0; u < 8; ++u)
-#pragma unroll
-      for (int w = 0; w < 8; ++w) acc[u][w] = 0.f;
-#pragma unroll 2
-    for (int d = 0; d < D; ++d) {
-      const float4 a0 = *reinterpret_cast<const float4*>(&qT[d][8 * qr]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&qT[d][8 * qr + 4]);
-      const float4 c0 = *reinterpret_cast<const float4*>(&kT[d][8 * tc]);
-      const float4 c1 = *reinterpret_cast<const float4*>(&kT[d][8 * tc + 4]);
-      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-#pragma unroll
-        for (int w = 0; w < 8; ++w) acc[u][w] = fmaf(av[u], cv[w], acc[u][w]);
-    }
-  };
-
-  // pass 1: running maximum m and sum of exponentials l per query-head row (the 8
-  // lanes of a lane group hold the same values)
-  float m[8], l[8];
-#pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    m[u] = -INFINITY;
-    l[u] = 0.f;
-  }
-  for (int jt0 = n_init; jt0 <= j_hi; jt0 += kScTile) {
-    tile_scores(jt0);
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      float mx = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < 8; ++w)
-        if (jt0 + 8 * tc + w <= jmax[u]) mx = fmaxf(mx, acc[u][w] * inv_sqrt_d);
-#pragma unroll
-      for (int off = 1; off < 8; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-      const bool any = mx > -INFINITY;  // the row has candidates in this tile
-      const float mn = any ? fmaxf(m[u], mx) : m[u];
-      float sum = 0.f;
-#pragma unroll
-      for (int w = 0; w < 8; ++w)
-        if (jt0 + 8 * tc + w <= jmax[u]) sum += expf(acc[u][w] * inv_sqrt_d - mn);
-#pragma unroll
-      for (int off = 1; off < 8; off <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-      if (any) {
-        l[u] = l[u] * expf(m[u] - mn) + sum;  // expf(-inf) = 0 on a row's first tile
-        m[u] = mn;
-      }
-    }
-  }
-  float inv_l[8];
-#pragma unroll
-  for (int u = 0; u < 8; ++u) inv_l[u] = l[u] > 0.f ? 1.0f / l[u] : 0.f;
-
-  // pass 2: p = exp(s - m) / l, summed over the G heads of each query row
-  float* srow_base = scores + ((int64_t)b * Hkv + hk) * rows_pass * (int64_t)nb;
-  for (int jt0 = n_init; jt0 <= j_hi; jt0 += kScTile) {
-    tile_scores(jt0);
-#pragma unroll
-    for (int w = 0; w < 8; ++w) {
-      const int j = jt0 + 8 * tc + w;
-      float ps[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        ps[u] = j <= jmax[u] ? expf(acc[u][w] * inv_sqrt_d - m[u]) * inv_l[u] : 0.f;
-#pragma unroll
-      for (int a = 0; a < 8; a += GIN) {
-        float hsum = 0.f;
-#pragma unroll
-        for (int v = 0; v < GIN; ++v) hsum += ps[a + v];
-        if (G >= 16) hsum += __shfl_xor_sync(0xffffffffu, hsum, 8);
-        if (G >= 32) hsum += __shfl_xor_sync(0xffffffffu, hsum, 16);
-        // the first thread of the query row's lane set writes
-        const bool writer = G <= 8 || (qr & (G / 8 - 1)) == 0;
-        const int t = t0 + (8 * qr + a) / G;
-        if (writer && j <= jmax[a])
-          srow_base[(int64_t)(t - r_begin) * nb + (j - n_init)] = hsum;
-      }
-    }
-  }
 }
 
 }  // namespace sala

@@ -155,9 +155,10 @@ def test_workspace_queries(lib):
     # topk <= 64: block means only (scores and top-k fused)
     n = sala.sparse_select_workspace(1, 131072, 32, 2, 128, 64, 64)
     assert means <= n <= means + 1024
-    # larger topk: plus a score scratch bounded by 1 GiB
+    # larger topk: plus a score scratch bounded by 1 GiB and the means' third bf16 part
     n = sala.sparse_select_workspace(1, 131072, 32, 2, 128, 64, 100)
-    assert means + (1 << 29) <= n <= means + (1 << 30) + 4096
+    means3 = means + nb * 2 * 128 * 2
+    assert means3 + (1 << 29) <= n <= means3 + (1 << 30) + 4096
     assert sala.sparse_select_workspace(1, 1 << 20, 32, 2, 128, 64, 200) <= (1 << 30) + (1 << 26)
     # fp16 copy of v, then 128 partial maxima and 128 partial sums of squares, one
     # exponent and one outlier flag per (sequence, KV head), each part 256-byte aligned
@@ -188,7 +189,8 @@ def test_head_softmax_workspace_has_score_scratch():
     nb = 131072 // 64
     means = nb * 2 * 128 * (4 + 2 + 2)
     n = sala.sparse_select_head_softmax_workspace(1, 131072, 32, 2, 128)
-    assert means + (1 << 29) <= n <= means + (1 << 30) + 4096
+    means3 = means + nb * 2 * 128 * 2  # hi / lo / lo2 bf16 parts of the means
+    assert means3 + (1 << 29) <= n <= means3 + (1 << 30) + 4096
     assert n == sala.sparse_select_workspace(1, 131072, 32, 2, 128, 64, 100)
     assert sala.sparse_select_head_softmax_workspace(1, 0, 32, 2, 128) == 0
 
@@ -221,7 +223,7 @@ def test_row_window_workspace_queries():
     assert n == sala.sparse_select_workspace(1, 131072, 32, 2, 128, 64, 64)
     assert means <= n <= means + 1024
     hs = sala.sparse_select_rows_workspace(1, 64, 131072, 32, 2, 128, score="head_softmax")
-    assert hs == means + 2 * 64 * nb * 4
+    assert hs == means + 2 * 64 * nb * 4 + nb * 2 * 128 * 2  # + the means' third part
     full = sala.sparse_select_rows_workspace(1, 131072, 131072, 32, 2, 128, score="head_softmax")
     assert full == sala.sparse_select_head_softmax_workspace(1, 131072, 32, 2, 128)
     assert sala.sparse_select_rows_workspace(1, 64, 0, 32, 2, 128) == 0
