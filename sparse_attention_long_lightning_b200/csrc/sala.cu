@@ -139,30 +139,29 @@ namespace sala {
 // Per-head softmax-normalised scores on tcgen05 for group size G (a power of two up to
 // 32): one persistent CTA per SM over the rows [geo.r0, geo.r1) of a score pass.
 template <int D, int G>
-static bool launch_hsm_tc(cudaStream_t st, const CUtensorMap& tq, const CUtensorMap& th,
-                          const CUtensorMap& tm, const CUtensorMap& tl, float* scores, HtGeom geo,
-                          int rows_pass, float scale_log2) {
+static bool launch_hsm_tc(cudaStream_t st, const __nv_bfloat16* q, sala_strides sq,
+                          const CUtensorMap& th, const CUtensorMap& tm, const CUtensorMap& tl,
+                          float* scores, HtGeom geo, int rows_pass) {
   auto kern = select_hsm_tc_kernel<D, G>;
   if (!set_smem(kern, HtSmem<D>::bytes)) return false;
   geo.R = kHtLanes / G;
   geo.nitems = (geo.r1 - geo.r0 + geo.R - 1) / geo.R * geo.hb;
   const int grid = std::max(1, std::min(geo.nitems, num_sms()));
   geo.nrounds = (geo.nitems + grid - 1) / grid;
-  kern<<<grid, kHtThreads, HtSmem<D>::bytes, st>>>(tq, th, tm, tl, scores, geo, rows_pass,
-                                                   scale_log2);
+  kern<<<grid, kHtThreads, HtSmem<D>::bytes, st>>>(q, sq, th, tm, tl, scores, geo, rows_pass);
   return true;
 }
 template <int D>
-static bool launch_hsm_tc_g(int G, cudaStream_t st, const CUtensorMap& tq, const CUtensorMap& th,
-                            const CUtensorMap& tm, const CUtensorMap& tl, float* scores,
-                            const HtGeom& geo, int rows_pass, float sl) {
+static bool launch_hsm_tc_g(int G, cudaStream_t st, const __nv_bfloat16* q, sala_strides sq,
+                            const CUtensorMap& th, const CUtensorMap& tm, const CUtensorMap& tl,
+                            float* scores, const HtGeom& geo, int rows_pass) {
   switch (G) {
-    case 1: return launch_hsm_tc<D, 1>(st, tq, th, tm, tl, scores, geo, rows_pass, sl);
-    case 2: return launch_hsm_tc<D, 2>(st, tq, th, tm, tl, scores, geo, rows_pass, sl);
-    case 4: return launch_hsm_tc<D, 4>(st, tq, th, tm, tl, scores, geo, rows_pass, sl);
-    case 8: return launch_hsm_tc<D, 8>(st, tq, th, tm, tl, scores, geo, rows_pass, sl);
-    case 16: return launch_hsm_tc<D, 16>(st, tq, th, tm, tl, scores, geo, rows_pass, sl);
-    case 32: return launch_hsm_tc<D, 32>(st, tq, th, tm, tl, scores, geo, rows_pass, sl);
+    case 1: return launch_hsm_tc<D, 1>(st, q, sq, th, tm, tl, scores, geo, rows_pass);
+    case 2: return launch_hsm_tc<D, 2>(st, q, sq, th, tm, tl, scores, geo, rows_pass);
+    case 4: return launch_hsm_tc<D, 4>(st, q, sq, th, tm, tl, scores, geo, rows_pass);
+    case 8: return launch_hsm_tc<D, 8>(st, q, sq, th, tm, tl, scores, geo, rows_pass);
+    case 16: return launch_hsm_tc<D, 16>(st, q, sq, th, tm, tl, scores, geo, rows_pass);
+    case 32: return launch_hsm_tc<D, 32>(st, q, sq, th, tm, tl, scores, geo, rows_pass);
     default: return false;
   }
 }
@@ -630,21 +629,23 @@ static sala_status sparse_select_impl(const void* q, const void* k, int B, int T
   float* scores = reinterpret_cast<float*>(wsb + L.score_off);
   const int G = Hq / Hkv;
   const float inv_sqrt_d = 1.0f / std::sqrt((float)D);
+  // per-head softmax: the bf16 parts carry the means times log2(e) / sqrt(D), so the
+  // MMAs give the scores in the log2 domain of the exponentials
+  const float part_scale = mode == 1 ? inv_sqrt_d * 1.4426950408889634f : 1.0f;
   if (L.nb > 0) {
     dim3 gm(L.nb, Hkv, B);
     if (D == 128)
       block_means_kernel<128><<<gm, 128, 0, st>>>((const __nv_bfloat16*)k, kbar, khi, klo, klo2,
-                                                   L.nb, Hkv, sk);
+                                                   part_scale, L.nb, Hkv, sk);
     else
       block_means_kernel<64><<<gm, 64, 0, st>>>((const __nv_bfloat16*)k, kbar, khi, klo, klo2,
-                                                 L.nb, Hkv, sk);
+                                                 part_scale, L.nb, Hkv, sk);
     SALA_CHECK_LAUNCH();
   }
-  CUtensorMap hq, hh, hm, hl;  // per-head softmax path: q, and the means' three bf16 parts
+  CUtensorMap hh, hm, hl;  // per-head softmax path: the means' three bf16 parts
   if (mode == 1 && L.nb > 0) {
     const sala_strides skb{(int64_t)L.nb * Hkv * D, (int64_t)Hkv * D, (int64_t)D};
-    if (!make_tmap_bhtd(&hq, q, B, T, Hq, D, sq, kHtLanes / G, G) ||
-        !make_tmap_bhtd(&hh, khi, B, L.nb, Hkv, D, skb, kHtN) ||
+    if (!make_tmap_bhtd(&hh, khi, B, L.nb, Hkv, D, skb, kHtN) ||
         !make_tmap_bhtd(&hm, klo, B, L.nb, Hkv, D, skb, kHtN) ||
         !make_tmap_bhtd(&hl, klo2, B, L.nb, Hkv, D, skb, kHtN))
       return SALA_ERR_CUDA;
@@ -681,17 +682,18 @@ static sala_status sparse_select_impl(const void* q, const void* k, int B, int T
       HtGeom geo{};
       geo.r0 = r0;
       geo.r1 = r1;
+      geo.Tq = T;
       geo.qpos0 = qpos0;
       geo.nb = L.nb;
       geo.Hkv = Hkv;
       geo.hb = Hkv * B;
       geo.n_init = n_init;
       geo.n_local = n_local;
-      const float sl = inv_sqrt_d * 1.4426950408889634f;
-      const bool ok = D == 128 ? launch_hsm_tc_g<128>(G, st, hq, hh, hm, hl, scores, geo,
-                                                      L.rows_pass, sl)
-                               : launch_hsm_tc_g<64>(G, st, hq, hh, hm, hl, scores, geo,
-                                                     L.rows_pass, sl);
+      const __nv_bfloat16* qb = (const __nv_bfloat16*)q;
+      const bool ok = D == 128 ? launch_hsm_tc_g<128>(G, st, qb, sq, hh, hm, hl, scores, geo,
+                                                      L.rows_pass)
+                               : launch_hsm_tc_g<64>(G, st, qb, sq, hh, hm, hl, scores, geo,
+                                                     L.rows_pass);
       if (!ok) return SALA_ERR_CUDA;
       SALA_CHECK_LAUNCH();
     } else if (L.nb > 0) {

@@ -65,14 +65,16 @@ inline SelLayout sel_layout(int B, int T, int Tk, int Hkv, int D) {
 
 // ---- kernel 1: block means.  grid (nb, Hkv, B), block D threads.
 // Writes the fp32 mean and its split into bf16 high and low parts (hi + lo
-// carries 16 significant bits: the tensor-core scoring operand); with klo2, also
-// the third part lo2 = mean - hi - lo, so that hi + lo + lo2 is the fp32 mean exactly
+// carries 16 significant bits: the tensor-core scoring operand); with klo2, the
+// parts are those of x = mean * part_scale (one fp32 rounding; 1 leaves the mean as it
+// is) and include the third part lo2 = x - hi - lo, so that hi + lo + lo2 is x exactly
 // (each remainder is exact in fp32 and has at most 8 significant bits left at the end).
 template <int D>
 __global__ void __launch_bounds__(D)
 block_means_kernel(const __nv_bfloat16* __restrict__ k, float* __restrict__ kbar,
                    __nv_bfloat16* __restrict__ khi, __nv_bfloat16* __restrict__ klo,
-                   __nv_bfloat16* __restrict__ klo2, int nb, int Hkv, sala_strides sk) {
+                   __nv_bfloat16* __restrict__ klo2, float part_scale, int nb, int Hkv,
+                   sala_strides sk) {
   const int j = blockIdx.x, hk = blockIdx.y, b = blockIdx.z, d = threadIdx.x;
   const __nv_bfloat16* src = k + b * sk.b + (int64_t)j * kSelBlk * sk.t + hk * sk.h + d;
   float acc = 0.f;
@@ -81,9 +83,10 @@ block_means_kernel(const __nv_bfloat16* __restrict__ k, float* __restrict__ kbar
   const float m = acc * (1.0f / kSelBlk);
   const int64_t o = (((int64_t)b * nb + j) * Hkv + hk) * D + d;
   kbar[o] = m;
-  const __nv_bfloat16 h = __float2bfloat16_rn(m);
+  const float x = klo2 ? m * part_scale : m;
+  const __nv_bfloat16 h = __float2bfloat16_rn(x);
   khi[o] = h;
-  const float r1 = m - __bfloat162float(h);
+  const float r1 = x - __bfloat162float(h);
   const __nv_bfloat16 lo = __float2bfloat16_rn(r1);
   klo[o] = lo;
   if (klo2) klo2[o] = __float2bfloat16_rn(r1 - __bfloat162float(lo));

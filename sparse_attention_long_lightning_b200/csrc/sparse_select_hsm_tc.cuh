@@ -11,23 +11,31 @@
 //
 // Design (sm_100a).  An item is R = 128 / G consecutive query rows of one KV head: its
 // R x G (query row, head) pairs are the M = 128 rows of the MMAs, so TMEM lane l =
-// (row l / G, head l % G) and each consumer thread owns one head of one row.  A TMA box
-// of q [B, T, Hq, D] with G heads x R rows lands exactly in that order (the A operand,
-// q as stored: bf16 is exact).  The block means (fp32) are split into three bf16 parts
-// hi + mid + lo = Kbar exactly (8 significant bits each), so
-//   S = q.lo + q.mid + q.hi
-// (24 MMAs of N = 64 per 64-candidate tile at D = 128) is the fp32 dot product up to
-// the accumulation order.  Every item is scored twice: pass 1 keeps each thread's
+// (row l / G, head l % G) and each consumer thread owns one head of one row.  The A
+// operand (q as stored: bf16 is exact) sits in TMEM, so the MMAs of a tile read only the
+// block means from shared memory.  The block means times log2(e)/sqrt(D) (one fp32
+// rounding: the scores come out in the log2 domain of the exponentials) are split into
+// three bf16 parts hi + mid + lo = that value exactly (8 significant bits each); a tile's three parts are
+// stacked as the N = 192 rows of the B operand, so 8 MMAs (D = 128) give q.hi, q.mid and
+// q.lo side by side in TMEM and the consumers form S = (q.lo + q.mid) + q.hi: the fp32
+// dot product up to the summation order (fewer, wider MMAs: each MMA instruction has a
+// fixed cost that N = 64 products did not cover).  Every item is scored twice: pass 1 keeps each thread's
 // running maximum and sum of exponentials (online, in registers: no cross-thread work),
 // pass 2 recomputes S, forms p = exp(s - m) / l, and the G threads of a query row sum
 // their heads' p by a butterfly reduce-scatter (after which lane g of the row's group
 // holds the sums of candidates g * 64/G .. (g + 1) * 64/G - 1 of the tile) and store
 // them, coalesced, into the scratch row.
-//   issuer (warp 4, one thread): TMA of the items' q tiles (two A buffers) and of the
-//     block-mean tiles (3-stage ring, hi / mid / lo), and the MMAs into one of 4 TMEM
-//     score buffers, running ahead of the consumers by the ring depth;
-//   consumers (warps 0-3): tcgen05.ld of a tile's 64 scores, buffer release (per-warp
-//     arrival), then the pass's arithmetic.
+//   producers (warps 9-12): thread l loads lane l's query-head row of the next item
+//     and stores it into its TMEM lane (two A buffers), overlapping the current item;
+//   copier (warp 13, one thread): TMA of the block-mean tiles (4-stage ring, hi / mid /
+//     lo per 64-dim half), running ahead by the ring depth;
+//   issuer (warp 8, one thread): the MMAs of each tile into one of 2 TMEM score buffers;
+//   consumers (warps 0-7): warps w and w + 4 read TMEM lane quadrant w, each one half
+//     (32 candidates) of every tile: tcgen05.ld, buffer release (per-warp arrival), then
+//     the pass's arithmetic; at the end of pass 1 the two threads of a lane merge their
+//     halves' (max, sum) through shared memory (a bounded mbarrier wait, per item
+//     parity), so pass 2 normalises with the row's full sum.  Two warps per scheduler
+//     hide each other's latency.
 // All waits are bounded: a wait that runs out raises SALA_ERR_TIMEOUT, and the kernel
 // drains its copies and MMAs before it frees TMEM and returns.
 #pragma once
@@ -38,23 +46,38 @@ namespace sala {
 
 constexpr int kHtLanes = 128;   // (query row, head) pairs per item = TMEM lanes
 constexpr int kHtN = 64;        // candidates per tile
-constexpr int kHtStages = 3;    // block-mean tile ring
-constexpr int kHtAcc = 4;       // TMEM score buffers
-constexpr int kHtThreads = kHtLanes + 32;
+constexpr int kHtHalf = kHtN / 2;  // candidates of a tile per consumer thread
+constexpr int kHtStages = 4;    // block-mean tile ring
+constexpr int kHtAcc = 2;       // TMEM score buffers (3 x kHtN columns each)
+constexpr int kHtConsumers = 8; // two warps per TMEM lane quadrant (one per tile half)
+constexpr int kHtThreads = kHtConsumers * 32 + 32 + kHtLanes + 32;  // consumers, issuer,
+                                                                    // producers, copier
+constexpr int kHtCopier = kHtConsumers + 1 + kHtLanes / 32;        // the copier's warp
+
+// 2^x on the transcendental unit (relative error about 2^-22; subnormal results kept)
+__device__ __forceinline__ float ht_exp2(float x) {
+  float y;
+  asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 template <int D>
 struct HtSmem {
   static constexpr int kHalfB = kHtN * 128;         // 64 candidates x 64 dims, bf16
-  static constexpr int kPartB = (D / 64) * kHalfB;  // one of hi / mid / lo
-  static constexpr int kStage = 3 * kPartB;
-  static constexpr int kAHalf = kHtLanes * 128;     // 128 lanes x 64 dims, bf16
-  static constexpr int kA = (D / 64) * kAHalf;
+  static constexpr int kHalf3 = 3 * kHalfB;         // hi, mid, lo of one 64-dim half
+  static constexpr int kStage = (D / 64) * kHalf3;
   static constexpr size_t kB = 0;                                    // [stages]
-  static constexpr size_t kAoff = kB + kHtStages * size_t(kStage);   // [2]
-  static constexpr size_t kBars = kAoff + 2 * size_t(kA);
-  // full[S], stage_free[S], mma_done[A], acc_free[A], a_full[2], a_free[2], drain
-  static constexpr int kNumBars = 2 * kHtStages + 2 * kHtAcc + 4 + 1;
-  static constexpr size_t bytes = 1024 + kBars + kNumBars * 8 + 16;
+  static constexpr size_t kBars = kB + kHtStages * size_t(kStage);
+  // full[S], stage_free[S], mma_done[A], acc_free[A], a_full[2], a_free[2], drain,
+  // pair[4 quadrants][2 item parities]
+  static constexpr int kNumBars = 2 * kHtStages + 2 * kHtAcc + 4 + 1 + 8;
+  // [2 item parities][2 tile halves][128 lanes] x (max, sum): the two warps of a lane
+  // quadrant combine their halves' running softmax state at the end of pass 1
+  static constexpr size_t kComb = kBars + kNumBars * 8 + 16;
+  static constexpr size_t need = 1024 + kComb + 2 * 2 * kHtLanes * 8;
+  // at least half of the SM's shared memory, so that one CTA per SM holds all 512 TMEM
+  // columns (a second CTA's allocation would wait for the first to finish)
+  static constexpr size_t bytes = need > 120 * 1024 ? need : 120 * 1024;
   static_assert(bytes <= 232448, "fits one CTA per SM");
 };
 
@@ -67,7 +90,7 @@ struct HtCursor {
 };
 
 struct HtGeom {
-  int R, r0, r1, qpos0, nb, Hkv, hb, nitems, nrounds, n_init, n_local;
+  int R, r0, r1, Tq, qpos0, nb, Hkv, hb, nitems, nrounds, n_init, n_local;
   __device__ int item_of(int r) const {
     return r * (int)gridDim.x + ((r & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x);
   }
@@ -113,9 +136,9 @@ struct HtGeom {
 // Sum of the G lanes' values of one query row, scattered: each step at distance d
 // (G / 2, G / 4, .., 1) adds the partner's half of the N values the lane still holds and
 // keeps the half selected by (lane & d); lane g of the group ends with the sums of
-// entries g * kHtN / G .. (g + 1) * kHtN / G - 1 in s[0 ..].
+// entries g * N / G .. (g + 1) * N / G - 1 in s[0 ..].
 template <int G, int N>
-__device__ __forceinline__ void ht_reduce_scatter(float (&s)[kHtN], int lane) {
+__device__ __forceinline__ void ht_reduce_scatter(float (&s)[kHtHalf], int lane) {
   if constexpr (G > 1) {
     constexpr int d = G / 2, half = N / 2;
     const bool upper = (lane & d) != 0;
@@ -131,14 +154,14 @@ __device__ __forceinline__ void ht_reduce_scatter(float (&s)[kHtN], int lane) {
 
 template <int D, int G>
 __global__ void __launch_bounds__(kHtThreads, 1)
-select_hsm_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+select_hsm_tc_kernel(const __nv_bfloat16* __restrict__ q, sala_strides sq,
                      const __grid_constant__ CUtensorMap tm_hi,
                      const __grid_constant__ CUtensorMap tm_mid,
                      const __grid_constant__ CUtensorMap tm_lo, float* __restrict__ scores,
-                     const HtGeom geo, int rows_pass, float scale_log2) {
+                     const HtGeom geo, int rows_pass) {
   using L = HtSmem<D>;
   constexpr int kK = D / 16;  // k-steps
-  constexpr uint32_t kId = umma_idesc_bf16(128, kHtN, false, false);
+  constexpr uint32_t kId = umma_idesc_bf16(128, 3 * kHtN, false, false);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -149,7 +172,8 @@ select_hsm_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint64_t* a_full = acc_free + kHtAcc;                          // [2] q tile landed
   uint64_t* a_free = a_full + 2;                                 // [2] q tile's MMAs done
   uint64_t* drain = a_free + 2;                                  // every MMA done (exit)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* pair = drain + 1;                                    // [4][2] halves merged
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pair + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -160,93 +184,86 @@ select_hsm_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
     for (int i = 0; i < kHtAcc; ++i) {
       mbar_init(&mma_done[i], 1);
-      mbar_init(&acc_free[i], kHtLanes / 32);
+      mbar_init(&acc_free[i], kHtConsumers);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&a_full[i], 1);
+      mbar_init(&a_full[i], kHtLanes);
       mbar_init(&a_free[i], 1);
     }
     mbar_init(drain, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(&pair[i], 64);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0) tc_alloc(tmem_slot, kHtAcc * kHtN);
+  constexpr int kAcols = D / 2;  // TMEM columns of one A buffer (bf16 pairs)
+  constexpr uint32_t kCols = 2 * kAcols + kHtAcc * 3 * kHtN <= 256 ? 256 : 512;
+  static_assert(2 * kAcols + kHtAcc * 3 * kHtN <= 512, "TMEM columns");
+  if (warp == 0) tc_alloc(tmem_slot, kCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tD = *tmem_slot;
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tD = tmem + 2 * kAcols;  // [kHtAcc] x (hi, mid, lo) x kHtN columns
 
-  if (warp == 4) {
-    // ================= issuer: TMA (q tiles, block-mean tiles) and the score MMAs
+  if (warp == kHtCopier) {
+    // ================= copier: block-mean tiles (hi, mid, lo per 64-dim half) by TMA
     if ((tid & 31) == 0) {
-      prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_hi);
       prefetch_tmap(&tm_mid);
       prefetch_tmap(&tm_lo);
-      HtCursor tc, mc;  // TMA cursor (runs ahead), MMA cursor
+      HtCursor tc;
       geo.begin(tc);
-      geo.begin(mc);
-      int g_tma = 0, g_mma = 0, a_loads = 0;
+      int g_tma = 0;
       bool ok = true;
-      // issue the copies of the tile under the TMA cursor (and its item's q tile first)
-      auto tma_step = [&]() -> bool {
-        if (tc.pass == 0 && tc.i == 0) {
-          const int buf = tc.u & 1;
-          if (tc.u >= 2 && !mbar_wait(&a_free[buf], ((tc.u - 2) >> 1) & 1)) return false;
-          uint8_t* dst = smem + L::kAoff + buf * L::kA;
-          mbar_arrive_expect_tx(&a_full[buf], L::kA);
-#pragma unroll
-          for (int hf = 0; hf < D / 64; ++hf)
-            tma_load_4d(dst + hf * L::kAHalf, &tm_q, &a_full[buf], hf * 64, tc.hk * G, tc.t0,
-                        tc.b);
-          a_loads = tc.u + 1;
-        }
+      while (tc.valid && ok) {
         const int st = g_tma % kHtStages;
-        if (g_tma >= kHtStages &&
-            !mbar_wait(&stage_free[st], ((g_tma / kHtStages) + 1) & 1))
-          return false;
+        if (*abort_flag ||
+            (g_tma >= kHtStages && !mbar_wait(&stage_free[st], ((g_tma / kHtStages) + 1) & 1))) {
+          ok = false;
+          break;
+        }
         uint8_t* dst = smem + L::kB + st * L::kStage;
         const int j0 = geo.n_init + tc.i * kHtN;
         mbar_arrive_expect_tx(&full[st], L::kStage);
+        // per 64-dim half: hi, mid, lo (B operand rows 0-63, 64-127, 128-191)
 #pragma unroll
         for (int hf = 0; hf < D / 64; ++hf) {
-          tma_load_4d(dst + hf * L::kHalfB, &tm_hi, &full[st], hf * 64, tc.hk, j0, tc.b);
-          tma_load_4d(dst + L::kPartB + hf * L::kHalfB, &tm_mid, &full[st], hf * 64, tc.hk, j0,
-                      tc.b);
-          tma_load_4d(dst + 2 * L::kPartB + hf * L::kHalfB, &tm_lo, &full[st], hf * 64, tc.hk,
-                      j0, tc.b);
+          uint8_t* h3 = dst + hf * L::kHalf3;
+          tma_load_4d(h3, &tm_hi, &full[st], hf * 64, tc.hk, j0, tc.b);
+          tma_load_4d(h3 + L::kHalfB, &tm_mid, &full[st], hf * 64, tc.hk, j0, tc.b);
+          tma_load_4d(h3 + 2 * L::kHalfB, &tm_lo, &full[st], hf * 64, tc.hk, j0, tc.b);
         }
         ++g_tma;
         geo.next(tc);
-        return true;
-      };
+      }
+      if (!ok) *abort_flag = 1;
+      // every copy landed before the CTA releases its shared memory
+      for (int x = g_tma > kHtStages ? g_tma - kHtStages : 0; x < g_tma; ++x)
+        mbar_wait(&full[x % kHtStages], (x / kHtStages) & 1);
+    }
+  } else if (warp == kHtConsumers) {
+    // ================= issuer: the score MMAs of each tile
+    if ((tid & 31) == 0) {
+      HtCursor mc;
+      geo.begin(mc);
+      int g_mma = 0;
+      bool ok = true;
       auto desc = [&](uint32_t base, int kk, int half_bytes) {
         return umma_desc_sw128(base + (kk >> 2) * half_bytes + (kk & 3) * 32, 16, 1024);
       };
-      for (int x = 0; x < kHtStages - 1 && tc.valid && ok; ++x) ok = tma_step();
       while (mc.valid && ok) {
-        if (tc.valid) ok = tma_step();
-        if (!ok) break;
         const int buf = mc.u & 1, st = g_mma % kHtStages, ab = g_mma % kHtAcc;
-        if (mc.pass == 0 && mc.i == 0) ok = mbar_wait(&a_full[buf], (mc.u >> 1) & 1);
+        if (mc.pass == 0 && mc.i == 0) ok = !*abort_flag && mbar_wait(&a_full[buf], (mc.u >> 1) & 1);
         ok = ok && mbar_wait(&full[st], (g_mma / kHtStages) & 1) &&
              (g_mma < kHtAcc || mbar_wait(&acc_free[ab], ((g_mma / kHtAcc) + 1) & 1));
         if (!ok) break;
         tc_fence_after();
-        const uint32_t a = smem_u32(smem + L::kAoff + buf * L::kA);
+        const uint32_t a = tmem + buf * kAcols;  // A in TMEM: k-step kk at columns 8 kk
         const uint32_t bh = smem_u32(smem + L::kB + st * L::kStage);
-        const uint32_t d = tD + kHtN * ab;
-        // smallest part first: lo, mid, hi
+        const uint32_t d = tD + 3 * kHtN * ab;
 #pragma unroll
         for (int kk = 0; kk < kK; ++kk)
-          tc_mma_ss(d, desc(a, kk, L::kAHalf), desc(bh + 2 * L::kPartB, kk, L::kHalfB), kId,
-                    kk > 0 ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < kK; ++kk)
-          tc_mma_ss(d, desc(a, kk, L::kAHalf), desc(bh + L::kPartB, kk, L::kHalfB), kId, 1u);
-#pragma unroll
-        for (int kk = 0; kk < kK; ++kk)
-          tc_mma_ss(d, desc(a, kk, L::kAHalf), desc(bh, kk, L::kHalfB), kId, 1u);
+          tc_mma_ts(d, a + 8 * kk, desc(bh, kk, L::kHalf3), kId, kk > 0 ? 1u : 0u);
         tc_commit(&mma_done[ab]);
         tc_commit(&stage_free[st]);
         const bool last_of_item = mc.pass == 1 && mc.i == mc.ntiles - 1;
@@ -255,25 +272,64 @@ select_hsm_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         geo.next(mc);
       }
       if (!ok) *abort_flag = 1;
-      // wind down: every MMA complete and every copy landed before TMEM is freed
+      // wind down: every MMA complete before TMEM is freed
       tc_commit(drain);
       mbar_wait(drain, 0);
-      for (int x = g_tma > kHtStages ? g_tma - kHtStages : 0; x < g_tma; ++x)
-        mbar_wait(&full[x % kHtStages], (x / kHtStages) & 1);
-      for (int x = a_loads > 2 ? a_loads - 2 : 0; x < a_loads; ++x)
-        mbar_wait(&a_full[x & 1], (x >> 1) & 1);
+    }
+  } else if (warp > kHtConsumers) {
+    // ================= producers (warps 9-12): lane l's query-head row of each item into its TMEM lane
+    const int l = 32 * (warp & 3) + (tid & 31);  // this warp's TMEM lane quadrant is warp % 4
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    const int rrow = l / G, head = l % G;
+    HtCursor c;
+    geo.begin(c);
+    while (c.valid) {
+      const int buf = c.u & 1;
+      if (*abort_flag || (c.u >= 2 && !mbar_wait(&a_free[buf], ((c.u - 2) >> 1) & 1))) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const int t = c.t0 + rrow;
+      const bool in = t < geo.Tq;
+      const __nv_bfloat16* qp = q + c.b * sq.b + (int64_t)(in ? t : 0) * sq.t +
+                                (int64_t)(c.hk * G + head) * sq.h;
+#pragma unroll
+      for (int hf = 0; hf < D / 64; ++hf) {
+        uint32_t w[32];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+          const uint4 v = in ? __ldg(reinterpret_cast<const uint4*>(qp + hf * 64 + 8 * x))
+                             : make_uint4(0u, 0u, 0u, 0u);
+          w[4 * x] = v.x;
+          w[4 * x + 1] = v.y;
+          w[4 * x + 2] = v.z;
+          w[4 * x + 3] = v.w;
+        }
+        tc_st32(tmem + buf * kAcols + 32 * hf + lane_off, w);
+      }
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(&a_full[buf]);
+      // the next scoring item
+      c.pass = 1;
+      c.i = c.ntiles - 1;
+      geo.next(c);
     }
   } else {
-    // ================= consumers: thread l = (row l / G, head l % G) of the item
-    const int l = tid;
+    // ================= consumers: thread (l, half) with l = (row l / G, head l % G)
+    const int quad = warp & 3, half = warp >> 2;
+    const int l = 32 * quad + (tid & 31);
     const int rrow = l / G, gl = l % G;  // row within the item, lane within the row's group
-    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
-    constexpr int per = kHtN / G;        // candidates each lane stores per tile
+    const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
+    constexpr int per = kHtHalf / G;     // candidates each lane stores per tile half
+    float2* comb = reinterpret_cast<float2*>(smem + L::kComb);  // [parity][half][lane]
     HtCursor c;
     geo.begin(c);
     int g = 0;
-    float m = -INFINITY, lsum = 0.f, inv_l = 0.f;
-    while (c.valid) {
+    float m = -INFINITY, lsum = 0.f, mp = -INFINITY;
+    bool ok = true;
+    while (c.valid && ok) {
       const int t = c.t0 + rrow;                      // query row (local)
       const bool live = t < geo.r1;
       const int cblk = (geo.qpos0 + t) / kSelBlk;
@@ -285,61 +341,87 @@ select_hsm_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       const int ab = g % kHtAcc;
       const bool landed = !*abort_flag && mbar_wait(&mma_done[ab], (g / kHtAcc) & 1);
       if (__any_sync(0xffffffffu, !landed)) {
-        *abort_flag = 1;
+        ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t sv[2][32];
-      tc_ld32(tD + kHtN * ab + lane_off, sv[0]);
-      tc_ld32(tD + kHtN * ab + 32 + lane_off, sv[1]);
+      uint32_t sh[kHtHalf], sm[kHtHalf], sl[kHtHalf];  // q.hi, q.mid, q.lo
+      const uint32_t col = tD + 3 * kHtN * ab + kHtHalf * half + lane_off;
+      tc_ld32(col, sh);
+      tc_ld32(col + kHtN, sm);
+      tc_ld32(col + 2 * kHtN, sl);
       tc_wait_ld();
       tc_fence_before();
       __syncwarp();
       if ((tid & 31) == 0) mbar_arrive(&acc_free[ab]);
-      const int j0 = geo.n_init + c.i * kHtN;
-      float s[kHtN];
+      const int j0 = geo.n_init + c.i * kHtN + kHtHalf * half;  // this half's first candidate
+      float s[kHtHalf];  // scores, log2 domain (-inf: not a candidate of the row)
 #pragma unroll
-      for (int x = 0; x < kHtN; ++x) {
-        const bool in = j0 + x <= jmax;
-        s[x] = in ? __uint_as_float(sv[x >> 5][x & 31]) * scale_log2 : -INFINITY;
+      for (int x = 0; x < kHtHalf; ++x)
+        s[x] = (__uint_as_float(sl[x]) + __uint_as_float(sm[x])) + __uint_as_float(sh[x]);
+      if (j0 + kHtHalf - 1 > jmax) {  // the row's candidates end inside this half tile
+#pragma unroll
+        for (int x = 0; x < kHtHalf; ++x) s[x] = j0 + x <= jmax ? s[x] : -INFINITY;
       }
       if (c.pass == 0) {
-        float mt = -INFINITY;
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int x = 0; x < kHtN; ++x) mt = fmaxf(mt, s[x]);
+        for (int x = 0; x < kHtHalf; ++x) mx[x & 3] = fmaxf(mx[x & 3], s[x]);
+        const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
         if (mt > -INFINITY) {
           const float mn = fmaxf(m, mt);
-          float acc = 0.f;
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int x = 0; x < kHtN; ++x) acc += exp2f(s[x] - mn);  // exp2(-inf) = 0
-          lsum = lsum * exp2f(m - mn) + acc;                       // 0 on the row's first tile
+          for (int x = 0; x < kHtHalf; ++x) acc[x & 3] += ht_exp2(s[x] - mn);  // exp2(-inf) = 0
+          lsum = lsum * ht_exp2(m - mn) + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
           m = mn;
         }
-        if (c.i == c.ntiles - 1) inv_l = lsum > 0.f ? 1.0f / lsum : 0.f;
+        if (c.i == c.ntiles - 1) {
+          // merge with the other half's (max, sum) of the same lane
+          const int par = c.u & 1;
+          comb[(par * 2 + half) * kHtLanes + l] = make_float2(m, lsum);
+          mbar_arrive(&pair[quad * 2 + par]);
+          const bool merged = mbar_wait(&pair[quad * 2 + par], (c.u >> 1) & 1);
+          if (__any_sync(0xffffffffu, !merged)) {  // leave the loop as a whole warp
+            ok = false;
+            break;
+          }
+          const float2 o = comb[(par * 2 + (half ^ 1)) * kHtLanes + l];
+          const float ma = fmaxf(m, o.x);
+          const float la = ma == -INFINITY ? 0.f : lsum * ht_exp2(m - ma) + o.y * ht_exp2(o.x - ma);
+          // p = exp2(s - ma) / la = exp2(s - mp); -inf marks a row without candidates
+          mp = la > 0.f ? ma + log2f(la) : -INFINITY;
+        }
       } else {
-        // p (0 for candidates outside the row, also when the row has none: m = -inf)
+        // p (exp2(-inf) = 0 for candidates outside the row; all 0 for a row without any)
+        if (mp == -INFINITY) {
 #pragma unroll
-        for (int x = 0; x < kHtN; ++x) s[x] = s[x] == -INFINITY ? 0.f : exp2f(s[x] - m) * inv_l;
-        ht_reduce_scatter<G, kHtN>(s, l);
+          for (int x = 0; x < kHtHalf; ++x) s[x] = 0.f;
+        } else {
+#pragma unroll
+          for (int x = 0; x < kHtHalf; ++x) s[x] = ht_exp2(s[x] - mp);
+        }
+        ht_reduce_scatter<G, kHtHalf>(s, l);
         // lane gl of the row holds candidates j0 + gl * per .. j0 + gl * per + per - 1
         if (live) {
           float* srow = scores + (((int64_t)c.b * geo.Hkv + c.hk) * rows_pass + (t - geo.r0)) *
                                      (int64_t)geo.nb;
           const int jb = j0 + gl * per;
 #pragma unroll
-          for (int x = 0; x < kHtN; ++x)
-            if (x < per && jb + x <= jmax) srow[jb + x - geo.n_init] = s[x];
+          for (int x = 0; x < per; ++x)
+            if (jb + x <= jmax) srow[jb + x - geo.n_init] = s[x];
         }
       }
       ++g;
       geo.next(c);
     }
+    if (!ok) *abort_flag = 1;
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tc_dealloc(*tmem_slot, kHtAcc * kHtN);
+    tc_dealloc(tmem, kCols);
   }
 }
 
