@@ -201,12 +201,15 @@ sala_status sala_sparse_select(const void *q, const void *k, int B, int T, int H
  * Everything else (candidates, top `topk` with ties -> smaller j, init blocks,
  * local window, sorted, -1 padded) is as in sala_sparse_select.  Each head's p sums
  * to 1, so a row's scores sum to G; with G = 1 the choice equals sala_sparse_select's.
- * fp32 arithmetic (expf, IEEE division): a decision between two scores closer than
- * about 1e-5 of their size may differ from exact arithmetic.
+ * fp32-equivalent arithmetic (dot products on tensor cores from an exact three-part
+ * bf16 split of the fp32 block means, fp32 exponentials of about 2^-22 relative error):
+ * a decision between two scores closer than about 1e-5 of their size may differ from
+ * exact arithmetic.
  *
  *   arguments, layouts and ownership as sala_sparse_select; ws of
- *   >= sala_sparse_select_head_softmax_workspace() bytes (block means and a score
- *   scratch of at most 1 GiB); G = Hq / Hkv must be 1, 2, 4, 8, 16 or 32.
+ *   >= sala_sparse_select_head_softmax_workspace() bytes (block means with their three
+ *   bf16 parts and a score scratch of at most 1 GiB); G = Hq / Hkv must be 1, 2, 4, 8,
+ *   16 or 32.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
  */
 size_t sala_sparse_select_head_softmax_workspace(int B, int T, int Hq, int Hkv, int D,
