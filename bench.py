@@ -38,7 +38,7 @@ if ROOT not in sys.path:
 
 METRIC = "Hybrid-attn prefill tokens/s at 128K (lightning+sparse); % of roofline"
 # DRAM read + write bytes per launch of a kernel, by T (see the comment where it is used)
-NCU_TRAFFIC = {131072: {"attn": 8322618624 + 1098238720}}
+NCU_TRAFFIC = {131072: {"attn": 8369097472 + 1124515072}}
 B, H, HKV, D = 1, 32, 2, 128
 CHUNK, BLOCK, TOPK, N_INIT, N_LOCAL = 128, 64, 64, 1, 2
 SPARSE_LAYERS = (2, 6)
