@@ -50,8 +50,10 @@ typedef enum {
     SALA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
     SALA_ERR_TIMEOUT = 4,      /* a device-side bounded wait ran out */
     SALA_ERR_WORKSPACE = 5,    /* workspace missing or smaller than required */
-    SALA_ERR_RANGE = 6         /* a non-finite value reached a result on the device, or a
+    SALA_ERR_RANGE = 6,        /* a non-finite value reached a result on the device, or a
                                   decode position lies outside the cache */
+    SALA_ERR_BOUNDS = 7        /* debug builds only (SALA_DEBUG): a device-side index
+                                  check failed and its access was skipped */
 } sala_status;
 
 typedef enum { SALA_F32 = 0, SALA_BF16 = 1 } sala_dtype;
@@ -431,11 +433,24 @@ sala_status sala_selftest_wait_timeout(long long cycles, void *stream);
 
 /*
  * Synchronise `stream`, then read and clear the device error word of the
- * current device.  Returns SALA_OK, SALA_ERR_RANGE or SALA_ERR_TIMEOUT (the
- * first condition raised since the last call), or SALA_ERR_CUDA if the
- * synchronisation itself failed.
+ * current device.  Returns SALA_OK, SALA_ERR_RANGE, SALA_ERR_TIMEOUT or (debug
+ * builds) SALA_ERR_BOUNDS (the first condition raised since the last call), or
+ * SALA_ERR_CUDA if the synchronisation itself failed.
  */
 sala_status sala_get_device_error(void *stream);
+
+/*
+ * Device index checks.  The library built with SALA_DEBUG defined (libsala_debug.so;
+ * the same kernels and arithmetic) checks, before the access, the indices that data
+ * or arithmetic select: every block index an attention row reads (in [-1, key
+ * blocks)), every per-row selection buffer slot and output position, every score
+ * scratch slot and every decode block index.  A failed check skips its access and
+ * raises SALA_ERR_BOUNDS in the device error word instead of faulting.
+ * Returns the source line of the first failed check since the last call and clears it
+ * (0: none) after synchronising the current device; -1 in the release library, which
+ * compiles the checks out.  Errors: none (a failed synchronisation reads as 0).
+ */
+int sala_debug_bounds_line(void);
 
 #ifdef __cplusplus
 }

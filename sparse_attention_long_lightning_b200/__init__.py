@@ -20,13 +20,16 @@ __all__ = [
     "lightning_prefill_noalloc", "lightning_projection", "lightning_prefill_prepared",
     "lightning_decode", "sparse_select", "sparse_select_workspace", "sparse_select_head_softmax_workspace", "sparse_attn",
     "sparse_attn_workspace",
-    "get_device_error", "selftest_wait_timeout", "sparse_decode", "sparse_decode_workspace",
+    "get_device_error", "debug_bounds_line", "selftest_wait_timeout", "sparse_decode", "sparse_decode_workspace",
     "sparse_block_means", "lightning_state", "state_prefix_sum", "status_string", "version",
     "set_tracing",
     "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsala.so")
+# SALA_LIBRARY=debug loads libsala_debug.so (the same kernels with device index checks,
+# built with SALA_DEBUG); any other non-empty value is a path to the library
+LIB_DEBUG_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsala_debug.so")
 SALA_F32, SALA_BF16 = 0, 1
 _lib = None
 
@@ -80,7 +83,8 @@ def load_library(path: Optional[str] = None):
     global _lib
     if _lib is not None:
         return _lib
-    p = path or LIB_PATH
+    env = os.environ.get("SALA_LIBRARY", "")
+    p = path or (LIB_DEBUG_PATH if env == "debug" else env) or LIB_PATH
     if not os.path.exists(p):
         raise OSError(f"libsala.so not found at {p}; build it with "
                       "`python -m sparse_attention_long_lightning_b200.build`")
@@ -144,6 +148,8 @@ def load_library(path: Optional[str] = None):
     lib.sala_sparse_attn_rows.restype = i
     lib.sala_get_device_error.argtypes = [vp]
     lib.sala_get_device_error.restype = i
+    lib.sala_debug_bounds_line.argtypes = []
+    lib.sala_debug_bounds_line.restype = i
     lib.sala_selftest_wait_timeout.argtypes = [ctypes.c_longlong, vp]
     lib.sala_selftest_wait_timeout.restype = i
     _lib = _Lib(lib)
@@ -546,3 +552,9 @@ def selftest_wait_timeout(cycles=20_000_000, stream=None):
 def get_device_error(stream=None) -> int:
     """Synchronise the stream and read/clear the device error word (0 = none)."""
     return int(load_library().sala_get_device_error(_stream(stream)))
+
+
+def debug_bounds_line() -> int:
+    """Source line of the first failed device index check since the last call (0: none;
+    -1: the release library, which has no checks).  Clears it."""
+    return int(load_library().sala_debug_bounds_line())

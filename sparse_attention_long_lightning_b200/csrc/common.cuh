@@ -18,6 +18,22 @@ __device__ __forceinline__ void raise_device_error(int code) {
   atomicCAS(&g_device_error, 0, code);
 }
 
+// SALA_IN_BOUNDS(cond): true when cond holds.  Built with SALA_DEBUG, a false cond
+// records its source line (the first since the last read), raises SALA_ERR_BOUNDS and
+// yields false, so the caller skips the access; otherwise the check compiles to true and
+// cond is not evaluated.
+#ifdef SALA_DEBUG
+__device__ int g_bounds_line;
+__device__ __noinline__ bool bounds_failed(int line) {
+  atomicCAS(&g_bounds_line, 0, line);
+  raise_device_error(SALA_ERR_BOUNDS);
+  return false;
+}
+#define SALA_IN_BOUNDS(cond) ((cond) ? true : ::sala::bounds_failed(__LINE__))
+#else
+#define SALA_IN_BOUNDS(cond) true
+#endif
+
 template <typename T>
 struct Elem;
 template <>

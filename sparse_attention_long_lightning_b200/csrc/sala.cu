@@ -179,11 +179,18 @@ const char* sala_status_string(sala_status s) {
     case SALA_ERR_TIMEOUT: return "SALA_ERR_TIMEOUT";
     case SALA_ERR_WORKSPACE: return "SALA_ERR_WORKSPACE";
     case SALA_ERR_RANGE: return "SALA_ERR_RANGE";
+    case SALA_ERR_BOUNDS: return "SALA_ERR_BOUNDS";
   }
   return "SALA_ERR_UNKNOWN";
 }
 
-const char* sala_version(void) { return "sala-b200 0.1 (sm_100a)"; }
+const char* sala_version(void) {
+#ifdef SALA_DEBUG
+  return "sala-b200 0.1 (sm_100a, SALA_DEBUG index checks)";
+#else
+  return "sala-b200 0.1 (sm_100a)";
+#endif
+}
 
 // ------------------------------------------------------------------ Lightning prefill
 size_t sala_lightning_prefill_workspace(int B, int T, int H, int D, int chunk, sala_dtype dt) {
@@ -822,6 +829,7 @@ static sala_status sparse_attn_impl(const void* q, const void* k, const void* v,
   p.scale_log2 = sc * 1.4426950408889634f;
   p.rows = (int64_t)B * Hkv * T;
   p.qpos0 = qpos0;
+  p.nkb = (Tk + kSaBlk - 1) / kSaBlk;
   cudaStream_t st = as_stream(stream);
   const int64_t want = num_sms();
   const unsigned grid = (unsigned)std::min<int64_t>(want, p.rows);
@@ -1157,6 +1165,24 @@ sala_status sala_selftest_wait_timeout(long long cycles, void* stream) {
 }
 
 // ------------------------------------------------------------------ device error word
+int sala_debug_bounds_line(void) {
+#ifdef SALA_DEBUG
+  if (cudaDeviceSynchronize() != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  int line = 0;
+  if (cudaMemcpyFromSymbol(&line, g_bounds_line, sizeof(int)) != cudaSuccess) return 0;
+  if (line != 0) {
+    const int zero = 0;
+    (void)cudaMemcpyToSymbol(g_bounds_line, &zero, sizeof(int));
+  }
+  return line;
+#else
+  return -1;
+#endif
+}
+
 sala_status sala_get_device_error(void* stream) {
   if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) {
     (void)cudaGetLastError();

@@ -61,11 +61,14 @@ struct SaParams {
   float scale_log2;  // softmax scale * log2(e)
   int64_t rows;      // B * Hkv * T
   int64_t qpos0;     // sequence position of query row 0 (row t is position qpos0 + t)
+  int nkb;           // key blocks, ceil(Tk / 64): block indices lie in [-1, nkb)
 };
 
-// A selected block j takes part in row t iff j >= 0 and its first key is <= t.
-__device__ __forceinline__ bool sa_block_live(int j, int64_t t) {
-  return j >= 0 && (int64_t)j * kSaBlk <= t;
+// A selected block j takes part in row t iff j >= 0 and its first key is <= t.  (Debug
+// builds first check j against [-1, nkb): an index past the keys can only come from a
+// corrupted selection; the release rule already skips it as not live.)
+__device__ __forceinline__ bool sa_block_live(int j, int64_t t, int nkb) {
+  return SALA_IN_BOUNDS(j >= -1 && j < nkb) && j >= 0 && (int64_t)j * kSaBlk <= t;
 }
 
 // The first row >= r, in r's class modulo `stride`, of a (sequence, KV head) that this
@@ -141,7 +144,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const int32_t* ir = p.idx + r * p.n_sel;
         for (int e = 0; e < p.n_sel; ++e) {
           const int j = __ldg(ir + e);
-          if (!sa_block_live(j, tp)) continue;
+          if (!sa_block_live(j, tp, p.nkb)) continue;
           const int s = it % NS;
           if (*abort_flag || !mbar_wait(&empty[s], ((it / NS) & 1) ^ 1)) { ok = false; break; }
           uint8_t* st = stages + size_t(s) * L::kStage;
@@ -194,7 +197,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k,
       const int32_t* ir = p.idx + r * p.n_sel;
       for (int e0 = 0; e0 < p.n_sel; e0 += 32) {
         const int e = e0 + lane;
-        const bool live = e < p.n_sel && sa_block_live(__ldg(ir + e), tp);
+        const bool live = e < p.n_sel && sa_block_live(__ldg(ir + e), tp, p.nkb);
         nblk += __popc(__ballot_sync(0xffffffffu, live));
       }
     }

@@ -316,6 +316,7 @@ __global__ void __launch_bounds__(kSdAttnWarps * 32) sd_attn_kernel(const SdPara
   }
   auto issue = [&](int e) {  // K and V of chosen block e into ring slot (e - sb0) % S
     const int j = __ldg(ir + e);
+    if (!SALA_IN_BOUNDS(j >= 0 && j <= c)) return;  // a chosen block lies in [0, c]
     const uint32_t kb = smem_u32(smem + ((e - sb0) % kSdStages) * L::kBuf), vb = kb + L::kTile;
     const __nv_bfloat16* ks = p.k + b * p.sk.b + (int64_t)j * kSdBlk * p.sk.t + hk * p.sk.h;
     const __nv_bfloat16* vs = p.v + b * p.sv.b + (int64_t)j * kSdBlk * p.sv.t + hk * p.sv.h;

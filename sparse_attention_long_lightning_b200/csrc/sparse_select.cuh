@@ -156,7 +156,8 @@ block_scores_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
         const int j = jt0 + tx * 4 + w;
-        if (j <= jmax && j <= j_hi) srow[j - n_init] = acc[u][w] * inv_sqrt_d;
+        if (j <= jmax && j <= j_hi && SALA_IN_BOUNDS(j - n_init < nb && t - r_begin < rows_pass))
+          srow[j - n_init] = acc[u][w] * inv_sqrt_d;
       }
     }
   }
@@ -261,6 +262,7 @@ topk_select_kernel(const float* __restrict__ scores, int32_t* __restrict__ idx, 
   }
   // local window
   const int lo = max(n_init, c - n_local + 1);
+  if (!SALA_IN_BOUNDS(pos + max(0, c - lo + 1) <= n_sel)) return;
   for (int j = lo + lane; j <= c; j += 32) out[pos + (j - lo)] = j;
   pos += (c >= lo) ? c - lo + 1 : 0;
   for (int e = pos + lane; e < n_sel; e += 32) out[e] = -1;

@@ -409,7 +409,9 @@ select_hsm_tc_kernel(const __nv_bfloat16* __restrict__ q, sala_strides sq,
           const int jb = j0 + gl * per;
 #pragma unroll
           for (int x = 0; x < per; ++x)
-            if (jb + x <= jmax) srow[jb + x - geo.n_init] = s[x];
+            if (jb + x <= jmax &&
+                SALA_IN_BOUNDS(jb + x - geo.n_init < geo.nb && t - geo.r0 < rows_pass))
+              srow[jb + x - geo.n_init] = s[x];
         }
       }
       ++g;

@@ -488,7 +488,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constan
             const int j0 = n_init + i * kStcN + kStcSub * sub;
             auto append = [&](int cc, bool in_range) {  // predicated, no branch
               const float sc = __uint_as_float(sv[sub][cc]);
-              const bool p = in_range & (sc > thr);
+              const bool p = (in_range & (sc > thr)) && SALA_IN_BOUNDS(cnt < kStcCap);
               sts_f32_if(p, sA + cnt * (kStcRows * 4), sc);
               sts_u16_if(p, jA + cnt * (kStcRows * 2), (uint32_t)(j0 + cc));
               cnt += p ? 1 : 0;
@@ -519,7 +519,9 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constan
       if (buffered && cnt > topk)
         cnt = stc_compact(sA, jA, hA, sh16, cnt, topk, smin, smax, topk, &thr);  // exact
       // ---- this thread's row: init blocks, the kept candidates in block order, local window
-      if (live) {
+      if (live && SALA_IN_BOUNDS(min(n_init, c + 1) + (buffered ? cnt : max(n_row, 0)) +
+                                     max(0, c - max(n_init, c - n_local + 1) + 1) <=
+                                 n_sel)) {
         int32_t* out = idx + (((int64_t)it.b * Hkv + it.hk) * T + t) * n_sel;
         const int n_first = min(n_init, c + 1);
         for (int e = 0; e < n_first; ++e) out[e] = e;

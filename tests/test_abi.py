@@ -42,7 +42,20 @@ def test_status_strings(lib):
     assert sala.status_string(0) == "SALA_OK"
     assert sala.status_string(1) == "SALA_ERR_INVALID_ARG"
     assert sala.status_string(6) == "SALA_ERR_RANGE"
-    assert "sm_100a" in sala.version()
+    assert sala.status_string(7) == "SALA_ERR_BOUNDS"
+    assert "sm_100a" in sala.version() and "SALA_DEBUG" not in sala.version()
+    # the release library has no device index checks
+    assert sala.debug_bounds_line() == -1
+
+
+def test_debug_library_exports_every_declared_symbol():
+    """libsala_debug.so (SALA_DEBUG: device index checks) is the same ABI."""
+    path = sala_build.build(debug=True)
+    dbg = ctypes.CDLL(path)
+    for name in declared_symbols():
+        assert hasattr(dbg, name), name
+    dbg.sala_version.restype = ctypes.c_char_p
+    assert b"SALA_DEBUG" in dbg.sala_version()
 
 
 Z = sala.SalaStrides(0, 0, 0)
