@@ -390,8 +390,8 @@ sala_status sala_lightning_prefill_prepared(const void *qh, const void *kh, cons
                                             size_t workspace_bytes, void *stream);
 
 /*
- * Lightning prefill that allocates nothing (no counterpart in the paper: this is
- * a library convenience).  Some callers cannot hand the library a workspace:
+ * Lightning prefill that allocates nothing (not part of the method: a library
+ * convenience).  Some callers cannot hand the library a workspace:
  * code embedded in a host framework that owns all device memory and offers its
  * plugins no allocator, or a serving loop whose memory pool is frozen after
  * start-up and must not call cudaMalloc on the hot path.  This entry point takes
@@ -406,7 +406,7 @@ sala_status sala_lightning_prefill_prepared(const void *qh, const void *kh, cons
  * dtype/head_dim/chunk combinations need no scratch and behave exactly like
  * sala_lightning_prefill.
  * Set-up: the first call on each device looks up the device address of the
- * scratch array (so make that first call before any stream capture).
+ * scratch array.
  * Concurrency: every call on a device shares the one scratch array and leaves
  * its contents behind; calls that can overlap on the GPU (different streams,
  * or several threads) race on it and must be serialised by the caller.
