@@ -107,3 +107,58 @@ def test_sparse_decode_and_block_means_writes_stay_inside():
     torch.cuda.synchronize()
     assert sala.get_device_error() == 0
     assert kbar.intact() and out.intact() and idx.intact() and ws.intact()
+
+
+@pytest.mark.parametrize("score", ["group_sum", "head_softmax"])
+def test_row_window_calls_write_stay_inside(score):
+    """Selection and attention over a window of query rows (row-window entry points)."""
+    T, Hq, Hkv, D, topk = 64 * 40 + 29, 16, 2, 128, 16
+    a, b = 64 * 11 + 5, 64 * 31 + 3
+    s = inputs.sparse_inputs(1, T, Hq, Hkv, D, seed=61, device=DEV, gate=True)
+    n_sel = 1 + topk + 2
+    idx = Guarded((1, Hkv, b - a, n_sel), torch.int32)
+    ws = _ws(sala.sparse_select_rows_workspace(1, b - a, T, Hq, Hkv, D, 64, topk, score))
+    sala.sparse_select(s.q[:, a:b], s.k, topk=topk, out=idx.view, workspace=ws.view,
+                       score=score, q_pos0=a)
+    out = Guarded((1, b - a, Hq, D), torch.bfloat16)
+    wsa = _ws(sala.sparse_attn_workspace(1, T, Hkv, D))
+    sala.sparse_attn(s.q[:, a:b], s.k, s.v, idx.view, s.g[:, a:b], out=out.view,
+                     workspace=wsa.view, q_pos0=a)
+    torch.cuda.synchronize()
+    assert sala.get_device_error() == 0
+    assert idx.intact() and ws.intact() and out.intact() and wsa.intact()
+
+
+def test_projection_and_prepared_prefill_writes_stay_inside():
+    """The fused projection's four outputs, then the prepared prefill's output, state and
+    workspace, on ragged rows (2 x 301 tokens: a partial last tile)."""
+    B, T, hidden, H, D = 2, 301, 256, 2, 128
+    gen = inputs.generator(62, DEV)
+    x = inputs.randn((B, T, hidden), gen, device=DEV)
+    w = inputs.randn((4 * H * D, hidden), gen, device=DEV, scale=hidden ** -0.5)
+    outs = (Guarded((B, T, H, D), torch.float16), Guarded((B, T, H, D), torch.float16),
+            Guarded((B, T, H, D), torch.bfloat16), Guarded((B, T, H, D), torch.float16))
+    qh, kh, v, gate = sala.lightning_projection(x, w, heads=H, head_dim=D, pos0=5,
+                                                out=tuple(o.view for o in outs))
+    state = Guarded((B, H, D, D), torch.float32, init=torch.zeros((B, H, D, D)))
+    y = Guarded((B, T, H, D), torch.bfloat16)
+    ws = _ws(sala.lightning_prefill_workspace(B, T, H, D, 128))
+    sala.lightning_prefill_prepared(qh, kh, v, gate, state.view, out=y.view, workspace=ws.view)
+    torch.cuda.synchronize()
+    assert sala.get_device_error() == 0
+    assert all(o.intact() for o in outs) and state.intact() and y.intact() and ws.intact()
+
+
+def test_state_only_and_noalloc_writes_stay_inside():
+    """The state-only pass (sequence-parallel Lightning) and the allocation-free prefill."""
+    T, H, D = 128 * 3 + 77, 4, 128
+    x = inputs.lightning_inputs(1, T, H, D, seed=63, device=DEV)
+    state = Guarded((1, H, D, D), torch.float32, init=torch.zeros((1, H, D, D)))
+    ws = _ws(sala.lightning_prefill_workspace(1, T, H, D, 128))
+    sala.lightning_state(x.k, x.v, state.view, workspace=ws.view, pos0=128)
+    st2 = Guarded((1, H, D, D), torch.float32, init=torch.zeros((1, H, D, D)))
+    out = Guarded((1, T, H, D), torch.bfloat16)
+    sala.lightning_prefill_noalloc(x.q, x.k, x.v, x.g, st2.view, out.view)
+    torch.cuda.synchronize()
+    assert sala.get_device_error() == 0
+    assert state.intact() and ws.intact() and st2.intact() and out.intact()
