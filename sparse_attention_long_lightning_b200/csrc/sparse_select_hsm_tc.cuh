@@ -25,17 +25,17 @@
 // their heads' p by a butterfly reduce-scatter (after which lane g of the row's group
 // holds the sums of candidates g * 64/G .. (g + 1) * 64/G - 1 of the tile) and store
 // them, coalesced, into the scratch row.
-//   producers (warps 9-12): thread l loads lane l's query-head row of the next item
+//   producers (warps 17-20): thread l loads lane l's query-head row of the next item
 //     and stores it into its TMEM lane (two A buffers), overlapping the current item;
-//   copier (warp 13, one thread): TMA of the block-mean tiles (4-stage ring, hi / mid /
+//   copier (warp 21, one thread): TMA of the block-mean tiles (4-stage ring, hi / mid /
 //     lo per 64-dim half), running ahead by the ring depth;
-//   issuer (warp 8, one thread): the MMAs of each tile into one of 2 TMEM score buffers;
-//   consumers (warps 0-7): warps w and w + 4 read TMEM lane quadrant w, each one half
-//     (32 candidates) of every tile: tcgen05.ld, buffer release (per-warp arrival), then
-//     the pass's arithmetic; at the end of pass 1 the two threads of a lane merge their
-//     halves' (max, sum) through shared memory (a bounded mbarrier wait, per item
-//     parity), so pass 2 normalises with the row's full sum.  Two warps per scheduler
-//     hide each other's latency.
+//   issuer (warp 16, one thread): the MMAs of each tile into one of 2 TMEM score buffers;
+//   consumers (warps 0-15): warps w, w + 4, w + 8, w + 12 read TMEM lane quadrant w % 4,
+//     each one quarter (16 candidates) of every tile: tcgen05.ld, buffer release
+//     (per-warp arrival), then the pass's arithmetic; at the end of pass 1 the four
+//     threads of a lane merge their parts' (max, sum) through shared memory in a fixed
+//     order (a bounded mbarrier wait, per item parity), so pass 2 normalises with the
+//     row's full sum.  Four warps per scheduler hide each other's latency.
 // All waits are bounded: a wait that runs out raises SALA_ERR_TIMEOUT, and the kernel
 // drains its copies and MMAs before it frees TMEM and returns.
 #pragma once
@@ -46,10 +46,10 @@ namespace sala {
 
 constexpr int kHtLanes = 128;   // (query row, head) pairs per item = TMEM lanes
 constexpr int kHtN = 64;        // candidates per tile
-constexpr int kHtHalf = kHtN / 2;  // candidates of a tile per consumer thread
+constexpr int kHtPart = kHtN / 4;  // candidates of a tile per consumer thread
 constexpr int kHtStages = 4;    // block-mean tile ring
 constexpr int kHtAcc = 2;       // TMEM score buffers (3 x kHtN columns each)
-constexpr int kHtConsumers = 8; // two warps per TMEM lane quadrant (one per tile half)
+constexpr int kHtConsumers = 16; // four warps per TMEM lane quadrant (16 columns each)
 constexpr int kHtThreads = kHtConsumers * 32 + 32 + kHtLanes + 32;  // consumers, issuer,
                                                                     // producers, copier
 constexpr int kHtCopier = kHtConsumers + 1 + kHtLanes / 32;        // the copier's warp
@@ -69,12 +69,12 @@ struct HtSmem {
   static constexpr size_t kB = 0;                                    // [stages]
   static constexpr size_t kBars = kB + kHtStages * size_t(kStage);
   // full[S], stage_free[S], mma_done[A], acc_free[A], a_full[2], a_free[2], drain,
-  // pair[4 quadrants][2 item parities]
+  // merged[4 quadrants][2 item parities]
   static constexpr int kNumBars = 2 * kHtStages + 2 * kHtAcc + 4 + 1 + 8;
-  // [2 item parities][2 tile halves][128 lanes] x (max, sum): the two warps of a lane
-  // quadrant combine their halves' running softmax state at the end of pass 1
+  // [2 item parities][4 tile parts][128 lanes] x (max, sum): the four warps of a lane
+  // quadrant combine their parts' running softmax state at the end of pass 1
   static constexpr size_t kComb = kBars + kNumBars * 8 + 16;
-  static constexpr size_t need = 1024 + kComb + 2 * 2 * kHtLanes * 8;
+  static constexpr size_t need = 1024 + kComb + 2 * 4 * kHtLanes * 8;
   // at least half of the SM's shared memory, so that one CTA per SM holds all 512 TMEM
   // columns (a second CTA's allocation would wait for the first to finish)
   static constexpr size_t bytes = need > 120 * 1024 ? need : 120 * 1024;
@@ -137,18 +137,26 @@ struct HtGeom {
 // (G / 2, G / 4, .., 1) adds the partner's half of the N values the lane still holds and
 // keeps the half selected by (lane & d); lane g of the group ends with the sums of
 // entries g * N / G .. (g + 1) * N / G - 1 in s[0 ..].
+// When G > N the last steps have one value left: lanes d apart add theirs (both keep
+// the sum), so lanes g and g ^ d .. hold the same entry (entry g * N / G rounded down).
 template <int G, int N>
-__device__ __forceinline__ void ht_reduce_scatter(float (&s)[kHtHalf], int lane) {
+__device__ __forceinline__ void ht_reduce_scatter(float (&s)[kHtPart], int lane) {
   if constexpr (G > 1) {
-    constexpr int d = G / 2, half = N / 2;
-    const bool upper = (lane & d) != 0;
+    constexpr int d = G / 2;
+    if constexpr (N > 1) {
+      constexpr int half = N / 2;
+      const bool upper = (lane & d) != 0;
 #pragma unroll
-    for (int x = 0; x < half; ++x) {
-      const float send = upper ? s[x] : s[x + half];
-      const float keep = upper ? s[x + half] : s[x];
-      s[x] = keep + __shfl_xor_sync(0xffffffffu, send, d);
+      for (int x = 0; x < half; ++x) {
+        const float send = upper ? s[x] : s[x + half];
+        const float keep = upper ? s[x + half] : s[x];
+        s[x] = keep + __shfl_xor_sync(0xffffffffu, send, d);
+      }
+      ht_reduce_scatter<d, half>(s, lane);
+    } else {
+      s[0] += __shfl_xor_sync(0xffffffffu, s[0], d);
+      ht_reduce_scatter<d, 1>(s, lane);
     }
-    ht_reduce_scatter<d, half>(s, lane);
   }
 }
 
@@ -191,7 +199,7 @@ select_hsm_tc_kernel(const __nv_bfloat16* __restrict__ q, sala_strides sq,
       mbar_init(&a_free[i], 1);
     }
     mbar_init(drain, 1);
-    for (int i = 0; i < 8; ++i) mbar_init(&pair[i], 64);
+    for (int i = 0; i < 8; ++i) mbar_init(&pair[i], 4 * 32);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -317,13 +325,15 @@ select_hsm_tc_kernel(const __nv_bfloat16* __restrict__ q, sala_strides sq,
       geo.next(c);
     }
   } else {
-    // ================= consumers: thread (l, half) with l = (row l / G, head l % G)
-    const int quad = warp & 3, half = warp >> 2;
+    // ================= consumers: thread (l, part) with l = (row l / G, head l % G)
+    const int quad = warp & 3, part = warp >> 2;
     const int l = 32 * quad + (tid & 31);
     const int rrow = l / G, gl = l % G;  // row within the item, lane within the row's group
     const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
-    constexpr int per = kHtHalf / G;     // candidates each lane stores per tile half
-    float2* comb = reinterpret_cast<float2*>(smem + L::kComb);  // [parity][half][lane]
+    // after the reduce-scatter: `per` sums per lane, shared by `rep` lanes
+    constexpr int per = kHtPart / G > 0 ? kHtPart / G : 1;
+    constexpr int rep = G / kHtPart > 0 ? G / kHtPart : 1;
+    float2* comb = reinterpret_cast<float2*>(smem + L::kComb);  // [parity][part][lane]
     HtCursor c;
     geo.begin(c);
     int g = 0;
@@ -345,50 +355,57 @@ select_hsm_tc_kernel(const __nv_bfloat16* __restrict__ q, sala_strides sq,
         break;
       }
       tc_fence_after();
-      uint32_t sh[kHtHalf], sm[kHtHalf], sl[kHtHalf];  // q.hi, q.mid, q.lo
-      const uint32_t col = tD + 3 * kHtN * ab + kHtHalf * half + lane_off;
-      tc_ld32(col, sh);
-      tc_ld32(col + kHtN, sm);
-      tc_ld32(col + 2 * kHtN, sl);
+      uint32_t sh[kHtPart], sm[kHtPart], sl[kHtPart];  // q.hi, q.mid, q.lo
+      const uint32_t col = tD + 3 * kHtN * ab + kHtPart * part + lane_off;
+      tc_ld16(col, sh);
+      tc_ld16(col + kHtN, sm);
+      tc_ld16(col + 2 * kHtN, sl);
       tc_wait_ld();
       tc_fence_before();
       __syncwarp();
       if ((tid & 31) == 0) mbar_arrive(&acc_free[ab]);
-      const int j0 = geo.n_init + c.i * kHtN + kHtHalf * half;  // this half's first candidate
-      float s[kHtHalf];  // scores, log2 domain (-inf: not a candidate of the row)
+      const int j0 = geo.n_init + c.i * kHtN + kHtPart * part;  // this part's first candidate
+      float s[kHtPart];  // scores, log2 domain (-inf: not a candidate of the row)
 #pragma unroll
-      for (int x = 0; x < kHtHalf; ++x)
+      for (int x = 0; x < kHtPart; ++x)
         s[x] = (__uint_as_float(sl[x]) + __uint_as_float(sm[x])) + __uint_as_float(sh[x]);
-      if (j0 + kHtHalf - 1 > jmax) {  // the row's candidates end inside this half tile
+      if (j0 + kHtPart - 1 > jmax) {  // the row's candidates end inside this part
 #pragma unroll
-        for (int x = 0; x < kHtHalf; ++x) s[x] = j0 + x <= jmax ? s[x] : -INFINITY;
+        for (int x = 0; x < kHtPart; ++x) s[x] = j0 + x <= jmax ? s[x] : -INFINITY;
       }
       if (c.pass == 0) {
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int x = 0; x < kHtHalf; ++x) mx[x & 3] = fmaxf(mx[x & 3], s[x]);
+        for (int x = 0; x < kHtPart; ++x) mx[x & 3] = fmaxf(mx[x & 3], s[x]);
         const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
         if (mt > -INFINITY) {
           const float mn = fmaxf(m, mt);
           float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int x = 0; x < kHtHalf; ++x) acc[x & 3] += ht_exp2(s[x] - mn);  // exp2(-inf) = 0
+          for (int x = 0; x < kHtPart; ++x) acc[x & 3] += ht_exp2(s[x] - mn);  // exp2(-inf) = 0
           lsum = lsum * ht_exp2(m - mn) + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
           m = mn;
         }
         if (c.i == c.ntiles - 1) {
-          // merge with the other half's (max, sum) of the same lane
+          // merge the four parts' (max, sum) of the same lane, in part order (so the
+          // four threads compute the same values)
           const int par = c.u & 1;
-          comb[(par * 2 + half) * kHtLanes + l] = make_float2(m, lsum);
+          comb[(par * 4 + part) * kHtLanes + l] = make_float2(m, lsum);
           mbar_arrive(&pair[quad * 2 + par]);
           const bool merged = mbar_wait(&pair[quad * 2 + par], (c.u >> 1) & 1);
           if (__any_sync(0xffffffffu, !merged)) {  // leave the loop as a whole warp
             ok = false;
             break;
           }
-          const float2 o = comb[(par * 2 + (half ^ 1)) * kHtLanes + l];
-          const float ma = fmaxf(m, o.x);
-          const float la = ma == -INFINITY ? 0.f : lsum * ht_exp2(m - ma) + o.y * ht_exp2(o.x - ma);
+          float2 o[4];
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) o[q4] = comb[(par * 4 + q4) * kHtLanes + l];
+          const float ma = fmaxf(fmaxf(o[0].x, o[1].x), fmaxf(o[2].x, o[3].x));
+          float la = 0.f;
+          if (ma != -INFINITY) {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) la += o[q4].y * ht_exp2(o[q4].x - ma);
+          }
           // p = exp2(s - ma) / la = exp2(s - mp); -inf marks a row without candidates
           mp = la > 0.f ? ma + log2f(la) : -INFINITY;
         }
@@ -396,17 +413,18 @@ select_hsm_tc_kernel(const __nv_bfloat16* __restrict__ q, sala_strides sq,
         // p (exp2(-inf) = 0 for candidates outside the row; all 0 for a row without any)
         if (mp == -INFINITY) {
 #pragma unroll
-          for (int x = 0; x < kHtHalf; ++x) s[x] = 0.f;
+          for (int x = 0; x < kHtPart; ++x) s[x] = 0.f;
         } else {
 #pragma unroll
-          for (int x = 0; x < kHtHalf; ++x) s[x] = ht_exp2(s[x] - mp);
+          for (int x = 0; x < kHtPart; ++x) s[x] = ht_exp2(s[x] - mp);
         }
-        ht_reduce_scatter<G, kHtHalf>(s, l);
-        // lane gl of the row holds candidates j0 + gl * per .. j0 + gl * per + per - 1
-        if (live) {
+        ht_reduce_scatter<G, kHtPart>(s, l);
+        // lane gl of the row holds candidates j0 + (gl / rep) * per .. + per - 1 (the
+        // first of each `rep` lanes that share them stores)
+        if (live && gl % rep == 0) {
           float* srow = scores + (((int64_t)c.b * geo.Hkv + c.hk) * rows_pass + (t - geo.r0)) *
                                      (int64_t)geo.nb;
-          const int jb = j0 + gl * per;
+          const int jb = j0 + (gl / rep) * per;
 #pragma unroll
           for (int x = 0; x < per; ++x)
             if (jb + x <= jmax &&
