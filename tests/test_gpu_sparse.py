@@ -254,3 +254,23 @@ def test_sparse_kvhead_parallel_single_rank_group():
     finally:
         dist.destroy_process_group()
     assert sala.get_device_error() == 0
+
+
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 127, 4288, 4289])
+def test_select_and_attn_edge_lengths(T):
+    """Sequence lengths at block and budget edges (one token; one block -1, 0, +1; the
+    dense-fallback limit 67 x 64 and one past it), two sequences, gated, selection and
+    attention against the oracle."""
+    B, Hq, Hkv, D, topk = 2, 16, 2, 128, 64
+    s = inputs.sparse_inputs(B, T, Hq, Hkv, D, seed=700 + T, gate=True)
+    dq, dk, dv, dg = (x.cuda() for x in (s.q, s.k, s.v, s.g))
+    idx = sala.sparse_select(dq, dk, topk=topk)
+    rows = np.arange(T) if T <= 512 else _sampled_rows(T, n_mid=256, seed=T)
+    ref, gap, sc = oracle.sparse_select(_np(s.q[:, rows]), _np(s.k), topk=topk, rows=rows,
+                                        want_scores=True)
+    check_index_sets(idx.cpu().numpy()[:, :, rows], ref, gap, sc, rows, topk=topk)
+    o = sala.sparse_attn(dq, dk, dv, idx, dg)
+    want = oracle.attention(_np(s.q[:, rows]), _np(s.k), _np(s.v), _np(s.g[:, rows]),
+                            idx=idx.cpu().numpy()[:, :, rows], rows=rows)
+    assert rel_err(_np(o[:, rows]), want, True) <= TOL_BF16
+    assert sala.get_device_error() == 0
