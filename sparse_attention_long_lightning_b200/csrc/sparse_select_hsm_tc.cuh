@@ -3,11 +3,10 @@
 // The per-head selection variant (MiniCPM-SALA tech-report mirror, section 02 (2): the
 // selection score is left open; this variant softmax-normalises each query head's
 // scores before the GQA group sums them):
-//   s_{h,j}  = (1/sqrt(D)) q_{t,h} . Kbar_j          h in group(hk), n_init <= j <= c - n_local
+//   s_{h,j}  = (1/sqrt(D)) q_{t,h} . Kbar_j        h in group(hk), n_init <= j <= c - n_local
 //   p_{h,j}  = exp(s_{h,j} - m_h) / sum_{j'} exp(s_{h,j'} - m_h),   m_h = max_j s_{h,j}
 //   score_j  = sum_{h in group(hk)} p_{h,j}
-// written into the same fp32 score scratch as block_scores_hsm_kernel, from which
-// topk_select_kernel picks the top-k.
+// written into the fp32 score scratch from which topk_select_kernel picks the top-k.
 //
 // Design (sm_100a).  An item is R = 128 / G consecutive query rows of one KV head: its
 // R x G (query row, head) pairs are the M = 128 rows of the MMAs, so TMEM lane l =
@@ -15,16 +14,17 @@
 // operand (q as stored: bf16 is exact) sits in TMEM, so the MMAs of a tile read only the
 // block means from shared memory.  The block means times log2(e)/sqrt(D) (one fp32
 // rounding: the scores come out in the log2 domain of the exponentials) are split into
-// three bf16 parts hi + mid + lo = that value exactly (8 significant bits each); a tile's three parts are
-// stacked as the N = 192 rows of the B operand, so 8 MMAs (D = 128) give q.hi, q.mid and
-// q.lo side by side in TMEM and the consumers form S = (q.lo + q.mid) + q.hi: the fp32
-// dot product up to the summation order (fewer, wider MMAs: each MMA instruction has a
-// fixed cost that N = 64 products did not cover).  Every item is scored twice: pass 1 keeps each thread's
-// running maximum and sum of exponentials (online, in registers: no cross-thread work),
-// pass 2 recomputes S, forms p = exp(s - m) / l, and the G threads of a query row sum
-// their heads' p by a butterfly reduce-scatter (after which lane g of the row's group
-// holds the sums of candidates g * 64/G .. (g + 1) * 64/G - 1 of the tile) and store
-// them, coalesced, into the scratch row.
+// three bf16 parts hi + mid + lo = that value exactly (8 significant bits each).  A
+// tile's three parts are stacked as the N = 192 rows of the B operand, so 8 MMAs
+// (D = 128) give q.hi, q.mid and q.lo side by side in TMEM and the consumers form
+// S = (q.lo + q.mid) + q.hi: the fp32 dot product up to the summation order (fewer,
+// wider MMAs: each MMA instruction has a fixed cost that N = 64 products did not cover).
+// Every item is scored twice: pass 1 keeps each thread's running maximum and sum of
+// exponentials (online, in registers), pass 2 recomputes S, forms
+// p = exp2(s - (m + log2 l)), and the G threads of a query row sum their heads' p by a
+// butterfly reduce-scatter over the thread's 16 candidates (lane g of the row's group
+// ends with the sums of 16 / G of them, or shares one with G / 16 - 1 other lanes when
+// G = 32) and store them, coalesced, into the scratch row.
 //   producers (warps 17-20): thread l loads lane l's query-head row of the next item
 //     and stores it into its TMEM lane (two A buffers), overlapping the current item;
 //   copier (warp 21, one thread): TMA of the block-mean tiles (4-stage ring, hi / mid /
@@ -35,7 +35,7 @@
 //     (per-warp arrival), then the pass's arithmetic; at the end of pass 1 the four
 //     threads of a lane merge their parts' (max, sum) through shared memory in a fixed
 //     order (a bounded mbarrier wait, per item parity), so pass 2 normalises with the
-//     row's full sum.  Four warps per scheduler hide each other's latency.
+//     row's full sum.
 // All waits are bounded: a wait that runs out raises SALA_ERR_TIMEOUT, and the kernel
 // drains its copies and MMAs before it frees TMEM and returns.
 #pragma once
