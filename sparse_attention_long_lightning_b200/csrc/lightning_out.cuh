@@ -177,7 +177,9 @@ __device__ __forceinline__ void lo_store32(const uint32_t (&r)[32], const uint4*
 // S [384,512).
 // kPrepared: q and k arrive already normalised and rotated as fp16 and the gate tensor
 // holds sigmoid(g) as fp16 (the projection epilogue's outputs), so the PREP warps only
-// convert v.
+// convert v; they then also write each chunk's gated output (reading O from TMEM with the
+// CONV warps' lane mapping), which takes that phase off the CONV warps: O buffer x is
+// handed back through o_free[x], and the chunk's S-operand exponent arrives in e_ring[x].
 template <bool kPrepared>
 __global__ void __launch_bounds__(kTcThreads, 1)
 lightning_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
@@ -207,6 +209,14 @@ lightning_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
   volatile int* conv_abort = reinterpret_cast<volatile int*>(misc + 108);
   float* red = reinterpret_cast<float*>(misc + 112);           // [16]
   double* inv_freq = reinterpret_cast<double*>(misc + 192);    // [64]
+  // prepared operands only: the PREP warps write each chunk's output, so O buffer x is
+  // handed back (o_free[x], count 8), P V of the chunk in O buffer x has its own barrier
+  // (mma2b[x]), and the S-operand exponent of the chunk reaches them through e_ring[x]
+  // (e_ready[x])
+  uint64_t* o_free = reinterpret_cast<uint64_t*>(misc + 704);  // [2]
+  uint64_t* mma2b = o_free + 2;                                // [2]
+  uint64_t* e_ready = o_free + 4;                              // [2]
+  int* e_ring = reinterpret_cast<int*>(misc + 752);            // [2]
   // [2][32]: (base angle, inv_freq) of rotation pairs i, i + 1 at item lo_ang_item(i)
   __shared__ float4 ang_tab[2 * 32];
 
@@ -237,6 +247,13 @@ lightning_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
     mbar_init(mma1_bar, 1);
     mbar_init(mma2_bar, 1);
     mbar_init(drain_bar, 1);
+    if constexpr (kPrepared) {
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&o_free[i], kLoPrepThreads / 32);
+        mbar_init(&mma2b[i], 1);
+        mbar_init(&e_ready[i], 1);
+      }
+    }
     smax[0] = smax[1] = 0u;
     *prep_abort = 0;
     *conv_abort = 0;
@@ -345,6 +362,38 @@ lightning_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
     // ------------------------------------------------------------------ PREP
     const int prow = tid >> 1, phf = tid & 1;
     bool fail = false;
+    // prepared operands: PREP only converts v, so it also writes the gated output of each
+    // chunk (TMEM lane row prow_o, columns 64 * pch ..), which the CONV warps otherwise do
+    const int prow_o = 32 * (warp & 3) + lane, pch = warp >> 2;
+    const uint32_t plane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    auto output_chunk = [&](int uu) -> bool {
+      const int ob = uu & 1;
+      const int64_t t = (int64_t)(c_begin + uu) * kTcC + prow_o;
+      uint4 gq[8] = {};
+      if (p.g != nullptr && t < p.T) {
+        const uint4* gp = reinterpret_cast<const uint4*>(p.g + b * p.sg.b + t * p.sg.t +
+                                                         (int64_t)h * p.sg.h + 64 * pch);
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) gq[c8] = __ldg(gp + c8);
+      }
+      if (!mbar_wait(&mma2b[ob], (uu >> 1) & 1) || !mbar_wait(&e_ready[ob], (uu >> 1) & 1))
+        return false;
+      tc_fence_after();
+      const float os = pow2i(e_ring[ob]) * oscale;
+      __nv_bfloat16* orow = p.o + b * p.so.b + t * p.so.t + (int64_t)h * p.so.h + 64 * pch;
+      const uint32_t t_o = t_o0 + 128 * ob + plane_off + 64 * pch;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t r[32];
+        tc_ld32(t_o + 32 * hh, r);
+        tc_wait_ld();
+        if (t < p.T) lo_store32<kPrepared>(r, gq + 4 * hh, p.g != nullptr, os, orow + 32 * hh, bad);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_free[ob]);  // O buffer ob may take chunk uu + 2
+      return true;
+    };
     for (int u = 0; u < nchunks; ++u) {
       const int s = u & 1;
       uint8_t* st = stages + s * L::kStageBytes;
@@ -358,8 +407,14 @@ lightning_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
       __syncwarp();
       if (lane == 0) mbar_arrive(&prep_done[s]);
       if (u + 1 < nchunks) fill_angles(u + 1);  // the other table; its last reader was prep(u-1)
+      if constexpr (kPrepared) {
+        if (u > 0 && !fail) fail = !output_chunk(u - 1);
+      }
       if (fail) *prep_abort = 1;
       if (named_bar_or(2, kLoPrepThreads, fail) && *prep_abort) break;
+    }
+    if constexpr (kPrepared) {
+      if (nchunks > 0 && !*prep_abort && !output_chunk(nchunks - 1)) *prep_abort = 1;
     }
   } else {
     // ------------------------------------------------------------------ CONV
@@ -379,8 +434,17 @@ lightning_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
         smax[(u + 1) & 1] = 0u;  // last read before the previous barrier; next written below
         // operands prepared; P V of chunk u-1 (which reads the TMEM columns the score MMA
         // overwrites) has completed
-        const bool ok = mbar_wait(&prep_done[s], (u >> 1) & 1) &&
-                        (u == 0 || mbar_wait(mma2_bar, (u - 1) & 1));
+        bool ok = mbar_wait(&prep_done[s], (u >> 1) & 1) &&
+                  (u == 0 || mbar_wait(mma2_bar, (u - 1) & 1));
+        if constexpr (kPrepared) {
+          // O buffer s held chunk u - 2, whose output the PREP warps write; then the
+          // exponent of this chunk's S operand for that output
+          ok = ok && (u < 2 || mbar_wait(&o_free[s], ((u - 2) >> 1) & 1));
+          if (ok) {
+            e_ring[s] = e_cur;
+            mbar_arrive(&e_ready[s]);
+          }
+        }
         fail |= !ok;
         if (ok) {
           tc_fence_after();
@@ -398,7 +462,12 @@ lightning_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
         }
       }
       // ---- output of chunk u-1 once its P V has landed; refill its stage with chunk u+1
-      if (u > 0) {
+      if (u > 0 && kPrepared) {
+        fail |= !mbar_wait(mma2_bar, (u - 1) & 1);
+        tc_fence_after();
+        if (iss && !fail && v_issued < nchunks) issue_v(v_issued++);  // v of chunk u-1 is free
+      }
+      if (u > 0 && !kPrepared) {
         fail |= !mbar_wait(mma2_bar, (u - 1) & 1);
         tc_fence_after();
         if (iss && !fail && v_issued < nchunks) issue_v(v_issued++);  // v of chunk u-1 is free
@@ -414,7 +483,7 @@ lightning_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
                               bad);
         }
       }
-      {
+      if (!kPrepared) {
         // gate of chunk u for its output (next iteration)
         const int64_t t = (int64_t)(c_begin + u) * kTcC + trow;
         if (gated && t < p.T) {
@@ -475,6 +544,7 @@ lightning_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
         for (int kk = 0; kk < 8; ++kk)
           tc_mma_ts(t_o, t_p + 8 * kk + (kk >= 4 ? 32 : 0), tc_desc_mn(sV, kk), kIdPV, 1u);
         tc_commit(mma2_bar);
+        if constexpr (kPrepared) tc_commit(&mma2b[s]);  // the PREP warps' output of chunk u
       }
       e_prev = e_cur;
       // ---- S(u) -> fp16 operand of chunk u+1 (its last reader, Qh S_op of chunk u, is done)
@@ -505,8 +575,8 @@ lightning_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
       tc_fence_before();
       named_bar_sync(1, kLoConvThreads);  // S operand written, output reads of O done
     }
-    // ---- output of the last chunk
-    if (nchunks > 0 && !*conv_abort) {
+    // ---- output of the last chunk (the PREP warps write it for prepared operands)
+    if (!kPrepared && nchunks > 0 && !*conv_abort) {
       const int u = nchunks;
       const bool ok = mbar_wait(mma2_bar, (u - 1) & 1);
       tc_fence_after();
